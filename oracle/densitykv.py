@@ -1,0 +1,256 @@
+"""DensityKV online bank update, one (layer) admit step at a time, fp64.
+
+Follows DensityKV App. B.1 "Online Bank Update", §3 "Online Density-Constrained
+Bank Update" and App. E (default policy), in the pages' order:
+
+1. every head keeps its own bank of exact (id, key, value) entries, at most M
+   (App. B.1; App. D: independent layer-head banks, M = 9,360);
+2. the finalised block's tokens are candidates; each is scored by its density
+   against the head's bank, normalised by the mean of the bank's frozen
+   insertion baselines ("mean-normalised insertion disturbance", lower first;
+   App. E candidate ordering);
+3. the admitted count P is the largest prefix feasible for every head of the
+   layer (synchronised admission, App. E cross-head synchronisation); each head
+   admits its own P lowest-scoring candidates;
+4. bank entries whose projected density ratio crosses tau are evicted first
+   (threshold-first eviction, App. E); capacity eviction then removes the
+   highest-ratio entries until the bank fits M (§3, "mandatory or highest-density
+   states until capacity is released");
+5. co-admitted candidates set their insertion baselines together, after the
+   update (App. B.1: mutual interactions among the admitted block do not reject
+   one another; only growth from later blocks counts); baselines of older entries
+   stay frozen (App. E: fixed insertion-time references).
+
+Readings taken where the pages are silent (each is a parameter or a plain choice):
+
+* density: ``oracle.density`` (phi = (||a-b||^2/h + eps)^(-s/2), self excluded by id);
+* disturbance score of candidate c in head h: rho_B(c) / mean_{i in B} rho0_i;
+  candidate feasible iff score <= tau; if the bank is empty or its mean baseline
+  is 0, every candidate is feasible with score 0;
+* the prefix is ordered by (score ascending, id ascending);
+* P = min(min_h P_h, M, N) with P_h the number of feasible candidates of head h
+  (``sync_heads=False``: each head uses its own min(P_h, M, N));
+* projected ratio of entry i: (rho_i + sum_{c in A_h} phi(c, i)) / rho0_i, with
+  rho_i its density within the current bank; ratio 0 when rho0_i = 0;
+  mandatory iff ratio > tau;
+* capacity evictions E_cap = max(0, |B| - |mandatory| + P - M) among the
+  non-mandatory entries, by (ratio descending, id ascending: older first);
+* after the update every density is recomputed from scratch over the new bank;
+  new entries take rho0 = that density.
+
+Nothing here is incremental: the CUDA path's incremental maintenance (App. B.1:
+"exact update in O(N M d_k)") is checked against these from-scratch values.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import List, Optional
+
+import numpy as np
+
+from .density import density
+
+
+@dataclasses.dataclass
+class Params:
+    capacity: int
+    tau: float = 2.0
+    eps: float = 1e-3
+    s: float = 2.0
+    h: float = 0.0           # distance scale; 0 => head_dim
+    sync_heads: bool = True
+
+    def scale(self, d: int) -> float:
+        return float(self.h) if self.h > 0 else float(d)
+
+
+@dataclasses.dataclass
+class HeadBank:
+    ids: np.ndarray          # int64 [n]
+    K: np.ndarray            # float64 [n][d]
+    V: np.ndarray            # float64 [n][d]
+    rho0: np.ndarray         # float64 [n] frozen insertion baselines
+
+    @staticmethod
+    def empty(d: int) -> "HeadBank":
+        return HeadBank(np.zeros(0, np.int64), np.zeros((0, d)), np.zeros((0, d)), np.zeros(0))
+
+    @property
+    def size(self) -> int:
+        return int(self.ids.shape[0])
+
+
+@dataclasses.dataclass
+class AdmitResult:
+    banks: List[HeadBank]
+    P: int
+    P_h: np.ndarray                  # feasible count per head
+    rho_cand: List[np.ndarray]       # rho_B(c) per head, [N]
+    score: List[np.ndarray]          # disturbance score per head, [N]
+    admitted: List[np.ndarray]       # candidate indices admitted per head (selection order)
+    rho_cur: List[np.ndarray]        # density of old entries within the old bank
+    proj: List[np.ndarray]           # sum over admitted of phi(c, i), per old entry
+    ratio: List[np.ndarray]          # projected ratio per old entry
+    mandatory: List[np.ndarray]      # bool per old entry
+    evicted: List[np.ndarray]        # bool per old entry (mandatory or capacity)
+    n_capacity: np.ndarray           # capacity evictions per head
+    rho_new: List[np.ndarray]        # from-scratch density of the new bank entries
+    near_ties: int                   # decisions with relative margin < tie_margin
+    margins: dict
+
+
+def _lex_order(primary: np.ndarray, ids: np.ndarray) -> np.ndarray:
+    """Indices sorted by (primary ascending, id ascending)."""
+    return np.lexsort((np.asarray(ids), np.asarray(primary)))
+
+
+def admit(banks: List[HeadBank], cand_ids: np.ndarray, candK: np.ndarray, candV: np.ndarray,
+          p: Params, tie_margin: float = 1e-4) -> AdmitResult:
+    """One admit step for one layer.  candK/candV [H][N][d] (storage precision)."""
+    H = len(banks)
+    cand_ids = np.asarray(cand_ids, dtype=np.int64)
+    N = cand_ids.shape[0]
+    d = candK.shape[-1]
+    h = p.scale(d)
+    kw = dict(h=h, eps=p.eps, s=p.s)
+    M = p.capacity
+
+    # -- step 2: candidate densities against the bank, disturbance scores ------------
+    rho_cand, score, feas = [], [], []
+    for hh in range(H):
+        b = banks[hh]
+        rc = density(candK[hh], b.K, row_ids=cand_ids, col_ids=b.ids, **kw)
+        mean0 = float(b.rho0.mean()) if b.size else 0.0
+        sc = rc / mean0 if mean0 > 0 else np.zeros(N)
+        rho_cand.append(rc)
+        score.append(sc)
+        feas.append(sc <= p.tau)
+    P_h = np.array([int(f.sum()) for f in feas])
+
+    # -- step 3: largest feasible prefix, synchronised across heads --------------------
+    if p.sync_heads:
+        P_all = [int(min(P_h.min(), M, N))] * H
+    else:
+        P_all = [int(min(P_h[hh], M, N)) for hh in range(H)]
+    admitted = []
+    for hh in range(H):
+        order = _lex_order(score[hh], cand_ids)
+        admitted.append(order[:P_all[hh]])
+
+    # -- step 4: projected growth, threshold-first and capacity eviction ---------------
+    rho_cur, proj, ratio, mand, evicted, n_cap = [], [], [], [], [], []
+    for hh in range(H):
+        b = banks[hh]
+        A = admitted[hh]
+        rcur = density(b.K, b.K, row_ids=b.ids, col_ids=b.ids, **kw)
+        pj = density(b.K, candK[hh][A], row_ids=b.ids, col_ids=cand_ids[A], **kw)
+        rhat = rcur + pj
+        with np.errstate(divide="ignore", invalid="ignore"):
+            rt = np.where(b.rho0 > 0, rhat / np.where(b.rho0 > 0, b.rho0, 1.0), 0.0)
+        md = rt > p.tau
+        ecap = max(0, b.size - int(md.sum()) + len(A) - M)
+        ev = md.copy()
+        if ecap:
+            rest = np.nonzero(~md)[0]
+            order = _lex_order(-rt[rest], b.ids[rest])
+            ev[rest[order[:ecap]]] = True
+        rho_cur.append(rcur)
+        proj.append(pj)
+        ratio.append(rt)
+        mand.append(md)
+        evicted.append(ev)
+        n_cap.append(ecap)
+
+    # -- step 5: new bank, baselines of co-admitted entries set together ---------------
+    new_banks, rho_new = [], []
+    for hh in range(H):
+        b = banks[hh]
+        keep = ~evicted[hh]
+        A = admitted[hh]
+        ids = np.concatenate([b.ids[keep], cand_ids[A]])
+        K = np.concatenate([b.K[keep], np.asarray(candK[hh][A], np.float64)])
+        V = np.concatenate([b.V[keep], np.asarray(candV[hh][A], np.float64)])
+        rn = density(K, K, row_ids=ids, col_ids=ids, **kw)
+        n_old = int(keep.sum())
+        rho0 = np.concatenate([b.rho0[keep], rn[n_old:]])
+        new_banks.append(HeadBank(ids, K, V, rho0))
+        rho_new.append(rn)
+
+    margins = _margins(p, score, P_h, P_all, admitted, ratio, mand, evicted, n_cap, banks, cand_ids)
+    near = sum(int((m < tie_margin).sum()) for m in margins.values())
+    return AdmitResult(new_banks, P_all[0] if p.sync_heads else -1, P_h, rho_cand, score, admitted,
+                       rho_cur, proj, ratio, mand, evicted, np.array(n_cap), rho_new, near, margins)
+
+
+def _rel(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    with np.errstate(invalid="ignore"):
+        r = np.abs(a - b) / np.maximum(np.abs(b), 1e-300)
+    return np.where(np.isnan(r), np.inf, r)
+
+
+def _margins(p, score, P_h, P_all, admitted, ratio, mand, evicted, n_cap, banks, cand_ids):
+    """Relative margins of every decision that a rounding difference could flip.
+
+    * admission threshold: |score - tau| / tau for each candidate;
+    * admission cut (when P is below a head's feasible count): relative gap between
+      the last admitted and the first rejected score of that head;
+    * eviction threshold: |ratio - tau| / tau per bank entry;
+    * capacity cut: relative gap between the last capacity-evicted and the first
+      kept non-mandatory ratio."""
+    out = {"adm_thr": [], "adm_cut": [], "ev_thr": [], "ev_cut": []}
+    for hh in range(len(score)):
+        if banks[hh].size and banks[hh].rho0.mean() > 0:
+            out["adm_thr"].append(_rel(score[hh], p.tau))
+        P = P_all[hh]
+        if 0 < P < int(P_h[hh]):
+            order = _lex_order(score[hh], cand_ids)
+            a, b = score[hh][order[P - 1]], score[hh][order[P]]
+            out["adm_cut"].append(np.array([_rel(b, a) if a != 0 else 1.0]))
+        if banks[hh].size:
+            out["ev_thr"].append(_rel(ratio[hh], p.tau))
+        if n_cap[hh] > 0:
+            rest = np.nonzero(~mand[hh])[0]
+            order = _lex_order(-ratio[hh][rest], banks[hh].ids[rest])
+            if n_cap[hh] < rest.size:
+                a = ratio[hh][rest[order[n_cap[hh] - 1]]]
+                b = ratio[hh][rest[order[n_cap[hh]]]]
+                out["ev_cut"].append(np.array([_rel(b, a) if a != 0 else 1.0]))
+    return {k: (np.concatenate(v) if v else np.zeros(0)) for k, v in out.items()}
+
+
+def densities_from_scratch(bank: HeadBank, p: Params) -> np.ndarray:
+    d = bank.K.shape[-1]
+    return density(bank.K, bank.K, row_ids=bank.ids, col_ids=bank.ids, h=p.scale(d), eps=p.eps, s=p.s)
+
+
+def attention_set(bank: HeadBank, sinkK, sinkV, winK, winV):
+    """K/V read by the current chunk: [sink | bank | local window] (DensityKV Fig. 2)."""
+    K = np.concatenate([np.asarray(sinkK, np.float64), bank.K, np.asarray(winK, np.float64)])
+    V = np.concatenate([np.asarray(sinkV, np.float64), bank.V, np.asarray(winV, np.float64)])
+    return K, V
+
+
+def rollout(layer_inputs, p: Params, steps: int, attend: bool = True, tie_margin: float = 1e-4,
+            on_step: Optional[callable] = None):
+    """Run admit (+ attention) for steps 1..steps of one layer; returns per-step results."""
+    from .attention import attention
+    w = layer_inputs.w
+    H = len(layer_inputs.heads)
+    banks = [HeadBank.empty(w.head_dim) for _ in range(H)]
+    results = []
+    for i in range(1, steps + 1):
+        x = layer_inputs.step(i)
+        r = admit(banks, x["cand_ids"], x["candK"], x["candV"], p, tie_margin)
+        banks = r.banks
+        outs = None
+        if attend:
+            outs = []
+            for hh in range(H):
+                K, V = attention_set(banks[hh], x["sinkK"][hh], x["sinkV"][hh], x["winK"][hh], x["winV"][hh])
+                outs.append(attention(x["Q"][hh], K, V))
+        rec = {"step": i, "admit": r, "attn": outs, "inputs": x}
+        if on_step is not None:
+            on_step(rec)
+        results.append(rec)
+    return results

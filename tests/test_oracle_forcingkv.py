@@ -1,0 +1,116 @@
+"""Pins of the oracle's Forcing-KV hybrid prune (reading notes §3.3, §3.4, §3.5).
+
+Hand-built frames with known cosines, partition counts of the 4x4 segmentation of
+a 30x52 frame, the r = 1 and identical-frame special cases, the static-head set
+[sink, transition, current chunk] and the FIFO length of the dynamic history."""
+import math
+
+import numpy as np
+import pytest
+
+import kvgen
+from oracle import forcingkv as fkv
+
+
+def test_segment_partition_480p():
+    segs = fkv.segments(30, 52, 4, 4)
+    assert len(segs) == 8 * 13 == 104
+    sizes = np.array([s.size for s in segs])
+    assert (sizes == 16).sum() == 91 and (sizes == 8).sum() == 13
+    allt = np.sort(np.concatenate(segs))
+    np.testing.assert_array_equal(allt, np.arange(1560))
+    # segment 0 = rows 0..3, cols 0..3 in row-major order
+    np.testing.assert_array_equal(segs[0], [0, 1, 2, 3, 52, 53, 54, 55, 104, 105, 106, 107, 156, 157, 158, 159])
+    assert fkv.keep_count(104, 0.7) == 72      # floor(72.8)
+    assert fkv.keep_count(6, 0.3) == 1         # the pages' default n=6, r=0.3
+    assert fkv.keep_count(104, 1.0) == 104
+
+
+def test_hand_built_cosines_and_bottom_k():
+    # frame 2 x 4 tokens, 2 x 2 segments -> segment 0 = tokens {0,1,4,5}, segment 1 = {2,3,6,7}
+    Kt = np.array([[1, 0]] * 8, dtype=np.float64)
+    Kn = Kt.copy()
+    Kn[[2, 3, 6, 7]] = [0, 1]                     # segment 1 turns 90 degrees: cos 0
+    Kn[[0]] = [1, 1]                              # one token of segment 0 at 45 degrees
+    segs = fkv.segments(2, 4, 2, 2)
+    np.testing.assert_array_equal(segs[1], [2, 3, 6, 7])
+    sim = fkv.segment_similarity(Kt, Kn, segs)
+    assert sim[0] == pytest.approx((3 + 1 / math.sqrt(2)) / 4, rel=1e-14)
+    assert sim[1] == pytest.approx(0.0, abs=1e-15)
+    # the least similar segment is kept
+    np.testing.assert_array_equal(fkv.bottom_k(sim, 1), [1])
+    # opposite direction counts as least similar (cos -1)
+    Kn2 = Kt.copy()
+    Kn2[[0, 1, 4, 5]] = [-2, 0]
+    sim2 = fkv.segment_similarity(Kt, Kn2, segs)
+    np.testing.assert_allclose(sim2, [-1.0, 1.0], rtol=1e-15)
+    np.testing.assert_array_equal(fkv.bottom_k(sim2, 1), [0])
+    # zero-norm tokens give cos 0 (norm product clamped), not NaN
+    assert fkv.token_cosine(np.zeros((1, 2)), np.ones((1, 2)))[0] == 0.0
+
+
+def test_bottom_k_ties_take_lower_index_and_sorted_output():
+    sim = np.array([0.5, 0.2, 0.5, 0.2, 0.9])
+    np.testing.assert_array_equal(fkv.bottom_k(sim, 3), [0, 1, 3])
+    np.testing.assert_array_equal(fkv.bottom_k(np.ones(6), 4), [0, 1, 2, 3])
+
+
+def _run(w, steps, labels, retention=None):
+    L = kvgen.LayerInputs(w, 0)
+    p = fkv.Params(w.frame_h, w.frame_w, w.seg_h, w.seg_w,
+                   w.retention if retention is None else retention, w.hist_frames)
+    states = [fkv.HeadState(bool(s)) for s in labels]
+    out = []
+    for i in range(1, steps + 1):
+        x = L.step(i, forcing=True)
+        fkv.prune_hybrid(states, p, x["newK"], x["newV"], x["new_ids"], x["nextK"])
+        out.append((i, x, [fkv.history(st, w.head_dim) for st in states]))
+    return L, p, states, out
+
+
+def test_static_heads_keep_sink_transition_chunk():
+    w = kvgen.WORKLOADS["forcing_mid"]
+    L, p, states, out = _run(w, 4, [1, 0, 1, 0])
+    for i, x, hist in out:
+        last = (i - 1) * w.chunk_frames + w.chunk_frames - 1
+        for hh in (0, 2):
+            ids, K, V = hist[hh]
+            np.testing.assert_array_equal(ids, kvgen.token_ids(w, [last]))
+            Kall, _ = fkv.attention_set(states[hh], x["sinkK"][hh], x["sinkV"][hh], x["winK"][hh], x["winV"][hh])
+        assert Kall.shape[0] == 5 * w.F                      # sink + transition + 3-frame chunk
+
+
+def test_retention_one_keeps_everything_and_ring_is_fifo():
+    w = kvgen.WORKLOADS["forcing_mid"]
+    L, p, states, out = _run(w, 5, [0, 0, 0, 0], retention=1.0)
+    for i, x, hist in out:
+        frames = list(range(1, i * w.chunk_frames))[-w.hist_frames:]
+        for hh in range(4):
+            np.testing.assert_array_equal(np.sort(hist[hh][0]), kvgen.token_ids(w, frames))
+            # inside a frame, tokens come segment by segment (segments ascending)
+            segs = fkv.segments(w.frame_h, w.frame_w, w.seg_h, w.seg_w)
+            first = hist[hh][0][:w.F] - frames[0] * w.F
+            np.testing.assert_array_equal(first, np.concatenate(segs))
+
+
+def test_identical_frames_tie_to_lowest_segments():
+    p = fkv.Params(4, 8, 2, 2, 0.5, 3)
+    st = [fkv.HeadState(False)]
+    # one-hot keys: every cosine is exactly 1 in floating point, so all segments tie
+    K = np.tile(np.eye(16)[np.arange(32) % 16][None], (1, 2, 1))
+    fkv.prune_hybrid(st, p, K, K, np.arange(64), K[:, :32])
+    for sim, keep in zip(st[0].sims, st[0].kept):
+        np.testing.assert_allclose(sim, 1.0, rtol=1e-14)
+        np.testing.assert_array_equal(keep, [0, 1, 2, 3])
+
+
+def test_dynamic_direction_uses_successor_frame():
+    """The last new frame is compared with the next chunk's first frame (successor t+1)."""
+    p = fkv.Params(2, 2, 1, 1, 0.5, 4)   # 4 one-token segments, keep 2
+    st = [fkv.HeadState(False)]
+    f0 = np.array([[1, 0], [1, 0], [1, 0], [1, 0]], float)
+    nxt = np.array([[1, 0], [0, 1], [-1, 0], [1, 1]], float)     # cos 1, 0, -1, 1/sqrt2
+    fkv.prune_hybrid(st, p, f0[None], f0[None], np.arange(4), nxt[None])
+    np.testing.assert_allclose(st[0].sims[0], [1, 0, -1, 1 / math.sqrt(2)], atol=1e-15)
+    np.testing.assert_array_equal(st[0].kept[0], [1, 2])
+    np.testing.assert_array_equal(st[0].ring[0].ids, [1, 2])
