@@ -1,0 +1,221 @@
+/*
+ * kvb -- historical KV-bank management for chunk-by-chunk autoregressive video
+ * diffusion, and attention of the current chunk over the retained history.
+ * Hand-written sm_100a (B200) kernels behind a plain C ABI.
+ *
+ * Two cache policies are implemented:
+ *
+ *  - DensityKV ("DensityKV: Density-Guided KV Cache Compression for Long Video
+ *    Generation"): per-(layer, head) banks of exact K/V pairs, at most M per
+ *    head (App. B.1 "Online Bank Update"), updated after every finalised block by
+ *    Soft-Riesz density over post-RoPE keys (§3 "Soft-Riesz Density"): candidates
+ *    are ordered by mean-normalised disturbance, the largest prefix feasible for
+ *    every head is admitted (synchronised admission, App. E), bank entries whose
+ *    projected growth ratio crosses tau are evicted first, then the highest-ratio
+ *    entries until the bank fits M (§3), co-admitted entries set their insertion
+ *    baselines together (App. B.1).
+ *  - Forcing-KV ("Forcing-KV: Hybrid KV Cache Compression for Efficient
+ *    Autoregressive Video Diffusion Models"): static heads attend [sink,
+ *    transition frame, current chunk] (§3.3); dynamic heads keep, per history
+ *    frame, the BottomK(floor(r n)) segments least similar (mean token cosine) to
+ *    the same segment of the next frame (§3.4, §3.5).
+ *
+ * Formulas where the pages give none (the readings this library implements):
+ *   phi(x) = (x + eps)^(-s/2),  x = ||a - b||^2 / h   (h = dist_scale, 0 => d)
+ *   rho_B(c) = sum_{i in B} phi(x(c, k_i))
+ *   score(c) = rho_B(c) / mean_{i in B} rho0_i        (feasible iff <= tau;
+ *              an empty bank or a zero mean baseline makes every candidate
+ *              feasible with score 0)
+ *   P = min(min_h #feasible_h, M, N) (sync_heads=1); each head admits its P
+ *       lowest (score, id)
+ *   ratio_i = (rho_i + sum_{c in A_h} phi(c, i)) / rho0_i  (0 if rho0_i = 0);
+ *       evicted: every ratio_i > tau, then max(0, |B|-|mandatory|+P-M) more by
+ *       (ratio descending, id ascending)
+ *   new entries: rho0 = rho = density within the updated bank.
+ *
+ * Conventions
+ *  - All device pointers are caller-owned device memory, head-major and
+ *    contiguous: a [H][L][d] tensor is H*L*d elements, row d contiguous.  Key
+ *    and value element type is the bank's dtype (bf16 or f32); ids are int32.
+ *  - `stream` is a cudaStream_t (passed as void*).  Every call is asynchronous on
+ *    that stream unless its comment says it synchronises.
+ *  - The library never allocates device memory.  The caller provides one device
+ *    workspace (size from kvb_workspace_size, 256-byte aligned) that holds every
+ *    bank, the scratch of every step and a device status word.  Host-side state
+ *    (the opaque kvb_bank) is malloc'd by kvb_bank_create and freed by destroy.
+ *  - Argument errors return before anything is launched.  Device-side failures
+ *    (a bounded wait that gave up, an index a kernel refused) are latched into
+ *    the status word and reported by kvb_device_status; kernels never trap.
+ *  - Token ids must be unique across a layer's bank and the candidate block.
+ */
+#ifndef KVB_H
+#define KVB_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVB_API __attribute__((visibility("default")))
+#else
+#define KVB_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVB_OK = 0,
+  KVB_E_INVAL = 1,          /* bad argument (null, size out of range, ...); nothing launched */
+  KVB_E_WORKSPACE = 2,      /* workspace null, too small or not 256-byte aligned */
+  KVB_E_CUDA = 3,           /* a CUDA runtime call (launch, memcpy, attribute) failed */
+  KVB_E_DEVICE_TIMEOUT = 4, /* a kernel's bounded wait gave up (latched on device) */
+  KVB_E_DEVICE_BOUNDS = 5,  /* a kernel refused an out-of-range index (latched on device) */
+  KVB_E_STATE = 6,          /* call not valid for this bank (wrong method, layer, ...) */
+  KVB_E_UNSUPPORTED = 7     /* valid but not implemented here (e.g. head_dim not 64/128) */
+} kvb_status;
+
+typedef enum { KVB_BF16 = 0, KVB_F32 = 1 } kvb_dtype;
+
+typedef enum { KVB_DENSITYKV = 0, KVB_FORCINGKV = 1 } kvb_method;
+
+typedef struct {
+  kvb_method method;
+  kvb_dtype dtype;        /* storage/compute input type of K, V, Q, O */
+  int32_t layers;         /* number of independent layers held by the bank */
+  int32_t heads;          /* H, 1..64 */
+  int32_t head_dim;       /* d: 64 or 128 */
+  /* DensityKV */
+  int32_t capacity;       /* M per (layer, head), >= 1 */
+  int32_t max_candidates; /* upper bound on N of kvb_admit */
+  float tau;              /* growth bound (DensityKV App. D default 2.0) */
+  float eps;              /* Soft-Riesz regulariser */
+  float s;                /* Soft-Riesz decay exponent */
+  float dist_scale;       /* h; 0 => head_dim */
+  int32_t sync_heads;     /* 1: shared admitted count across heads (App. E default) */
+  /* Forcing-KV */
+  int32_t frame_h, frame_w; /* token grid of one latent frame; F = frame_h*frame_w */
+  int32_t seg_h, seg_w;     /* segment tile (edge segments are partial) */
+  int32_t hist_frames;      /* frames of pruned history kept by dynamic heads */
+  int32_t max_new_frames;   /* upper bound on the frames pushed per kvb_prune_hybrid */
+  float retention;          /* r: each frame keeps floor(r * n_segments) segments */
+  /* attention */
+  int32_t max_queries;      /* upper bound on Nq of kvb_attend */
+} kvb_config;
+
+/* Per-(layer, head) counters of the last kvb_admit / kvb_prune_hybrid. */
+typedef struct {
+  int32_t admitted;      /* P (DensityKV) or kept tokens pushed (Forcing-KV) */
+  int32_t feasible;      /* candidates with score <= tau (DensityKV) */
+  int32_t mandatory;     /* evictions with ratio > tau */
+  int32_t capacity_evicted;
+  int32_t size;          /* bank size after the update (ring size for Forcing-KV) */
+  int32_t reserved[3];
+} kvb_admit_stats;
+
+typedef struct kvb_bank kvb_bank; /* opaque, host-side */
+
+/* Bytes of device workspace kvb_bank_create needs for `cfg`; 0 if cfg is invalid. */
+KVB_API size_t kvb_workspace_size(const kvb_config* cfg);
+
+/* Bind a bank to a caller-owned workspace (>= kvb_workspace_size bytes, 256-B
+ * aligned).  Clears the status word and every bank to empty with async memsets
+ * on `stream`.  *out receives a host handle.  KVB_E_INVAL / KVB_E_WORKSPACE /
+ * KVB_E_UNSUPPORTED on bad config or workspace; KVB_E_CUDA if the device is not
+ * an sm_100 part. */
+KVB_API kvb_status kvb_bank_create(const kvb_config* cfg, void* workspace, size_t workspace_bytes,
+                           void* stream, kvb_bank** out);
+
+/* Free the host handle (the workspace stays the caller's). */
+KVB_API kvb_status kvb_bank_destroy(kvb_bank* bank);
+
+/* DensityKV admit of one finalised block into layer `layer` (App. B.1):
+ * candK, candV: device [H][N][d]; cand_ids: device [N] int32 (new ids);
+ * 1 <= N <= max_candidates.  Launches the density Gram passes, selection,
+ * eviction and compaction on `stream`; no host synchronisation. */
+KVB_API kvb_status kvb_admit(kvb_bank* bank, int32_t layer, const void* candK, const void* candV,
+                     const int32_t* cand_ids, int32_t N, void* stream);
+
+/* Forcing-KV history update with the frames of a finalised chunk (§3.3-§3.5):
+ * head_is_static: host [H] (1 static, 0 dynamic); newK/newV: device
+ * [H][n_frames*F][d] (frames oldest first; the sink frame is never passed);
+ * nextK: device [H][F][d], the first frame of the next chunk (successor of the
+ * last new frame); new_ids: device [n_frames*F] int32.  Static heads take the
+ * last new frame as their transition frame; dynamic heads push each new frame's
+ * BottomK segments into their FIFO of hist_frames frames. */
+KVB_API kvb_status kvb_prune_hybrid(kvb_bank* bank, int32_t layer, const uint8_t* head_is_static,
+                            const void* newK, const void* newV, const void* nextK,
+                            const int32_t* new_ids, int32_t n_frames, void* stream);
+
+/* Attention of the current chunk's queries over [sink | history(layer) | window]:
+ * Q, O: device [H][Nq][d]; sinkK/V [H][Ls][d]; winK/V [H][Lw][d]; lse: device
+ * [H][Nq] f32 (natural log) or NULL.  O = softmax(Q K^T / sqrt(d)) V, no mask.
+ * History is the DensityKV bank, or for Forcing-KV the transition frame (static
+ * heads) / the pruned FIFO (dynamic heads).  1 <= Nq <= max_queries. */
+KVB_API kvb_status kvb_attend(kvb_bank* bank, int32_t layer, const void* Q, int32_t Nq,
+                      const void* sinkK, const void* sinkV, int32_t Ls,
+                      const void* winK, const void* winV, int32_t Lw,
+                      void* O, float* lse, void* stream);
+
+/* Copy the counters of `layer` (H entries) to host memory.  Synchronises `stream`. */
+KVB_API kvb_status kvb_read_stats(kvb_bank* bank, int32_t layer, kvb_admit_stats* host_out, void* stream);
+
+/* Export one (layer, head) DensityKV bank, or Forcing-KV history, into caller
+ * device buffers of capacity rows (M for DensityKV, hist_frames*F for
+ * Forcing-KV): ids [cap] int32, rho/rho0 [cap] f32 (may be NULL; zero for
+ * Forcing-KV), K/V [cap][d].  *size (host) receives the entry count.  Rows are in
+ * the bank's slot order (Forcing-KV: oldest frame first).  Synchronises `stream`. */
+KVB_API kvb_status kvb_bank_export(kvb_bank* bank, int32_t layer, int32_t head, int32_t* ids, float* rho,
+                           float* rho0, void* K, void* V, int32_t* size, void* stream);
+
+/* Load one (layer, head) DensityKV bank from caller device buffers (size <= M):
+ * ids, rho (current density within the bank), rho0 (frozen baselines), K, V.
+ * Replaces the bank's contents; used for checkpoint/resume and stepwise tests. */
+KVB_API kvb_status kvb_bank_import(kvb_bank* bank, int32_t layer, int32_t head, const int32_t* ids,
+                           const float* rho, const float* rho0, const void* K, const void* V,
+                           int32_t size, void* stream);
+
+/* Synchronise `stream` and return the first latched device error (KVB_OK if none). */
+KVB_API kvb_status kvb_device_status(kvb_bank* bank, void* stream);
+
+/* Static string for a status code. */
+KVB_API const char* kvb_status_string(kvb_status st);
+
+/* ------------------------------------------------------------------------------
+ * Operation-level entry points: the same kernels on caller buffers, for callers
+ * that manage their own caches.  They use the scratch of a caller workspace.
+ * ---------------------------------------------------------------------------- */
+
+/* Bytes of scratch kvb_density needs for these sizes (0 on invalid sizes). */
+KVB_API size_t kvb_density_workspace_size(int32_t heads, int32_t n_rows, int32_t n_cols, int32_t head_dim,
+                                  kvb_dtype dtype);
+
+/* Soft-Riesz density of every row against every column, per head (DensityKV §3):
+ *   out[h][r] = sum_{c < n_cols} phi(||rows[h][r] - cols[h][c]||^2 / h_scale)
+ * rows [H][n_rows][d], cols [H][n_cols][d] device; out [H][n_rows] f32 device.
+ * If `exclude_diagonal` is nonzero, rows and cols must be the same set in the same
+ * order (n_rows == n_cols) and the pair c == r is skipped (a key's density within
+ * its own bank).  dist_scale 0 => head_dim.  workspace: device scratch of
+ * kvb_density_workspace_size bytes, 256-B aligned.  The first 4 bytes of the
+ * workspace are this call's device status word (zeroed by the call, then set to a
+ * kvb_status code by a kernel that gives up; read it with a copy after a sync). */
+KVB_API kvb_status kvb_density(const void* rows, int32_t n_rows, const void* cols, int32_t n_cols,
+                       int32_t heads, int32_t head_dim, kvb_dtype dtype, float dist_scale,
+                       float eps, float s, int32_t exclude_diagonal, float* out,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* Segment-wise cosine similarity of Forcing-KV (§3.4): for every head and every
+ * frame t < n_frames, sim[h][t][j] = mean over the tokens p of segment j of
+ * cos(K[h][t][p], succ[h][t][p]) with succ = frame t+1 of K, or `nextK` for the
+ * last frame.  K [H][n_frames*F][d], nextK [H][F][d]; sim [H][n_frames][n_seg]
+ * f32 with n_seg = ceil(frame_h/seg_h)*ceil(frame_w/seg_w), segments row-major.
+ * cos(a, b) = a.b / max(|a| |b|, 1e-8). */
+KVB_API kvb_status kvb_segment_cosine(const void* K, const void* nextK, int32_t heads, int32_t n_frames,
+                              int32_t frame_h, int32_t frame_w, int32_t seg_h, int32_t seg_w,
+                              int32_t head_dim, kvb_dtype dtype, float* sim, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVB_H */

@@ -1,0 +1,503 @@
+// Soft-Riesz density Gram on the 5th-generation tensor cores.
+//
+// DensityKV §3 "Soft-Riesz Density" / App. B.1: every admit step needs, per head,
+// sums of phi(||a - b||^2 / h) over candidate x bank (and bank x admitted, bank x
+// evicted, admitted x admitted) pairs: O(N M d_k).  With the norm expansion
+//     ||a - b||^2 / h = ||a||^2/h + ||b||^2/h - (2/h) a.b
+// the a.b part is a dense bf16 contraction (tcgen05.mma, fp32 accumulate in TMEM)
+// and the rest is an epilogue on CUDA cores: one FADD + FFMA + FMNMX per pair, then
+// phi.  For the default s = 2 the reciprocals of four pairs share one MUFU op:
+//     1/t0 + 1/t1 + 1/t2 + 1/t3 = ((t0+t1) t2 t3 + (t2+t3) t0 t1) / (t0 t1 t2 t3)
+// which keeps the special-function unit off the critical path.
+//
+// Work unit = (head, 256-row block, chunk of column tiles).  A persistent grid of
+// one CTA per SM walks a contiguous range of units; within a unit the CTA keeps
+// the 256 rows resident in shared memory and streams 128-row column tiles through
+// a 4-stage TMA ring.  Warp roles: 0 = TMA producer, 1 = MMA issuer, 2 = TMEM
+// owner, 4..11 = epilogue (two row tiles x four TMEM lane quarters, one thread per
+// row: row sums need no cross-thread reduction).  TMEM holds 2 row tiles x 2
+// buffers x 128 fp32 columns = all 512 columns.
+#include <climits>
+
+#include "gram.cuh"
+#include "kvb_device.cuh"
+#include "sm100.cuh"
+
+namespace kvb {
+using namespace sm100;
+
+namespace {
+
+constexpr int kStages = 4;
+
+struct alignas(8) GramBars {
+  uint64_t a_full, a_empty;
+  uint64_t full[kStages], empty[kStages];
+  uint64_t acc_full[2], acc_empty[2];
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr int kBarBytes = 256;
+static_assert(sizeof(GramBars) <= kBarBytes, "barrier block overflows its reservation");
+
+__device__ __forceinline__ int set_n(const GramSet& s, int h) { return s.n_dev ? s.n_dev[h] : s.n_uni; }
+__device__ __forceinline__ int set_off(const GramSet& s, int h) { return s.off_dev ? s.off_dev[h] : s.off_uni; }
+
+// Position in the (head, row block, column tile) step sequence.
+struct Cursor {
+  int h, rb, j;          // current step
+  int RB, CT;            // row blocks / column tiles of head h
+  int nR, nC, rOff, cOff;
+};
+
+__device__ __forceinline__ void head_dims(const GramArgs& a, int h, int& RB, int& CT) {
+  const int nR = set_n(a.rows, h), nC = set_n(a.cols, h);
+  RB = nC > 0 ? (nR + kGramRowBlock - 1) / kGramRowBlock : 0;
+  CT = nR > 0 ? (nC + kGramColTile - 1) / kGramColTile : 0;
+}
+
+__device__ __forceinline__ long long total_steps(const GramArgs& a) {
+  long long T = 0;
+  for (int h = 0; h < a.H; ++h) {
+    int RB, CT;
+    head_dims(a, h, RB, CT);
+    T += static_cast<long long>(RB) * CT;
+  }
+  return T;
+}
+
+__device__ __forceinline__ int active_grid(const GramArgs& a, long long T) {
+  long long g = T / a.min_steps;
+  if (g > a.grid) g = a.grid;
+  if (g < 1) g = 1;
+  return static_cast<int>(g);
+}
+
+__device__ __forceinline__ void cursor_load_head(const GramArgs& a, Cursor& c) {
+  head_dims(a, c.h, c.RB, c.CT);
+  c.nR = set_n(a.rows, c.h);
+  c.nC = set_n(a.cols, c.h);
+  c.rOff = set_off(a.rows, c.h);
+  c.cOff = set_off(a.cols, c.h);
+}
+
+// position the cursor at step L (0 <= L < T)
+__device__ __forceinline__ void cursor_seek(const GramArgs& a, long long L, Cursor& c) {
+  for (c.h = 0; c.h < a.H; ++c.h) {
+    head_dims(a, c.h, c.RB, c.CT);
+    const long long n = static_cast<long long>(c.RB) * c.CT;
+    if (L < n) break;
+    L -= n;
+  }
+  cursor_load_head(a, c);
+  c.rb = static_cast<int>(L / c.CT);
+  c.j = static_cast<int>(L % c.CT);
+}
+
+__device__ __forceinline__ void cursor_next(const GramArgs& a, Cursor& c) {
+  if (++c.j < c.CT) return;
+  c.j = 0;
+  if (++c.rb < c.RB) return;
+  c.rb = 0;
+  do {
+    ++c.h;
+    if (c.h >= a.H) return;
+    head_dims(a, c.h, c.RB, c.CT);
+  } while (c.RB * c.CT == 0);
+  cursor_load_head(a, c);
+}
+
+// the CTA (of G_eff) whose range contains step L
+__device__ __forceinline__ int cta_of(long long L, long long T, int G) {
+  return static_cast<int>(((L + 1) * G - 1) / T);
+}
+
+__device__ __forceinline__ int nact_of(const Cursor& c) {
+  return (c.nR - c.rb * kGramRowBlock > kGramRowTile) ? 2 : 1;
+}
+
+// phi for one pair given t = x + eps (already clamped to >= eps)
+template <int SMODE>
+__device__ __forceinline__ float phi_t(float t, float nhs) {
+  if constexpr (SMODE == 2) return rcp_approx(t);
+  else if constexpr (SMODE == 1) return rsqrt_approx(t);
+  else return ex2_approx(nhs * lg2_approx(t));
+}
+
+template <int SMODE>
+__global__ void __launch_bounds__(kGramThreads, 1)
+    gram_bf16_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmC,
+                     const GramArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int nbox = a.d / 64;
+  const uint32_t tileBytes = static_cast<uint32_t>(kGramRowTile) * a.d * 2;
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + 2 * tileBytes;
+  GramBars* bars = reinterpret_cast<GramBars*>(sB + kStages * tileBytes);
+  // [8 warps][2][128] column terms, 16-byte aligned for float4 reads
+  float* sColTerm = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kBarBytes);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->a_full, 1);
+    mbar_init(&bars->a_empty, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->acc_full[b], 1);
+      mbar_init(&bars->acc_empty[b], 8);
+    }
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort = &bars->abort;
+
+  const long long T = total_steps(a);
+  const int G = active_grid(a, T);
+  const int cta = blockIdx.x;
+  const long long L0 = (cta < G) ? (T * cta) / G : 0;
+  const long long L1 = (cta < G) ? (T * (cta + 1)) / G : 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmR);
+      prefetch_tmap(&tmC);
+      int it = 0, aload = 0;
+      bool ok = true;
+      Cursor c;
+      if (L0 < L1) cursor_seek(a, L0, c);
+      for (long long L = L0; L < L1; ++L, cursor_next(a, c)) {
+        if (L == L0 || c.j == 0) {
+          if (aload > 0 && !(ok = mbar_wait(&bars->a_empty, (aload - 1) & 1, abort, a.status))) break;
+          const int nact = nact_of(c);
+          mbar_arrive_expect_tx(&bars->a_full, nact * tileBytes);
+          for (int r = 0; r < nact; ++r)
+            for (int k = 0; k < nbox; ++k)
+              tma_load_3d(sA + r * tileBytes + k * 16384, &tmR, &bars->a_full, k * 64,
+                          c.rOff + c.rb * kGramRowBlock + r * kGramRowTile, c.h);
+          ++aload;
+        }
+        const int s = it % kStages;
+        if (!(ok = mbar_wait(&bars->empty[s], ((it / kStages) & 1) ^ 1, abort, a.status))) break;
+        mbar_arrive_expect_tx(&bars->full[s], tileBytes);
+        for (int k = 0; k < nbox; ++k)
+          tma_load_3d(sB + s * tileBytes + k * 16384, &tmC, &bars->full[s], k * 64, c.cOff + c.j * kGramColTile,
+                      c.h);
+        ++it;
+      }
+      if (!ok) {
+        // abort path: let the copies already issued land before the CTA exits
+        for (int k = max(0, it - kStages); k < it; ++k)
+          mbar_wait_drain(&bars->full[k % kStages], (k / kStages) & 1, 200000000ull);
+        if (aload > 0) mbar_wait_drain(&bars->a_full, (aload - 1) & 1, 200000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, kGramColTile, 0, 0);
+      const uint32_t aBase = smem_u32(sA), bBase = smem_u32(sB);
+      int it = 0, t = 0, aload = 0;
+      bool ok = true;
+      Cursor c;
+      if (L0 < L1) cursor_seek(a, L0, c);
+      for (long long L = L0; L < L1; ++L) {
+        const int nact = nact_of(c);
+        if (L == L0 || c.j == 0) {
+          if (!(ok = mbar_wait(&bars->a_full, aload & 1, abort, a.status))) break;
+          tc_fence_after();
+          ++aload;
+        }
+        const int s = it % kStages;
+        const int b = t & 1;
+        if (!(ok = mbar_wait(&bars->full[s], (it / kStages) & 1, abort, a.status))) break;
+        if (!(ok = mbar_wait(&bars->acc_empty[b], ((t >> 1) & 1) ^ 1, abort, a.status))) break;
+        tc_fence_after();
+        for (int r = 0; r < nact; ++r) {
+          const uint32_t dcol = tmem + static_cast<uint32_t>((r * 2 + b) * kGramColTile);
+          for (int kk = 0; kk < a.d / 16; ++kk) {
+            const uint32_t koff = static_cast<uint32_t>((kk >> 2) * 16384 + (kk & 3) * 32);
+            const uint64_t ad = sdesc_sw128(aBase + r * tileBytes + koff, 16, 1024);
+            const uint64_t bd = sdesc_sw128(bBase + s * tileBytes + koff, 16, 1024);
+            mma_f16_ss(dcol, ad, bd, idesc, kk > 0 ? 1u : 0u);
+          }
+        }
+        mma_commit(&bars->empty[s]);
+        mma_commit(&bars->acc_full[b]);
+        ++it;
+        ++t;
+        const bool last_of_block = (L + 1 == L1) || (c.j + 1 == c.CT);
+        if (last_of_block) mma_commit(&bars->a_empty);
+        cursor_next(a, c);
+      }
+      if (!ok && t > 0) {
+        // abort path: make sure no MMA still writes TMEM when it is freed
+        mma_commit(&bars->a_empty);
+        mbar_wait_drain(&bars->acc_full[(t - 1) & 1], ((t - 1) >> 1) & 1, 200000000ull);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - 4;
+    const int r = e >> 2;          // row tile
+    const int q = warp & 3;        // TMEM lane quarter (warp_id % 4)
+    const int row_in_tile = q * 32 + lane;
+    const float ks = a.kscale, eps = a.eps, nhs = -0.5f * a.s;
+    int t = 0;
+    bool ok = true;
+    Cursor c;
+    if (L0 < L1) cursor_seek(a, L0, c);
+    float acc_pos = 0.f, acc_neg = 0.f, ra = 0.f;
+    int row = 0, nneg = 0, diag = 0, rt0 = 0;
+    bool active = false, valid_row = false;
+    long long Lblock = L0;  // first step of the current row block
+    for (long long L = L0; L < L1; ++L) {
+      if (L == L0 || c.j == 0) {
+        Lblock = L - c.j;
+        rt0 = c.rb * kGramRowBlock + r * kGramRowTile;
+        row = rt0 + row_in_tile;
+        active = r < nact_of(c);
+        valid_row = active && row < c.nR;
+        ra = valid_row ? a.rowTerm[static_cast<size_t>(c.h) * a.ldRT + c.rOff + row] : 0.f;
+        nneg = a.nneg_dev ? a.nneg_dev[c.h] : a.nneg_uni;
+        diag = a.use_diag ? (a.diag_dev ? a.diag_dev[c.h] : a.diag_uni) : INT_MIN / 2;
+        acc_pos = 0.f;
+        acc_neg = 0.f;
+      }
+      const int b = t & 1;
+      const int c0 = c.j * kGramColTile;
+      if (*abort) {
+        ok = false;
+        break;
+      }
+      // this warp's copy of the tile's column terms (no cross-warp barrier, so an
+      // aborting warp can never strand another one)
+      float* cb = sColTerm + (e * 2 + b) * kGramColTile;
+#pragma unroll
+      for (int i = lane; i < kGramColTile; i += 32) {
+        const long idx = static_cast<long>(c.cOff) + c0 + i;
+        cb[i] = (idx < a.ldCT) ? a.colTerm[static_cast<size_t>(c.h) * a.ldCT + idx] : 0.f;
+      }
+      __syncwarp();
+      if (!(ok = mbar_wait(&bars->acc_full[b], (t >> 1) & 1, abort, a.status))) break;
+      tc_fence_after();
+      if (active) {
+        const bool tail = c0 + kGramColTile > c.nC;
+        const bool allneg = c0 + kGramColTile <= nneg;
+        const bool mixed = (c0 < nneg) && !allneg;
+        // diagonal columns of this row tile: [rt0 + diag, rt0 + diag + 128)
+        const bool diag_hit =
+            a.use_diag && (rt0 + diag < c0 + kGramColTile) && (rt0 + diag + kGramRowTile > c0);
+        const bool masked = tail || mixed || diag_hit;
+        const uint32_t taddr =
+            tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>((r * 2 + b) * kGramColTile);
+        float tile_acc = 0.f;
+#pragma unroll 1
+        for (int cc = 0; cc < kGramColTile / 32; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(taddr + cc * 32, v);
+          tmem_wait_ld();
+          if (!masked) {
+            if constexpr (SMODE == 2) {
+#pragma unroll
+              for (int k = 0; k < 32; k += 4) {
+                const float4 cbv = *reinterpret_cast<const float4*>(cb + cc * 32 + k);
+                const float t0 = fmaxf(fmaf(__uint_as_float(v[k + 0]), ks, ra + cbv.x), eps);
+                const float t1 = fmaxf(fmaf(__uint_as_float(v[k + 1]), ks, ra + cbv.y), eps);
+                const float t2 = fmaxf(fmaf(__uint_as_float(v[k + 2]), ks, ra + cbv.z), eps);
+                const float t3 = fmaxf(fmaf(__uint_as_float(v[k + 3]), ks, ra + cbv.w), eps);
+                const float p01 = t0 * t1, p23 = t2 * t3;
+                const float num = fmaf(t2 + t3, p01, (t0 + t1) * p23);
+                tile_acc = fmaf(num, rcp_approx(p01 * p23), tile_acc);
+              }
+            } else {
+#pragma unroll
+              for (int k = 0; k < 32; k += 4) {
+                const float4 cbv = *reinterpret_cast<const float4*>(cb + cc * 32 + k);
+                tile_acc += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 0]), ks, ra + cbv.x), eps), nhs);
+                tile_acc += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 1]), ks, ra + cbv.y), eps), nhs);
+                tile_acc += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 2]), ks, ra + cbv.z), eps), nhs);
+                tile_acc += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 3]), ks, ra + cbv.w), eps), nhs);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              const int col = c0 + cc * 32 + k;
+              const float tv = fmaxf(fmaf(__uint_as_float(v[k]), ks, ra + cb[cc * 32 + k]), eps);
+              const bool valid = (col < c.nC) && (col != row + diag);
+              const float ph = valid ? phi_t<SMODE>(tv, nhs) : 0.f;
+              if (col < nneg) acc_neg += ph;
+              else acc_pos += ph;
+            }
+          }
+        }
+        if (!masked) {
+          if (allneg) acc_neg += tile_acc;
+          else acc_pos += tile_acc;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->acc_empty[b]);
+      ++t;
+      const bool last_of_block = (L + 1 == L1) || (c.j + 1 == c.CT);
+      if (last_of_block && valid_row) {
+        const int slot = cta - cta_of(Lblock, T, G);
+        if (slot >= 0 && slot < a.slots)
+          a.partial[(static_cast<size_t>(slot) * a.H + c.h) * a.ldOut + row] = acc_pos - acc_neg;
+        else
+          latch_status(a.status, 5 /* KVB_E_DEVICE_BOUNDS */);
+      }
+      cursor_next(a, c);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// -------------------------------------------------------------------- f32 path
+// One warp per row, 32 columns per step staged in shared memory, direct
+// differences in fp32 (no norm expansion), same masks and phi as above.
+constexpr int kF32Warps = 8;
+constexpr int kF32Cols = 32;
+
+__global__ void __launch_bounds__(kF32Warps * 32) gram_f32_kernel(const GramArgs a) {
+  extern __shared__ float sh[];  // [kF32Warps][d] rows + [kF32Cols][d + 1] cols
+  const int d = a.d;
+  float* sRow = sh;
+  float* sCol = sh + kF32Warps * d;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  const int nR = set_n(a.rows, h), nC = set_n(a.cols, h);
+  const int rOff = set_off(a.rows, h), cOff = set_off(a.cols, h);
+  const int row = blockIdx.x * kF32Warps + warp;
+  if (blockIdx.x * kF32Warps >= nR) return;
+  const float inv_h = -0.5f * a.kscale;
+  const float nhs = -0.5f * a.s;
+  const int nneg = a.nneg_dev ? a.nneg_dev[h] : a.nneg_uni;
+  const int diag = a.use_diag ? (a.diag_dev ? a.diag_dev[h] : a.diag_uni) : INT_MIN / 2;
+  for (int k = lane; k < d; k += 32)
+    sRow[warp * d + k] = (row < nR) ? a.R32[(static_cast<size_t>(h) * a.ldR + rOff + row) * d + k] : 0.f;
+  float acc = 0.f;
+  for (int c0 = 0; c0 < nC; c0 += kF32Cols) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < kF32Cols * d; i += blockDim.x) {
+      const int cc = i / d, k = i % d;
+      const int col = c0 + cc;
+      sCol[cc * (d + 1) + k] = (col < nC) ? a.C32[(static_cast<size_t>(h) * a.ldC + cOff + col) * d + k] : 0.f;
+    }
+    __syncthreads();
+    const int col = c0 + lane;
+    float dist = 0.f;
+    for (int k = 0; k < d; ++k) {
+      const float df = sRow[warp * d + k] - sCol[lane * (d + 1) + k];
+      dist = fmaf(df, df, dist);
+    }
+    const float tv = fmaf(dist, inv_h, a.eps);
+    float ph = 0.f;
+    if (col < nC && col != row + diag) {
+      ph = (a.s == 2.f) ? 1.f / tv : powf(tv, nhs);
+      if (col < nneg) ph = -ph;
+    }
+    acc += ph;
+  }
+  acc = warp_sum(acc);
+  if (lane == 0 && row < nR) a.partial[static_cast<size_t>(h) * a.ldOut + row] = acc;
+}
+
+__global__ void gram_reduce_kernel(const GramArgs a, float* out, int ldOut) {
+  const int h = blockIdx.y;
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  const int nR = set_n(a.rows, h);
+  if (r >= nR) return;
+  int RB, CT;
+  head_dims(a, h, RB, CT);
+  float acc = 0.f;
+  if (CT > 0) {
+    const long long T = total_steps(a);
+    const int G = active_grid(a, T);
+    long long before = 0;
+    for (int g = 0; g < h; ++g) {
+      int rb2, ct2;
+      head_dims(a, g, rb2, ct2);
+      before += static_cast<long long>(rb2) * ct2;
+    }
+    const long long Lb = before + static_cast<long long>(r / kGramRowBlock) * CT;
+    const int first = cta_of(Lb, T, G), last = cta_of(Lb + CT - 1, T, G);
+    for (int sl = 0; sl <= last - first && sl < a.slots; ++sl)
+      acc += a.partial[(static_cast<size_t>(sl) * a.H + h) * a.ldOut + r];
+  }
+  out[static_cast<size_t>(h) * ldOut + r] = acc;
+}
+
+}  // namespace
+
+size_t gram_smem_bytes(int d) {
+  const size_t tile = static_cast<size_t>(kGramRowTile) * d * 2;
+  return 1024 + (2 + kStages) * tile + kBarBytes + 16 * kGramColTile * sizeof(float);
+}
+
+void gram_plan(GramArgs& a, int max_col_tiles, int n_sm) {
+  a.grid = n_sm;
+  a.slots = 8;
+  const int m = (max_col_tiles + a.slots - 2) / (a.slots - 1);
+  a.min_steps = m < 1 ? 1 : m;
+}
+
+cudaError_t launch_gram_bf16(const GramArgs& a, const CUtensorMap& tmR, const CUtensorMap& tmC, int n_sm,
+                             cudaStream_t st) {
+  (void)n_sm;
+  const size_t smem = gram_smem_bytes(a.d);
+  const int grid = a.grid;
+  if (grid <= 0) return cudaSuccess;
+  cudaError_t e;
+  if (a.s == 2.f) {
+    e = cudaFuncSetAttribute(gram_bf16_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    gram_bf16_kernel<2><<<grid, kGramThreads, smem, st>>>(tmR, tmC, a);
+  } else if (a.s == 1.f) {
+    e = cudaFuncSetAttribute(gram_bf16_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    gram_bf16_kernel<1><<<grid, kGramThreads, smem, st>>>(tmR, tmC, a);
+  } else {
+    e = cudaFuncSetAttribute(gram_bf16_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    gram_bf16_kernel<0><<<grid, kGramThreads, smem, st>>>(tmR, tmC, a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gram_f32(const GramArgs& a, cudaStream_t st) {
+  const int maxR = a.max_rows;
+  dim3 grid((maxR + kF32Warps - 1) / kF32Warps, a.H);
+  const size_t smem = sizeof(float) * (kF32Warps * a.d + kF32Cols * (a.d + 1));
+  gram_f32_kernel<<<grid, kF32Warps * 32, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gram_reduce(const GramArgs& a, float* out, int ldOut, cudaStream_t st) {
+  const int maxR = a.max_rows;
+  dim3 grid((maxR + 255) / 256, a.H);
+  gram_reduce_kernel<<<grid, 256, 0, st>>>(a, out, ldOut);
+  return cudaGetLastError();
+}
+
+}  // namespace kvb

@@ -1,0 +1,45 @@
+// Host-side helpers: status mapping, device properties, TMA descriptors and a
+// bump carver for caller workspaces.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/kvb.h"
+
+namespace kvb {
+
+struct DeviceInfo {
+  int device = -1;
+  int n_sm = 0;
+  int cc_major = 0;
+  int cc_minor = 0;
+};
+
+// Properties of the current device (cached per device).  false if unavailable.
+bool current_device(DeviceInfo* out);
+
+// 3D tiled tensor map over a bf16 [heads][rows][d] buffer, box 64 x box_rows x 1,
+// 128-byte swizzle, zero fill out of bounds.
+bool make_tmap_bf16(CUtensorMap* m, const void* base, int d, long long rows, int heads, int box_rows);
+
+inline kvb_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVB_OK : KVB_E_CUDA; }
+
+// Bump allocation inside a caller workspace, 256-byte aligned pieces.
+struct Carver {
+  uintptr_t base = 0;
+  size_t used = 0;
+  explicit Carver(void* p = nullptr) : base(reinterpret_cast<uintptr_t>(p)) {}
+  template <typename T>
+  T* take(size_t count) {
+    used = (used + 255) & ~size_t(255);
+    T* p = reinterpret_cast<T*>(base + used);
+    used += count * sizeof(T);
+    return base ? p : nullptr;
+  }
+  size_t bytes() const { return (used + 255) & ~size_t(255); }
+};
+
+}  // namespace kvb
