@@ -1,0 +1,427 @@
+// DensityKV admit step, the parts that are not a density contraction
+// (DensityKV App. B.1 "Online Bank Update", §3, App. E default policy):
+//
+//   count     per head: mean frozen baseline of the bank, number of candidates
+//             whose disturbance score rho_B(c) / mean rho0 is <= tau
+//   select    P = min over heads (synchronised prefix) of the feasible counts,
+//             capped by M and N; each head keeps its P lowest (score, id) keys
+//             (radix select over 64-bit composite keys: exact, tie-free)
+//   evict     projected ratio (rho_i + sum_A phi) / rho0_i; every entry above tau
+//             is evicted, then max(0, |B| - mandatory + P - M) more by (ratio
+//             descending, id ascending) -- another radix select
+//   compact   admitted entries fill the evicted slots below the new size, then
+//             append; surviving entries beyond the new size move into the
+//             remaining holes, so every bank stays dense in [0, size)
+//   finalize  incremental densities: survivors rho + sum_A phi - sum_E phi,
+//             new entries rho_B(c) - sum_E phi + sum_{A, c' != c} phi, and new
+//             baselines rho0 = rho (co-admitted entries set them together)
+//
+// The selection kernels run one 1024-thread CTA per head (latency-bound, a few
+// microseconds); the row movers use one warp per 256-byte K/V row.
+#include <climits>
+
+#include "admit.cuh"
+#include "kvb_device.cuh"
+
+namespace kvb {
+namespace {
+
+constexpr int kSelThreads = 1024;
+
+struct SelShared {
+  unsigned int hist[256];
+  unsigned long long prefix, mask;
+  int kRem;
+  int done;
+  int warp_tot[32];
+  float fred[32];
+};
+
+__device__ __forceinline__ float block_sum(float v, SelShared* S) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) S->fred[w] = v;
+  __syncthreads();
+  float t = 0.f;
+  if (w == 0) {
+    t = (l < static_cast<int>(blockDim.x >> 5)) ? S->fred[l] : 0.f;
+    t = warp_sum(t);
+    if (l == 0) S->fred[0] = t;
+  }
+  __syncthreads();
+  t = S->fred[0];
+  __syncthreads();
+  return t;
+}
+
+// exclusive scan over the block; *total receives the sum
+__device__ __forceinline__ int block_excl_scan(int v, SelShared* S, int* total) {
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (l >= o) incl += t;
+  }
+  __syncthreads();
+  if (l == 31) S->warp_tot[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    const int nw = blockDim.x >> 5;
+    int x = (l < nw) ? S->warp_tot[l] : 0;
+    int xi = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, xi, o);
+      if (l >= o) xi += t;
+    }
+    if (l < nw) S->warp_tot[l] = xi - x;  // exclusive warp offsets
+    if (l == nw - 1) S->kRem = xi;        // reuse as total holder
+  }
+  __syncthreads();
+  const int res = S->warp_tot[w] + incl - v;
+  *total = S->kRem;
+  __syncthreads();
+  return res;
+}
+
+// Write, in ascending order, every i in [lo, hi) with pred(i) to out; returns count.
+template <class Pred>
+__device__ int block_compact(int lo, int hi, Pred pred, int* out, SelShared* S) {
+  const int n = hi > lo ? hi - lo : 0;
+  const int chunk = (n + blockDim.x - 1) / blockDim.x;
+  const int b = lo + threadIdx.x * chunk, e = min(hi, b + chunk);
+  int cnt = 0;
+  for (int i = b; i < e; ++i) cnt += pred(i) ? 1 : 0;
+  int total;
+  int pos = block_excl_scan(cnt, S, &total);
+  if (out)
+    for (int i = b; i < e; ++i)
+      if (pred(i)) out[pos++] = i;
+  __syncthreads();
+  return total;
+}
+
+// Radix select of the k smallest 64-bit keys among {i < n : keep(i)} (1 <= k <
+// count).  On return S->prefix / S->mask define the selection:
+// keep(i) && (key(i) & mask) <= prefix.  Keys are unique (they carry the id).
+template <class KeyFn, class KeepFn>
+__device__ void block_radix_select(int n, int k, KeyFn key, KeepFn keep, SelShared* S) {
+  if (threadIdx.x == 0) {
+    S->prefix = 0ull;
+    S->mask = 0ull;
+    S->kRem = k;
+    S->done = 0;
+  }
+  __syncthreads();
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) S->hist[i] = 0u;
+    __syncthreads();
+    const unsigned long long prefix = S->prefix, mask = S->mask;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      if (!keep(i)) continue;
+      const unsigned long long kk = key(i);
+      if ((kk & mask) == prefix) atomicAdd(&S->hist[(kk >> shift) & 0xFFull], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      unsigned int loc[8];
+      unsigned int s = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        loc[j] = S->hist[lane * 8 + j];
+        s += loc[j];
+      }
+      unsigned int incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const unsigned int excl = incl - s;
+      const unsigned int kr = static_cast<unsigned int>(S->kRem);
+      __syncwarp();
+      if (excl < kr && kr <= incl) {
+        unsigned int c = excl;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (c + loc[j] >= kr) {
+            S->prefix = prefix | (static_cast<unsigned long long>(lane * 8 + j) << shift);
+            S->mask = mask | (0xFFull << shift);
+            S->kRem = static_cast<int>(kr - c);
+            if (loc[j] == kr - c) S->done = 1;
+            break;
+          }
+          c += loc[j];
+        }
+      }
+    }
+    __syncthreads();
+    if (S->done) break;
+  }
+}
+
+__device__ __forceinline__ float score_of(float rhoB, float mean0) {
+  return mean0 > 0.f ? __fdiv_rn(rhoB, mean0) : 0.f;
+}
+__device__ __forceinline__ float ratio_of(float rho, float proj, float rho0) {
+  return rho0 > 0.f ? __fdiv_rn(rho + proj, rho0) : 0.f;
+}
+
+// -------------------------------------------------------------------- kernels
+__global__ void __launch_bounds__(kSelThreads) admit_count_kernel(const AdmitPlan p) {
+  __shared__ SelShared S;
+  const int h = blockIdx.x;
+  const int n = p.size[h];
+  float s = 0.f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) s += p.rho0[static_cast<size_t>(h) * p.M + i];
+  const float sum = block_sum(s, &S);
+  const float mean0 = n > 0 ? sum / static_cast<float>(n) : 0.f;
+  const float* rb = p.rhoB + static_cast<size_t>(h) * p.ldN;
+  int cnt = 0;
+  for (int c = threadIdx.x; c < p.N; c += blockDim.x) cnt += (score_of(rb[c], mean0) <= p.tau) ? 1 : 0;
+  int total;
+  block_excl_scan(cnt, &S, &total);
+  if (threadIdx.x == 0) {
+    p.mean0[h] = mean0;
+    p.feasible[h] = total;
+    p.n_old[h] = n;
+  }
+}
+
+__global__ void __launch_bounds__(kSelThreads) admit_select_kernel(const AdmitPlan p) {
+  __shared__ SelShared S;
+  const int h = blockIdx.x;
+  int Pt = p.feasible[h];
+  if (p.sync_heads)
+    for (int g = 0; g < p.H; ++g) Pt = min(Pt, p.feasible[g]);
+  const int P = min(Pt, min(p.M, p.N));
+  const float mean0 = p.mean0[h];
+  const float* rb = p.rhoB + static_cast<size_t>(h) * p.ldN;
+  int* out = p.adm_idx + static_cast<size_t>(h) * p.ldN;
+  auto key = [&](int c) -> unsigned long long {
+    return (static_cast<unsigned long long>(float_key(score_of(rb[c], mean0))) << 32) |
+           static_cast<unsigned int>(p.cand_ids[c]);
+  };
+  auto all = [](int) { return true; };
+  if (P >= p.N) {
+    for (int c = threadIdx.x; c < p.N; c += blockDim.x) out[c] = c;
+  } else if (P > 0) {
+    block_radix_select(p.N, P, key, all, &S);
+    const unsigned long long prefix = S.prefix, mask = S.mask;
+    const int got = block_compact(0, p.N, [&](int c) { return (key(c) & mask) <= prefix; }, out, &S);
+    if (threadIdx.x == 0 && got != P) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
+  }
+  if (threadIdx.x == 0) {
+    p.P[h] = P;
+    p.stats[h].admitted = P;
+    p.stats[h].feasible = p.feasible[h];
+  }
+}
+
+// one warp per 16-byte-chunked row copy
+__device__ __forceinline__ void copy_row(void* dst, const void* src, int row_bytes, int lane) {
+  const uint4* s = static_cast<const uint4*>(src);
+  uint4* d = static_cast<uint4*>(dst);
+  for (int o = lane; o < row_bytes / 16; o += 32) d[o] = s[o];
+}
+
+__global__ void gather_admitted_kernel(const AdmitPlan p) {
+  const int h = blockIdx.y;
+  const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (w >= p.P[h]) return;
+  const int c = p.adm_idx[static_cast<size_t>(h) * p.ldN + w];
+  const size_t dst = static_cast<size_t>(h) * p.ldEA + p.M + w;
+  copy_row(static_cast<char*>(p.EA) + dst * p.row_bytes,
+           static_cast<const char*>(p.candK) + (static_cast<size_t>(h) * p.N + c) * p.row_bytes, p.row_bytes, lane);
+  if (lane == 0) p.EAterm[dst] = p.cterm[static_cast<size_t>(h) * p.ldN + c];
+}
+
+__global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPlan p) {
+  __shared__ SelShared S;
+  const int h = blockIdx.x;
+  const int n = p.n_old[h];
+  const int Ph = p.P[h];
+  const size_t base = static_cast<size_t>(h) * p.M;
+  const float* rho = p.rho + base;
+  const float* rho0 = p.rho0 + base;
+  const float* proj = p.proj + base;
+  const int* ids = p.ids + base;
+  int* evflag = p.tail + base;  // per-slot flags live in the tail array until the tail list is built
+  auto ratio = [&](int i) { return ratio_of(rho[i], proj[i], rho0[i]); };
+  // mandatory evictions: projected growth above tau
+  int cnt = 0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const bool m = ratio(i) > p.tau;
+    evflag[i] = m ? 1 : 0;
+    cnt += m ? 1 : 0;
+  }
+  int n_mand;
+  block_excl_scan(cnt, &S, &n_mand);
+  const int ecap = max(0, n - n_mand + Ph - p.M);
+  const int n_free = n - n_mand;
+  if (ecap > 0) {
+    auto key = [&](int i) -> unsigned long long {
+      return (static_cast<unsigned long long>(~float_key(ratio(i))) << 32) | static_cast<unsigned int>(ids[i]);
+    };
+    auto keep = [&](int i) { return evflag[i] == 0; };
+    if (ecap >= n_free) {
+      for (int i = threadIdx.x; i < n; i += blockDim.x) evflag[i] = 1;
+    } else {
+      block_radix_select(n, ecap, key, keep, &S);
+      const unsigned long long prefix = S.prefix, mask = S.mask;
+      for (int i = threadIdx.x; i < n; i += blockDim.x)
+        if (evflag[i] == 0 && (key(i) & mask) <= prefix) evflag[i] = 2;
+    }
+  }
+  __syncthreads();
+  const int E = n_mand + min(ecap, n_free);
+  const int n_new = n - E + Ph;
+  int* ev = p.ev_slot + base;
+  const int gotE = block_compact(0, n, [&](int i) { return evflag[i] != 0; }, ev, &S);
+  const int nh = block_compact(0, n, [&](int i) { return evflag[i] != 0 && i < n_new; }, nullptr, &S);
+  // survivors at or above the new size move into holes; list them (ascending)
+  __shared__ int s_ntail;
+  {
+    // count first (flags are still needed), then write the list over the flag array
+    const int nt = block_compact(n_new < n ? n_new : n, n, [&](int i) { return evflag[i] == 0; }, nullptr, &S);
+    if (threadIdx.x == 0) s_ntail = nt;
+  }
+  __syncthreads();
+  // the tail list is short; build it in the newp scratch and copy it over the flags
+  int* tmp = p.newp + base;
+  block_compact(n_new < n ? n_new : n, n, [&](int i) { return evflag[i] == 0; }, tmp, &S);
+  for (int k = threadIdx.x; k < s_ntail; k += blockDim.x) evflag[k] = tmp[k];
+  __syncthreads();
+  // every slot of the new bank starts as an old, unmoved entry
+  const int top = max(n, n_new);
+  for (int i = threadIdx.x; i < top; i += blockDim.x) tmp[i] = -1;
+  if (threadIdx.x == 0) {
+    if (gotE != E) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
+    p.E[h] = E;
+    p.nhole[h] = nh;
+    p.ntail[h] = s_ntail;
+    p.EAoff[h] = p.M - E;
+    p.EAcnt[h] = E;
+    p.size[h] = n_new;
+    p.stats[h].mandatory = n_mand;
+    p.stats[h].capacity_evicted = E - n_mand;
+    p.stats[h].size = n_new;
+  }
+}
+
+__global__ void gather_evicted_kernel(const AdmitPlan p) {
+  const int h = blockIdx.y;
+  const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int E = p.E[h];
+  if (w >= E) return;
+  const int slot = p.ev_slot[static_cast<size_t>(h) * p.M + w];
+  const size_t src = static_cast<size_t>(h) * p.M + slot;
+  const size_t dst = static_cast<size_t>(h) * p.ldEA + (p.M - E) + w;
+  copy_row(static_cast<char*>(p.EA) + dst * p.row_bytes, static_cast<const char*>(p.K) + src * p.row_bytes,
+           p.row_bytes, lane);
+  if (lane == 0) p.EAterm[dst] = p.term[src];
+}
+
+// moves: [0, P) admitted candidates, [P, P + ntail) surviving tail entries
+__global__ void compact_kernel(const AdmitPlan p) {
+  const int h = blockIdx.y;
+  const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int P = p.P[h], nt = p.ntail[h], nh = p.nhole[h], n_old = p.n_old[h];
+  const size_t base = static_cast<size_t>(h) * p.M;
+  const int* hole = p.ev_slot + base;  // evicted slots ascending: the first nh are holes
+  if (w < P) {
+    const int dst = (w < nh) ? hole[w] : n_old + (w - nh);
+    if (dst < 0 || dst >= p.M) {
+      if (lane == 0) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
+      return;
+    }
+    const int c = p.adm_idx[static_cast<size_t>(h) * p.ldN + w];
+    const size_t srow = static_cast<size_t>(h) * p.N + c;
+    copy_row(static_cast<char*>(p.K) + (base + dst) * p.row_bytes,
+             static_cast<const char*>(p.candK) + srow * p.row_bytes, p.row_bytes, lane);
+    copy_row(static_cast<char*>(p.V) + (base + dst) * p.row_bytes,
+             static_cast<const char*>(p.candV) + srow * p.row_bytes, p.row_bytes, lane);
+    if (lane == 0) {
+      p.ids[base + dst] = p.cand_ids[c];
+      p.term[base + dst] = p.cterm[static_cast<size_t>(h) * p.ldN + c];
+      p.rho[base + dst] = p.rhoB[static_cast<size_t>(h) * p.ldN + c];
+      p.newp[base + dst] = w;
+    }
+  } else if (w < P + nt) {
+    const int k = w - P;
+    const int src = p.tail[base + k];
+    const int dst = hole[P + k];
+    if (src < 0 || src >= p.M || dst < 0 || dst >= p.M) {
+      if (lane == 0) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
+      return;
+    }
+    copy_row(static_cast<char*>(p.K) + (base + dst) * p.row_bytes,
+             static_cast<const char*>(p.K) + (base + src) * p.row_bytes, p.row_bytes, lane);
+    copy_row(static_cast<char*>(p.V) + (base + dst) * p.row_bytes,
+             static_cast<const char*>(p.V) + (base + src) * p.row_bytes, p.row_bytes, lane);
+    if (lane == 0) {
+      p.ids[base + dst] = p.ids[base + src];
+      p.term[base + dst] = p.term[base + src];
+      p.rho0[base + dst] = p.rho0[base + src];
+      p.rho[base + dst] = p.rho[base + src] + p.proj[base + src];
+      p.newp[base + dst] = -2;
+    }
+  }
+}
+
+__global__ void finalize_kernel(const AdmitPlan p) {
+  const int h = blockIdx.y;
+  const int s = blockIdx.x * blockDim.x + threadIdx.x;
+  const int n_new = p.size[h];
+  if (s >= n_new) return;
+  const size_t i = static_cast<size_t>(h) * p.M + s;
+  const int tag = p.newp[i];
+  float v = p.rho[i] + p.sub[i];
+  if (tag == -1) {
+    v += p.proj[i];
+  } else if (tag >= 0) {
+    v += p.coadm[static_cast<size_t>(h) * p.ldN + tag];
+    p.rho0[i] = v;
+  }
+  p.rho[i] = v;
+}
+
+}  // namespace
+
+cudaError_t launch_admit_count(const AdmitPlan& p, cudaStream_t st) {
+  admit_count_kernel<<<p.H, kSelThreads, 0, st>>>(p);
+  return cudaGetLastError();
+}
+cudaError_t launch_admit_select(const AdmitPlan& p, cudaStream_t st) {
+  admit_select_kernel<<<p.H, kSelThreads, 0, st>>>(p);
+  return cudaGetLastError();
+}
+cudaError_t launch_gather_admitted(const AdmitPlan& p, int maxP, cudaStream_t st) {
+  if (maxP <= 0) return cudaSuccess;
+  gather_admitted_kernel<<<dim3((maxP + 7) / 8, p.H), 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+cudaError_t launch_evict_select(const AdmitPlan& p, cudaStream_t st) {
+  evict_select_kernel<<<p.H, kSelThreads, 0, st>>>(p);
+  return cudaGetLastError();
+}
+cudaError_t launch_gather_evicted(const AdmitPlan& p, cudaStream_t st) {
+  gather_evicted_kernel<<<dim3((p.M + 7) / 8, p.H), 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+cudaError_t launch_compact(const AdmitPlan& p, cudaStream_t st) {
+  compact_kernel<<<dim3((p.N + p.M + 7) / 8, p.H), 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+cudaError_t launch_finalize(const AdmitPlan& p, cudaStream_t st) {
+  finalize_kernel<<<dim3((p.M + 255) / 256, p.H), 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace kvb

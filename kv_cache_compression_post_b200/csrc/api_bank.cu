@@ -1,16 +1,432 @@
-// Bank-level C entry points (placeholder until the admit pipeline lands).
-#include "host_util.h"
+// Bank-level C entry points: create/destroy, kvb_admit (DensityKV), export /
+// import, counters and the device status word.  Forcing-KV's prune and the
+// attention entry point live in api_forcing.cu and api_attend.cu.
+#include <climits>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "admit.cuh"
+#include "bank.h"
+#include "gram.cuh"
+#include "small_kernels.cuh"
+
+using namespace kvb;
+
+namespace {
+
+bool config_ok(const kvb_config* c) {
+  if (!c) return false;
+  if (c->method != KVB_DENSITYKV && c->method != KVB_FORCINGKV) return false;
+  if (c->dtype != KVB_BF16 && c->dtype != KVB_F32) return false;
+  if (c->layers < 1 || c->heads < 1 || c->heads > 64) return false;
+  if (c->head_dim != 64 && c->head_dim != 128) return false;
+  if (c->max_queries < 1) return false;
+  if (c->method == KVB_DENSITYKV) {
+    if (c->capacity < 1 || c->max_candidates < 1) return false;
+    if (!(c->eps > 0.f) || !std::isfinite(c->eps) || !(c->s >= 0.f) || !std::isfinite(c->s)) return false;
+    if (!(c->tau > 0.f) || !(c->dist_scale >= 0.f)) return false;
+  } else {
+    if (c->frame_h < 1 || c->frame_w < 1 || c->seg_h < 1 || c->seg_w < 1) return false;
+    if (c->hist_frames < 1 || c->max_new_frames < 1) return false;
+    if (!(c->retention >= 0.f && c->retention <= 1.f)) return false;
+  }
+  return true;
+}
+
+}  // namespace
+
+size_t kvb_bank::layout(void* base) {
+  Carver c(base);
+  const kvb_config& g = cfg;
+  const size_t L = g.layers, H = g.heads, d = g.head_dim;
+  status = c.take<int>(64);
+  if (g.method == KVB_DENSITYKV) {
+    const size_t M = g.capacity, N = g.max_candidates;
+    ldN = static_cast<int>(N);
+    ldEA = static_cast<int>(M + N);
+    ldPart = static_cast<int>(M > N ? M : N);
+    K = c.take<char>(L * H * M * d * elem);
+    V = c.take<char>(L * H * M * d * elem);
+    ids = c.take<int>(L * H * M);
+    rho = c.take<float>(L * H * M);
+    rho0 = c.take<float>(L * H * M);
+    term = c.take<float>(L * H * M);
+    size = c.take<int>(L * H);
+    stats = c.take<kvb_admit_stats>(L * H);
+    cterm = c.take<float>(H * N);
+    rhoB = c.take<float>(H * N);
+    mean0 = c.take<float>(H);
+    feasible = c.take<int>(H);
+    P = c.take<int>(H);
+    E = c.take<int>(H);
+    n_old = c.take<int>(H);
+    nhole = c.take<int>(H);
+    ntail = c.take<int>(H);
+    EAoff = c.take<int>(H);
+    EAcnt = c.take<int>(H);
+    adm_idx = c.take<int>(H * N);
+    EA = c.take<char>(H * (M + N) * d * elem);
+    EAterm = c.take<float>(H * (M + N) + 128);
+    proj = c.take<float>(H * M);
+    ev_slot = c.take<int>(H * M);
+    tail = c.take<int>(H * M);
+    newp = c.take<int>(H * M);
+    sub = c.take<float>(H * M);
+    coadm = c.take<float>(H * N);
+    partial = c.take<float>(8 * H * static_cast<size_t>(ldPart));
+  } else {
+    F = g.frame_h * g.frame_w;
+    n_seg = ((g.frame_h + g.seg_h - 1) / g.seg_h) * ((g.frame_w + g.seg_w - 1) / g.seg_w);
+    ring_cap = g.hist_frames * F;
+    const size_t nf = g.max_new_frames;
+    tK = c.take<char>(L * H * F * d * elem);
+    tV = c.take<char>(L * H * F * d * elem);
+    tids = c.take<int>(L * H * F);
+    tlen = c.take<int>(L * H);
+    rK = c.take<char>(L * H * static_cast<size_t>(ring_cap) * d * elem);
+    rV = c.take<char>(L * H * static_cast<size_t>(ring_cap) * d * elem);
+    rids = c.take<int>(L * H * static_cast<size_t>(ring_cap));
+    fstart = c.take<int>(L * H * g.hist_frames);
+    fcount = c.take<int>(L * H * g.hist_frames);
+    rstate = c.take<int>(L * H * 4);
+    is_static = c.take<uint8_t>(L * H);
+    stats = c.take<kvb_admit_stats>(L * H);
+    sims = c.take<float>(H * nf * n_seg);
+    keep = c.take<int>(H * nf * n_seg);
+    seg_tok = c.take<int>(n_seg + 1);
+    seg_list = c.take<int>(F);
+    plan = c.take<int>(H * nf * F);
+    plan_n = c.take<int>(H);
+  }
+  return c.bytes();
+}
 
 extern "C" {
-size_t kvb_workspace_size(const kvb_config*) { return 0; }
-kvb_status kvb_bank_create(const kvb_config*, void*, size_t, void*, kvb_bank**) { return KVB_E_UNSUPPORTED; }
-kvb_status kvb_bank_destroy(kvb_bank*) { return KVB_E_UNSUPPORTED; }
-kvb_status kvb_admit(kvb_bank*, int32_t, const void*, const void*, const int32_t*, int32_t, void*) { return KVB_E_UNSUPPORTED; }
-kvb_status kvb_prune_hybrid(kvb_bank*, int32_t, const uint8_t*, const void*, const void*, const void*, const int32_t*, int32_t, void*) { return KVB_E_UNSUPPORTED; }
-kvb_status kvb_attend(kvb_bank*, int32_t, const void*, int32_t, const void*, const void*, int32_t, const void*, const void*, int32_t, void*, float*, void*) { return KVB_E_UNSUPPORTED; }
-kvb_status kvb_read_stats(kvb_bank*, int32_t, kvb_admit_stats*, void*) { return KVB_E_UNSUPPORTED; }
-kvb_status kvb_bank_export(kvb_bank*, int32_t, int32_t, int32_t*, float*, float*, void*, void*, int32_t*, void*) { return KVB_E_UNSUPPORTED; }
-kvb_status kvb_bank_import(kvb_bank*, int32_t, int32_t, const int32_t*, const float*, const float*, const void*, const void*, int32_t, void*) { return KVB_E_UNSUPPORTED; }
-kvb_status kvb_device_status(kvb_bank*, void*) { return KVB_E_UNSUPPORTED; }
-kvb_status kvb_segment_cosine(const void*, const void*, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, kvb_dtype, float*, void*) { return KVB_E_UNSUPPORTED; }
+
+size_t kvb_workspace_size(const kvb_config* cfg) {
+  if (!config_ok(cfg)) return 0;
+  kvb_bank b;
+  b.cfg = *cfg;
+  b.elem = cfg->dtype == KVB_BF16 ? 2 : 4;
+  return b.layout(nullptr);
 }
+
+// implemented in api_forcing.cu
+kvb_status kvb_forcing_init(kvb_bank* b, cudaStream_t st);
+
+kvb_status kvb_bank_create(const kvb_config* cfg, void* workspace, size_t workspace_bytes, void* stream,
+                           kvb_bank** out) {
+  if (!out || !config_ok(cfg)) return KVB_E_INVAL;
+  *out = nullptr;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return KVB_E_WORKSPACE;
+  DeviceInfo dev;
+  if (!current_device(&dev)) return KVB_E_CUDA;
+  if (dev.cc_major != 10) return KVB_E_UNSUPPORTED;
+  kvb_bank* b = new (std::nothrow) kvb_bank();
+  if (!b) return KVB_E_INVAL;
+  b->cfg = *cfg;
+  b->elem = cfg->dtype == KVB_BF16 ? 2 : 4;
+  b->row_bytes = cfg->head_dim * b->elem;
+  b->h = cfg->dist_scale > 0.f ? cfg->dist_scale : static_cast<float>(cfg->head_dim);
+  const size_t need = b->layout(nullptr);
+  if (workspace_bytes < need) {
+    delete b;
+    return KVB_E_WORKSPACE;
+  }
+  b->ws = workspace;
+  b->ws_bytes = workspace_bytes;
+  b->layout(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t LH = static_cast<size_t>(cfg->layers) * cfg->heads;
+  cudaError_t e = cudaMemsetAsync(b->status, 0, sizeof(int), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(b->stats, 0, LH * sizeof(kvb_admit_stats), st);
+  if (cfg->method == KVB_DENSITYKV) {
+    if (e == cudaSuccess) e = cudaMemsetAsync(b->size, 0, LH * sizeof(int), st);
+  } else if (e == cudaSuccess) {
+    const kvb_status fs = kvb_forcing_init(b, st);
+    if (fs != KVB_OK) {
+      delete b;
+      return fs;
+    }
+  }
+  if (e != cudaSuccess) {
+    delete b;
+    return KVB_E_CUDA;
+  }
+  *out = b;
+  return KVB_OK;
+}
+
+kvb_status kvb_bank_destroy(kvb_bank* bank) {
+  if (!bank) return KVB_E_INVAL;
+  delete bank;
+  return KVB_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// One density pass: out[h][r] = sum over the column set of sign * phi, through the
+// tcgen05 kernel (bf16) or the CUDA-core kernel (f32).
+struct Pass {
+  const void* R;       // rows buffer [H][ldR][d]
+  long long ldR;
+  GramSet rows;
+  const float* rowTerm;
+  int ldRT;
+  const void* C;
+  long long ldC;
+  GramSet cols;
+  const float* colTerm;
+  int ldCT;
+  int max_rows;
+  int max_cols;
+  int use_diag = 0;
+  int nneg = 0;
+  float* out;
+  int ldOut;
+};
+
+cudaError_t run_pass(kvb_bank* b, const Pass& ps, const DeviceInfo& dev, cudaStream_t st) {
+  const kvb_config& g = b->cfg;
+  GramArgs a;
+  a.H = g.heads;
+  a.d = g.head_dim;
+  a.rows = ps.rows;
+  a.cols = ps.cols;
+  a.rowTerm = ps.rowTerm;
+  a.ldRT = ps.ldRT;
+  a.colTerm = ps.colTerm;
+  a.ldCT = ps.ldCT;
+  a.use_diag = ps.use_diag;
+  a.diag_uni = 0;
+  a.nneg_uni = ps.nneg;
+  a.kscale = -2.f / b->h;
+  a.eps = g.eps;
+  a.s = g.s;
+  a.max_rows = ps.max_rows;
+  a.status = b->status;
+  if (g.dtype == KVB_F32) {
+    a.R32 = static_cast<const float*>(ps.R);
+    a.C32 = static_cast<const float*>(ps.C);
+    a.ldR = static_cast<int>(ps.ldR);
+    a.ldC = static_cast<int>(ps.ldC);
+    a.partial = ps.out;
+    a.ldOut = ps.ldOut;
+    return launch_gram_f32(a, st);
+  }
+  CUtensorMap tmR, tmC;
+  if (!make_tmap_bf16(&tmR, ps.R, g.head_dim, ps.ldR, g.heads, 128) ||
+      !make_tmap_bf16(&tmC, ps.C, g.head_dim, ps.ldC, g.heads, 128))
+    return cudaErrorInvalidValue;
+  a.partial = b->partial;
+  a.ldOut = b->ldPart;
+  gram_plan(a, (ps.max_cols + 127) / 128, dev.n_sm);
+  cudaError_t e = launch_gram_bf16(a, tmR, tmC, dev.n_sm, st);
+  if (e == cudaSuccess) e = launch_gram_reduce(a, ps.out, ps.ldOut, st);
+  return e;
+}
+
+}  // namespace
+
+extern "C" kvb_status kvb_admit(kvb_bank* b, int32_t layer, const void* candK, const void* candV,
+                                const int32_t* cand_ids, int32_t N, void* stream) {
+  if (!b) return KVB_E_INVAL;
+  const kvb_config& g = b->cfg;
+  if (g.method != KVB_DENSITYKV) return KVB_E_STATE;
+  if (layer < 0 || layer >= g.layers || N < 1 || N > g.max_candidates) return KVB_E_INVAL;
+  if (!candK || !candV || !cand_ids) return KVB_E_INVAL;
+  DeviceInfo dev;
+  if (!current_device(&dev)) return KVB_E_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int H = g.heads, M = g.capacity, d = g.head_dim;
+  const size_t lo = static_cast<size_t>(layer) * H * M;  // slot offset of this layer
+
+  AdmitPlan p;
+  p.H = H;
+  p.M = M;
+  p.N = N;
+  p.d = d;
+  p.dtype = g.dtype;
+  p.row_bytes = b->row_bytes;
+  p.tau = g.tau;
+  p.sync_heads = g.sync_heads;
+  p.K = b->K + lo * b->row_bytes;
+  p.V = b->V + lo * b->row_bytes;
+  p.ids = b->ids + lo;
+  p.rho = b->rho + lo;
+  p.rho0 = b->rho0 + lo;
+  p.term = b->term + lo;
+  p.size = b->size + static_cast<size_t>(layer) * H;
+  p.stats = b->stats + static_cast<size_t>(layer) * H;
+  p.candK = candK;
+  p.candV = candV;
+  p.cand_ids = cand_ids;
+  p.cterm = b->cterm;
+  p.rhoB = b->rhoB;
+  p.mean0 = b->mean0;
+  p.feasible = b->feasible;
+  p.P = b->P;
+  p.adm_idx = b->adm_idx;
+  p.EA = b->EA;
+  p.EAterm = b->EAterm;
+  p.ldEA = b->ldEA;
+  p.EAoff = b->EAoff;
+  p.EAcnt = b->EAcnt;
+  p.proj = b->proj;
+  p.ev_slot = b->ev_slot;
+  p.E = b->E;
+  p.n_old = b->n_old;
+  p.hole = b->ev_slot;
+  p.nhole = b->nhole;
+  p.tail = b->tail;
+  p.ntail = b->ntail;
+  p.newp = b->newp;
+  p.sub = b->sub;
+  p.coadm = b->coadm;
+  p.ldN = b->ldN;
+  p.status = b->status;
+
+  const float inv_h = 1.f / b->h;
+  cudaError_t e = launch_row_terms(candK, g.dtype, H, N, d, N, nullptr, N, inv_h, 0.f, b->cterm, b->ldN, st);
+
+  // pass 1: candidate density against the bank, rho_B(c)
+  if (e == cudaSuccess) {
+    Pass ps{candK, N, GramSet{N, nullptr, 0, nullptr}, b->cterm, b->ldN,
+            p.K, M, GramSet{0, p.size, 0, nullptr}, p.term, M, N, M};
+    ps.out = b->rhoB;
+    ps.ldOut = b->ldN;
+    e = run_pass(b, ps, dev, st);
+  }
+  if (e == cudaSuccess) e = launch_admit_count(p, st);
+  if (e == cudaSuccess) e = launch_admit_select(p, st);
+  if (e == cudaSuccess) e = launch_gather_admitted(p, N < M ? N : M, st);
+  // pass 2: projected growth of every bank entry from the admitted block
+  if (e == cudaSuccess) {
+    Pass ps{p.K, M, GramSet{0, p.size, 0, nullptr}, p.term, M,
+            b->EA, b->ldEA, GramSet{0, b->P, M, nullptr}, b->EAterm, b->ldEA, M, N};
+    ps.out = b->proj;
+    ps.ldOut = M;
+    e = run_pass(b, ps, dev, st);
+  }
+  if (e == cudaSuccess) e = launch_evict_select(p, st);
+  if (e == cudaSuccess) e = launch_gather_evicted(p, st);
+  if (e == cudaSuccess) e = launch_compact(p, st);
+  // pass 3a: every entry of the new bank loses its evicted neighbours
+  if (e == cudaSuccess) {
+    Pass ps{p.K, M, GramSet{0, p.size, 0, nullptr}, p.term, M,
+            b->EA, b->ldEA, GramSet{0, b->EAcnt, 0, b->EAoff}, b->EAterm, b->ldEA, M, M};
+    ps.nneg = INT_MAX;
+    ps.out = b->sub;
+    ps.ldOut = M;
+    e = run_pass(b, ps, dev, st);
+  }
+  // pass 3b: co-admitted entries see one another (self excluded)
+  if (e == cudaSuccess) {
+    Pass ps{b->EA, b->ldEA, GramSet{0, b->P, M, nullptr}, b->EAterm, b->ldEA,
+            b->EA, b->ldEA, GramSet{0, b->P, M, nullptr}, b->EAterm, b->ldEA, N, N};
+    ps.use_diag = 1;
+    ps.out = b->coadm;
+    ps.ldOut = b->ldN;
+    e = run_pass(b, ps, dev, st);
+  }
+  if (e == cudaSuccess) e = launch_finalize(p, st);
+  return cuda_status(e);
+}
+
+extern "C" {
+
+kvb_status kvb_read_stats(kvb_bank* b, int32_t layer, kvb_admit_stats* host_out, void* stream) {
+  if (!b || !host_out || layer < 0 || layer >= b->cfg.layers) return KVB_E_INVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int H = b->cfg.heads;
+  cudaError_t e = cudaMemcpyAsync(host_out, b->stats + static_cast<size_t>(layer) * H,
+                                  sizeof(kvb_admit_stats) * H, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  return cuda_status(e);
+}
+
+kvb_status kvb_device_status(kvb_bank* b, void* stream) {
+  if (!b) return KVB_E_INVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, b->status, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return KVB_E_CUDA;
+  return static_cast<kvb_status>(v);
+}
+
+// implemented in api_forcing.cu
+kvb_status kvb_forcing_export(kvb_bank* b, int32_t layer, int32_t head, int32_t* ids, void* K, void* V,
+                              int32_t* size, cudaStream_t st);
+
+kvb_status kvb_bank_export(kvb_bank* b, int32_t layer, int32_t head, int32_t* ids, float* rho, float* rho0,
+                           void* K, void* V, int32_t* size, void* stream) {
+  if (!b || !size || layer < 0 || layer >= b->cfg.layers || head < 0 || head >= b->cfg.heads)
+    return KVB_E_INVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (b->cfg.method == KVB_FORCINGKV) return kvb_forcing_export(b, layer, head, ids, K, V, size, st);
+  const int M = b->cfg.capacity;
+  const size_t slot0 = (static_cast<size_t>(layer) * b->cfg.heads + head) * M;
+  int n = 0;
+  cudaError_t e = cudaMemcpyAsync(&n, b->size + static_cast<size_t>(layer) * b->cfg.heads + head, sizeof(int),
+                                  cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return KVB_E_CUDA;
+  if (n < 0 || n > M) return KVB_E_DEVICE_BOUNDS;
+  *size = n;
+  if (n == 0) return KVB_OK;
+  if (ids && e == cudaSuccess)
+    e = cudaMemcpyAsync(ids, b->ids + slot0, sizeof(int) * n, cudaMemcpyDeviceToDevice, st);
+  if (rho && e == cudaSuccess)
+    e = cudaMemcpyAsync(rho, b->rho + slot0, sizeof(float) * n, cudaMemcpyDeviceToDevice, st);
+  if (rho0 && e == cudaSuccess)
+    e = cudaMemcpyAsync(rho0, b->rho0 + slot0, sizeof(float) * n, cudaMemcpyDeviceToDevice, st);
+  if (K && e == cudaSuccess)
+    e = cudaMemcpyAsync(K, b->K + slot0 * b->row_bytes, static_cast<size_t>(n) * b->row_bytes,
+                        cudaMemcpyDeviceToDevice, st);
+  if (V && e == cudaSuccess)
+    e = cudaMemcpyAsync(V, b->V + slot0 * b->row_bytes, static_cast<size_t>(n) * b->row_bytes,
+                        cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  return cuda_status(e);
+}
+
+kvb_status kvb_bank_import(kvb_bank* b, int32_t layer, int32_t head, const int32_t* ids, const float* rho,
+                           const float* rho0, const void* K, const void* V, int32_t size, void* stream) {
+  if (!b || layer < 0 || layer >= b->cfg.layers || head < 0 || head >= b->cfg.heads) return KVB_E_INVAL;
+  if (b->cfg.method != KVB_DENSITYKV) return KVB_E_STATE;
+  const int M = b->cfg.capacity;
+  if (size < 0 || size > M) return KVB_E_INVAL;
+  if (size > 0 && (!ids || !rho || !rho0 || !K || !V)) return KVB_E_INVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t slot0 = (static_cast<size_t>(layer) * b->cfg.heads + head) * M;
+  cudaError_t e = cudaSuccess;
+  if (size > 0) {
+    e = cudaMemcpyAsync(b->ids + slot0, ids, sizeof(int) * size, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(b->rho + slot0, rho, sizeof(float) * size, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(b->rho0 + slot0, rho0, sizeof(float) * size, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(b->K + slot0 * b->row_bytes, K, static_cast<size_t>(size) * b->row_bytes,
+                          cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(b->V + slot0 * b->row_bytes, V, static_cast<size_t>(size) * b->row_bytes,
+                          cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess)
+      e = launch_row_terms(b->K + slot0 * b->row_bytes, b->cfg.dtype, 1, size, b->cfg.head_dim, size, nullptr,
+                           size, 1.f / b->h, 0.f, b->term + slot0, size, st);
+  }
+  // the size word comes from host memory; the call synchronises before returning
+  int host_size = size;
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(b->size + static_cast<size_t>(layer) * b->cfg.heads + head, &host_size, sizeof(int),
+                        cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  return cuda_status(e);
+}
+
+}  // extern "C"

@@ -106,7 +106,7 @@ kvb_status kvb_density(const void* rows, int32_t n_rows, const void* cols, int32
     return cuda_status(launch_gram_f32(a, st));
   }
   if (n_cols == 0) return cuda_status(cudaMemsetAsync(out, 0, sizeof(float) * heads * n_rows, st));
-  cudaError_t e = launch_row_terms(rows, dtype, heads, n_rows, head_dim, n_rows, nullptr, n_rows, 1.f / h, eps,
+  cudaError_t e = launch_row_terms(rows, dtype, heads, n_rows, head_dim, n_rows, nullptr, n_rows, 1.f / h, 0.f,
                                    L.rowTerm, n_rows, st);
   if (e == cudaSuccess)
     e = launch_row_terms(cols, dtype, heads, n_cols, head_dim, n_cols, nullptr, n_cols, 1.f / h, 0.f, L.colTerm,

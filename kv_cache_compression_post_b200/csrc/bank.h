@@ -1,0 +1,78 @@
+// Host-side bank object: where every array of the bank lives in the caller's
+// workspace.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/kvb.h"
+#include "host_util.h"
+
+struct kvb_bank {
+  kvb_config cfg;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  int elem = 2;             // bytes per K/V element
+  int row_bytes = 0;        // d * elem
+  float h = 0.f;            // distance scale
+  int F = 0;                // tokens per frame (Forcing-KV)
+  int n_seg = 0;            // segments per frame (Forcing-KV)
+  int ring_cap = 0;         // tokens a dynamic head's FIFO can hold
+  int* status = nullptr;
+
+  // ---- DensityKV, per layer: base pointers of layer 0 and strides
+  char* K = nullptr;        // [L][H][M][d]
+  char* V = nullptr;
+  int* ids = nullptr;       // [L][H][M]
+  float* rho = nullptr;
+  float* rho0 = nullptr;
+  float* term = nullptr;
+  int* size = nullptr;      // [L][H]
+  kvb_admit_stats* stats = nullptr;  // [L][H]
+
+  // ---- DensityKV scratch (shared by layers)
+  int ldN = 0, ldEA = 0, ldPart = 0;
+  float* cterm = nullptr;
+  float* rhoB = nullptr;
+  float* mean0 = nullptr;
+  int* feasible = nullptr;
+  int* P = nullptr;
+  int* E = nullptr;
+  int* n_old = nullptr;
+  int* nhole = nullptr;
+  int* ntail = nullptr;
+  int* EAoff = nullptr;
+  int* EAcnt = nullptr;
+  int* adm_idx = nullptr;
+  char* EA = nullptr;
+  float* EAterm = nullptr;
+  float* proj = nullptr;
+  int* ev_slot = nullptr;
+  int* tail = nullptr;
+  int* newp = nullptr;
+  float* sub = nullptr;
+  float* coadm = nullptr;
+  float* partial = nullptr;
+
+  // ---- Forcing-KV, per layer
+  char* tK = nullptr;       // [L][H][F][d] transition frame (static heads)
+  char* tV = nullptr;
+  int* tids = nullptr;      // [L][H][F]
+  int* tlen = nullptr;      // [L][H] transition length (0 before the first prune)
+  char* rK = nullptr;       // [L][H][ring_cap][d] FIFO of pruned frames (dynamic heads)
+  char* rV = nullptr;
+  int* rids = nullptr;      // [L][H][ring_cap]
+  int* fstart = nullptr;    // [L][H][hist_frames] ring position of each stored frame
+  int* fcount = nullptr;    // [L][H][hist_frames]
+  int* rstate = nullptr;    // [L][H][4]: first frame slot, frames held, token start, tokens held
+  uint8_t* is_static = nullptr;  // [L][H] labels of the last prune
+  // ---- Forcing-KV scratch
+  float* sims = nullptr;    // [H][max_new_frames][n_seg]
+  int* keep = nullptr;      // [H][max_new_frames][n_seg] kept segment ids, ascending
+  int* seg_tok = nullptr;   // [n_seg + 1] token offsets of each segment in segment-major order
+  int* seg_list = nullptr;  // [F] token index (row-major) in segment-major order
+  int* plan = nullptr;      // [H][max_new_frames*F] source token -> ring position
+  int* plan_n = nullptr;    // [H]
+
+  size_t layout(void* base);  // carve (base may be null to measure); returns bytes
+};

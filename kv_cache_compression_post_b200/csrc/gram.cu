@@ -271,7 +271,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
         row = rt0 + row_in_tile;
         active = r < nact_of(c);
         valid_row = active && row < c.nR;
-        ra = valid_row ? a.rowTerm[static_cast<size_t>(c.h) * a.ldRT + c.rOff + row] : 0.f;
+        ra = (valid_row ? a.rowTerm[static_cast<size_t>(c.h) * a.ldRT + c.rOff + row] : 0.f) + eps;
         nneg = a.nneg_dev ? a.nneg_dev[c.h] : a.nneg_uni;
         diag = a.use_diag ? (a.diag_dev ? a.diag_dev[c.h] : a.diag_uni) : INT_MIN / 2;
         acc_pos = 0.f;

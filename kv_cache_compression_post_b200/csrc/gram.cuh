@@ -27,7 +27,7 @@ struct GramArgs {
   int H = 0;
   int d = 0;
   GramSet rows, cols;
-  const float* rowTerm = nullptr;  // [H][ldRT]: ||r||^2/h + eps   (indexed off+r)
+  const float* rowTerm = nullptr;  // [H][ldRT]: ||r||^2/h         (indexed off+r)
   int ldRT = 0;
   const float* colTerm = nullptr;  // [H][ldCT]: ||c||^2/h         (indexed off+c)
   int ldCT = 0;

@@ -13,7 +13,7 @@ import os
 from typing import Optional
 
 __all__ = [
-    "KvbError", "kvb_config", "kvb_admit_stats", "make_config", "lib", "LIB_PATH",
+    "KvbError", "kvb_config", "kvb_admit_stats", "make_config", "lib", "LIB_PATH", "Bank",
     "KVB_BF16", "KVB_F32", "KVB_DENSITYKV", "KVB_FORCINGKV",
     "kvb_workspace_size", "kvb_bank_create", "kvb_bank_destroy", "kvb_admit", "kvb_prune_hybrid",
     "kvb_attend", "kvb_read_stats", "kvb_bank_export", "kvb_bank_import", "kvb_device_status",
@@ -145,7 +145,10 @@ def kvb_prune_hybrid(bank: int, layer: int, head_is_static, newK, newV, nextK, n
                      stream=None) -> None:
     """head_is_static: host bytes / bytearray / numpy uint8 array of length H."""
     import numpy as np
-    arr = np.ascontiguousarray(np.asarray(head_is_static, dtype=np.uint8))
+    if isinstance(head_is_static, (bytes, bytearray)):
+        arr = np.frombuffer(bytes(head_is_static), dtype=np.uint8).copy()
+    else:
+        arr = np.ascontiguousarray(np.asarray(head_is_static, dtype=np.uint8))
     _check(lib.kvb_prune_hybrid(bank, layer, arr.ctypes.data, _ptr(newK), _ptr(newV), _ptr(nextK),
                                 _ptr(new_ids), n_frames, _stream(stream)), "kvb_prune_hybrid")
 
@@ -195,3 +198,63 @@ def kvb_segment_cosine(K, nextK, heads: int, n_frames: int, frame_h: int, frame_
                        head_dim: int, dtype: int, sim, stream=None) -> None:
     _check(lib.kvb_segment_cosine(_ptr(K), _ptr(nextK), heads, n_frames, frame_h, frame_w, seg_h, seg_w, head_dim,
                                   dtype, _ptr(sim), _stream(stream)), "kvb_segment_cosine")
+
+
+class Bank:
+    """A kvb bank whose workspace is a torch uint8 tensor on the current device.
+
+    Marshalling only: every method calls the C entry point of the same name."""
+
+    def __init__(self, cfg: kvb_config, stream=None):
+        import torch
+        self.cfg = cfg
+        self.nbytes = kvb_workspace_size(cfg)
+        if self.nbytes == 0:
+            raise KvbError(1, "kvb_workspace_size")
+        self._buf = torch.empty(self.nbytes + 256, dtype=torch.uint8, device="cuda")
+        self.ws = (self._buf.data_ptr() + 255) & ~255
+        self.handle = kvb_bank_create(cfg, self.ws, self.nbytes, stream)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            kvb_bank_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def admit(self, layer, candK, candV, cand_ids, stream=None):
+        kvb_admit(self.handle, layer, candK, candV, cand_ids, cand_ids.shape[0], stream)
+
+    def prune_hybrid(self, layer, head_is_static, newK, newV, nextK, new_ids, n_frames, stream=None):
+        kvb_prune_hybrid(self.handle, layer, head_is_static, newK, newV, nextK, new_ids, n_frames, stream)
+
+    def attend(self, layer, Q, sinkK, sinkV, winK, winV, O, lse=None, stream=None):
+        kvb_attend(self.handle, layer, Q, Q.shape[1], sinkK, sinkV, sinkK.shape[1], winK, winV, winK.shape[1],
+                   O, lse, stream)
+
+    def stats(self, layer, stream=None):
+        return kvb_read_stats(self.handle, layer, self.cfg.heads, stream)
+
+    def status(self, stream=None) -> int:
+        return kvb_device_status(self.handle, stream)
+
+    def export(self, layer, head, stream=None):
+        """(ids, rho, rho0, K, V) torch tensors of one (layer, head) bank or history."""
+        import torch
+        cap = self.cfg.capacity if self.cfg.method == KVB_DENSITYKV else \
+            self.cfg.hist_frames * self.cfg.frame_h * self.cfg.frame_w
+        dt = torch.bfloat16 if self.cfg.dtype == KVB_BF16 else torch.float32
+        ids = torch.empty(cap, dtype=torch.int32, device="cuda")
+        rho = torch.zeros(cap, dtype=torch.float32, device="cuda")
+        rho0 = torch.zeros(cap, dtype=torch.float32, device="cuda")
+        K = torch.empty(cap, self.cfg.head_dim, dtype=dt, device="cuda")
+        V = torch.empty(cap, self.cfg.head_dim, dtype=dt, device="cuda")
+        n = kvb_bank_export(self.handle, layer, head, ids, rho, rho0, K, V, stream)
+        return ids[:n], rho[:n], rho0[:n], K[:n], V[:n]
+
+    def import_(self, layer, head, ids, rho, rho0, K, V, stream=None):
+        kvb_bank_import(self.handle, layer, head, ids, rho, rho0, K, V, int(ids.shape[0]), stream)

@@ -97,6 +97,8 @@ class AdmitResult:
     rho_new: List[np.ndarray]        # from-scratch density of the new bank entries
     near_ties: int                   # decisions with relative margin < tie_margin
     margins: dict
+    tie_cand_ids: List[set] = None   # per head: candidate ids in a near-tie decision
+    tie_bank_ids: List[set] = None   # per head: old bank ids in a near-tie decision
 
 
 def _lex_order(primary: np.ndarray, ids: np.ndarray) -> np.ndarray:
@@ -178,8 +180,9 @@ def admit(banks: List[HeadBank], cand_ids: np.ndarray, candK: np.ndarray, candV:
 
     margins = _margins(p, score, P_h, P_all, admitted, ratio, mand, evicted, n_cap, banks, cand_ids)
     near = sum(int((m < tie_margin).sum()) for m in margins.values())
+    tc, tb = _tie_ids(p, score, P_h, P_all, ratio, mand, n_cap, banks, cand_ids, tie_margin)
     return AdmitResult(new_banks, P_all[0] if p.sync_heads else -1, P_h, rho_cand, score, admitted,
-                       rho_cur, proj, ratio, mand, evicted, np.array(n_cap), rho_new, near, margins)
+                       rho_cur, proj, ratio, mand, evicted, np.array(n_cap), rho_new, near, margins, tc, tb)
 
 
 def _rel(a, b):
@@ -217,6 +220,37 @@ def _margins(p, score, P_h, P_all, admitted, ratio, mand, evicted, n_cap, banks,
                 b = ratio[hh][rest[order[n_cap[hh]]]]
                 out["ev_cut"].append(np.array([_rel(b, a) if a != 0 else 1.0]))
     return {k: (np.concatenate(v) if v else np.zeros(0)) for k, v in out.items()}
+
+
+def _tie_ids(p, score, P_h, P_all, ratio, mand, n_cap, banks, cand_ids, m):
+    """Ids whose admit/evict decision could flip under a relative perturbation < m."""
+    tc, tb = [], []
+    for hh in range(len(score)):
+        c, b = set(), set()
+        if banks[hh].size and banks[hh].rho0.mean() > 0:
+            c |= set(cand_ids[_rel(score[hh], p.tau) < m].tolist())
+        P = P_all[hh]
+        if 0 < P < int(P_h[hh]):
+            order = _lex_order(score[hh], cand_ids)
+            lo, hi = score[hh][order[P - 1]], score[hh][order[P]]
+            close = np.abs(score[hh] - lo) <= m * max(abs(lo), 1e-300)
+            if _rel(hi, lo) < m:
+                c |= set(cand_ids[close | (np.abs(score[hh] - hi) <= m * max(abs(hi), 1e-300))].tolist())
+        ids = banks[hh].ids
+        if banks[hh].size:
+            b |= set(ids[_rel(ratio[hh], p.tau) < m].tolist())
+        if n_cap[hh] > 0:
+            rest = np.nonzero(~mand[hh])[0]
+            order = _lex_order(-ratio[hh][rest], ids[rest])
+            if n_cap[hh] < rest.size:
+                lo = ratio[hh][rest[order[n_cap[hh] - 1]]]
+                hi = ratio[hh][rest[order[n_cap[hh]]]]
+                if _rel(hi, lo) < m:
+                    r = ratio[hh]
+                    b |= set(ids[(np.abs(r - lo) <= m * abs(lo)) | (np.abs(r - hi) <= m * abs(hi))].tolist())
+        tc.append(c)
+        tb.append(b)
+    return tc, tb
 
 
 def densities_from_scratch(bank: HeadBank, p: Params) -> np.ndarray:

@@ -1,0 +1,145 @@
+"""GPU parity of the DensityKV admit step (kvb_admit) against the fp64 oracle.
+
+* tiny fp32 workload (2 heads, d 64, M 384): the whole 7-step rollout runs on the
+  GPU from an empty bank; every step's bank must equal the oracle's exactly (id
+  sets), densities within 1e-4, K/V pairing intact.  This workload has no
+  near-tie decision (checked).
+* mid bf16 workload (4 heads, d 128, 170-token frames, M 900: several 128-row
+  tiles with ragged tails): stepwise -- the oracle's bank before step i is
+  imported, one GPU step runs, and its bank is compared with the oracle's step
+  i; id sets may differ only on decisions within 1e-4 of their threshold or cut.
+"""
+import numpy as np
+import pytest
+
+import kvgen
+from oracle import densitykv as dkv
+from tests.gpu_util import dev_ids, dev_tensor, host
+
+pytestmark = pytest.mark.gpu
+
+RTOL = 1e-4
+
+
+def _cfg(w, tau=None, sync=1, layers=1):
+    import kv_cache_compression_post_b200 as kvb
+    return kvb.make_config(method=kvb.KVB_DENSITYKV, dtype=kvb.KVB_BF16 if w.dtype == "bf16" else kvb.KVB_F32,
+                           layers=layers, heads=w.heads, head_dim=w.head_dim, capacity=w.capacity,
+                           max_candidates=w.chunk_tokens, tau=w.tau if tau is None else tau, eps=w.eps, s=w.s,
+                           sync_heads=sync, max_queries=w.chunk_tokens)
+
+
+def _export(bank, layer, H):
+    out = []
+    for hh in range(H):
+        ids, rho, rho0, K, V = bank.export(layer, hh)
+        out.append(dict(ids=host(ids).astype(np.int64), rho=host(rho).astype(np.float64),
+                        rho0=host(rho0).astype(np.float64), K=host(K), V=host(V)))
+    return out
+
+
+def _compare(g, r, hh, exact=True, tie_ids=frozenset()):
+    """g: exported GPU bank of head hh; r: oracle AdmitResult after the same step."""
+    ob = r.banks[hh]
+    gs, os_ = set(g["ids"].tolist()), set(ob.ids.tolist())
+    diff = gs ^ os_
+    if exact:
+        assert not diff, f"head {hh}: ids differ {sorted(diff)[:10]}"
+    else:
+        assert diff <= set(tie_ids), f"head {hh}: ids differ outside near ties: {sorted(diff - set(tie_ids))[:10]}"
+    # K/V pairing through the carried ids
+    np.testing.assert_array_equal(kvgen.untag_ids(g["V"]), g["ids"])
+    if diff:
+        return False
+    order = np.argsort(g["ids"])
+    oo = np.argsort(ob.ids)
+    np.testing.assert_array_equal(g["K"][order], ob.K[oo].astype(np.float32))
+    np.testing.assert_allclose(g["rho"][order], r.rho_new[hh][oo], rtol=RTOL)
+    np.testing.assert_allclose(g["rho0"][order], ob.rho0[oo], rtol=RTOL)
+    return True
+
+
+def test_tiny_rollout_matches_oracle_exactly():
+    import torch
+    import kv_cache_compression_post_b200 as kvb
+    w = kvgen.WORKLOADS["tiny"]
+    L = kvgen.LayerInputs(w, 0, tagged=True)
+    p = dkv.Params(capacity=w.capacity, tau=w.tau, eps=w.eps, s=w.s)
+    bank = kvb.Bank(_cfg(w))
+    banks = [dkv.HeadBank.empty(w.head_dim) for _ in range(w.heads)]
+    for i in range(1, w.n_chunks):
+        x = L.step(i)
+        r = dkv.admit(banks, x["cand_ids"], x["candK"], x["candV"], p)
+        assert r.near_ties == 0
+        bank.admit(0, dev_tensor(x["candK"], "f32"), dev_tensor(x["candV"], "f32"), dev_ids(x["cand_ids"]))
+        torch.cuda.synchronize()
+        assert bank.status() == 0
+        st = bank.stats(0)
+        g = _export(bank, 0, w.heads)
+        for hh in range(w.heads):
+            _compare(g[hh], r, hh, exact=True)
+            assert st[hh]["admitted"] == len(r.admitted[hh])
+            assert st[hh]["mandatory"] == int(r.mandatory[hh].sum())
+            assert st[hh]["capacity_evicted"] == int(r.n_capacity[hh])
+            assert st[hh]["size"] == r.banks[hh].size
+        banks = r.banks
+    bank.close()
+
+
+def _import(bank, banks, p, w):
+    import torch
+    for hh, b in enumerate(banks):
+        n = b.size
+        if n == 0:
+            bank.import_(0, hh, torch.zeros(0, dtype=torch.int32, device="cuda"), None, None, None, None)
+            continue
+        rho = dkv.densities_from_scratch(b, p)
+        bank.import_(0, hh, dev_ids(b.ids), dev_tensor(rho, "f32"), dev_tensor(b.rho0, "f32"),
+                     dev_tensor(b.K, w.dtype), dev_tensor(b.V, w.dtype))
+
+
+@pytest.mark.parametrize("tau,sync", [(2.0, 1), (1.0, 1), (1.0, 0)])
+def test_mid_stepwise_matches_oracle(tau, sync):
+    import torch
+    import kv_cache_compression_post_b200 as kvb
+    w = kvgen.WORKLOADS["mid"]
+    L = kvgen.LayerInputs(w, 0, tagged=True)
+    p = dkv.Params(capacity=w.capacity, tau=tau, eps=w.eps, s=w.s, sync_heads=bool(sync))
+    bank = kvb.Bank(_cfg(w, tau=tau, sync=sync))
+    banks = [dkv.HeadBank.empty(w.head_dim) for _ in range(w.heads)]
+    exact_steps = 0
+    for i in range(1, w.n_chunks):
+        x = L.step(i)
+        r = dkv.admit(banks, x["cand_ids"], x["candK"], x["candV"], p)
+        _import(bank, banks, p, w)
+        bank.admit(0, dev_tensor(x["candK"], w.dtype), dev_tensor(x["candV"], w.dtype), dev_ids(x["cand_ids"]))
+        torch.cuda.synchronize()
+        assert bank.status() == 0
+        g = _export(bank, 0, w.heads)
+        all_exact = True
+        for hh in range(w.heads):
+            ties = r.tie_cand_ids[hh] | r.tie_bank_ids[hh]
+            all_exact &= _compare(g[hh], r, hh, exact=False, tie_ids=ties)
+        exact_steps += int(all_exact)
+        banks = r.banks
+    assert exact_steps >= (w.n_chunks - 1) // 2
+    bank.close()
+
+
+def test_admit_argument_errors():
+    import torch
+    import kv_cache_compression_post_b200 as kvb
+    w = kvgen.WORKLOADS["mid"]
+    bank = kvb.Bank(_cfg(w))
+    K = torch.zeros(w.heads, 10, w.head_dim, dtype=torch.bfloat16, device="cuda")
+    ids = torch.arange(10, dtype=torch.int32, device="cuda")
+    with pytest.raises(kvb.KvbError) as e:
+        kvb.kvb_admit(bank.handle, 1, K, K, ids, 10)          # layer out of range
+    assert e.value.status == 1
+    with pytest.raises(kvb.KvbError) as e:
+        kvb.kvb_admit(bank.handle, 0, K, K, ids, w.chunk_tokens + 1)   # N above max_candidates
+    assert e.value.status == 1
+    with pytest.raises(kvb.KvbError) as e:
+        kvb.kvb_prune_hybrid(bank.handle, 0, bytes(w.heads), K, K, K, ids, 1)  # wrong method
+    assert e.value.status in (6, 7)
+    bank.close()
