@@ -92,6 +92,7 @@ size_t kvb_bank::layout(void* base) {
     fcount = c.take<int>(L * H * g.hist_frames);
     rstate = c.take<int>(L * H * 4);
     is_static = c.take<uint8_t>(L * H);
+    aseg = c.take<int>(L * 4 * H);
     stats = c.take<kvb_admit_stats>(L * H);
     sims = c.take<float>(H * nf * n_seg);
     keep = c.take<int>(H * nf * n_seg);
@@ -143,7 +144,12 @@ kvb_status kvb_bank_create(const kvb_config* cfg, void* workspace, size_t worksp
   cudaError_t e = cudaMemsetAsync(b->status, 0, sizeof(int), st);
   if (e == cudaSuccess) e = cudaMemsetAsync(b->stats, 0, LH * sizeof(kvb_admit_stats), st);
   if (cfg->method == KVB_DENSITYKV) {
+    // rows past a bank's size are read by full attention tiles (and masked): keep
+    // them finite by starting from zeros
+    const size_t kv = LH * cfg->capacity * static_cast<size_t>(b->row_bytes);
     if (e == cudaSuccess) e = cudaMemsetAsync(b->size, 0, LH * sizeof(int), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(b->K, 0, kv, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(b->V, 0, kv, st);
   } else if (e == cudaSuccess) {
     const kvb_status fs = kvb_forcing_init(b, st);
     if (fs != KVB_OK) {

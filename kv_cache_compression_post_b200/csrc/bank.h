@@ -66,6 +66,7 @@ struct kvb_bank {
   int* fcount = nullptr;    // [L][H][hist_frames]
   int* rstate = nullptr;    // [L][H][4]: first frame slot, frames held, token start, tokens held
   uint8_t* is_static = nullptr;  // [L][H] labels of the last prune
+  int* aseg = nullptr;      // [L][4][H]: transition length, ring part-1 start, part-1 length, part-2 length
   // ---- Forcing-KV scratch
   float* sims = nullptr;    // [H][max_new_frames][n_seg]
   int* keep = nullptr;      // [H][max_new_frames][n_seg] kept segment ids, ascending

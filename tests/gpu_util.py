@@ -27,3 +27,16 @@ def workspace(nbytes):
 def aligned_ptr(buf):
     p = buf.data_ptr()
     return (p + 255) & ~255
+
+
+def import_oracle_banks(bank, banks, params, w, layer=0):
+    """Load oracle HeadBanks (with from-scratch densities) into a GPU bank."""
+    import torch
+    from oracle import densitykv as dkv
+    for hh, b in enumerate(banks):
+        if b.size == 0:
+            bank.import_(layer, hh, torch.zeros(0, dtype=torch.int32, device="cuda"), None, None, None, None)
+            continue
+        rho = dkv.densities_from_scratch(b, params)
+        bank.import_(layer, hh, dev_ids(b.ids), dev_tensor(rho, "f32"), dev_tensor(b.rho0, "f32"),
+                     dev_tensor(b.K, w.dtype), dev_tensor(b.V, w.dtype))
