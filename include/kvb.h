@@ -178,6 +178,10 @@ KVB_API kvb_status kvb_bank_import(kvb_bank* bank, int32_t layer, int32_t head, 
 /* Synchronise `stream` and return the first latched device error (KVB_OK if none). */
 KVB_API kvb_status kvb_device_status(kvb_bank* bank, void* stream);
 
+/* Number of kernels the library has launched in this process (all entry points,
+ * all devices); a diagnostic for callers that account launches. */
+KVB_API unsigned long long kvb_launch_count(void);
+
 /* Static string for a status code. */
 KVB_API const char* kvb_status_string(kvb_status st);
 

@@ -21,6 +21,7 @@
 #include <climits>
 
 #include "admit.cuh"
+#include "host_util.h"
 #include "kvb_device.cuh"
 
 namespace kvb {
@@ -395,31 +396,38 @@ __global__ void finalize_kernel(const AdmitPlan p) {
 }  // namespace
 
 cudaError_t launch_admit_count(const AdmitPlan& p, cudaStream_t st) {
+  note_launch();
   admit_count_kernel<<<p.H, kSelThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_admit_select(const AdmitPlan& p, cudaStream_t st) {
+  note_launch();
   admit_select_kernel<<<p.H, kSelThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_gather_admitted(const AdmitPlan& p, int maxP, cudaStream_t st) {
   if (maxP <= 0) return cudaSuccess;
+  note_launch();
   gather_admitted_kernel<<<dim3((maxP + 7) / 8, p.H), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_evict_select(const AdmitPlan& p, cudaStream_t st) {
+  note_launch();
   evict_select_kernel<<<p.H, kSelThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_gather_evicted(const AdmitPlan& p, cudaStream_t st) {
+  note_launch();
   gather_evicted_kernel<<<dim3((p.M + 7) / 8, p.H), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_compact(const AdmitPlan& p, cudaStream_t st) {
+  note_launch();
   compact_kernel<<<dim3((p.N + p.M + 7) / 8, p.H), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_finalize(const AdmitPlan& p, cudaStream_t st) {
+  note_launch();
   finalize_kernel<<<dim3((p.M + 255) / 256, p.H), 256, 0, st>>>(p);
   return cudaGetLastError();
 }

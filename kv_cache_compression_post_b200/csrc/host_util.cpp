@@ -2,6 +2,7 @@
 
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 
 namespace kvb {
@@ -21,6 +22,12 @@ void load_encode() {
     g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
 }
 }  // namespace
+
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 bool current_device(DeviceInfo* out) {
   int dev = -1;
@@ -54,3 +61,5 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, int d, long long rows, int
 }
 
 }  // namespace kvb
+
+extern "C" unsigned long long kvb_launch_count(void) { return kvb::g_launches.load(std::memory_order_relaxed); }

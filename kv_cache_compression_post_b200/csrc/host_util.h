@@ -25,6 +25,9 @@ bool current_device(DeviceInfo* out);
 // 128-byte swizzle, zero fill out of bounds.
 bool make_tmap_bf16(CUtensorMap* m, const void* base, int d, long long rows, int heads, int box_rows);
 
+// Count of kernel launches issued by the library in this process.
+void note_launch();
+
 inline kvb_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVB_OK : KVB_E_CUDA; }
 
 // Bump allocation inside a caller workspace, 256-byte aligned pieces.

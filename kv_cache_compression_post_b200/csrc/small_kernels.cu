@@ -1,5 +1,6 @@
 #include <cuda_bf16.h>
 
+#include "host_util.h"
 #include "kvb_device.cuh"
 #include "small_kernels.cuh"
 
@@ -31,6 +32,7 @@ cudaError_t launch_row_terms(const void* X, kvb_dtype dtype, int H, long long ld
                              cudaStream_t st) {
   if (max_n <= 0 || H <= 0) return cudaSuccess;
   dim3 grid((max_n + 7) / 8, H);
+  note_launch();
   if (dtype == KVB_BF16)
     row_terms_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), ldX, d, n_uni, n_dev, inv_h, add,
                                            out, ldOut);

@@ -17,7 +17,7 @@ __all__ = [
     "KVB_BF16", "KVB_F32", "KVB_DENSITYKV", "KVB_FORCINGKV",
     "kvb_workspace_size", "kvb_bank_create", "kvb_bank_destroy", "kvb_admit", "kvb_prune_hybrid",
     "kvb_attend", "kvb_read_stats", "kvb_bank_export", "kvb_bank_import", "kvb_device_status",
-    "kvb_status_string", "kvb_density_workspace_size", "kvb_density", "kvb_segment_cosine",
+    "kvb_status_string", "kvb_launch_count", "kvb_density_workspace_size", "kvb_density", "kvb_segment_cosine",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvb.so")
@@ -84,6 +84,7 @@ _SIGS = {
     "kvb_bank_import": (ctypes.c_int, [_vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp]),
     "kvb_device_status": (ctypes.c_int, [_vp, _vp]),
     "kvb_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "kvb_launch_count": (ctypes.c_ulonglong, []),
     "kvb_density_workspace_size": (_sz, [_i32, _i32, _i32, _i32, ctypes.c_int]),
     "kvb_density": (ctypes.c_int, [_vp, _i32, _vp, _i32, _i32, _i32, ctypes.c_int, _f, _f, _f, _i32, _vp, _vp,
                                    _sz, _vp]),
@@ -116,6 +117,10 @@ def _stream(s) -> Optional[int]:
 def _check(st: int, where: str) -> None:
     if st != 0:
         raise KvbError(st, where)
+
+
+def kvb_launch_count() -> int:
+    return int(lib.kvb_launch_count())
 
 
 def kvb_status_string(status: int) -> str:

@@ -23,8 +23,11 @@ standing in for the generator's activations):
   -- DensityKV, Supplementary "Post-RoPE Attention Geometry": the backbones zero
   the temporal RoPE coordinate of non-local memory keys.  Window keys, sink keys
   and queries use their true frame index.  Forcing-KV caches keep true indices.
-* Seeds: numpy PCG64 from SeedSequence([workload, layer, head, stream]),
-  stream 0 = keys, 1 = values, 2 = queries, 3 = head labels.
+* Seeds: numpy PCG64.  Keys: one generator per (workload, layer, head) from
+  SeedSequence([workload, layer, head, 0]) drawing frames in order; values and
+  queries: SeedSequence([workload, layer, head, stream, frame]) per frame
+  (stream 1 = values, 2 = queries); head labels: SeedSequence([workload, layer,
+  0, 3]).
 """
 from __future__ import annotations
 
@@ -121,12 +124,11 @@ def rng_for(w: Workload, layer: int, head: int, stream: int, seed_offset: int = 
 # storage precision
 # ---------------------------------------------------------------------------------
 def round_bf16(x: np.ndarray) -> np.ndarray:
-    """Round float32 values to the nearest bfloat16 (ties to even); returns float32."""
+    """Round finite float32 values to the nearest bfloat16 (ties to even); returns float32."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    u = (u + 0x7FFF + lsb) & 0xFFFF0000
-    return u.astype(np.uint32).view(np.float32).reshape(x.shape)
+    u = x.view(np.uint32)
+    u = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) & np.uint32(0xFFFF0000)
+    return u.view(np.float32).reshape(x.shape)
 
 
 def to_storage(w: Workload, x: np.ndarray) -> np.ndarray:
@@ -165,11 +167,15 @@ def rope_angles(d: int, t: np.ndarray, r: np.ndarray, c: np.ndarray) -> np.ndarr
     return ang
 
 
-def apply_rope(x: np.ndarray, ang: np.ndarray) -> np.ndarray:
-    """Rotate interleaved pairs (x[2k], x[2k+1]) of x [..., n_tok, d] by ang [n_tok, d/2]."""
+def apply_rope(x: np.ndarray, ang) -> np.ndarray:
+    """Rotate interleaved pairs (x[2k], x[2k+1]) of x [..., n_tok, d] by ang [n_tok, d/2]
+    (or by a precomputed (cos, sin) pair)."""
     x = np.asarray(x, dtype=np.float32)
-    cos = np.cos(ang).astype(np.float32)
-    sin = np.sin(ang).astype(np.float32)
+    if isinstance(ang, tuple):
+        cos, sin = ang
+    else:
+        cos = np.cos(ang).astype(np.float32)
+        sin = np.sin(ang).astype(np.float32)
     x0 = x[..., 0::2]
     x1 = x[..., 1::2]
     out = np.empty_like(x)
@@ -181,15 +187,30 @@ def apply_rope(x: np.ndarray, ang: np.ndarray) -> np.ndarray:
 # ---------------------------------------------------------------------------------
 # per-(layer, head) raw streams
 # ---------------------------------------------------------------------------------
+class _FrameDraws:
+    """i.i.d. N(0,1) frames of one stream, each frame seeded on its own."""
+
+    def __init__(self, w, layer, head, stream, seed_offset):
+        self.key = (w.wid + 1000 * seed_offset, layer, head, stream)
+        self.shape = (w.F, w.head_dim)
+
+    def __getitem__(self, t):
+        if isinstance(t, (list, tuple, np.ndarray)):
+            return np.stack([self[int(u)] for u in t])
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([*self.key, int(t)])))
+        return g.standard_normal(self.shape, dtype=np.float32)
+
+
 class HeadStream:
-    """Raw (pre-RoPE) keys, values and queries of one (layer, head), frames [0, T)."""
+    """Raw (pre-RoPE) keys, values and queries of one (layer, head), frames [0, T).
+
+    Keys follow the AR(1) recurrence (one generator, frames drawn in order); values
+    and queries are drawn per frame from SeedSequence([..., stream, frame])."""
 
     def __init__(self, w: Workload, layer: int, head: int, n_frames: int, seed_offset: int = 0):
         F, d = w.F, w.head_dim
         self.w = w
         rk = rng_for(w, layer, head, STREAM_K, seed_offset)
-        rv = rng_for(w, layer, head, STREAM_V, seed_offset)
-        rq = rng_for(w, layer, head, STREAM_Q, seed_offset)
         K = np.empty((n_frames, F, d), dtype=np.float32)
         if w.background_rows > 0:
             rows = np.repeat(np.arange(w.frame_h), w.frame_w)
@@ -202,8 +223,8 @@ class HeadStream:
         for t in range(1, n_frames):
             K[t] = a * K[t - 1] + b * rk.standard_normal((F, d), dtype=np.float32)
         self.K = K
-        self.V = rv.standard_normal((n_frames, F, d), dtype=np.float32)
-        self.Q = rq.standard_normal((n_frames, F, d), dtype=np.float32)
+        self.V = _FrameDraws(w, layer, head, STREAM_V, seed_offset)
+        self.Q = _FrameDraws(w, layer, head, STREAM_Q, seed_offset)
 
 
 def token_ids(w: Workload, frames) -> np.ndarray:
@@ -217,14 +238,27 @@ def _grid(w: Workload):
     return r, c
 
 
+_ROT_CACHE: dict = {}
+
+
+def frame_rotation(w: Workload, t: int):
+    """(cos, sin) [F][d/2] float32 of frame index t (cached)."""
+    key = (w.frame_h, w.frame_w, w.head_dim, int(t))
+    if key not in _ROT_CACHE:
+        if len(_ROT_CACHE) > 256:
+            _ROT_CACHE.clear()
+        r, c = _grid(w)
+        ang = rope_angles(w.head_dim, np.full(w.F, float(t)), r, c)
+        _ROT_CACHE[key] = (np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32))
+    return _ROT_CACHE[key]
+
+
 def rotated_frames(w: Workload, raw: np.ndarray, frames, memory: bool) -> np.ndarray:
     """Apply 3D RoPE to raw[frames] ([n][F][d]); memory=True zeroes the frame index."""
     frames = list(frames)
-    r, c = _grid(w)
     out = np.empty((len(frames), w.F, w.head_dim), dtype=np.float32)
     for i, t in enumerate(frames):
-        tt = np.zeros(w.F) if memory else np.full(w.F, float(t))
-        out[i] = apply_rope(raw[t], rope_angles(w.head_dim, tt, r, c))
+        out[i] = apply_rope(raw[t], frame_rotation(w, 0 if memory else t))
     return out
 
 
@@ -292,10 +326,9 @@ class LayerInputs:
 
     def queries(self, frames) -> np.ndarray:
         w = self.w
-        r, c = _grid(w)
         out = []
         for s in self.streams:
-            qs = [apply_rope(s.Q[t], rope_angles(w.head_dim, np.full(w.F, float(t)), r, c)) for t in frames]
+            qs = [apply_rope(s.Q[t], frame_rotation(w, t)) for t in frames]
             out.append(np.concatenate(qs, axis=0))
         return to_storage(w, np.stack(out))
 
