@@ -208,6 +208,27 @@ KVB_API kvb_status kvb_density(const void* rows, int32_t n_rows, const void* col
                        float eps, float s, int32_t exclude_diagonal, float* out,
                        void* workspace, size_t workspace_bytes, void* stream);
 
+/* kvb_density for callers that cannot allocate device memory.  (The pages have
+ * no counterpart: this is an interface for a host application whose allocator
+ * owns all device memory and forbids allocations outside it, or for a
+ * latency-critical loop that must not pay for an allocation, and which therefore
+ * cannot hand the library a scratch workspace.)
+ * Same inputs, outputs and results as kvb_density with dtype KVB_BF16; the
+ * scratch lives in one 4 MiB array inside the library's device image, held by
+ * every GPU that loads the library until the process exits.  Sizes are rejected
+ * with KVB_E_WORKSPACE (nothing launched) unless
+ *   256 + 4*H*n_rows + 4*(H*n_cols + 128) + 32*H*n_rows  (each term rounded up
+ *   to 256 bytes)  <=  4 MiB.
+ * The first call on a device looks up the array's address with that device
+ * current: make it before any stream capture.  All calls on a device share the
+ * array (it keeps the last call's contents); calls that overlap on the GPU race,
+ * so order them on one stream.  status_out: device int32 (may be NULL) that
+ * receives this call's device status (zeroed by the call). */
+KVB_API kvb_status kvb_density_noalloc(const void* rows, int32_t n_rows, const void* cols, int32_t n_cols,
+                                       int32_t heads, int32_t head_dim, kvb_dtype dtype, float dist_scale,
+                                       float eps, float s, int32_t exclude_diagonal, float* out,
+                                       int32_t* status_out, void* stream);
+
 /* Segment-wise cosine similarity of Forcing-KV (§3.4): for every head and every
  * frame t < n_frames, sim[h][t][j] = mean over the tokens p of segment j of
  * cos(K[h][t][p], succ[h][t][p]) with succ = frame t+1 of K, or `nextK` for the

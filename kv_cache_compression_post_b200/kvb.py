@@ -17,7 +17,7 @@ __all__ = [
     "KVB_BF16", "KVB_F32", "KVB_DENSITYKV", "KVB_FORCINGKV",
     "kvb_workspace_size", "kvb_bank_create", "kvb_bank_destroy", "kvb_admit", "kvb_prune_hybrid",
     "kvb_attend", "kvb_read_stats", "kvb_bank_export", "kvb_bank_import", "kvb_device_status",
-    "kvb_status_string", "kvb_launch_count", "kvb_density_workspace_size", "kvb_density", "kvb_segment_cosine",
+    "kvb_status_string", "kvb_launch_count", "kvb_density_workspace_size", "kvb_density", "kvb_density_noalloc", "kvb_segment_cosine",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvb.so")
@@ -88,6 +88,8 @@ _SIGS = {
     "kvb_density_workspace_size": (_sz, [_i32, _i32, _i32, _i32, ctypes.c_int]),
     "kvb_density": (ctypes.c_int, [_vp, _i32, _vp, _i32, _i32, _i32, ctypes.c_int, _f, _f, _f, _i32, _vp, _vp,
                                    _sz, _vp]),
+    "kvb_density_noalloc": (ctypes.c_int, [_vp, _i32, _vp, _i32, _i32, _i32, ctypes.c_int, _f, _f, _f, _i32, _vp,
+                                           _vp, _vp]),
     "kvb_segment_cosine": (ctypes.c_int, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_int, _vp,
                                           _vp]),
 }
@@ -197,6 +199,15 @@ def kvb_density(rows, n_rows: int, cols, n_cols: int, heads: int, head_dim: int,
     _check(lib.kvb_density(_ptr(rows), n_rows, _ptr(cols), n_cols, heads, head_dim, dtype, dist_scale, eps, s,
                            exclude_diagonal, _ptr(out), _ptr(workspace), workspace_bytes, _stream(stream)),
            "kvb_density")
+
+
+def kvb_density_noalloc(rows, n_rows: int, cols, n_cols: int, heads: int, head_dim: int, dtype: int,
+                        dist_scale: float, eps: float, s: float, exclude_diagonal: int, out, status_out=None,
+                        stream=None) -> None:
+    """kvb_density without a workspace (scratch in a fixed device array of the library)."""
+    _check(lib.kvb_density_noalloc(_ptr(rows), n_rows, _ptr(cols), n_cols, heads, head_dim, dtype, dist_scale, eps,
+                                   s, exclude_diagonal, _ptr(out), _ptr(status_out), _stream(stream)),
+           "kvb_density_noalloc")
 
 
 def kvb_segment_cosine(K, nextK, heads: int, n_frames: int, frame_h: int, frame_w: int, seg_h: int, seg_w: int,
