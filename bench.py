@@ -62,7 +62,18 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index: int):
-        self.index = index
+        self.index = str(index)
+        try:
+            # the process may see a remapped device 0: address the GPU by PCI bus id
+            import torch
+            pr = torch.cuda.get_device_properties(index)
+            bus = getattr(pr, "pci_bus_id", None)
+            dom = getattr(pr, "pci_domain_id", 0)
+            dv = getattr(pr, "pci_device_id", 0)
+            if bus is not None:
+                self.index = f"{dom:08X}:{bus:02X}:{dv:02X}.0"
+        except Exception:
+            pass
         self.proc = None
         self.file = None
 
