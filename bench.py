@@ -82,7 +82,11 @@ class ClockSampler:
             self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.file, stderr=subprocess.DEVNULL)
+                 "-lms", "20"], stdout=self.file, stderr=subprocess.DEVNULL)
+            # nvidia-smi needs about a second before its first sample: wait for it
+            t0 = time.time()
+            while time.time() - t0 < 10 and os.path.getsize(self.file.name) == 0:
+                time.sleep(0.05)
         except Exception:
             self.proc = None
 
