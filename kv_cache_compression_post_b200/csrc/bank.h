@@ -72,7 +72,7 @@ struct kvb_bank {
   int* keep = nullptr;      // [H][max_new_frames][n_seg] kept segment ids, ascending
   int* seg_tok = nullptr;   // [n_seg + 1] token offsets of each segment in segment-major order
   int* seg_list = nullptr;  // [F] token index (row-major) in segment-major order
-  int* plan = nullptr;      // [H][max_new_frames*F] source token -> ring position
+  int* plan = nullptr;      // [H][max_new_frames*F][2] (source row, ring position) pairs
   int* plan_n = nullptr;    // [H]
 
   size_t layout(void* base);  // carve (base may be null to measure); returns bytes

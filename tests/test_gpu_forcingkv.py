@@ -1,0 +1,122 @@
+"""GPU parity of the Forcing-KV path against the fp64 oracle (Forcing-KV reading
+notes §3.3-§3.5): segment-wise cosine, per-frame BottomK into the dynamic heads'
+FIFO, the static heads' transition frame, and hybrid attention."""
+import numpy as np
+import pytest
+
+import kvgen
+from oracle import forcingkv as fkv
+from oracle.attention import attention
+from tests.gpu_util import dev_ids, dev_tensor, host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("name,dtype,H,nf", [("forcing_mid", "bf16", 4, 3), ("forcing480", "bf16", 2, 3),
+                                             ("forcing_mid", "f32", 2, 2), ("wan1080", "bf16", 1, 2)])
+def test_segment_cosine_matches_oracle(name, dtype, H, nf):
+    import torch
+    import kv_cache_compression_post_b200 as kvb
+    w = kvgen.WORKLOADS[name]
+    L = kvgen.LayerInputs(w, 0, n_chunks=2, heads=range(H))
+    frames = list(range(1, 1 + nf))
+    K = L.keys(frames, memory=False)
+    if dtype == "f32":
+        K = K + np.float32(1e-3) * np.random.default_rng(0).standard_normal(K.shape).astype(np.float32)
+    nxt = L.keys([1 + nf], memory=False)
+    segs = fkv.segments(w.frame_h, w.frame_w, w.seg_h, w.seg_w)
+    sim = torch.full((H, nf, len(segs)), float("nan"), device="cuda")
+    kvb.kvb_segment_cosine(dev_tensor(K, dtype), dev_tensor(nxt, dtype), H, nf, w.frame_h, w.frame_w, w.seg_h,
+                           w.seg_w, w.head_dim, kvb.KVB_BF16 if dtype == "bf16" else kvb.KVB_F32, sim)
+    torch.cuda.synchronize()
+    got = host(sim)
+    for hh in range(H):
+        Kf = K[hh].reshape(nf, w.F, -1)
+        for t in range(nf):
+            succ = Kf[t + 1] if t + 1 < nf else nxt[hh]
+            ref = fkv.segment_similarity(Kf[t], succ, segs)
+            np.testing.assert_allclose(got[hh, t], ref, atol=2e-6, rtol=0)
+
+
+def _cfg(w, layers=1):
+    import kv_cache_compression_post_b200 as kvb
+    return kvb.make_config(method=kvb.KVB_FORCINGKV, dtype=kvb.KVB_BF16, layers=layers, heads=w.heads,
+                           head_dim=w.head_dim, frame_h=w.frame_h, frame_w=w.frame_w, seg_h=w.seg_h,
+                           seg_w=w.seg_w, hist_frames=w.hist_frames, max_new_frames=w.chunk_frames,
+                           retention=w.retention, max_queries=w.chunk_tokens)
+
+
+def _kept_near_tie(sim, k, margin=1e-4):
+    order = np.lexsort((np.arange(sim.size), sim))
+    if k == 0 or k >= sim.size:
+        return False
+    a, b = sim[order[k - 1]], sim[order[k]]
+    return abs(b - a) <= margin * max(abs(a), 1e-3)
+
+
+def _rollout(name, steps, labels, sample_rows=None):
+    import torch
+    import kv_cache_compression_post_b200 as kvb
+    w = kvgen.WORKLOADS[name]
+    H = len(labels)
+    L = kvgen.LayerInputs(w, 0, n_chunks=steps + 2, heads=range(H))
+    p = fkv.Params(w.frame_h, w.frame_w, w.seg_h, w.seg_w, w.retention, w.hist_frames)
+    states = [fkv.HeadState(bool(s)) for s in labels]
+    import dataclasses
+    bank = kvb.Bank(_cfg(dataclasses.replace(w, heads=H)))
+    rng = np.random.default_rng(0)
+    tie_frames = [set() for _ in range(H)]   # frames pushed with a near-tie BottomK decision
+    for i in range(1, steps + 1):
+        x = L.step(i, forcing=True)
+        nf = len(x["new_ids"]) // w.F
+        fkv.prune_hybrid(states, p, x["newK"], x["newV"], x["new_ids"], x["nextK"])
+        new_frames = [int(f) for f in x["new_ids"][::w.F] // w.F]
+        for hh in range(H):
+            if not states[hh].static:
+                for f, s in zip(new_frames, states[hh].sims):
+                    if _kept_near_tie(s, fkv.keep_count(s.size, w.retention)):
+                        tie_frames[hh].add(f)
+        bank.prune_hybrid(0, np.array(labels, np.uint8), dev_tensor(x["newK"], "bf16"), dev_tensor(x["newV"], "bf16"),
+                          dev_tensor(x["nextK"], "bf16"), dev_ids(x["new_ids"]), nf)
+        Q = dev_tensor(x["Q"], "bf16")
+        O = torch.empty_like(Q)
+        lse = torch.empty(H, Q.shape[1], device="cuda")
+        bank.attend(0, Q, dev_tensor(x["sinkK"], "bf16"), dev_tensor(x["sinkV"], "bf16"),
+                    dev_tensor(x["winK"], "bf16"), dev_tensor(x["winV"], "bf16"), O, lse)
+        torch.cuda.synchronize()
+        assert bank.status() == 0
+        O = host(O)
+        st = bank.stats(0)
+        for hh in range(H):
+            ids, _, _, K, V = bank.export(0, hh)
+            gid, gK, gV = host(ids).astype(np.int64), host(K), host(V)
+            oid, oK, oV = fkv.history(states[hh], w.head_dim)
+            gf, of = gid // w.F, oid // w.F
+            assert sorted(set(gf.tolist())) == sorted(set(of.tolist()))   # same frames held
+            clean = True
+            for f in sorted(set(of.tolist())):
+                if f in tie_frames[hh]:
+                    clean = False
+                    continue
+                np.testing.assert_array_equal(gid[gf == f], oid[of == f])
+                np.testing.assert_array_equal(gK[gf == f], oK[of == f].astype(np.float32))
+                np.testing.assert_array_equal(gV[gf == f], oV[of == f].astype(np.float32))
+            if clean:
+                assert st[hh]["size"] == len(oid)
+                Kall, Vall = fkv.attention_set(states[hh], x["sinkK"][hh], x["sinkV"][hh], x["winK"][hh],
+                                               x["winV"][hh])
+                rows = np.arange(Q.shape[1]) if sample_rows is None else \
+                    np.sort(rng.choice(Q.shape[1], sample_rows, replace=False))
+                O_ref, _ = attention(x["Q"][hh][rows], Kall, Vall)
+                np.testing.assert_allclose(O[hh][rows], O_ref, atol=2e-2, rtol=0)
+    bank.close()
+
+
+def test_forcing_mid_rollout_matches_oracle():
+    # hist_frames 7 < frames pushed: the FIFO wraps and drops old frames
+    _rollout("forcing_mid", 4, [1, 0, 1, 0])
+
+
+def test_forcing480_full_size_sampled():
+    # 480P, 4 heads (2 static, 2 dynamic), 8 chunks: the 21-frame FIFO fills up
+    _rollout("forcing480", 8, [0, 1, 0, 1], sample_rows=16)
