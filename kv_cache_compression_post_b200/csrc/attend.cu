@@ -223,7 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const float sl2 = a.scale * 1.4426950408889634f;  // scale * log2(e)
-    float m = -INFINITY, l = 0.f;
+    const float thr_raw = kRescaleThreshold / sl2;     // rescale threshold in raw score units
+    float m = -INFINITY, l = 0.f;                      // m: running max of the raw scores
     bool ok = true;
     for (int j = 0; j < T; ++j) {
       int s, row, nv;
@@ -231,38 +232,59 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int sb = j & 1;
       if (!(ok = mbar_wait(&bars->s_full[sb], (j >> 1) & 1, abort, a.status))) break;
       tc_fence_after();
-      float x[kTile];
-#pragma unroll
-      for (int c = 0; c < kTile / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tS + sb * kTile + lane_off + c * 32, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int k = 0; k < 32; ++k) x[c * 32 + k] = (c * 32 + k < nv) ? __uint_as_float(v[k]) * sl2 : -INFINITY;
-      }
+      // all four 32-column loads in flight before one wait
+      uint32_t v0[32], v1[32], v2[32], v3[32];
+      tmem_ld32(tS + sb * kTile + lane_off + 0, v0);
+      tmem_ld32(tS + sb * kTile + lane_off + 32, v1);
+      tmem_ld32(tS + sb * kTile + lane_off + 64, v2);
+      tmem_ld32(tS + sb * kTile + lane_off + 96, v3);
+      tmem_wait_ld_reg(v0);  // the first wait covers all four loads; the others
+      tmem_wait_ld_reg(v1);  // only tie the registers to it
+      tmem_wait_ld_reg(v2);
+      tmem_wait_ld_reg(v3);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->s_empty[sb]);
-      float mt = x[0];
+      float x[kTile];
 #pragma unroll
-      for (int k = 1; k < kTile; ++k) mt = fmaxf(mt, x[k]);
+      for (int k = 0; k < 32; ++k) {
+        x[k] = __uint_as_float(v0[k]);
+        x[32 + k] = __uint_as_float(v1[k]);
+        x[64 + k] = __uint_as_float(v2[k]);
+        x[96 + k] = __uint_as_float(v3[k]);
+      }
+      if (nv < kTile) {  // the last tile of a segment: keys past its end do not exist
+#pragma unroll
+        for (int k = 0; k < kTile; ++k)
+          if (k >= nv) x[k] = -INFINITY;
+      }
+      // row max of the raw scores, eight independent chains
+      float mx[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = x[i];
+#pragma unroll
+      for (int k = 8; k < kTile; ++k) mx[k & 7] = fmaxf(mx[k & 7], x[k]);
+      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       float alpha = 1.f;
       bool resc = false;
       if (j == 0) {
         m = mt;
-      } else if (mt > m + kRescaleThreshold) {
-        alpha = ex2_approx(m - mt);
+      } else if (mt > m + thr_raw) {
+        alpha = ex2_approx((m - mt) * sl2);
         m = mt;
         resc = true;
       }
-      float rs = 0.f;
+      // p = 2^((s - m) * scale * log2 e): one FFMA and one ex2 per score
+      const float nb = -m * sl2;
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[kTile / 2];
 #pragma unroll
       for (int k = 0; k < kTile; k += 2) {
-        const float p0 = ex2_approx(x[k] - m), p1 = ex2_approx(x[k + 1] - m);
-        rs += p0 + p1;
+        const float p0 = ex2_approx(fmaf(x[k], sl2, nb)), p1 = ex2_approx(fmaf(x[k + 1], sl2, nb));
+        rs4[(k >> 1) & 3] += p0 + p1;
         pk[k >> 1] = pack_bf16(p0, p1);
       }
+      const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       if (j >= 1) {
         // P buffer free and O final for tile j-1
         if (!(ok = mbar_wait(&bars->o_ready, (j - 1) & 1, abort, a.status))) break;
@@ -271,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < d / 32; ++c) {
             uint32_t v[32];
             tmem_ld32(tO + lane_off + c * 32, v);
-            tmem_wait_ld();
+            tmem_wait_ld_reg(v);
 #pragma unroll
             for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
             tmem_st32(tO + lane_off + c * 32, v);
@@ -303,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t v[32];
         if (T > 0) {
           tmem_ld32(tO + lane_off + c * 32, v);
-          tmem_wait_ld();
+          tmem_wait_ld_reg(v);
         } else {
 #pragma unroll
           for (int k = 0; k < 32; ++k) v[k] = 0u;
@@ -321,7 +343,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (a.lse && qrow < a.Nq)
-        a.lse[static_cast<size_t>(h) * a.Nq + qrow] = (T > 0) ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+        a.lse[static_cast<size_t>(h) * a.Nq + qrow] =
+            (T > 0) ? (m * sl2 + __log2f(l)) * 0.6931471805599453f : -INFINITY;
     }
   }
 

@@ -262,6 +262,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
     Cursor c;
     if (L0 < L1) cursor_seek(a, L0, c);
     float acc_pos = 0.f, acc_neg = 0.f, ra = 0.f;
+    float cbn[4] = {0.f, 0.f, 0.f, 0.f};  // next tile's column terms (prefetched)
     int row = 0, nneg = 0, diag = 0, rt0 = 0;
     bool active = false, valid_row = false;
     long long Lblock = L0;  // first step of the current row block
@@ -285,16 +286,31 @@ __global__ void __launch_bounds__(kGramThreads, 1)
         break;
       }
       // this warp's copy of the tile's column terms (no cross-warp barrier, so an
-      // aborting warp can never strand another one)
+      // aborting warp can never strand another one); the values were fetched one
+      // tile ahead so their L2 latency overlaps the previous tile
       float* cb = sColTerm + (e * 2 + b) * kGramColTile;
+      if (L == L0) {
 #pragma unroll
-      for (int i = lane; i < kGramColTile; i += 32) {
-        const long idx = static_cast<long>(c.cOff) + c0 + i;
-        cb[i] = (idx < a.ldCT) ? a.colTerm[static_cast<size_t>(c.h) * a.ldCT + idx] : 0.f;
+        for (int i = 0; i < 4; ++i) {
+          const long idx = static_cast<long>(c.cOff) + c0 + lane + 32 * i;
+          cbn[i] = (idx < a.ldCT) ? a.colTerm[static_cast<size_t>(c.h) * a.ldCT + idx] : 0.f;
+        }
       }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) cb[lane + 32 * i] = cbn[i];
       __syncwarp();
+      if (L + 1 < L1) {
+        Cursor cn = c;
+        cursor_next(a, cn);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const long idx = static_cast<long>(cn.cOff) + cn.j * kGramColTile + lane + 32 * i;
+          cbn[i] = (idx < a.ldCT) ? a.colTerm[static_cast<size_t>(cn.h) * a.ldCT + idx] : 0.f;
+        }
+      }
       if (!(ok = mbar_wait(&bars->acc_full[b], (t >> 1) & 1, abort, a.status))) break;
       tc_fence_after();
+      bool released = false;
       if (active) {
         const bool tail = c0 + kGramColTile > c.nC;
         const bool allneg = c0 + kGramColTile <= nneg;
@@ -305,55 +321,82 @@ __global__ void __launch_bounds__(kGramThreads, 1)
         const bool masked = tail || mixed || diag_hit;
         const uint32_t taddr =
             tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>((r * 2 + b) * kGramColTile);
-        float tile_acc = 0.f;
-#pragma unroll 1
-        for (int cc = 0; cc < kGramColTile / 32; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(taddr + cc * 32, v);
-          tmem_wait_ld();
-          if (!masked) {
-            if constexpr (SMODE == 2) {
+        float acc0 = 0.f, acc1 = 0.f;
+        auto fast = [&](const uint32_t (&v)[32], int cc) {
+          if constexpr (SMODE == 2) {
 #pragma unroll
-              for (int k = 0; k < 32; k += 4) {
-                const float4 cbv = *reinterpret_cast<const float4*>(cb + cc * 32 + k);
-                const float t0 = fmaxf(fmaf(__uint_as_float(v[k + 0]), ks, ra + cbv.x), eps);
-                const float t1 = fmaxf(fmaf(__uint_as_float(v[k + 1]), ks, ra + cbv.y), eps);
-                const float t2 = fmaxf(fmaf(__uint_as_float(v[k + 2]), ks, ra + cbv.z), eps);
-                const float t3 = fmaxf(fmaf(__uint_as_float(v[k + 3]), ks, ra + cbv.w), eps);
-                const float p01 = t0 * t1, p23 = t2 * t3;
-                const float num = fmaf(t2 + t3, p01, (t0 + t1) * p23);
-                tile_acc = fmaf(num, rcp_approx(p01 * p23), tile_acc);
-              }
-            } else {
-#pragma unroll
-              for (int k = 0; k < 32; k += 4) {
-                const float4 cbv = *reinterpret_cast<const float4*>(cb + cc * 32 + k);
-                tile_acc += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 0]), ks, ra + cbv.x), eps), nhs);
-                tile_acc += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 1]), ks, ra + cbv.y), eps), nhs);
-                tile_acc += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 2]), ks, ra + cbv.z), eps), nhs);
-                tile_acc += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 3]), ks, ra + cbv.w), eps), nhs);
-              }
+            for (int k = 0; k < 32; k += 8) {
+              const float4 ca = *reinterpret_cast<const float4*>(cb + cc * 32 + k);
+              const float4 cbv = *reinterpret_cast<const float4*>(cb + cc * 32 + k + 4);
+              const float t0 = fmaxf(fmaf(__uint_as_float(v[k + 0]), ks, ra + ca.x), eps);
+              const float t1 = fmaxf(fmaf(__uint_as_float(v[k + 1]), ks, ra + ca.y), eps);
+              const float t2 = fmaxf(fmaf(__uint_as_float(v[k + 2]), ks, ra + ca.z), eps);
+              const float t3 = fmaxf(fmaf(__uint_as_float(v[k + 3]), ks, ra + ca.w), eps);
+              const float t4 = fmaxf(fmaf(__uint_as_float(v[k + 4]), ks, ra + cbv.x), eps);
+              const float t5 = fmaxf(fmaf(__uint_as_float(v[k + 5]), ks, ra + cbv.y), eps);
+              const float t6 = fmaxf(fmaf(__uint_as_float(v[k + 6]), ks, ra + cbv.z), eps);
+              const float t7 = fmaxf(fmaf(__uint_as_float(v[k + 7]), ks, ra + cbv.w), eps);
+              const float p01 = t0 * t1, p23 = t2 * t3, p45 = t4 * t5, p67 = t6 * t7;
+              const float na = fmaf(t2 + t3, p01, (t0 + t1) * p23);
+              const float nb2 = fmaf(t6 + t7, p45, (t4 + t5) * p67);
+              acc0 = fmaf(na, rcp_approx(p01 * p23), acc0);
+              acc1 = fmaf(nb2, rcp_approx(p45 * p67), acc1);
             }
           } else {
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              const int col = c0 + cc * 32 + k;
-              const float tv = fmaxf(fmaf(__uint_as_float(v[k]), ks, ra + cb[cc * 32 + k]), eps);
-              const bool valid = (col < c.nC) && (col != row + diag);
-              const float ph = valid ? phi_t<SMODE>(tv, nhs) : 0.f;
-              if (col < nneg) acc_neg += ph;
-              else acc_pos += ph;
+            for (int k = 0; k < 32; k += 4) {
+              const float4 cbv = *reinterpret_cast<const float4*>(cb + cc * 32 + k);
+              acc0 += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 0]), ks, ra + cbv.x), eps), nhs);
+              acc1 += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 1]), ks, ra + cbv.y), eps), nhs);
+              acc0 += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 2]), ks, ra + cbv.z), eps), nhs);
+              acc1 += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 3]), ks, ra + cbv.w), eps), nhs);
             }
           }
-        }
+        };
+        auto slow = [&](const uint32_t (&v)[32], int cc) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const int col = c0 + cc * 32 + k;
+            const float tv = fmaxf(fmaf(__uint_as_float(v[k]), ks, ra + cb[cc * 32 + k]), eps);
+            const bool valid = (col < c.nC) && (col != row + diag);
+            const float ph = valid ? phi_t<SMODE>(tv, nhs) : 0.f;
+            if (col < nneg) acc_neg += ph;
+            else acc_pos += ph;
+          }
+        };
+        auto process = [&](const uint32_t (&v)[32], int cc) {
+          if (masked) slow(v, cc);
+          else fast(v, cc);
+        };
+        // chunk cc+1 is in flight while chunk cc is processed
+        uint32_t va[32], vb[32];
+        tmem_ld32(taddr + 0, va);
+        tmem_wait_ld_reg(va);
+        tmem_ld32(taddr + 32, vb);
+        process(va, 0);
+        tmem_wait_ld_reg(vb);
+        tmem_ld32(taddr + 64, va);
+        process(vb, 1);
+        tmem_wait_ld_reg(va);
+        tmem_ld32(taddr + 96, vb);
+        process(va, 2);
+        tmem_wait_ld_reg(vb);
+        // every column of the accumulator is in registers: hand the buffer back
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->acc_empty[b]);
+        released = true;
+        process(vb, 3);
         if (!masked) {
-          if (allneg) acc_neg += tile_acc;
-          else acc_pos += tile_acc;
+          if (allneg) acc_neg += acc0 + acc1;
+          else acc_pos += acc0 + acc1;
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->acc_empty[b]);
+      if (!released) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->acc_empty[b]);
+      }
       ++t;
       const bool last_of_block = (L + 1 == L1) || (c.j + 1 == c.CT);
       if (last_of_block && valid_row) {
