@@ -217,8 +217,8 @@ KVB_API kvb_status kvb_density(const void* rows, int32_t n_rows, const void* col
  * scratch lives in one 4 MiB array inside the library's device image, held by
  * every GPU that loads the library until the process exits.  Sizes are rejected
  * with KVB_E_WORKSPACE (nothing launched) unless
- *   256 + 4*H*n_rows + 4*(H*n_cols + 128) + 32*H*n_rows  (each term rounded up
- *   to 256 bytes)  <=  4 MiB.
+ *   256 + 64*H*n_rows + 64*H*n_cols + 64*H*n_rows  (each term rounded up to
+ *   256 bytes)  <=  4 MiB.
  * The first call on a device looks up the array's address with that device
  * current: make it before any stream capture.  All calls on a device share the
  * array (it keeps the last call's contents); calls that overlap on the GPU race,

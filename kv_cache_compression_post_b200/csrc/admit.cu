@@ -228,6 +228,10 @@ __device__ __forceinline__ void copy_row(void* dst, const void* src, int row_byt
   uint4* d = static_cast<uint4*>(dst);
   for (int o = lane; o < row_bytes / 16; o += 32) d[o] = s[o];
 }
+// 64-byte augmented row, lanes 0..3
+__device__ __forceinline__ void copy_aug(uint16_t* dst, const uint16_t* src, int lane) {
+  if (lane < 4) reinterpret_cast<uint4*>(dst)[lane] = reinterpret_cast<const uint4*>(src)[lane];
+}
 
 __global__ void gather_admitted_kernel(const AdmitPlan p) {
   const int h = blockIdx.y;
@@ -238,7 +242,7 @@ __global__ void gather_admitted_kernel(const AdmitPlan p) {
   const size_t dst = static_cast<size_t>(h) * p.ldEA + p.M + w;
   copy_row(static_cast<char*>(p.EA) + dst * p.row_bytes,
            static_cast<const char*>(p.candK) + (static_cast<size_t>(h) * p.N + c) * p.row_bytes, p.row_bytes, lane);
-  if (lane == 0) p.EAterm[dst] = p.cterm[static_cast<size_t>(h) * p.ldN + c];
+  copy_aug(p.EAaug + dst * 32, p.caug + (static_cast<size_t>(h) * p.ldN + c) * 32, lane);
 }
 
 __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPlan p) {
@@ -325,7 +329,7 @@ __global__ void gather_evicted_kernel(const AdmitPlan p) {
   const size_t dst = static_cast<size_t>(h) * p.ldEA + (p.M - E) + w;
   copy_row(static_cast<char*>(p.EA) + dst * p.row_bytes, static_cast<const char*>(p.K) + src * p.row_bytes,
            p.row_bytes, lane);
-  if (lane == 0) p.EAterm[dst] = p.term[src];
+  copy_aug(p.EAaug + dst * 32, p.aug + src * 32, lane);
 }
 
 // moves: [0, P) admitted candidates, [P, P + ntail) surviving tail entries
@@ -348,9 +352,9 @@ __global__ void compact_kernel(const AdmitPlan p) {
              static_cast<const char*>(p.candK) + srow * p.row_bytes, p.row_bytes, lane);
     copy_row(static_cast<char*>(p.V) + (base + dst) * p.row_bytes,
              static_cast<const char*>(p.candV) + srow * p.row_bytes, p.row_bytes, lane);
+    copy_aug(p.aug + (base + dst) * 32, p.caug + (static_cast<size_t>(h) * p.ldN + c) * 32, lane);
     if (lane == 0) {
       p.ids[base + dst] = p.cand_ids[c];
-      p.term[base + dst] = p.cterm[static_cast<size_t>(h) * p.ldN + c];
       p.rho[base + dst] = p.rhoB[static_cast<size_t>(h) * p.ldN + c];
       p.newp[base + dst] = w;
     }
@@ -366,9 +370,9 @@ __global__ void compact_kernel(const AdmitPlan p) {
              static_cast<const char*>(p.K) + (base + src) * p.row_bytes, p.row_bytes, lane);
     copy_row(static_cast<char*>(p.V) + (base + dst) * p.row_bytes,
              static_cast<const char*>(p.V) + (base + src) * p.row_bytes, p.row_bytes, lane);
+    copy_aug(p.aug + (base + dst) * 32, p.aug + (base + src) * 32, lane);
     if (lane == 0) {
       p.ids[base + dst] = p.ids[base + src];
-      p.term[base + dst] = p.term[base + src];
       p.rho0[base + dst] = p.rho0[base + src];
       p.rho[base + dst] = p.rho[base + src] + p.proj[base + src];
       p.newp[base + dst] = -2;

@@ -5,7 +5,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
-#include "../../include/kvb.h"
+#include "kvb.h"
 
 namespace kvb {
 
@@ -23,7 +23,7 @@ struct AdmitPlan {
   int* ids = nullptr;
   float* rho = nullptr;
   float* rho0 = nullptr;
-  float* term = nullptr;    // ||k||^2 / h
+  uint16_t* aug = nullptr;  // [H][M][32] augmented rows of the keys (norm terms for the MMA)
   int* size = nullptr;      // [H]
   kvb_admit_stats* stats = nullptr;  // [H]
   // candidates (caller)
@@ -31,14 +31,14 @@ struct AdmitPlan {
   const void* candV = nullptr;
   const int* cand_ids = nullptr;
   // scratch
-  const float* cterm = nullptr;  // [H][N] candidate ||c||^2 / h
+  const uint16_t* caug = nullptr;  // [H][Nmax][32] augmented candidate rows
   float* rhoB = nullptr;         // [H][Nmax]  density against the bank
   float* mean0 = nullptr;        // [H]
   int* feasible = nullptr;       // [H]
   int* P = nullptr;              // [H] admitted count
   int* adm_idx = nullptr;        // [H][Nmax] admitted candidate indices (ascending)
   void* EA = nullptr;            // [H][M + Nmax][d] evicted keys at [M - E, M), admitted at [M, M + P)
-  float* EAterm = nullptr;       // [H][M + Nmax]
+  uint16_t* EAaug = nullptr;     // [H][M + Nmax][32]
   int ldEA = 0;                  // M + Nmax
   int* EAoff = nullptr;          // [H] M - E_h
   int* EAcnt = nullptr;          // [H] E_h (pass 3a column count)

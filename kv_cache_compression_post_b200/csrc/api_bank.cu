@@ -52,10 +52,10 @@ size_t kvb_bank::layout(void* base) {
     ids = c.take<int>(L * H * M);
     rho = c.take<float>(L * H * M);
     rho0 = c.take<float>(L * H * M);
-    term = c.take<float>(L * H * M);
+    aug = c.take<uint16_t>(L * H * M * 32);
     size = c.take<int>(L * H);
     stats = c.take<kvb_admit_stats>(L * H);
-    cterm = c.take<float>(H * N);
+    caug = c.take<uint16_t>(H * N * 32);
     rhoB = c.take<float>(H * N);
     mean0 = c.take<float>(H);
     feasible = c.take<int>(H);
@@ -68,14 +68,14 @@ size_t kvb_bank::layout(void* base) {
     EAcnt = c.take<int>(H);
     adm_idx = c.take<int>(H * N);
     EA = c.take<char>(H * (M + N) * d * elem);
-    EAterm = c.take<float>(H * (M + N) + 128);
+    EAaug = c.take<uint16_t>(H * (M + N) * 32);
     proj = c.take<float>(H * M);
     ev_slot = c.take<int>(H * M);
     tail = c.take<int>(H * M);
     newp = c.take<int>(H * M);
     sub = c.take<float>(H * M);
     coadm = c.take<float>(H * N);
-    partial = c.take<float>(8 * H * static_cast<size_t>(ldPart));
+    partial = c.take<float>(16 * H * static_cast<size_t>(ldPart));
   } else {
     F = g.frame_h * g.frame_w;
     n_seg = ((g.frame_h + g.seg_h - 1) / g.seg_h) * ((g.frame_w + g.seg_w - 1) / g.seg_w);
@@ -181,13 +181,11 @@ struct Pass {
   const void* R;       // rows buffer [H][ldR][d]
   long long ldR;
   GramSet rows;
-  const float* rowTerm;
-  int ldRT;
+  const uint16_t* Raug;  // [H][ldR][32] augmented rows of R
   const void* C;
   long long ldC;
   GramSet cols;
-  const float* colTerm;
-  int ldCT;
+  const uint16_t* Caug;  // [H][ldC][32]
   int max_rows;
   int max_cols;
   int use_diag = 0;
@@ -203,10 +201,6 @@ cudaError_t run_pass(kvb_bank* b, const Pass& ps, const DeviceInfo& dev, cudaStr
   a.d = g.head_dim;
   a.rows = ps.rows;
   a.cols = ps.cols;
-  a.rowTerm = ps.rowTerm;
-  a.ldRT = ps.ldRT;
-  a.colTerm = ps.colTerm;
-  a.ldCT = ps.ldCT;
   a.use_diag = ps.use_diag;
   a.diag_uni = 0;
   a.nneg_uni = ps.nneg;
@@ -224,14 +218,15 @@ cudaError_t run_pass(kvb_bank* b, const Pass& ps, const DeviceInfo& dev, cudaStr
     a.ldOut = ps.ldOut;
     return launch_gram_f32(a, st);
   }
-  CUtensorMap tmR, tmC;
+  CUtensorMap tmR, tmC, tmRa, tmCa;
   if (!make_tmap_bf16(&tmR, ps.R, g.head_dim, ps.ldR, g.heads, 128) ||
-      !make_tmap_bf16(&tmC, ps.C, g.head_dim, ps.ldC, g.heads, 128))
+      !make_tmap_bf16(&tmC, ps.C, g.head_dim, ps.ldC, g.heads, 128) ||
+      !make_tmap_aug(&tmRa, ps.Raug, ps.ldR, g.heads, 128) || !make_tmap_aug(&tmCa, ps.Caug, ps.ldC, g.heads, 128))
     return cudaErrorInvalidValue;
   a.partial = b->partial;
   a.ldOut = b->ldPart;
   gram_plan(a, (ps.max_cols + 127) / 128, dev.n_sm);
-  cudaError_t e = launch_gram_bf16(a, tmR, tmC, dev.n_sm, st);
+  cudaError_t e = launch_gram_bf16(a, tmR, tmC, tmRa, tmCa, st);
   if (e == cudaSuccess) e = launch_gram_reduce(a, ps.out, ps.ldOut, st);
   return e;
 }
@@ -265,20 +260,20 @@ extern "C" kvb_status kvb_admit(kvb_bank* b, int32_t layer, const void* candK, c
   p.ids = b->ids + lo;
   p.rho = b->rho + lo;
   p.rho0 = b->rho0 + lo;
-  p.term = b->term + lo;
+  p.aug = b->aug + lo * 32;
   p.size = b->size + static_cast<size_t>(layer) * H;
   p.stats = b->stats + static_cast<size_t>(layer) * H;
   p.candK = candK;
   p.candV = candV;
   p.cand_ids = cand_ids;
-  p.cterm = b->cterm;
+  p.caug = b->caug;
   p.rhoB = b->rhoB;
   p.mean0 = b->mean0;
   p.feasible = b->feasible;
   p.P = b->P;
   p.adm_idx = b->adm_idx;
   p.EA = b->EA;
-  p.EAterm = b->EAterm;
+  p.EAaug = b->EAaug;
   p.ldEA = b->ldEA;
   p.EAoff = b->EAoff;
   p.EAcnt = b->EAcnt;
@@ -296,13 +291,12 @@ extern "C" kvb_status kvb_admit(kvb_bank* b, int32_t layer, const void* candK, c
   p.ldN = b->ldN;
   p.status = b->status;
 
-  const float inv_h = 1.f / b->h;
-  cudaError_t e = launch_row_terms(candK, g.dtype, H, N, d, N, nullptr, N, inv_h, 0.f, b->cterm, b->ldN, st);
+  cudaError_t e = cudaSuccess;
+  if (g.dtype == KVB_BF16) e = launch_aug_rows(candK, g.dtype, H, N, d, N, nullptr, N, b->caug, b->ldN, st);
 
   // pass 1: candidate density against the bank, rho_B(c)
   if (e == cudaSuccess) {
-    Pass ps{candK, N, GramSet{N, nullptr, 0, nullptr}, b->cterm, b->ldN,
-            p.K, M, GramSet{0, p.size, 0, nullptr}, p.term, M, N, M};
+    Pass ps{candK, N, GramSet{N, nullptr, 0, nullptr}, b->caug, p.K, M, GramSet{0, p.size, 0, nullptr}, p.aug, N, M};
     ps.out = b->rhoB;
     ps.ldOut = b->ldN;
     e = run_pass(b, ps, dev, st);
@@ -312,8 +306,7 @@ extern "C" kvb_status kvb_admit(kvb_bank* b, int32_t layer, const void* candK, c
   if (e == cudaSuccess) e = launch_gather_admitted(p, N < M ? N : M, st);
   // pass 2: projected growth of every bank entry from the admitted block
   if (e == cudaSuccess) {
-    Pass ps{p.K, M, GramSet{0, p.size, 0, nullptr}, p.term, M,
-            b->EA, b->ldEA, GramSet{0, b->P, M, nullptr}, b->EAterm, b->ldEA, M, N};
+    Pass ps{p.K, M, GramSet{0, p.size, 0, nullptr}, p.aug, b->EA, b->ldEA, GramSet{0, b->P, M, nullptr}, b->EAaug, M, N};
     ps.out = b->proj;
     ps.ldOut = M;
     e = run_pass(b, ps, dev, st);
@@ -323,8 +316,8 @@ extern "C" kvb_status kvb_admit(kvb_bank* b, int32_t layer, const void* candK, c
   if (e == cudaSuccess) e = launch_compact(p, st);
   // pass 3a: every entry of the new bank loses its evicted neighbours
   if (e == cudaSuccess) {
-    Pass ps{p.K, M, GramSet{0, p.size, 0, nullptr}, p.term, M,
-            b->EA, b->ldEA, GramSet{0, b->EAcnt, 0, b->EAoff}, b->EAterm, b->ldEA, M, M};
+    Pass ps{p.K, M, GramSet{0, p.size, 0, nullptr}, p.aug, b->EA, b->ldEA, GramSet{0, b->EAcnt, 0, b->EAoff}, b->EAaug,
+            M, M};
     ps.nneg = INT_MAX;
     ps.out = b->sub;
     ps.ldOut = M;
@@ -332,8 +325,8 @@ extern "C" kvb_status kvb_admit(kvb_bank* b, int32_t layer, const void* candK, c
   }
   // pass 3b: co-admitted entries see one another (self excluded)
   if (e == cudaSuccess) {
-    Pass ps{b->EA, b->ldEA, GramSet{0, b->P, M, nullptr}, b->EAterm, b->ldEA,
-            b->EA, b->ldEA, GramSet{0, b->P, M, nullptr}, b->EAterm, b->ldEA, N, N};
+    Pass ps{b->EA, b->ldEA, GramSet{0, b->P, M, nullptr}, b->EAaug, b->EA, b->ldEA, GramSet{0, b->P, M, nullptr}, b->EAaug,
+            N, N};
     ps.use_diag = 1;
     ps.out = b->coadm;
     ps.ldOut = b->ldN;
@@ -422,9 +415,9 @@ kvb_status kvb_bank_import(kvb_bank* b, int32_t layer, int32_t head, const int32
     if (e == cudaSuccess)
       e = cudaMemcpyAsync(b->V + slot0 * b->row_bytes, V, static_cast<size_t>(size) * b->row_bytes,
                           cudaMemcpyDeviceToDevice, st);
-    if (e == cudaSuccess)
-      e = launch_row_terms(b->K + slot0 * b->row_bytes, b->cfg.dtype, 1, size, b->cfg.head_dim, size, nullptr,
-                           size, 1.f / b->h, 0.f, b->term + slot0, size, st);
+    if (e == cudaSuccess && b->cfg.dtype == KVB_BF16)
+      e = launch_aug_rows(b->K + slot0 * b->row_bytes, b->cfg.dtype, 1, size, b->cfg.head_dim, size, nullptr, size,
+                          b->aug + slot0 * 32, size, st);
   }
   // the size word comes from host memory; the call synchronises before returning
   int host_size = size;

@@ -13,8 +13,8 @@ namespace {
 
 struct DensityLayout {
   int* status = nullptr;
-  float* rowTerm = nullptr;
-  float* colTerm = nullptr;
+  uint16_t* rowAug = nullptr;
+  uint16_t* colAug = nullptr;
   float* partial = nullptr;
   size_t bytes = 0;
 };
@@ -24,9 +24,9 @@ DensityLayout density_layout(void* ws, int H, int nR, int nC, kvb_dtype dtype) {
   DensityLayout L;
   L.status = c.take<int>(64);
   if (dtype == KVB_BF16) {
-    L.rowTerm = c.take<float>(static_cast<size_t>(H) * nR);
-    L.colTerm = c.take<float>(static_cast<size_t>(H) * nC + 128);
-    L.partial = c.take<float>(static_cast<size_t>(8) * H * nR);
+    L.rowAug = c.take<uint16_t>(static_cast<size_t>(H) * nR * 32);
+    L.colAug = c.take<uint16_t>(static_cast<size_t>(H) * nC * 32);
+    L.partial = c.take<float>(static_cast<size_t>(16) * H * nR);
   }
   L.bytes = c.bytes();
   return L;
@@ -106,24 +106,19 @@ kvb_status kvb_density(const void* rows, int32_t n_rows, const void* cols, int32
     return cuda_status(launch_gram_f32(a, st));
   }
   if (n_cols == 0) return cuda_status(cudaMemsetAsync(out, 0, sizeof(float) * heads * n_rows, st));
-  cudaError_t e = launch_row_terms(rows, dtype, heads, n_rows, head_dim, n_rows, nullptr, n_rows, 1.f / h, 0.f,
-                                   L.rowTerm, n_rows, st);
+  cudaError_t e = launch_aug_rows(rows, dtype, heads, n_rows, head_dim, n_rows, nullptr, n_rows, L.rowAug, n_rows, st);
   if (e == cudaSuccess)
-    e = launch_row_terms(cols, dtype, heads, n_cols, head_dim, n_cols, nullptr, n_cols, 1.f / h, 0.f, L.colTerm,
-                         n_cols, st);
+    e = launch_aug_rows(cols, dtype, heads, n_cols, head_dim, n_cols, nullptr, n_cols, L.colAug, n_cols, st);
   if (e != cudaSuccess) return KVB_E_CUDA;
-  CUtensorMap tmR, tmC;
+  CUtensorMap tmR, tmC, tmRa, tmCa;
   if (!make_tmap_bf16(&tmR, rows, head_dim, n_rows, heads, 128) ||
-      !make_tmap_bf16(&tmC, cols, head_dim, n_cols, heads, 128))
+      !make_tmap_bf16(&tmC, cols, head_dim, n_cols, heads, 128) || !make_tmap_aug(&tmRa, L.rowAug, n_rows, heads, 128) ||
+      !make_tmap_aug(&tmCa, L.colAug, n_cols, heads, 128))
     return KVB_E_INVAL;
-  a.rowTerm = L.rowTerm;
-  a.ldRT = n_rows;
-  a.colTerm = L.colTerm;
-  a.ldCT = n_cols;
   a.partial = L.partial;
   a.ldOut = n_rows;
   gram_plan(a, (n_cols + 127) / 128, dev.n_sm);
-  e = launch_gram_bf16(a, tmR, tmC, dev.n_sm, st);
+  e = launch_gram_bf16(a, tmR, tmC, tmRa, tmCa, st);
   if (e == cudaSuccess) e = launch_gram_reduce(a, out, n_rows, st);
   return cuda_status(e);
 }

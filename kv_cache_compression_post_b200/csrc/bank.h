@@ -5,7 +5,7 @@
 #include <cstddef>
 #include <cstdint>
 
-#include "../../include/kvb.h"
+#include "kvb.h"
 #include "host_util.h"
 
 struct kvb_bank {
@@ -26,13 +26,13 @@ struct kvb_bank {
   int* ids = nullptr;       // [L][H][M]
   float* rho = nullptr;
   float* rho0 = nullptr;
-  float* term = nullptr;
+  uint16_t* aug = nullptr;  // [L][H][M][32] augmented rows of the bank keys
   int* size = nullptr;      // [L][H]
   kvb_admit_stats* stats = nullptr;  // [L][H]
 
   // ---- DensityKV scratch (shared by layers)
   int ldN = 0, ldEA = 0, ldPart = 0;
-  float* cterm = nullptr;
+  uint16_t* caug = nullptr; // [H][Nmax][32] augmented candidate rows
   float* rhoB = nullptr;
   float* mean0 = nullptr;
   int* feasible = nullptr;
@@ -45,7 +45,7 @@ struct kvb_bank {
   int* EAcnt = nullptr;
   int* adm_idx = nullptr;
   char* EA = nullptr;
-  float* EAterm = nullptr;
+  uint16_t* EAaug = nullptr; // [H][M + Nmax][32]
   float* proj = nullptr;
   int* ev_slot = nullptr;
   int* tail = nullptr;

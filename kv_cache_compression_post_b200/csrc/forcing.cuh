@@ -4,7 +4,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
-#include "../../include/kvb.h"
+#include "kvb.h"
 
 namespace kvb {
 

@@ -3,19 +3,21 @@
 // DensityKV §3 "Soft-Riesz Density" / App. B.1: every admit step needs, per head,
 // sums of phi(||a - b||^2 / h) over candidate x bank (and bank x admitted, bank x
 // evicted, admitted x admitted) pairs: O(N M d_k).  With the norm expansion
-//     ||a - b||^2 / h = ||a||^2/h + ||b||^2/h - (2/h) a.b
-// the a.b part is a dense bf16 contraction (tcgen05.mma, fp32 accumulate in TMEM)
-// and the rest is an epilogue on CUDA cores: one FADD + FFMA + FMNMX per pair, then
-// phi.  For the default s = 2 the reciprocals of four pairs share one MUFU op:
+//     -||a - b||^2 / 2 = a.b - ||a||^2/2 - ||b||^2/2
+// the whole right-hand side is one bf16 contraction: each key carries 32 extra
+// bf16 values ("augmented row": -||k||^2/2 split exactly into three bf16 parts,
+// plus ones), and one extra K=16 MMA step adds both norm terms, so the fp32 TMEM
+// accumulator holds -||a - b||^2 / 2 for every pair.  The epilogue on CUDA cores is
+// then t = max(acc * (-2/h) + eps, eps) and phi(t); for the default s = 2 the
+// reciprocals of four pairs share one MUFU op:
 //     1/t0 + 1/t1 + 1/t2 + 1/t3 = ((t0+t1) t2 t3 + (t2+t3) t0 t1) / (t0 t1 t2 t3)
-// which keeps the special-function unit off the critical path.
 //
-// Work unit = (head, 256-row block, chunk of column tiles).  A persistent grid of
-// one CTA per SM walks a contiguous range of units; within a unit the CTA keeps
-// the 256 rows resident in shared memory and streams 128-row column tiles through
-// a 4-stage TMA ring.  Warp roles: 0 = TMA producer, 1 = MMA issuer, 2 = TMEM
-// owner, 4..11 = epilogue (two row tiles x four TMEM lane quarters, one thread per
-// row: row sums need no cross-thread reduction).  TMEM holds 2 row tiles x 2
+// Work = the sequence of (head, 256-row block, 128-column tile) steps, split evenly
+// over a persistent grid (one CTA per SM).  A CTA keeps its 256 rows (two 128-row
+// MMA tiles) in shared memory and streams column tiles through a 4-stage TMA ring.
+// Warp roles: 0 = TMA producer, 1 = MMA issuer, 2 = TMEM owner, 4..19 = epilogue
+// (2 row tiles x 4 TMEM lane quarters x 2 column halves; one thread per row and
+// half, so row sums need no cross-thread reduction).  TMEM holds 2 row tiles x 2
 // buffers x 128 fp32 columns = all 512 columns.
 #include <climits>
 
@@ -40,6 +42,8 @@ struct alignas(8) GramBars {
 };
 constexpr int kBarBytes = 256;
 static_assert(sizeof(GramBars) <= kBarBytes, "barrier block overflows its reservation");
+constexpr uint32_t kAugTileBytes = kGramRowTile * 32;   // 128 rows x 16 bf16
+constexpr int kEpiWarps = 16;
 
 __device__ __forceinline__ int set_n(const GramSet& s, int h) { return s.n_dev ? s.n_dev[h] : s.n_uni; }
 __device__ __forceinline__ int set_off(const GramSet& s, int h) { return s.off_dev ? s.off_dev[h] : s.off_uni; }
@@ -128,16 +132,17 @@ __device__ __forceinline__ float phi_t(float t, float nhs) {
 template <int SMODE>
 __global__ void __launch_bounds__(kGramThreads, 1)
     gram_bf16_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmC,
+                     const __grid_constant__ CUtensorMap tmRa, const __grid_constant__ CUtensorMap tmCa,
                      const GramArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nbox = a.d / 64;
   const uint32_t tileBytes = static_cast<uint32_t>(kGramRowTile) * a.d * 2;
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + 2 * tileBytes;
-  GramBars* bars = reinterpret_cast<GramBars*>(sB + kStages * tileBytes);
-  // [8 warps][2][128] column terms, 16-byte aligned for float4 reads
-  float* sColTerm = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kBarBytes);
+  uint8_t* sA = smem;                                  // 2 row tiles
+  uint8_t* sB = sA + 2 * tileBytes;                    // kStages column tiles
+  uint8_t* sAa = sB + kStages * tileBytes;             // 2 augmented row tiles
+  uint8_t* sBa = sAa + 2 * kAugTileBytes;              // kStages augmented column tiles
+  GramBars* bars = reinterpret_cast<GramBars*>(sBa + kStages * kAugTileBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -151,7 +156,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->acc_full[b], 1);
-      mbar_init(&bars->acc_empty[b], 8);
+      mbar_init(&bars->acc_empty[b], kEpiWarps);
     }
     bars->abort = 0;
     fence_barrier_init();
@@ -176,6 +181,8 @@ __global__ void __launch_bounds__(kGramThreads, 1)
     if (lane == 0) {
       prefetch_tmap(&tmR);
       prefetch_tmap(&tmC);
+      prefetch_tmap(&tmRa);
+      prefetch_tmap(&tmCa);
       int it = 0, aload = 0;
       bool ok = true;
       Cursor c;
@@ -184,19 +191,20 @@ __global__ void __launch_bounds__(kGramThreads, 1)
         if (L == L0 || c.j == 0) {
           if (aload > 0 && !(ok = mbar_wait(&bars->a_empty, (aload - 1) & 1, abort, a.status))) break;
           const int nact = nact_of(c);
-          mbar_arrive_expect_tx(&bars->a_full, nact * tileBytes);
-          for (int r = 0; r < nact; ++r)
-            for (int k = 0; k < nbox; ++k)
-              tma_load_3d(sA + r * tileBytes + k * 16384, &tmR, &bars->a_full, k * 64,
-                          c.rOff + c.rb * kGramRowBlock + r * kGramRowTile, c.h);
+          mbar_arrive_expect_tx(&bars->a_full, nact * (tileBytes + kAugTileBytes));
+          for (int r = 0; r < nact; ++r) {
+            const int y = c.rOff + c.rb * kGramRowBlock + r * kGramRowTile;
+            for (int k = 0; k < nbox; ++k) tma_load_3d(sA + r * tileBytes + k * 16384, &tmR, &bars->a_full, k * 64, y, c.h);
+            tma_load_3d(sAa + r * kAugTileBytes, &tmRa, &bars->a_full, 0, y, c.h);  // row form
+          }
           ++aload;
         }
         const int s = it % kStages;
         if (!(ok = mbar_wait(&bars->empty[s], ((it / kStages) & 1) ^ 1, abort, a.status))) break;
-        mbar_arrive_expect_tx(&bars->full[s], tileBytes);
-        for (int k = 0; k < nbox; ++k)
-          tma_load_3d(sB + s * tileBytes + k * 16384, &tmC, &bars->full[s], k * 64, c.cOff + c.j * kGramColTile,
-                      c.h);
+        mbar_arrive_expect_tx(&bars->full[s], tileBytes + kAugTileBytes);
+        const int y = c.cOff + c.j * kGramColTile;
+        for (int k = 0; k < nbox; ++k) tma_load_3d(sB + s * tileBytes + k * 16384, &tmC, &bars->full[s], k * 64, y, c.h);
+        tma_load_3d(sBa + s * kAugTileBytes, &tmCa, &bars->full[s], 16, y, c.h);  // column form
         ++it;
       }
       if (!ok) {
@@ -211,6 +219,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, kGramColTile, 0, 0);
       const uint32_t aBase = smem_u32(sA), bBase = smem_u32(sB);
+      const uint32_t aaBase = smem_u32(sAa), baBase = smem_u32(sBa);
       int it = 0, t = 0, aload = 0;
       bool ok = true;
       Cursor c;
@@ -235,6 +244,9 @@ __global__ void __launch_bounds__(kGramThreads, 1)
             const uint64_t bd = sdesc_sw128(bBase + s * tileBytes + koff, 16, 1024);
             mma_f16_ss(dcol, ad, bd, idesc, kk > 0 ? 1u : 0u);
           }
+          // the norm terms: one more K=16 step over the augmented rows
+          mma_f16_ss(dcol, sdesc_sw32(aaBase + r * kAugTileBytes, 256), sdesc_sw32(baBase + s * kAugTileBytes, 256),
+                     idesc, 1u);
         }
         mma_commit(&bars->empty[s]);
         mma_commit(&bars->acc_full[b]);
@@ -253,16 +265,16 @@ __global__ void __launch_bounds__(kGramThreads, 1)
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
     const int e = warp - 4;
-    const int r = e >> 2;          // row tile
     const int q = warp & 3;        // TMEM lane quarter (warp_id % 4)
+    const int r = (e >> 2) & 1;    // row tile
+    const int hf = e >> 3;         // column half of every 128-column tile
     const int row_in_tile = q * 32 + lane;
     const float ks = a.kscale, eps = a.eps, nhs = -0.5f * a.s;
     int t = 0;
     bool ok = true;
     Cursor c;
     if (L0 < L1) cursor_seek(a, L0, c);
-    float acc_pos = 0.f, acc_neg = 0.f, ra = 0.f;
-    float cbn[4] = {0.f, 0.f, 0.f, 0.f};  // next tile's column terms (prefetched)
+    float acc_pos = 0.f, acc_neg = 0.f;
     int row = 0, nneg = 0, diag = 0, rt0 = 0;
     bool active = false, valid_row = false;
     long long Lblock = L0;  // first step of the current row block
@@ -273,69 +285,38 @@ __global__ void __launch_bounds__(kGramThreads, 1)
         row = rt0 + row_in_tile;
         active = r < nact_of(c);
         valid_row = active && row < c.nR;
-        ra = (valid_row ? a.rowTerm[static_cast<size_t>(c.h) * a.ldRT + c.rOff + row] : 0.f) + eps;
         nneg = a.nneg_dev ? a.nneg_dev[c.h] : a.nneg_uni;
         diag = a.use_diag ? (a.diag_dev ? a.diag_dev[c.h] : a.diag_uni) : INT_MIN / 2;
         acc_pos = 0.f;
         acc_neg = 0.f;
       }
       const int b = t & 1;
-      const int c0 = c.j * kGramColTile;
-      if (*abort) {
-        ok = false;
-        break;
-      }
-      // this warp's copy of the tile's column terms (no cross-warp barrier, so an
-      // aborting warp can never strand another one); the values were fetched one
-      // tile ahead so their L2 latency overlaps the previous tile
-      float* cb = sColTerm + (e * 2 + b) * kGramColTile;
-      if (L == L0) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const long idx = static_cast<long>(c.cOff) + c0 + lane + 32 * i;
-          cbn[i] = (idx < a.ldCT) ? a.colTerm[static_cast<size_t>(c.h) * a.ldCT + idx] : 0.f;
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) cb[lane + 32 * i] = cbn[i];
-      __syncwarp();
-      if (L + 1 < L1) {
-        Cursor cn = c;
-        cursor_next(a, cn);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const long idx = static_cast<long>(cn.cOff) + cn.j * kGramColTile + lane + 32 * i;
-          cbn[i] = (idx < a.ldCT) ? a.colTerm[static_cast<size_t>(cn.h) * a.ldCT + idx] : 0.f;
-        }
-      }
+      const int c0 = c.j * kGramColTile + hf * 64;  // first column of this thread's half
       if (!(ok = mbar_wait(&bars->acc_full[b], (t >> 1) & 1, abort, a.status))) break;
       tc_fence_after();
       bool released = false;
       if (active) {
-        const bool tail = c0 + kGramColTile > c.nC;
-        const bool allneg = c0 + kGramColTile <= nneg;
+        const bool tail = c0 + 64 > c.nC;
+        const bool allneg = c0 + 64 <= nneg;
         const bool mixed = (c0 < nneg) && !allneg;
         // diagonal columns of this row tile: [rt0 + diag, rt0 + diag + 128)
-        const bool diag_hit =
-            a.use_diag && (rt0 + diag < c0 + kGramColTile) && (rt0 + diag + kGramRowTile > c0);
+        const bool diag_hit = a.use_diag && (rt0 + diag < c0 + 64) && (rt0 + diag + kGramRowTile > c0);
         const bool masked = tail || mixed || diag_hit;
-        const uint32_t taddr =
-            tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>((r * 2 + b) * kGramColTile);
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>((r * 2 + b) * kGramColTile + hf * 64);
         float acc0 = 0.f, acc1 = 0.f;
-        auto fast = [&](const uint32_t (&v)[32], int cc) {
+        auto fast = [&](const uint32_t (&v)[32]) {
           if constexpr (SMODE == 2) {
 #pragma unroll
             for (int k = 0; k < 32; k += 8) {
-              const float4 ca = *reinterpret_cast<const float4*>(cb + cc * 32 + k);
-              const float4 cbv = *reinterpret_cast<const float4*>(cb + cc * 32 + k + 4);
-              const float t0 = fmaxf(fmaf(__uint_as_float(v[k + 0]), ks, ra + ca.x), eps);
-              const float t1 = fmaxf(fmaf(__uint_as_float(v[k + 1]), ks, ra + ca.y), eps);
-              const float t2 = fmaxf(fmaf(__uint_as_float(v[k + 2]), ks, ra + ca.z), eps);
-              const float t3 = fmaxf(fmaf(__uint_as_float(v[k + 3]), ks, ra + ca.w), eps);
-              const float t4 = fmaxf(fmaf(__uint_as_float(v[k + 4]), ks, ra + cbv.x), eps);
-              const float t5 = fmaxf(fmaf(__uint_as_float(v[k + 5]), ks, ra + cbv.y), eps);
-              const float t6 = fmaxf(fmaf(__uint_as_float(v[k + 6]), ks, ra + cbv.z), eps);
-              const float t7 = fmaxf(fmaf(__uint_as_float(v[k + 7]), ks, ra + cbv.w), eps);
+              const float t0 = fmaxf(fmaf(__uint_as_float(v[k + 0]), ks, eps), eps);
+              const float t1 = fmaxf(fmaf(__uint_as_float(v[k + 1]), ks, eps), eps);
+              const float t2 = fmaxf(fmaf(__uint_as_float(v[k + 2]), ks, eps), eps);
+              const float t3 = fmaxf(fmaf(__uint_as_float(v[k + 3]), ks, eps), eps);
+              const float t4 = fmaxf(fmaf(__uint_as_float(v[k + 4]), ks, eps), eps);
+              const float t5 = fmaxf(fmaf(__uint_as_float(v[k + 5]), ks, eps), eps);
+              const float t6 = fmaxf(fmaf(__uint_as_float(v[k + 6]), ks, eps), eps);
+              const float t7 = fmaxf(fmaf(__uint_as_float(v[k + 7]), ks, eps), eps);
               const float p01 = t0 * t1, p23 = t2 * t3, p45 = t4 * t5, p67 = t6 * t7;
               const float na = fmaf(t2 + t3, p01, (t0 + t1) * p23);
               const float nb2 = fmaf(t6 + t7, p45, (t4 + t5) * p67);
@@ -344,12 +325,9 @@ __global__ void __launch_bounds__(kGramThreads, 1)
             }
           } else {
 #pragma unroll
-            for (int k = 0; k < 32; k += 4) {
-              const float4 cbv = *reinterpret_cast<const float4*>(cb + cc * 32 + k);
-              acc0 += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 0]), ks, ra + cbv.x), eps), nhs);
-              acc1 += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 1]), ks, ra + cbv.y), eps), nhs);
-              acc0 += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 2]), ks, ra + cbv.z), eps), nhs);
-              acc1 += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 3]), ks, ra + cbv.w), eps), nhs);
+            for (int k = 0; k < 32; k += 2) {
+              acc0 += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 0]), ks, eps), eps), nhs);
+              acc1 += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 1]), ks, eps), eps), nhs);
             }
           }
         };
@@ -357,36 +335,28 @@ __global__ void __launch_bounds__(kGramThreads, 1)
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
             const int col = c0 + cc * 32 + k;
-            const float tv = fmaxf(fmaf(__uint_as_float(v[k]), ks, ra + cb[cc * 32 + k]), eps);
+            const float tv = fmaxf(fmaf(__uint_as_float(v[k]), ks, eps), eps);
             const bool valid = (col < c.nC) && (col != row + diag);
             const float ph = valid ? phi_t<SMODE>(tv, nhs) : 0.f;
             if (col < nneg) acc_neg += ph;
             else acc_pos += ph;
           }
         };
-        auto process = [&](const uint32_t (&v)[32], int cc) {
-          if (masked) slow(v, cc);
-          else fast(v, cc);
-        };
-        // chunk cc+1 is in flight while chunk cc is processed
+        // chunk 1 is in flight while chunk 0 is processed
         uint32_t va[32], vb[32];
         tmem_ld32(taddr + 0, va);
         tmem_wait_ld_reg(va);
         tmem_ld32(taddr + 32, vb);
-        process(va, 0);
+        if (masked) slow(va, 0);
+        else fast(va);
         tmem_wait_ld_reg(vb);
-        tmem_ld32(taddr + 64, va);
-        process(vb, 1);
-        tmem_wait_ld_reg(va);
-        tmem_ld32(taddr + 96, vb);
-        process(va, 2);
-        tmem_wait_ld_reg(vb);
-        // every column of the accumulator is in registers: hand the buffer back
+        // every column this warp needs is in registers: hand the buffer back
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->acc_empty[b]);
         released = true;
-        process(vb, 3);
+        if (masked) slow(vb, 1);
+        else fast(vb);
         if (!masked) {
           if (allneg) acc_neg += acc0 + acc1;
           else acc_pos += acc0 + acc1;
@@ -400,7 +370,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
       ++t;
       const bool last_of_block = (L + 1 == L1) || (c.j + 1 == c.CT);
       if (last_of_block && valid_row) {
-        const int slot = cta - cta_of(Lblock, T, G);
+        const int slot = 2 * (cta - cta_of(Lblock, T, G)) + hf;
         if (slot >= 0 && slot < a.slots)
           a.partial[(static_cast<size_t>(slot) * a.H + c.h) * a.ldOut + row] = acc_pos - acc_neg;
         else
@@ -486,7 +456,8 @@ __global__ void gram_reduce_kernel(const GramArgs a, float* out, int ldOut) {
     }
     const long long Lb = before + static_cast<long long>(r / kGramRowBlock) * CT;
     const int first = cta_of(Lb, T, G), last = cta_of(Lb + CT - 1, T, G);
-    for (int sl = 0; sl <= last - first && sl < a.slots; ++sl)
+    const int n = 2 * (last - first + 1);  // two column halves per CTA
+    for (int sl = 0; sl < n && sl < a.slots; ++sl)
       acc += a.partial[(static_cast<size_t>(sl) * a.H + h) * a.ldOut + r];
   }
   out[static_cast<size_t>(h) * ldOut + r] = acc;
@@ -496,19 +467,20 @@ __global__ void gram_reduce_kernel(const GramArgs a, float* out, int ldOut) {
 
 size_t gram_smem_bytes(int d) {
   const size_t tile = static_cast<size_t>(kGramRowTile) * d * 2;
-  return 1024 + (2 + kStages) * tile + kBarBytes + 16 * kGramColTile * sizeof(float);
+  return 1024 + (2 + kStages) * (tile + kAugTileBytes) + kBarBytes;
 }
 
 void gram_plan(GramArgs& a, int max_col_tiles, int n_sm) {
+  // at most 8 CTAs cover a row block (every active CTA takes >= min_steps steps);
+  // each CTA writes one partial per column half
   a.grid = n_sm;
-  a.slots = 8;
-  const int m = (max_col_tiles + a.slots - 2) / (a.slots - 1);
+  a.slots = 16;
+  const int m = (max_col_tiles + 6) / 7;
   a.min_steps = m < 1 ? 1 : m;
 }
 
-cudaError_t launch_gram_bf16(const GramArgs& a, const CUtensorMap& tmR, const CUtensorMap& tmC, int n_sm,
-                             cudaStream_t st) {
-  (void)n_sm;
+cudaError_t launch_gram_bf16(const GramArgs& a, const CUtensorMap& tmR, const CUtensorMap& tmC,
+                             const CUtensorMap& tmRa, const CUtensorMap& tmCa, cudaStream_t st) {
   const size_t smem = gram_smem_bytes(a.d);
   const int grid = a.grid;
   if (grid <= 0) return cudaSuccess;
@@ -517,17 +489,17 @@ cudaError_t launch_gram_bf16(const GramArgs& a, const CUtensorMap& tmR, const CU
     e = cudaFuncSetAttribute(gram_bf16_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     note_launch();
-    gram_bf16_kernel<2><<<grid, kGramThreads, smem, st>>>(tmR, tmC, a);
+    gram_bf16_kernel<2><<<grid, kGramThreads, smem, st>>>(tmR, tmC, tmRa, tmCa, a);
   } else if (a.s == 1.f) {
     e = cudaFuncSetAttribute(gram_bf16_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     note_launch();
-    gram_bf16_kernel<1><<<grid, kGramThreads, smem, st>>>(tmR, tmC, a);
+    gram_bf16_kernel<1><<<grid, kGramThreads, smem, st>>>(tmR, tmC, tmRa, tmCa, a);
   } else {
     e = cudaFuncSetAttribute(gram_bf16_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     note_launch();
-    gram_bf16_kernel<0><<<grid, kGramThreads, smem, st>>>(tmR, tmC, a);
+    gram_bf16_kernel<0><<<grid, kGramThreads, smem, st>>>(tmR, tmC, tmRa, tmCa, a);
   }
   return cudaGetLastError();
 }

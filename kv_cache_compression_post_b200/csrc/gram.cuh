@@ -11,7 +11,7 @@ namespace kvb {
 constexpr int kGramRowTile = 128;      // rows per TMEM accumulator (M of the MMA)
 constexpr int kGramRowBlock = 256;     // rows per work unit (two accumulators)
 constexpr int kGramColTile = 128;      // columns per MMA (N)
-constexpr int kGramThreads = 384;      // 4 control warps + 8 epilogue warps
+constexpr int kGramThreads = 640;      // 4 control warps + 16 epilogue warps
 
 // A set of rows/cols: per head a count and a start row inside its buffer.  Each
 // field is either a uniform value or (if the pointer is non-null) a device array
@@ -27,10 +27,6 @@ struct GramArgs {
   int H = 0;
   int d = 0;
   GramSet rows, cols;
-  const float* rowTerm = nullptr;  // [H][ldRT]: ||r||^2/h         (indexed off+r)
-  int ldRT = 0;
-  const float* colTerm = nullptr;  // [H][ldCT]: ||c||^2/h         (indexed off+c)
-  int ldCT = 0;
   int use_diag = 0;                // exclude pair (r, c) with c == r + diag
   int diag_uni = 0;
   const int* diag_dev = nullptr;
@@ -41,7 +37,7 @@ struct GramArgs {
   float s = 2.f;
   int max_rows = 0;                // upper bound of the row count of any head
   int grid = 0;                    // CTAs launched
-  int slots = 0;                   // partial slots per row block
+  int slots = 0;                   // partial slots per row block (two column halves per CTA)
   int min_steps = 1;               // every active CTA takes at least this many steps
   float* partial = nullptr;        // [slots][H][ldOut]
   int ldOut = 0;
@@ -52,9 +48,11 @@ struct GramArgs {
   int ldR = 0, ldC = 0;
 };
 
-// bf16 operands through TMA: tensor maps over [H][rows][d] with 64x128 boxes.
-cudaError_t launch_gram_bf16(const GramArgs& a, const CUtensorMap& tmR, const CUtensorMap& tmC, int n_sm,
-                             cudaStream_t st);
+// bf16 operands through TMA: tensor maps over [H][rows][d] (64x128 boxes) and over
+// the augmented rows [H][rows][32] (16x128 boxes, see launch_aug_rows): the MMA
+// accumulates a.b - (||a||^2 + ||b||^2)/2 = -||a - b||^2 / 2 directly.
+cudaError_t launch_gram_bf16(const GramArgs& a, const CUtensorMap& tmR, const CUtensorMap& tmC,
+                             const CUtensorMap& tmRa, const CUtensorMap& tmCa, cudaStream_t st);
 // f32 operands, CUDA-core direct differences (small problems).
 cudaError_t launch_gram_f32(const GramArgs& a, cudaStream_t st);
 

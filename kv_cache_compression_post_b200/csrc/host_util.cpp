@@ -60,6 +60,20 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, int d, long long rows, int
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_aug(CUtensorMap* m, const void* base, long long rows, int heads, int box_rows) {
+  std::call_once(g_encode_once, load_encode);
+  if (!g_encode || !base || rows <= 0 || heads <= 0) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0) return false;
+  cuuint64_t dims[3] = {32, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(heads)};
+  cuuint64_t strides[2] = {64, static_cast<cuuint64_t>(rows) * 64};
+  cuuint32_t box[3] = {16, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace kvb
 
 extern "C" unsigned long long kvb_launch_count(void) { return kvb::g_launches.load(std::memory_order_relaxed); }

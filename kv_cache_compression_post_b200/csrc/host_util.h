@@ -7,7 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include "../../include/kvb.h"
+#include "kvb.h"
 
 namespace kvb {
 
@@ -24,6 +24,9 @@ bool current_device(DeviceInfo* out);
 // 3D tiled tensor map over a bf16 [heads][rows][d] buffer, box 64 x box_rows x 1,
 // 128-byte swizzle, zero fill out of bounds.
 bool make_tmap_bf16(CUtensorMap* m, const void* base, int d, long long rows, int heads, int box_rows);
+// Tensor map over the augmented rows [heads][rows][32] bf16 (64 bytes per row),
+// box 16 x box_rows x 1, 32-byte swizzle (one K=16 slice of an MMA operand).
+bool make_tmap_aug(CUtensorMap* m, const void* base, long long rows, int heads, int box_rows);
 
 // Count of kernel launches issued by the library in this process.
 void note_launch();

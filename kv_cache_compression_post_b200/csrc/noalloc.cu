@@ -52,17 +52,17 @@ void* scratch_address(int dev) {
 }
 
 struct NoAllocLayout {
-  size_t status = 0, rowTerm = 0, colTerm = 0, partial = 0, bytes = 0;
+  size_t status = 0, rowAug = 0, colAug = 0, partial = 0, bytes = 0;
 };
 
 NoAllocLayout noalloc_layout(int H, int nR, int nC) {
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
   NoAllocLayout L;
   L.status = 0;
-  L.rowTerm = up(L.status + 256);
-  L.colTerm = up(L.rowTerm + sizeof(float) * static_cast<size_t>(H) * nR);
-  L.partial = up(L.colTerm + sizeof(float) * (static_cast<size_t>(H) * nC + 128));
-  L.bytes = up(L.partial + sizeof(float) * static_cast<size_t>(8) * H * nR);
+  L.rowAug = up(L.status + 256);
+  L.colAug = up(L.rowAug + 64 * static_cast<size_t>(H) * nR);
+  L.partial = up(L.colAug + 64 * static_cast<size_t>(H) * nC);
+  L.bytes = up(L.partial + sizeof(float) * static_cast<size_t>(16) * H * nR);
   return L;
 }
 
@@ -88,23 +88,22 @@ extern "C" kvb_status kvb_density_noalloc(const void* rows, int32_t n_rows, cons
   if (!base) return KVB_E_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int* status = status_out ? status_out : reinterpret_cast<int*>(base + L.status);
-  float* rowTerm = reinterpret_cast<float*>(base + L.rowTerm);
-  float* colTerm = reinterpret_cast<float*>(base + L.colTerm);
+  uint16_t* rowAug = reinterpret_cast<uint16_t*>(base + L.rowAug);
+  uint16_t* colAug = reinterpret_cast<uint16_t*>(base + L.colAug);
   // the status word is the only piece that must start at zero on every call (the
-  // row terms and the partials are written in full before they are read)
+  // augmented rows and the partials are written in full before they are read)
   if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return KVB_E_CUDA;
   if (n_cols == 0) return cuda_status(cudaMemsetAsync(out, 0, sizeof(float) * heads * n_rows, st));
 
   const float h = dist_scale > 0.f ? dist_scale : static_cast<float>(head_dim);
-  cudaError_t e = launch_row_terms(rows, dtype, heads, n_rows, head_dim, n_rows, nullptr, n_rows, 1.f / h, 0.f,
-                                   rowTerm, n_rows, st);
+  cudaError_t e = launch_aug_rows(rows, dtype, heads, n_rows, head_dim, n_rows, nullptr, n_rows, rowAug, n_rows, st);
   if (e == cudaSuccess)
-    e = launch_row_terms(cols, dtype, heads, n_cols, head_dim, n_cols, nullptr, n_cols, 1.f / h, 0.f, colTerm,
-                         n_cols, st);
+    e = launch_aug_rows(cols, dtype, heads, n_cols, head_dim, n_cols, nullptr, n_cols, colAug, n_cols, st);
   if (e != cudaSuccess) return KVB_E_CUDA;
-  CUtensorMap tmR, tmC;
+  CUtensorMap tmR, tmC, tmRa, tmCa;
   if (!make_tmap_bf16(&tmR, rows, head_dim, n_rows, heads, 128) ||
-      !make_tmap_bf16(&tmC, cols, head_dim, n_cols, heads, 128))
+      !make_tmap_bf16(&tmC, cols, head_dim, n_cols, heads, 128) || !make_tmap_aug(&tmRa, rowAug, n_rows, heads, 128) ||
+      !make_tmap_aug(&tmCa, colAug, n_cols, heads, 128))
     return KVB_E_INVAL;
   GramArgs a;
   a.H = heads;
@@ -118,14 +117,10 @@ extern "C" kvb_status kvb_density_noalloc(const void* rows, int32_t n_rows, cons
   a.s = s;
   a.max_rows = n_rows;
   a.status = status;
-  a.rowTerm = rowTerm;
-  a.ldRT = n_rows;
-  a.colTerm = colTerm;
-  a.ldCT = n_cols;
   a.partial = reinterpret_cast<float*>(base + L.partial);
   a.ldOut = n_rows;
   gram_plan(a, (n_cols + 127) / 128, dev.n_sm);
-  e = launch_gram_bf16(a, tmR, tmC, dev.n_sm, st);
+  e = launch_gram_bf16(a, tmR, tmC, tmRa, tmCa, st);
   if (e == cudaSuccess) e = launch_gram_reduce(a, out, n_rows, st);
   return cuda_status(e);
 }

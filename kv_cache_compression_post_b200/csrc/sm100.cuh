@@ -179,14 +179,21 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 // Shared-memory matrix descriptor, 128-byte swizzle (PTX ISA tcgen05 matrix
 // descriptor): start address, leading and stride byte offsets (all >> 4), the
 // fixed sm_100 version field (1 at bit 46) and layout type 2 = SWIZZLE_128B.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes, uint32_t layout) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
   d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
   d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= static_cast<uint64_t>(1) << 46;
-  d |= static_cast<uint64_t>(2) << 61;
+  d |= static_cast<uint64_t>(layout & 7u) << 61;
   return d;
+}
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return sdesc(saddr, lbo_bytes, sbo_bytes, 2u);
+}
+// 32-byte swizzle (layout type 6): K-major rows of 32 bytes, 8-row groups SBO apart
+__device__ __forceinline__ uint64_t sdesc_sw32(uint32_t saddr, uint32_t sbo_bytes) {
+  return sdesc(saddr, 16, sbo_bytes, 6u);
 }
 
 // Instruction descriptor, kind::f16: f32 accumulator (bit 4), bf16 A and B (bits
