@@ -141,7 +141,8 @@ kvb_status kvb_bank_create(const kvb_config* cfg, void* workspace, size_t worksp
   b->layout(workspace);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t LH = static_cast<size_t>(cfg->layers) * cfg->heads;
-  cudaError_t e = cudaMemsetAsync(b->status, 0, sizeof(int), st);
+  // status word, and status[1] = the largest ||k||^2 ever stored (density clamp guard)
+  cudaError_t e = cudaMemsetAsync(b->status, 0, 2 * sizeof(int), st);
   if (e == cudaSuccess) e = cudaMemsetAsync(b->stats, 0, LH * sizeof(kvb_admit_stats), st);
   if (cfg->method == KVB_DENSITYKV) {
     // rows past a bank's size are read by full attention tiles (and masked): keep
@@ -220,12 +221,13 @@ cudaError_t run_pass(kvb_bank* b, const Pass& ps, const DeviceInfo& dev, cudaStr
   }
   CUtensorMap tmR, tmC, tmRa, tmCa;
   if (!make_tmap_bf16(&tmR, ps.R, g.head_dim, ps.ldR, g.heads, 128) ||
-      !make_tmap_bf16(&tmC, ps.C, g.head_dim, ps.ldC, g.heads, 128) ||
-      !make_tmap_aug(&tmRa, ps.Raug, ps.ldR, g.heads, 128) || !make_tmap_aug(&tmCa, ps.Caug, ps.ldC, g.heads, 128))
+      !make_tmap_bf16(&tmC, ps.C, g.head_dim, ps.ldC, g.heads, kGramColTile) ||
+      !make_tmap_aug(&tmRa, ps.Raug, ps.ldR, g.heads, 128) || !make_tmap_aug(&tmCa, ps.Caug, ps.ldC, g.heads, kGramColTile))
     return cudaErrorInvalidValue;
   a.partial = b->partial;
   a.ldOut = b->ldPart;
-  gram_plan(a, (ps.max_cols + 127) / 128, dev.n_sm);
+  a.norm_max = reinterpret_cast<const float*>(b->status + 1);
+  gram_plan(a, (ps.max_cols + kGramColTile - 1) / kGramColTile, dev.n_sm);
   cudaError_t e = launch_gram_bf16(a, tmR, tmC, tmRa, tmCa, st);
   if (e == cudaSuccess) e = launch_gram_reduce(a, ps.out, ps.ldOut, st);
   return e;
@@ -292,7 +294,9 @@ extern "C" kvb_status kvb_admit(kvb_bank* b, int32_t layer, const void* candK, c
   p.status = b->status;
 
   cudaError_t e = cudaSuccess;
-  if (g.dtype == KVB_BF16) e = launch_aug_rows(candK, g.dtype, H, N, d, N, nullptr, N, b->caug, b->ldN, st);
+  if (g.dtype == KVB_BF16)
+    e = launch_aug_rows(candK, g.dtype, H, N, d, N, nullptr, N, b->caug, b->ldN, reinterpret_cast<float*>(b->status + 1),
+                        st);
 
   // pass 1: candidate density against the bank, rho_B(c)
   if (e == cudaSuccess) {
@@ -417,7 +421,7 @@ kvb_status kvb_bank_import(kvb_bank* b, int32_t layer, int32_t head, const int32
                           cudaMemcpyDeviceToDevice, st);
     if (e == cudaSuccess && b->cfg.dtype == KVB_BF16)
       e = launch_aug_rows(b->K + slot0 * b->row_bytes, b->cfg.dtype, 1, size, b->cfg.head_dim, size, nullptr, size,
-                          b->aug + slot0 * 32, size, st);
+                          b->aug + slot0 * 32, size, reinterpret_cast<float*>(b->status + 1), st);
   }
   // the size word comes from host memory; the call synchronises before returning
   int host_size = size;

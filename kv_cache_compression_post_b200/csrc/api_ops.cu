@@ -81,7 +81,9 @@ kvb_status kvb_density(const void* rows, int32_t n_rows, const void* cols, int32
   if (!current_device(&dev)) return KVB_E_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float h = dist_scale > 0.f ? dist_scale : static_cast<float>(head_dim);
-  if (cudaMemsetAsync(L.status, 0, sizeof(int), st) != cudaSuccess) return KVB_E_CUDA;
+  // status word and the largest key norm seen (status[1]) start at zero
+  if (cudaMemsetAsync(L.status, 0, 2 * sizeof(int), st) != cudaSuccess) return KVB_E_CUDA;
+  float* norm_max = reinterpret_cast<float*>(L.status + 1);
 
   GramArgs a;
   a.H = heads;
@@ -106,18 +108,20 @@ kvb_status kvb_density(const void* rows, int32_t n_rows, const void* cols, int32
     return cuda_status(launch_gram_f32(a, st));
   }
   if (n_cols == 0) return cuda_status(cudaMemsetAsync(out, 0, sizeof(float) * heads * n_rows, st));
-  cudaError_t e = launch_aug_rows(rows, dtype, heads, n_rows, head_dim, n_rows, nullptr, n_rows, L.rowAug, n_rows, st);
+  cudaError_t e =
+      launch_aug_rows(rows, dtype, heads, n_rows, head_dim, n_rows, nullptr, n_rows, L.rowAug, n_rows, norm_max, st);
   if (e == cudaSuccess)
-    e = launch_aug_rows(cols, dtype, heads, n_cols, head_dim, n_cols, nullptr, n_cols, L.colAug, n_cols, st);
+    e = launch_aug_rows(cols, dtype, heads, n_cols, head_dim, n_cols, nullptr, n_cols, L.colAug, n_cols, norm_max, st);
+  a.norm_max = norm_max;
   if (e != cudaSuccess) return KVB_E_CUDA;
   CUtensorMap tmR, tmC, tmRa, tmCa;
   if (!make_tmap_bf16(&tmR, rows, head_dim, n_rows, heads, 128) ||
-      !make_tmap_bf16(&tmC, cols, head_dim, n_cols, heads, 128) || !make_tmap_aug(&tmRa, L.rowAug, n_rows, heads, 128) ||
-      !make_tmap_aug(&tmCa, L.colAug, n_cols, heads, 128))
+      !make_tmap_bf16(&tmC, cols, head_dim, n_cols, heads, kGramColTile) || !make_tmap_aug(&tmRa, L.rowAug, n_rows, heads, 128) ||
+      !make_tmap_aug(&tmCa, L.colAug, n_cols, heads, kGramColTile))
     return KVB_E_INVAL;
   a.partial = L.partial;
   a.ldOut = n_rows;
-  gram_plan(a, (n_cols + 127) / 128, dev.n_sm);
+  gram_plan(a, (n_cols + kGramColTile - 1) / kGramColTile, dev.n_sm);
   e = launch_gram_bf16(a, tmR, tmC, tmRa, tmCa, st);
   if (e == cudaSuccess) e = launch_gram_reduce(a, out, n_rows, st);
   return cuda_status(e);

@@ -8,17 +8,22 @@
 // bf16 values ("augmented row": -||k||^2/2 split exactly into three bf16 parts,
 // plus ones), and one extra K=16 MMA step adds both norm terms, so the fp32 TMEM
 // accumulator holds -||a - b||^2 / 2 for every pair.  The epilogue on CUDA cores is
-// then t = max(acc * (-2/h) + eps, eps) and phi(t); for the default s = 2 the
-// reciprocals of four pairs share one MUFU op:
-//     1/t0 + 1/t1 + 1/t2 + 1/t3 = ((t0+t1) t2 t3 + (t2+t3) t0 t1) / (t0 t1 t2 t3)
+// t = acc * (-2/h) + eps and phi(t).  For the default s = 2 four reciprocals share
+// one MUFU op,
+//     1/t0 + 1/t1 + 1/t2 + 1/t3 = ((t0+t1) t2 t3 + (t2+t3) t0 t1) / (t0 t1 t2 t3),
+// and the arithmetic runs two pairs per instruction (packed f32x2 FMA/MUL/ADD).
+// The clamp t >= eps is applied only when the largest key norm makes the fp32
+// rounding of x comparable to eps (a per-launch flag).
 //
-// Work = the sequence of (head, 256-row block, 128-column tile) steps, split evenly
+// Work = the sequence of (head, 256-row block, 256-column tile) steps, split evenly
 // over a persistent grid (one CTA per SM).  A CTA keeps its 256 rows (two 128-row
-// MMA tiles) in shared memory and streams column tiles through a 4-stage TMA ring.
-// Warp roles: 0 = TMA producer, 1 = MMA issuer, 2 = TMEM owner, 4..19 = epilogue
-// (2 row tiles x 4 TMEM lane quarters x 2 column halves; one thread per row and
-// half, so row sums need no cross-thread reduction).  TMEM holds 2 row tiles x 2
-// buffers x 128 fp32 columns = all 512 columns.
+// MMA tiles) in shared memory and streams 256-column tiles through a 2-stage TMA
+// ring.  Each row tile has one 128 x 256 fp32 accumulator in TMEM (N = 256 MMAs run
+// at full tensor rate); the two row tiles ping-pong: while the tensor core fills
+// one, the 8 epilogue warps of the other drain it.
+// Warp roles: 0 = TMA producer, 1 = MMA issuer, 2 = TMEM owner, 4..11 epilogue of
+// row tile 0, 12..19 of row tile 1 (4 TMEM lane quarters x 2 column halves; one
+// thread per row and half, so row sums need no cross-thread reduction).
 #include <climits>
 
 #include "gram.cuh"
@@ -31,19 +36,21 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kStages = 4;
+constexpr int kStages = 2;
+constexpr int kColTile = 256;   // columns per MMA (N) and per step
+constexpr int kEpiWarpsPerTile = 8;
+constexpr uint32_t kAugRowBytes = 32;  // 16 bf16 of the augmented row per operand row
 
 struct alignas(8) GramBars {
   uint64_t a_full, a_empty;
   uint64_t full[kStages], empty[kStages];
-  uint64_t acc_full[2], acc_empty[2];
+  uint64_t acc_full[2], acc_empty[2];   // per row tile
+  uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
 };
 constexpr int kBarBytes = 256;
 static_assert(sizeof(GramBars) <= kBarBytes, "barrier block overflows its reservation");
-constexpr uint32_t kAugTileBytes = kGramRowTile * 32;   // 128 rows x 16 bf16
-constexpr int kEpiWarps = 16;
 
 __device__ __forceinline__ int set_n(const GramSet& s, int h) { return s.n_dev ? s.n_dev[h] : s.n_uni; }
 __device__ __forceinline__ int set_off(const GramSet& s, int h) { return s.off_dev ? s.off_dev[h] : s.off_uni; }
@@ -58,7 +65,7 @@ struct Cursor {
 __device__ __forceinline__ void head_dims(const GramArgs& a, int h, int& RB, int& CT) {
   const int nR = set_n(a.rows, h), nC = set_n(a.cols, h);
   RB = nC > 0 ? (nR + kGramRowBlock - 1) / kGramRowBlock : 0;
-  CT = nR > 0 ? (nC + kGramColTile - 1) / kGramColTile : 0;
+  CT = nR > 0 ? (nC + kColTile - 1) / kColTile : 0;
 }
 
 __device__ __forceinline__ long long total_steps(const GramArgs& a) {
@@ -121,12 +128,40 @@ __device__ __forceinline__ int nact_of(const Cursor& c) {
   return (c.nR - c.rb * kGramRowBlock > kGramRowTile) ? 2 : 1;
 }
 
-// phi for one pair given t = x + eps (already clamped to >= eps)
+// phi for one pair given t = x + eps
 template <int SMODE>
 __device__ __forceinline__ float phi_t(float t, float nhs) {
   if constexpr (SMODE == 2) return rcp_approx(t);
   else if constexpr (SMODE == 1) return rsqrt_approx(t);
   else return ex2_approx(nhs * lg2_approx(t));
+}
+
+__device__ __forceinline__ float2 f2(uint32_t x, uint32_t y) { return make_float2(__uint_as_float(x), __uint_as_float(y)); }
+
+// Sum of phi over 32 accumulator columns (s = 2, packed f32x2, 8 MUFU ops):
+// t = acc * ks + eps; pairs (t_{2i}, t_{2i+1}) travel together, and each lane of a
+// float2 folds four reciprocals into one.
+template <bool CLAMP>
+__device__ __forceinline__ float2 sum_recip32(const uint32_t (&v)[32], float2 ks2, float2 eps2, float eps, float2 acc) {
+#pragma unroll
+  for (int k = 0; k < 32; k += 8) {
+    float2 A = __ffma2_rn(f2(v[k + 0], v[k + 1]), ks2, eps2);
+    float2 B = __ffma2_rn(f2(v[k + 2], v[k + 3]), ks2, eps2);
+    float2 C = __ffma2_rn(f2(v[k + 4], v[k + 5]), ks2, eps2);
+    float2 D = __ffma2_rn(f2(v[k + 6], v[k + 7]), ks2, eps2);
+    if constexpr (CLAMP) {
+      A = make_float2(fmaxf(A.x, eps), fmaxf(A.y, eps));
+      B = make_float2(fmaxf(B.x, eps), fmaxf(B.y, eps));
+      C = make_float2(fmaxf(C.x, eps), fmaxf(C.y, eps));
+      D = make_float2(fmaxf(D.x, eps), fmaxf(D.y, eps));
+    }
+    const float2 s = __fadd2_rn(A, B), p = __fmul2_rn(A, B);     // lane x: t0+t2, t0 t2; lane y: t1+t3, t1 t3
+    const float2 s2 = __fadd2_rn(C, D), p2 = __fmul2_rn(C, D);
+    const float2 num = __ffma2_rn(s, p2, __fmul2_rn(s2, p));      // (ta+tb) tc td + (tc+td) ta tb
+    const float2 den = __fmul2_rn(p, p2);
+    acc = __ffma2_rn(num, make_float2(rcp_approx(den.x), rcp_approx(den.y)), acc);
+  }
+  return acc;
 }
 
 template <int SMODE>
@@ -137,12 +172,14 @@ __global__ void __launch_bounds__(kGramThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nbox = a.d / 64;
-  const uint32_t tileBytes = static_cast<uint32_t>(kGramRowTile) * a.d * 2;
-  uint8_t* sA = smem;                                  // 2 row tiles
-  uint8_t* sB = sA + 2 * tileBytes;                    // kStages column tiles
-  uint8_t* sAa = sB + kStages * tileBytes;             // 2 augmented row tiles
-  uint8_t* sBa = sAa + 2 * kAugTileBytes;              // kStages augmented column tiles
-  GramBars* bars = reinterpret_cast<GramBars*>(sBa + kStages * kAugTileBytes);
+  const uint32_t aBytes = static_cast<uint32_t>(kGramRowTile) * a.d * 2;   // one 128-row tile
+  const uint32_t bBytes = static_cast<uint32_t>(kColTile) * a.d * 2;       // one 256-row column tile
+  const uint32_t aAug = kGramRowTile * kAugRowBytes, bAug = kColTile * kAugRowBytes;
+  uint8_t* sA = smem;                          // 2 row tiles
+  uint8_t* sB = sA + 2 * aBytes;               // kStages column tiles
+  uint8_t* sAa = sB + kStages * bBytes;        // 2 augmented row tiles
+  uint8_t* sBa = sAa + 2 * aAug;               // kStages augmented column tiles
+  GramBars* bars = reinterpret_cast<GramBars*>(sBa + kStages * bAug);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -154,10 +191,11 @@ __global__ void __launch_bounds__(kGramThreads, 1)
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->acc_full[b], 1);
-      mbar_init(&bars->acc_empty[b], kEpiWarps);
+    for (int r = 0; r < 2; ++r) {
+      mbar_init(&bars->acc_full[r], 1);
+      mbar_init(&bars->acc_empty[r], kEpiWarpsPerTile);
     }
+    mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     fence_barrier_init();
   }
@@ -191,20 +229,22 @@ __global__ void __launch_bounds__(kGramThreads, 1)
         if (L == L0 || c.j == 0) {
           if (aload > 0 && !(ok = mbar_wait(&bars->a_empty, (aload - 1) & 1, abort, a.status))) break;
           const int nact = nact_of(c);
-          mbar_arrive_expect_tx(&bars->a_full, nact * (tileBytes + kAugTileBytes));
+          mbar_arrive_expect_tx(&bars->a_full, nact * (aBytes + aAug));
           for (int r = 0; r < nact; ++r) {
             const int y = c.rOff + c.rb * kGramRowBlock + r * kGramRowTile;
-            for (int k = 0; k < nbox; ++k) tma_load_3d(sA + r * tileBytes + k * 16384, &tmR, &bars->a_full, k * 64, y, c.h);
-            tma_load_3d(sAa + r * kAugTileBytes, &tmRa, &bars->a_full, 0, y, c.h);  // row form
+            for (int k = 0; k < nbox; ++k)
+              tma_load_3d(sA + r * aBytes + k * (kGramRowTile * 128), &tmR, &bars->a_full, k * 64, y, c.h);
+            tma_load_3d(sAa + r * aAug, &tmRa, &bars->a_full, 0, y, c.h);  // row form
           }
           ++aload;
         }
         const int s = it % kStages;
         if (!(ok = mbar_wait(&bars->empty[s], ((it / kStages) & 1) ^ 1, abort, a.status))) break;
-        mbar_arrive_expect_tx(&bars->full[s], tileBytes + kAugTileBytes);
-        const int y = c.cOff + c.j * kGramColTile;
-        for (int k = 0; k < nbox; ++k) tma_load_3d(sB + s * tileBytes + k * 16384, &tmC, &bars->full[s], k * 64, y, c.h);
-        tma_load_3d(sBa + s * kAugTileBytes, &tmCa, &bars->full[s], 16, y, c.h);  // column form
+        mbar_arrive_expect_tx(&bars->full[s], bBytes + bAug);
+        const int y = c.cOff + c.j * kColTile;
+        for (int k = 0; k < nbox; ++k)
+          tma_load_3d(sB + s * bBytes + k * (kColTile * 128), &tmC, &bars->full[s], k * 64, y, c.h);
+        tma_load_3d(sBa + s * bAug, &tmCa, &bars->full[s], 16, y, c.h);  // column form
         ++it;
       }
       if (!ok) {
@@ -217,14 +257,15 @@ __global__ void __launch_bounds__(kGramThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, kGramColTile, 0, 0);
+      const uint32_t idesc = idesc_bf16_f32(128, kColTile, 0, 0);
       const uint32_t aBase = smem_u32(sA), bBase = smem_u32(sB);
       const uint32_t aaBase = smem_u32(sAa), baBase = smem_u32(sBa);
-      int it = 0, t = 0, aload = 0;
+      int it = 0, aload = 0;
+      int tr[2] = {0, 0};  // tiles issued into each row tile's accumulator
       bool ok = true;
       Cursor c;
       if (L0 < L1) cursor_seek(a, L0, c);
-      for (long long L = L0; L < L1; ++L) {
+      for (long long L = L0; L < L1 && ok; ++L) {
         const int nact = nact_of(c);
         if (L == L0 || c.j == 0) {
           if (!(ok = mbar_wait(&bars->a_full, aload & 1, abort, a.status))) break;
@@ -232,45 +273,49 @@ __global__ void __launch_bounds__(kGramThreads, 1)
           ++aload;
         }
         const int s = it % kStages;
-        const int b = t & 1;
         if (!(ok = mbar_wait(&bars->full[s], (it / kStages) & 1, abort, a.status))) break;
-        if (!(ok = mbar_wait(&bars->acc_empty[b], ((t >> 1) & 1) ^ 1, abort, a.status))) break;
-        tc_fence_after();
-        for (int r = 0; r < nact; ++r) {
-          const uint32_t dcol = tmem + static_cast<uint32_t>((r * 2 + b) * kGramColTile);
+        for (int r = 0; r < nact && ok; ++r) {
+          // the row tile's accumulator is free once its 8 epilogue warps hold it in registers
+          if (!(ok = mbar_wait(&bars->acc_empty[r], (tr[r] & 1) ^ 1, abort, a.status))) break;
+          tc_fence_after();
+          const uint32_t dcol = tmem + static_cast<uint32_t>(r * kColTile);
           for (int kk = 0; kk < a.d / 16; ++kk) {
-            const uint32_t koff = static_cast<uint32_t>((kk >> 2) * 16384 + (kk & 3) * 32);
-            const uint64_t ad = sdesc_sw128(aBase + r * tileBytes + koff, 16, 1024);
-            const uint64_t bd = sdesc_sw128(bBase + s * tileBytes + koff, 16, 1024);
-            mma_f16_ss(dcol, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            const uint32_t ka = static_cast<uint32_t>((kk >> 2) * (kGramRowTile * 128) + (kk & 3) * 32);
+            const uint32_t kb = static_cast<uint32_t>((kk >> 2) * (kColTile * 128) + (kk & 3) * 32);
+            mma_f16_ss(dcol, sdesc_sw128(aBase + r * aBytes + ka, 16, 1024), sdesc_sw128(bBase + s * bBytes + kb, 16, 1024),
+                       idesc, kk > 0 ? 1u : 0u);
           }
           // the norm terms: one more K=16 step over the augmented rows
-          mma_f16_ss(dcol, sdesc_sw32(aaBase + r * kAugTileBytes, 256), sdesc_sw32(baBase + s * kAugTileBytes, 256),
-                     idesc, 1u);
+          mma_f16_ss(dcol, sdesc_sw32(aaBase + r * aAug, 256), sdesc_sw32(baBase + s * bAug, 256), idesc, 1u);
+          mma_commit(&bars->acc_full[r]);
+          ++tr[r];
         }
+        if (!ok) break;
         mma_commit(&bars->empty[s]);
-        mma_commit(&bars->acc_full[b]);
         ++it;
-        ++t;
         const bool last_of_block = (L + 1 == L1) || (c.j + 1 == c.CT);
         if (last_of_block) mma_commit(&bars->a_empty);
         cursor_next(a, c);
       }
-      if (!ok && t > 0) {
-        // abort path: make sure no MMA still writes TMEM when it is freed
-        mma_commit(&bars->a_empty);
-        mbar_wait_drain(&bars->acc_full[(t - 1) & 1], ((t - 1) >> 1) & 1, 200000000ull);
+      if (!ok && (tr[0] + tr[1]) > 0) {
+        // abort path: no MMA may still write TMEM when it is freed (the commit
+        // arrives once every MMA issued by this thread has completed)
+        mma_commit(&bars->mma_done);
+        mbar_wait_drain(&bars->mma_done, 0, 200000000ull);
       }
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
     const int e = warp - 4;
-    const int q = warp & 3;        // TMEM lane quarter (warp_id % 4)
-    const int r = (e >> 2) & 1;    // row tile
-    const int hf = e >> 3;         // column half of every 128-column tile
+    const int r = e >> 3;            // row tile
+    const int q = warp & 3;          // TMEM lane quarter (warp_id % 4)
+    const int hf = (e >> 2) & 1;     // column half of the 256-column tile
     const int row_in_tile = q * 32 + lane;
     const float ks = a.kscale, eps = a.eps, nhs = -0.5f * a.s;
-    int t = 0;
+    const float2 ks2 = make_float2(ks, ks), eps2 = make_float2(eps, eps);
+    // clamp t >= eps only when fp32 rounding of x could reach eps / 2 (see header)
+    const bool clamp = a.norm_max ? (*a.norm_max) * 1e-4f >= eps * (-2.f / ks) : true;
+    int t = 0;                       // tiles seen by this row tile (phase of its barriers)
     bool ok = true;
     Cursor c;
     if (L0 < L1) cursor_seek(a, L0, c);
@@ -290,45 +335,25 @@ __global__ void __launch_bounds__(kGramThreads, 1)
         acc_pos = 0.f;
         acc_neg = 0.f;
       }
-      const int b = t & 1;
-      const int c0 = c.j * kGramColTile + hf * 64;  // first column of this thread's half
-      if (!(ok = mbar_wait(&bars->acc_full[b], (t >> 1) & 1, abort, a.status))) break;
-      tc_fence_after();
-      bool released = false;
       if (active) {
-        const bool tail = c0 + 64 > c.nC;
-        const bool allneg = c0 + 64 <= nneg;
+        if (!(ok = mbar_wait(&bars->acc_full[r], t & 1, abort, a.status))) break;
+        tc_fence_after();
+        const int c0 = c.j * kColTile + hf * 128;  // first column of this thread's half
+        const bool tail = c0 + 128 > c.nC;
+        const bool allneg = c0 + 128 <= nneg;
         const bool mixed = (c0 < nneg) && !allneg;
-        // diagonal columns of this row tile: [rt0 + diag, rt0 + diag + 128)
-        const bool diag_hit = a.use_diag && (rt0 + diag < c0 + 64) && (rt0 + diag + kGramRowTile > c0);
+        const bool diag_hit = a.use_diag && (rt0 + diag < c0 + 128) && (rt0 + diag + kGramRowTile > c0);
         const bool masked = tail || mixed || diag_hit;
-        const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) +
-                               static_cast<uint32_t>((r * 2 + b) * kGramColTile + hf * 64);
-        float acc0 = 0.f, acc1 = 0.f;
+        const uint32_t taddr =
+            tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(r * kColTile + hf * 128);
+        float2 acc2 = make_float2(0.f, 0.f);
+        float accs = 0.f;
         auto fast = [&](const uint32_t (&v)[32]) {
           if constexpr (SMODE == 2) {
-#pragma unroll
-            for (int k = 0; k < 32; k += 8) {
-              const float t0 = fmaxf(fmaf(__uint_as_float(v[k + 0]), ks, eps), eps);
-              const float t1 = fmaxf(fmaf(__uint_as_float(v[k + 1]), ks, eps), eps);
-              const float t2 = fmaxf(fmaf(__uint_as_float(v[k + 2]), ks, eps), eps);
-              const float t3 = fmaxf(fmaf(__uint_as_float(v[k + 3]), ks, eps), eps);
-              const float t4 = fmaxf(fmaf(__uint_as_float(v[k + 4]), ks, eps), eps);
-              const float t5 = fmaxf(fmaf(__uint_as_float(v[k + 5]), ks, eps), eps);
-              const float t6 = fmaxf(fmaf(__uint_as_float(v[k + 6]), ks, eps), eps);
-              const float t7 = fmaxf(fmaf(__uint_as_float(v[k + 7]), ks, eps), eps);
-              const float p01 = t0 * t1, p23 = t2 * t3, p45 = t4 * t5, p67 = t6 * t7;
-              const float na = fmaf(t2 + t3, p01, (t0 + t1) * p23);
-              const float nb2 = fmaf(t6 + t7, p45, (t4 + t5) * p67);
-              acc0 = fmaf(na, rcp_approx(p01 * p23), acc0);
-              acc1 = fmaf(nb2, rcp_approx(p45 * p67), acc1);
-            }
+            acc2 = clamp ? sum_recip32<true>(v, ks2, eps2, eps, acc2) : sum_recip32<false>(v, ks2, eps2, eps, acc2);
           } else {
 #pragma unroll
-            for (int k = 0; k < 32; k += 2) {
-              acc0 += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 0]), ks, eps), eps), nhs);
-              acc1 += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k + 1]), ks, eps), eps), nhs);
-            }
+            for (int k = 0; k < 32; ++k) accs += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k]), ks, eps), eps), nhs);
           }
         };
         auto slow = [&](const uint32_t (&v)[32], int cc) {
@@ -342,32 +367,35 @@ __global__ void __launch_bounds__(kGramThreads, 1)
             else acc_pos += ph;
           }
         };
-        // chunk 1 is in flight while chunk 0 is processed
+        auto process = [&](const uint32_t (&v)[32], int cc) {
+          if (masked) slow(v, cc);
+          else fast(v);
+        };
+        // 4 chunks of 32 columns; chunk c+1 is in flight while chunk c is processed
         uint32_t va[32], vb[32];
         tmem_ld32(taddr + 0, va);
         tmem_wait_ld_reg(va);
         tmem_ld32(taddr + 32, vb);
-        if (masked) slow(va, 0);
-        else fast(va);
+        process(va, 0);
         tmem_wait_ld_reg(vb);
-        // every column this warp needs is in registers: hand the buffer back
+        tmem_ld32(taddr + 64, va);
+        process(vb, 1);
+        tmem_wait_ld_reg(va);
+        tmem_ld32(taddr + 96, vb);
+        process(va, 2);
+        tmem_wait_ld_reg(vb);
+        // every column this warp needs is in registers: hand the accumulator back
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->acc_empty[b]);
-        released = true;
-        if (masked) slow(vb, 1);
-        else fast(vb);
+        if (lane == 0) mbar_arrive(&bars->acc_empty[r]);
+        process(vb, 3);
         if (!masked) {
-          if (allneg) acc_neg += acc0 + acc1;
-          else acc_pos += acc0 + acc1;
+          const float tile = acc2.x + acc2.y + accs;
+          if (allneg) acc_neg += tile;
+          else acc_pos += tile;
         }
+        ++t;
       }
-      if (!released) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->acc_empty[b]);
-      }
-      ++t;
       const bool last_of_block = (L + 1 == L1) || (c.j + 1 == c.CT);
       if (last_of_block && valid_row) {
         const int slot = 2 * (cta - cta_of(Lblock, T, G)) + hf;
@@ -466,8 +494,9 @@ __global__ void gram_reduce_kernel(const GramArgs a, float* out, int ldOut) {
 }  // namespace
 
 size_t gram_smem_bytes(int d) {
-  const size_t tile = static_cast<size_t>(kGramRowTile) * d * 2;
-  return 1024 + (2 + kStages) * (tile + kAugTileBytes) + kBarBytes;
+  const size_t a = static_cast<size_t>(kGramRowTile) * (d * 2 + kAugRowBytes);
+  const size_t b = static_cast<size_t>(kColTile) * (d * 2 + kAugRowBytes);
+  return 1024 + 2 * a + kStages * b + kBarBytes;
 }
 
 void gram_plan(GramArgs& a, int max_col_tiles, int n_sm) {

@@ -10,7 +10,7 @@ namespace kvb {
 
 constexpr int kGramRowTile = 128;      // rows per TMEM accumulator (M of the MMA)
 constexpr int kGramRowBlock = 256;     // rows per work unit (two accumulators)
-constexpr int kGramColTile = 128;      // columns per MMA (N)
+constexpr int kGramColTile = 256;      // columns per MMA (N) and per work step
 constexpr int kGramThreads = 640;      // 4 control warps + 16 epilogue warps
 
 // A set of rows/cols: per head a count and a start row inside its buffer.  Each
@@ -42,15 +42,18 @@ struct GramArgs {
   float* partial = nullptr;        // [slots][H][ldOut]
   int ldOut = 0;
   int* status = nullptr;
+  // largest ||k||^2 among the rows and columns (null: unknown, always clamp t >= eps)
+  const float* norm_max = nullptr;
   // f32 SIMT path only
   const float* R32 = nullptr;      // [H][ldR][d]
   const float* C32 = nullptr;      // [H][ldC][d]
   int ldR = 0, ldC = 0;
 };
 
-// bf16 operands through TMA: tensor maps over [H][rows][d] (64x128 boxes) and over
-// the augmented rows [H][rows][32] (16x128 boxes, see launch_aug_rows): the MMA
-// accumulates a.b - (||a||^2 + ||b||^2)/2 = -||a - b||^2 / 2 directly.
+// bf16 operands through TMA: tensor maps over [H][rows][d] and over the augmented
+// rows [H][rows][32] (see launch_aug_rows); row maps use 128-row boxes, column maps
+// 256-row boxes (kGramColTile).  The MMA accumulates a.b - (||a||^2 + ||b||^2)/2 =
+// -||a - b||^2 / 2 directly.
 cudaError_t launch_gram_bf16(const GramArgs& a, const CUtensorMap& tmR, const CUtensorMap& tmC,
                              const CUtensorMap& tmRa, const CUtensorMap& tmCa, cudaStream_t st);
 // f32 operands, CUDA-core direct differences (small problems).

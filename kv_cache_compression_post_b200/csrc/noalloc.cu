@@ -93,17 +93,21 @@ extern "C" kvb_status kvb_density_noalloc(const void* rows, int32_t n_rows, cons
   // the status word is the only piece that must start at zero on every call (the
   // augmented rows and the partials are written in full before they are read)
   if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return KVB_E_CUDA;
+  // the largest key norm of this call (decides whether t >= eps must be clamped)
+  float* norm_max = reinterpret_cast<float*>(base + L.status + 4);
+  if (cudaMemsetAsync(norm_max, 0, sizeof(float), st) != cudaSuccess) return KVB_E_CUDA;
   if (n_cols == 0) return cuda_status(cudaMemsetAsync(out, 0, sizeof(float) * heads * n_rows, st));
 
   const float h = dist_scale > 0.f ? dist_scale : static_cast<float>(head_dim);
-  cudaError_t e = launch_aug_rows(rows, dtype, heads, n_rows, head_dim, n_rows, nullptr, n_rows, rowAug, n_rows, st);
+  cudaError_t e =
+      launch_aug_rows(rows, dtype, heads, n_rows, head_dim, n_rows, nullptr, n_rows, rowAug, n_rows, norm_max, st);
   if (e == cudaSuccess)
-    e = launch_aug_rows(cols, dtype, heads, n_cols, head_dim, n_cols, nullptr, n_cols, colAug, n_cols, st);
+    e = launch_aug_rows(cols, dtype, heads, n_cols, head_dim, n_cols, nullptr, n_cols, colAug, n_cols, norm_max, st);
   if (e != cudaSuccess) return KVB_E_CUDA;
   CUtensorMap tmR, tmC, tmRa, tmCa;
   if (!make_tmap_bf16(&tmR, rows, head_dim, n_rows, heads, 128) ||
-      !make_tmap_bf16(&tmC, cols, head_dim, n_cols, heads, 128) || !make_tmap_aug(&tmRa, rowAug, n_rows, heads, 128) ||
-      !make_tmap_aug(&tmCa, colAug, n_cols, heads, 128))
+      !make_tmap_bf16(&tmC, cols, head_dim, n_cols, heads, kGramColTile) || !make_tmap_aug(&tmRa, rowAug, n_rows, heads, 128) ||
+      !make_tmap_aug(&tmCa, colAug, n_cols, heads, kGramColTile))
     return KVB_E_INVAL;
   GramArgs a;
   a.H = heads;
@@ -117,9 +121,10 @@ extern "C" kvb_status kvb_density_noalloc(const void* rows, int32_t n_rows, cons
   a.s = s;
   a.max_rows = n_rows;
   a.status = status;
+  a.norm_max = norm_max;
   a.partial = reinterpret_cast<float*>(base + L.partial);
   a.ldOut = n_rows;
-  gram_plan(a, (n_cols + 127) / 128, dev.n_sm);
+  gram_plan(a, (n_cols + kGramColTile - 1) / kGramColTile, dev.n_sm);
   e = launch_gram_bf16(a, tmR, tmC, tmRa, tmCa, st);
   if (e == cudaSuccess) e = launch_gram_reduce(a, out, n_rows, st);
   return cuda_status(e);

@@ -27,7 +27,7 @@ __global__ void row_terms_kernel(const T* __restrict__ X, long long ldX, int d, 
 
 template <typename T>
 __global__ void aug_rows_kernel(const T* __restrict__ X, long long ldX, int d, int n_uni, const int* n_dev,
-                                uint16_t* __restrict__ out, long long ldOut) {
+                                uint16_t* __restrict__ out, long long ldOut, float* norm_max) {
   const int h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * (blockDim.x >> 5) + warp;
@@ -40,6 +40,7 @@ __global__ void aug_rows_kernel(const T* __restrict__ X, long long ldX, int d, i
     acc = fmaf(v, v, acc);
   }
   acc = warp_sum(acc);
+  if (norm_max && lane == 0) atomicMax(reinterpret_cast<int*>(norm_max), __float_as_int(acc));
   const float nrm = -0.5f * acc;
   const __nv_bfloat16 hi = __float2bfloat16_rn(nrm);
   const __nv_bfloat16 mid = __float2bfloat16_rn(nrm - __bfloat162float(hi));
@@ -56,14 +57,15 @@ __global__ void aug_rows_kernel(const T* __restrict__ X, long long ldX, int d, i
 }  // namespace
 
 cudaError_t launch_aug_rows(const void* X, kvb_dtype dtype, int H, long long ldX, int d, int n_uni, const int* n_dev,
-                            int max_n, uint16_t* out, long long ldOut, cudaStream_t st) {
+                            int max_n, uint16_t* out, long long ldOut, float* norm_max, cudaStream_t st) {
   if (max_n <= 0 || H <= 0) return cudaSuccess;
   dim3 grid((max_n + 7) / 8, H);
   note_launch();
   if (dtype == KVB_BF16)
-    aug_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), ldX, d, n_uni, n_dev, out, ldOut);
+    aug_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), ldX, d, n_uni, n_dev, out, ldOut,
+                                          norm_max);
   else
-    aug_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const float*>(X), ldX, d, n_uni, n_dev, out, ldOut);
+    aug_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const float*>(X), ldX, d, n_uni, n_dev, out, ldOut, norm_max);
   return cudaGetLastError();
 }
 
