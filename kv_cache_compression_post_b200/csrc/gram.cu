@@ -138,13 +138,13 @@ __device__ __forceinline__ float phi_t(float t, float nhs) {
 
 __device__ __forceinline__ float2 f2(uint32_t x, uint32_t y) { return make_float2(__uint_as_float(x), __uint_as_float(y)); }
 
-// Sum of phi over 32 accumulator columns (s = 2, packed f32x2, 8 MUFU ops):
+// Sum of phi over 16 accumulator columns (s = 2, packed f32x2, 4 MUFU ops):
 // t = acc * ks + eps; pairs (t_{2i}, t_{2i+1}) travel together, and each lane of a
 // float2 folds four reciprocals into one.
 template <bool CLAMP>
-__device__ __forceinline__ float2 sum_recip32(const uint32_t (&v)[32], float2 ks2, float2 eps2, float eps, float2 acc) {
+__device__ __forceinline__ float2 sum_recip16(const uint32_t (&v)[16], float2 ks2, float2 eps2, float eps, float2 acc) {
 #pragma unroll
-  for (int k = 0; k < 32; k += 8) {
+  for (int k = 0; k < 16; k += 8) {
     float2 A = __ffma2_rn(f2(v[k + 0], v[k + 1]), ks2, eps2);
     float2 B = __ffma2_rn(f2(v[k + 2], v[k + 3]), ks2, eps2);
     float2 C = __ffma2_rn(f2(v[k + 4], v[k + 5]), ks2, eps2);
@@ -348,51 +348,49 @@ __global__ void __launch_bounds__(kGramThreads, 1)
             tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(r * kColTile + hf * 128);
         float2 acc2 = make_float2(0.f, 0.f);
         float accs = 0.f;
-        auto fast = [&](const uint32_t (&v)[32]) {
-          if constexpr (SMODE == 2) {
-            acc2 = clamp ? sum_recip32<true>(v, ks2, eps2, eps, acc2) : sum_recip32<false>(v, ks2, eps2, eps, acc2);
+        // masked tiles (ragged end, self pair, sign change) take an exact scalar path
+        auto chunk = [&](const uint32_t (&v)[16], int cc) {
+          const int cb = c0 + cc * 16;
+          if (SMODE == 2 && !masked) {
+            acc2 = clamp ? sum_recip16<true>(v, ks2, eps2, eps, acc2) : sum_recip16<false>(v, ks2, eps2, eps, acc2);
           } else {
 #pragma unroll
-            for (int k = 0; k < 32; ++k) accs += phi_t<SMODE>(fmaxf(fmaf(__uint_as_float(v[k]), ks, eps), eps), nhs);
+            for (int k = 0; k < 16; ++k) {
+              const int col = cb + k;
+              const float tv = fmaxf(fmaf(__uint_as_float(v[k]), ks, eps), eps);
+              const bool valid = (col < c.nC) && (col != row + diag);
+              const float ph = valid ? phi_t<SMODE>(tv, nhs) : 0.f;
+              if (masked && col < nneg) acc_neg += ph;
+              else accs += ph;
+            }
           }
         };
-        auto slow = [&](const uint32_t (&v)[32], int cc) {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const int col = c0 + cc * 32 + k;
-            const float tv = fmaxf(fmaf(__uint_as_float(v[k]), ks, eps), eps);
-            const bool valid = (col < c.nC) && (col != row + diag);
-            const float ph = valid ? phi_t<SMODE>(tv, nhs) : 0.f;
-            if (col < nneg) acc_neg += ph;
-            else acc_pos += ph;
+        // 8 chunks of 16 columns; chunk c+1 is in flight while chunk c is processed
+        uint32_t va[16], vb[16];
+        tmem_ld16(taddr + 0, va);
+        tmem_wait_ld_reg16(va);
+#pragma unroll 1
+        for (int cc = 0; cc < 8; cc += 2) {
+          tmem_ld16(taddr + (cc + 1) * 16, vb);
+          chunk(va, cc);
+          tmem_wait_ld_reg16(vb);
+          if (cc + 2 < 8) {
+            tmem_ld16(taddr + (cc + 2) * 16, va);
+          } else {
+            // every column this warp needs is in registers: hand the accumulator back
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->acc_empty[r]);
           }
-        };
-        auto process = [&](const uint32_t (&v)[32], int cc) {
-          if (masked) slow(v, cc);
-          else fast(v);
-        };
-        // 4 chunks of 32 columns; chunk c+1 is in flight while chunk c is processed
-        uint32_t va[32], vb[32];
-        tmem_ld32(taddr + 0, va);
-        tmem_wait_ld_reg(va);
-        tmem_ld32(taddr + 32, vb);
-        process(va, 0);
-        tmem_wait_ld_reg(vb);
-        tmem_ld32(taddr + 64, va);
-        process(vb, 1);
-        tmem_wait_ld_reg(va);
-        tmem_ld32(taddr + 96, vb);
-        process(va, 2);
-        tmem_wait_ld_reg(vb);
-        // every column this warp needs is in registers: hand the accumulator back
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->acc_empty[r]);
-        process(vb, 3);
+          chunk(vb, cc + 1);
+          if (cc + 2 < 8) tmem_wait_ld_reg16(va);
+        }
         if (!masked) {
           const float tile = acc2.x + acc2.y + accs;
           if (allneg) acc_neg += tile;
           else acc_pos += tile;
+        } else {
+          acc_pos += accs;
         }
         ++t;
       }
