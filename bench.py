@@ -177,29 +177,44 @@ def host_step(x, dt):
 
 
 def _cfg(w, kvb):
-    return kvb.make_config(method=kvb.KVB_DENSITYKV, dtype=kvb.KVB_BF16 if w.dtype == "bf16" else kvb.KVB_F32,
-                           layers=1, heads=w.heads, head_dim=w.head_dim, capacity=w.capacity,
-                           max_candidates=w.chunk_tokens, tau=w.tau, eps=w.eps, s=w.s, sync_heads=1,
-                           max_queries=w.chunk_tokens)
+    dt = kvb.KVB_BF16 if w.dtype == "bf16" else kvb.KVB_F32
+    if w.forcing:
+        return kvb.make_config(method=kvb.KVB_FORCINGKV, dtype=dt, layers=1, heads=w.heads, head_dim=w.head_dim,
+                               frame_h=w.frame_h, frame_w=w.frame_w, seg_h=w.seg_h, seg_w=w.seg_w,
+                               hist_frames=w.hist_frames, max_new_frames=w.chunk_frames, retention=w.retention,
+                               max_queries=w.chunk_tokens)
+    return kvb.make_config(method=kvb.KVB_DENSITYKV, dtype=dt, layers=1, heads=w.heads, head_dim=w.head_dim,
+                           capacity=w.capacity, max_candidates=w.chunk_tokens, tau=w.tau, eps=w.eps, s=w.s,
+                           sync_heads=1, max_queries=w.chunk_tokens)
 
 
-FIRST_TIMED = {"wan480": 19, "wan1080": 9, "mid": 4, "tiny": 4}
+# first timed chunk: steady state (DensityKV bank full; Forcing-KV ring of 21 frames full)
+FIRST_TIMED = {"wan480": 19, "wan1080": 9, "mid": 4, "tiny": 4, "forcing480": 8, "forcing_mid": 4}
 
 
 def attention_flops(w, sizes):
-    """4 * Nq * Lk * d summed over heads (Lk = sink + bank_h + window)."""
+    """4 * Nq * Lk * d summed over heads (Lk = sink + history_h + window)."""
     Nq = w.chunk_tokens
     return sum(4.0 * Nq * (w.F + s + w.chunk_tokens) * w.head_dim for s in sizes)
 
 
-def density_flops(w, N, st_before, st_after):
-    """Executed density work of one admit: 2d flops per pair over the four passes
-    (candidates x bank, bank x admitted, new bank x evicted, admitted x admitted)."""
-    f = 0.0
+def gram_pairs(N, st_before, st_after):
+    """Pairs of the four density passes of one admit, per pass (summed over heads):
+    candidates x bank, bank x admitted, new bank x evicted, admitted x admitted."""
+    out = [0.0, 0.0, 0.0, 0.0]
     for b0, s in zip(st_before, st_after):
         P, E = s["admitted"], s["mandatory"] + s["capacity_evicted"]
-        f += 2.0 * w.head_dim * (N * b0 + b0 * P + s["size"] * E + P * P)
-    return f
+        out[0] += N * b0
+        out[1] += b0 * P
+        out[2] += s["size"] * E
+        out[3] += P * P
+    return out
+
+
+def density_flops(w, N, st_before, st_after):
+    """Density work of one admit: 2d flops per pair over the four passes (the
+    projected-growth pass included)."""
+    return 2.0 * w.head_dim * sum(gram_pairs(N, st_before, st_after))
 
 
 def density_flops_algorithmic(w, N, st_before, st_after):
@@ -211,33 +226,114 @@ def density_flops_algorithmic(w, N, st_before, st_after):
     return f
 
 
-def run_densitykv(args, w, rank, world):
+def kernel_units(w, name, N, st_before, st_after, n_frames, labels):
+    """Algorithmic work of one step's launches of `name`: (bound, units, per-unit text)."""
+    row = w.head_dim * (2 if w.dtype == "bf16" else 4)
+    H = w.heads
+    if w.forcing:
+        dyn = [h for h in range(H) if not labels[h]]
+        sta = [h for h in range(H) if labels[h]]
+        if name == "attend_bf16_kernel":
+            return "tensor", attention_flops(w, [s["size"] for s in st_after]), "4*Nq*(Ls+hist_h+Lw)*d flops"
+        if name == "seg_cosine_kernel":
+            return "hbm", len(dyn) * ((n_frames + 1) * w.F * row + n_frames * 4 * w.n_segments), \
+                "dynamic heads x (n_frames+1 frames of K read + segment means written)"
+        if name == "prune_gather_kernel":
+            kept = sum(st_after[h]["admitted"] for h in dyn)
+            return "hbm", kept * (4 * row + 8), "kept tokens x (K,V read+write + id read+write)"
+        if name == "static_copy_kernel":
+            return "hbm", len(sta) * w.F * (4 * row + 8), "static heads x F x (K,V read+write + id)"
+        return "latency", None, "per-head bookkeeping (one CTA per head)"
+    pairs = gram_pairs(N, st_before, st_after)
+    P = sum(s["admitted"] for s in st_after)
+    E = sum(s["mandatory"] + s["capacity_evicted"] for s in st_after)
+    moved = sum(s.get("moved", 0) for s in st_after)
+    size = sum(s["size"] for s in st_after)
+    if name == "gram_bf16_kernel":
+        return "tensor", 2.0 * w.head_dim * sum(pairs), "2*d flops per pair over the four density passes"
+    if name == "attend_bf16_kernel":
+        return "tensor", attention_flops(w, [s["size"] for s in st_after]), "4*Nq*(Ls+|B_h|+Lw)*d flops"
+    if name == "aug_rows_kernel":
+        return "hbm", H * N * (row + 64), "candidates x (K row read + 64 B augmented row written)"
+    if name == "gather_admitted_kernel":
+        return "hbm", P * (2 * row + 128 + 4), "admitted x (K row + aug row, read+write)"
+    if name == "gather_evicted_kernel":
+        return "hbm", E * (2 * row + 128 + 4), "evicted x (K row + aug row, read+write)"
+    if name == "compact_kernel":
+        return "hbm", (P + moved) * (4 * row + 128 + 24), "(admitted + moved) x (K,V,aug rows read+write + ids/rho)"
+    if name == "finalize_kernel":
+        return "hbm", size * 24, "bank entries x (rho, sub, tag, growth in; rho, rho0 out)"
+    if name == "gram_reduce_kernel":
+        return "latency", None, "partial-sum reduction of the density passes"
+    return "latency", None, "selection (one CTA per head)"
+
+
+def kernel_table(w, records, steps, per_step_units, peaks):
+    """Per-kernel live timing (library launch trace, CUDA events on the launch
+    stream) against its roofline."""
+    agg = {}
+    for n, ms in records:
+        a = agg.setdefault(n, [0, 0.0])
+        a[0] += 1
+        a[1] += ms
+    total = sum(a[1] for a in agg.values())
+    out = []
+    for n, (cnt, ms) in sorted(agg.items(), key=lambda kv: -kv[1][1]):
+        bound, units, text = per_step_units.get(n, ("latency", None, ""))
+        e = {"kernel": n, "launches_per_step": round(cnt / steps, 2), "ms_per_step": round(ms / steps, 4),
+             "ms_per_launch": round(ms / cnt, 4), "share": round(ms / total, 4), "bound": bound, "algorithmic": text}
+        if units is not None and ms > 0:
+            if bound == "tensor":
+                ach = units / (ms / steps * 1e-3) / 1e12
+                e.update(achieved=round(ach, 2), unit="TFLOP/s", peak=peaks["bf16_tflops"],
+                         frac=round(ach / peaks["bf16_tflops"], 4))
+            else:
+                ach = units / (ms / steps * 1e-3) / 1e9
+                e.update(achieved=round(ach, 1), unit="GB/s", peak=peaks["hbm_gbs"],
+                         frac=round(ach / peaks["hbm_gbs"], 4), bytes_per_step=int(units))
+        out.append(e)
+    return out
+
+
+def run_workload(args, w, rank, world):
     import torch
     import kv_cache_compression_post_b200 as kvb
     dev = torch.cuda.current_device()
     first = FIRST_TIMED.get(w.name, 4)
-    n_dev_steps = args.warmup + args.steps
-    total_steps = first - 1 + n_dev_steps + args.steps  # pre-roll, device-timed, end-to-end
+    n_trace = min(3, args.steps)   # launch-traced steps after the timed ones (per-kernel times)
+    n_dev_steps = args.warmup + args.steps + n_trace
+    total_steps = first - 1 + n_dev_steps + args.steps  # pre-roll, device-timed, traced, end-to-end
     t0 = time.time()
     L = kvgen.LayerInputs(w, 0, n_chunks=total_steps + 2, seed_offset=rank)
     inputs = {}
     for i in range(1, first + n_dev_steps):
-        inputs[i] = upload_step(L.step(i), w.dtype)
-    hosted = {i: host_step(L.step(i), w.dtype) for i in range(first + n_dev_steps, total_steps + 1)}
+        inputs[i] = upload_step(L.step(i, forcing=w.forcing), w.dtype)
+    hosted = {i: host_step(L.step(i, forcing=w.forcing), w.dtype)
+              for i in range(first + n_dev_steps, total_steps + 1)}
     gen_s = time.time() - t0
 
     bank = kvb.Bank(_cfg(w, kvb))
+    labels = kvgen.head_labels(w, 0) if w.forcing else None
     stream = torch.cuda.current_stream()
     O = torch.empty_like(inputs[1]["Q"])
     lse = torch.empty(w.heads, w.chunk_tokens, device="cuda")
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
 
+    def update(x):
+        if w.forcing:
+            nf = x["new_ids"].shape[0] // w.F
+            bank.prune_hybrid(0, labels, x["newK"], x["newV"], x["nextK"], x["new_ids"], nf, stream)
+        else:
+            bank.admit(0, x["candK"], x["candV"], x["cand_ids"], stream)
+
     def step(x):
-        bank.admit(0, x["candK"], x["candV"], x["cand_ids"], stream)
+        update(x)
         bank.attend(0, x["Q"], x["sinkK"], x["sinkV"], x["winK"], x["winV"], O, lse, stream)
 
-    # pre-roll to steady state, then warm-up
-    for i in range(1, first + args.warmup):
+    # pre-roll to steady state (the history update alone), then warm-up
+    for i in range(1, first):
+        update(inputs[i])
+    for i in range(first, first + args.warmup):
         step(inputs[i])
     torch.cuda.synchronize()
     if bank.status() != 0:
@@ -247,30 +343,51 @@ def run_densitykv(args, w, rank, world):
     barrier(world)
     torch.cuda.synchronize()
     sampler.start()
-    per_step, adm_ms, att_ms, att_fl, den_fl, den_alg = [], [], [], [], [], []
+    per_step, upd_ms, att_ms, att_fl, den_fl, den_alg = [], [], [], [], [], []
+    units = {}
     launches0 = kvb.kvb_launch_count()
+    timed_end = first + args.warmup + args.steps
+    launches = None
     for i in range(first + args.warmup, first + n_dev_steps):
+        if i == timed_end:
+            # the timed steps are done; the next few steps run with the library's launch
+            # trace on (an event pair around every launch) for the per-kernel table
+            launches = kvb.kvb_launch_count() - launches0
+            clocks = sampler.stop()
+            kvb.kvb_trace_enable(True)
         x = inputs[i]
         flush.fill_(1.0)
         st_before = [s["size"] for s in bank.stats(0)]
         e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
         torch.cuda.synchronize()
         e0.record(stream)
-        bank.admit(0, x["candK"], x["candV"], x["cand_ids"], stream)
+        update(x)
         e1.record(stream)
         bank.attend(0, x["Q"], x["sinkK"], x["sinkV"], x["winK"], x["winV"], O, lse, stream)
         e2.record(stream)
         torch.cuda.synchronize()
         a_ms, t_ms = e0.elapsed_time(e1), e1.elapsed_time(e2)
         st = bank.stats(0)
-        adm_ms.append(a_ms)
-        att_ms.append(t_ms)
-        per_step.append(a_ms + t_ms)
-        att_fl.append(attention_flops(w, [s["size"] for s in st]))
-        den_fl.append(density_flops(w, x["cand_ids"].shape[0], st_before, st))
-        den_alg.append(density_flops_algorithmic(w, x["cand_ids"].shape[0], st_before, st))
-    launches = kvb.kvb_launch_count() - launches0
-    clocks = sampler.stop()
+        N = 0 if w.forcing else x["cand_ids"].shape[0]
+        nf = x["new_ids"].shape[0] // w.F if w.forcing else 0
+        if i < timed_end:
+            upd_ms.append(a_ms)
+            att_ms.append(t_ms)
+            per_step.append(a_ms + t_ms)
+            att_fl.append(attention_flops(w, [s["size"] for s in st]))
+            if not w.forcing:
+                den_fl.append(density_flops(w, N, st_before, st))
+                den_alg.append(density_flops_algorithmic(w, N, st_before, st))
+            continue
+        for name in ("gram_bf16_kernel", "attend_bf16_kernel", "aug_rows_kernel", "gather_admitted_kernel",
+                     "gather_evicted_kernel", "compact_kernel", "finalize_kernel", "gram_reduce_kernel",
+                     "admit_count_kernel", "admit_select_kernel", "evict_select_kernel", "seg_cosine_kernel",
+                     "prune_plan_kernel", "prune_gather_kernel", "static_copy_kernel"):
+            b, u, text = kernel_units(w, name, N, st_before, st, nf, labels)
+            prev = units.get(name)
+            units[name] = (b, None if u is None else (u + (prev[1] or 0.0) if prev else u), text)
+    records = kvb.kvb_trace_read()
+    kvb.kvb_trace_enable(False)
     barrier(world)
     status = bank.status()
     if status != 0:
@@ -301,34 +418,50 @@ def run_densitykv(args, w, rank, world):
     nh = len(hosted)
 
     peaks, peak_src = load_peaks()
+    per_step_units = {n: (b, (u / n_trace if u is not None else None), t) for n, (b, u, t) in units.items()}
+    kernels = kernel_table(w, records, n_trace, per_step_units, peaks)
     att_achieved = statistics.mean(f / (t * 1e-3) for f, t in zip(att_fl, att_ms)) / 1e12
-    den_achieved = statistics.mean(f / (t * 1e-3) for f, t in zip(den_fl, adm_ms)) / 1e12
-    dominant_attend = statistics.mean(att_ms) >= statistics.mean(adm_ms)
     bf16_peak = peaks["bf16_tflops"]
 
-    def roof(achieved, kernel, per_unit, traffic=None):
-        return {"bound": "tensor", "achieved": round(achieved, 2), "peak": bf16_peak, "unit": "TFLOP/s",
-                "frac": round(achieved / bf16_peak, 4), "traffic": traffic, "kernel": kernel,
-                "peak_source": f"{peak_src} bf16 burst", "algorithmic": per_unit}
+    def roof_of(k):
+        r = {"bound": k["bound"], "achieved": k.get("achieved"), "peak": k.get("peak"), "unit": k.get("unit"),
+             "frac": k.get("frac"), "traffic": None, "kernel": k["kernel"],
+             "launches_per_step": k["launches_per_step"], "ms_per_launch": k["ms_per_launch"],
+             "peak_source": f"{peak_src} " + ("bf16 burst" if k["bound"] == "tensor" else "HBM copy"),
+             "algorithmic": k["algorithmic"]}
+        return r
 
-    roof_att = roof(att_achieved, "attend_bf16_kernel (kvb_attend, 1 launch)",
-                    "4*Nq*(Ls+|B_h|+Lw)*d flops summed over heads")
-    roof_den = roof(den_achieved, "kvb_admit (4 density Gram launches + selection/compaction)",
-                    "2*d*(N|B| + |B|P + |B'|E + P^2) flops summed over heads")
+    # the dominant kernel: largest share of the step's device time (traced steps)
+    dominant = kernels[0]
+    others = [roof_of(k) for k in kernels[1:] if k.get("frac") is not None]
+    roof = roof_of(dominant)
+    if dominant["kernel"] == "attend_bf16_kernel":
+        # kvb_attend is this one launch: take its time from the timed steps themselves
+        roof.update(achieved=round(att_achieved, 2), frac=round(att_achieved / bf16_peak, 4),
+                    ms_per_launch=round(statistics.mean(att_ms), 4), timing="timed steps (events around the launch)")
+    else:
+        roof["timing"] = f"{n_trace} launch-traced steps right after the timed ones"
+    upd_name = "prune" if w.forcing else "admit"
+    breakdown = {f"{upd_name}_ms": round(statistics.mean(upd_ms), 4), "attend_ms": round(statistics.mean(att_ms), 4),
+                 "attend_tflops": round(att_achieved, 1), "attention_gflop": round(statistics.mean(att_fl) / 1e9, 1),
+                 "history_sizes": [s["size"] for s in bank.stats(0)]}
+    if not w.forcing:
+        den_achieved = statistics.mean(f / (t * 1e-3) for f, t in zip(den_fl, upd_ms)) / 1e12
+        breakdown.update(admit_density_tflops=round(den_achieved, 1),
+                         density_algorithmic_gflop=round(statistics.mean(den_alg) / 1e9, 1),
+                         density_executed_gflop=round(statistics.mean(den_fl) / 1e9, 1),
+                         admitted=[s["admitted"] for s in bank.stats(0)][:1])
+    else:
+        breakdown.update(static_heads=[int(v) for v in labels])
     return {
         "ms_per_step": total_ms / (world * args.steps),
         "e2e_ms": e2e_total / (world * nh),
         "h2d": h2d // nh, "d2h": d2h // nh,
         "clocks": clocks, "launches": launches,
-        "roofline": roof_att if dominant_attend else roof_den,
-        "roofline_other": roof_den if dominant_attend else roof_att,
-        "breakdown": {"admit_ms": round(statistics.mean(adm_ms), 4), "attend_ms": round(statistics.mean(att_ms), 4),
-                      "attend_tflops": round(att_achieved, 1), "admit_density_tflops": round(den_achieved, 1),
-                      "density_algorithmic_gflop": round(statistics.mean(den_alg) / 1e9, 1),
-                      "density_executed_gflop": round(statistics.mean(den_fl) / 1e9, 1),
-                      "attention_gflop": round(statistics.mean(att_fl) / 1e9, 1),
-                      "bank_sizes": [s["size"] for s in bank.stats(0)],
-                      "admitted": [s["admitted"] for s in bank.stats(0)][:1]},
+        "roofline": roof,
+        "roofline_other": others,
+        "kernels": kernels,
+        "breakdown": breakdown,
         "gen_s": round(gen_s, 1),
         "first_timed_chunk": first + args.warmup,
     }
@@ -382,21 +515,98 @@ def oracle_sample(w, reps: int = 1):
     return statistics.mean(times), sample, (os.cpu_count(), blas_threads)
 
 
+def oracle_sample_forcing(w, reps: int = 1):
+    """Time the fp64 Forcing-KV oracle on a bounded sample of one chunk-layer: the
+    hybrid prune of one static and one dynamic head (full), and attention of a
+    few queries over each head's history; scaled to the workload's head labels
+    and query count."""
+    from oracle import forcingkv as fkv
+    from oracle.attention import attention
+    first = FIRST_TIMED.get(w.name, 4)
+    labels = kvgen.head_labels(w, 0)
+    pick = [int(np.argmax(labels == 1)), int(np.argmax(labels == 0))]   # one static, one dynamic head
+    L = kvgen.LayerInputs(w, 0, n_chunks=first + 1, heads=pick)
+    p = fkv.Params(w.frame_h, w.frame_w, w.seg_h, w.seg_w, w.retention, w.hist_frames)
+    states = [fkv.HeadState(True), fkv.HeadState(False)]
+    for i in range(1, first):   # bring both heads to steady state (not timed)
+        x = L.step(i, forcing=True)
+        fkv.prune_hybrid(states, p, x["newK"], x["newV"], x["new_ids"], x["nextK"])
+    x = L.step(first, forcing=True)
+    qr = 2048
+    n_static = int(labels.sum())
+    times = []
+    for _ in range(reps):
+        st = [fkv.HeadState(True), fkv.HeadState(False)]
+        st[0].transition = states[0].transition
+        st[1].ring = type(states[1].ring)(states[1].ring)
+        t = time.perf_counter()
+        fkv.prune_hybrid(st[:1], p, x["newK"][:1], x["newV"][:1], x["new_ids"], x["nextK"][:1])
+        t1 = time.perf_counter()
+        fkv.prune_hybrid(st[1:], p, x["newK"][1:], x["newV"][1:], x["new_ids"], x["nextK"][1:])
+        t2 = time.perf_counter()
+        Ks, Vs = fkv.attention_set(st[0], x["sinkK"][0], x["sinkV"][0], x["winK"][0], x["winV"][0])
+        attention(x["Q"][0][:qr], Ks, Vs)
+        t3 = time.perf_counter()
+        Kd, Vd = fkv.attention_set(st[1], x["sinkK"][1], x["sinkV"][1], x["winK"][1], x["winV"][1])
+        attention(x["Q"][1][:qr], Kd, Vd)
+        t4 = time.perf_counter()
+        scale = w.chunk_tokens / qr
+        static_ms = (t1 - t) + (t3 - t2) * scale
+        dyn_ms = (t2 - t1) + (t4 - t3) * scale
+        times.append((n_static * static_ms + (w.heads - n_static) * dyn_ms) * 1e3)
+    sample = (f"chunk {first} of layer 0: Forcing-KV prune of one static and one dynamic head (full), attention of "
+              f"{qr} of {w.chunk_tokens} queries over {Ks.shape[0]} (static) and {Kd.shape[0]} (dynamic) keys; "
+              f"scaled by queries and by the layer's {n_static} static / {w.heads - n_static} dynamic heads")
+    return statistics.mean(times), sample
+
+
+def cpu_sample(w, reps: int = 1):
+    if w.forcing:
+        ms, sample = oracle_sample_forcing(w, reps)
+    else:
+        ms, sample, _ = oracle_sample(w, reps)
+    try:
+        from threadpoolctl import threadpool_info
+        blas_threads = max((p.get("num_threads", 1) for p in threadpool_info()), default=1)
+    except Exception:
+        blas_threads = None
+    return ms, sample, (os.cpu_count(), blas_threads)
+
+
 def run_reference(args, w, rank, world):
     if rank != 0:
         return
     t0 = time.time()
-    ms, sample, (cores, blas) = oracle_sample(w, reps=max(1, args.steps))
+    ms, sample, (cores, blas) = cpu_sample(w, reps=max(1, args.steps))
     line = {"impl": "reference", "metric": METRIC, "value": round(ms, 3), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "heads": w.heads, "head_dim": w.head_dim, "F": w.F,
-                       "N": w.chunk_tokens, "M": w.capacity},
+            "config": workload_config(w, args, world),
             "cpu_baseline": {"value": round(ms, 3), "unit": UNIT, "cores": cores, "blas_threads": blas,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(ms, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "wall_s": round(time.time() - t0, 1)}
     print(json.dumps(line), flush=True)
+
+
+def workload_config(w, args, world):
+    first = FIRST_TIMED.get(w.name, 4) + args.warmup
+    chunks = f"chunks {first}..{first + args.steps - 1}"
+    if w.forcing:
+        text = (f"{w.name}: Forcing-KV hybrid prune of the finalised chunk ({w.seg_h}x{w.seg_w} segments, r="
+                f"{w.retention}, {w.hist_frames}-frame history, Bernoulli(0.5) static heads) + attention of "
+                f"{w.chunk_tokens} queries over sink {w.F} + history + window {w.chunk_tokens}; {w.heads} heads, "
+                f"d={w.head_dim}, layer 0, {chunks}")
+        extra = {"seg": [w.seg_h, w.seg_w], "retention": w.retention, "hist_frames": w.hist_frames}
+    else:
+        text = (f"{w.name}: DensityKV admit of {w.chunk_tokens} candidates + attention of {w.chunk_tokens} "
+                f"queries over sink {w.F} + bank (M={w.capacity}) + window {w.chunk_tokens}; {w.heads} heads, "
+                f"d={w.head_dim}, 1 layer, {chunks}")
+        extra = {"M": w.capacity, "tau": w.tau}
+    cfg = {"workload": text, "heads": w.heads, "head_dim": w.head_dim, "F": w.F, "N": w.chunk_tokens}
+    cfg.update(extra)
+    cfg.update({"parallelism": f"replicas x{world}", "l2": "flushed (256 MB write) before each step"})
+    return cfg
 
 
 def main():
@@ -417,12 +627,12 @@ def main():
         return
     import torch
     torch.cuda.set_device(local)
-    r = run_densitykv(args, w, rank, world)
+    r = run_workload(args, w, rank, world)
     if rank != 0:
         return
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        ms, sample, (cores, blas) = oracle_sample(w, reps=1)
+        ms, sample, (cores, blas) = cpu_sample(w, reps=1)
         cpu = {"value": round(ms, 3), "unit": UNIT, "cores": cores, "blas_threads": blas, "kind": "oracle",
                "sample": sample}
     line = {
@@ -430,17 +640,13 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["ms_per_step"], 4),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16"
         else "f32", "data": "synthetic",
-        "config": {"workload": (f"{w.name}: DensityKV admit of {w.chunk_tokens} candidates + attention of "
-                                f"{w.chunk_tokens} queries over sink {w.F} + bank (M={w.capacity}) + window "
-                                f"{w.chunk_tokens}; {w.heads} heads, d={w.head_dim}, 1 layer, chunks "
-                                f"{r['first_timed_chunk']}..{r['first_timed_chunk'] + args.steps - 1}"),
-                   "heads": w.heads, "head_dim": w.head_dim, "F": w.F, "N": w.chunk_tokens, "M": w.capacity,
-                   "tau": w.tau, "parallelism": f"replicas x{world}", "l2": "flushed (256 MB write) before each step"},
+        "config": workload_config(w, args, world),
         "e2e": {"value": round(r["e2e_ms"], 4), "unit": UNIT, "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches"],
         "roofline": r["roofline"],
         "roofline_other": r["roofline_other"],
+        "kernels": r["kernels"],
         "breakdown": r["breakdown"],
         "clocks": r["clocks"],
         "cpu_baseline": cpu,

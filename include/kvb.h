@@ -110,7 +110,8 @@ typedef struct {
   int32_t mandatory;     /* evictions with ratio > tau */
   int32_t capacity_evicted;
   int32_t size;          /* bank size after the update (ring size for Forcing-KV) */
-  int32_t reserved[3];
+  int32_t moved;         /* DensityKV: surviving entries moved from the tail into holes */
+  int32_t reserved[2];
 } kvb_admit_stats;
 
 typedef struct kvb_bank kvb_bank; /* opaque, host-side */
@@ -181,6 +182,29 @@ KVB_API kvb_status kvb_device_status(kvb_bank* bank, void* stream);
 /* Number of kernels the library has launched in this process (all entry points,
  * all devices); a diagnostic for callers that account launches. */
 KVB_API unsigned long long kvb_launch_count(void);
+
+/* Launch tracing, a per-kernel timing aid.  While enabled, every kernel launch of
+ * the library is bracketed by a pair of CUDA events recorded on the stream the
+ * kernel is launched on, and the pair is kept with the kernel's name.  Meant for a
+ * single host thread driving the library.  Off by default.
+ *   kvb_trace_enable: switch tracing on (nonzero) or off; either way, drop the
+ *     records held so far.  Never fails.
+ *   kvb_trace_read: wait for the recorded events, write up to `max_records`
+ *     records in launch order into caller host memory `out`, set *n_out to the
+ *     number of records held (which may exceed max_records), then drop them all.
+ *     kernel: static name string owned by the library; ms: the launch's device
+ *     time in milliseconds, or -1 when its events could not be read (the call then
+ *     returns KVB_E_CUDA after filling the rest); device: CUDA ordinal.
+ *     KVB_E_INVAL if n_out is NULL or max_records < 0 or out is NULL with
+ *     max_records > 0.  At most 65536 launches are held; later ones are counted
+ *     by kvb_launch_count but not traced. */
+typedef struct {
+  const char* kernel;
+  float ms;
+  int32_t device;
+} kvb_trace_record;
+KVB_API kvb_status kvb_trace_enable(int32_t enable);
+KVB_API kvb_status kvb_trace_read(kvb_trace_record* out, int32_t max_records, int32_t* n_out);
 
 /* Static string for a status code. */
 KVB_API const char* kvb_status_string(kvb_status st);

@@ -315,6 +315,7 @@ __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPl
     p.stats[h].mandatory = n_mand;
     p.stats[h].capacity_evicted = E - n_mand;
     p.stats[h].size = n_new;
+    p.stats[h].moved = s_ntail;
   }
 }
 
@@ -400,38 +401,38 @@ __global__ void finalize_kernel(const AdmitPlan p) {
 }  // namespace
 
 cudaError_t launch_admit_count(const AdmitPlan& p, cudaStream_t st) {
-  note_launch();
+  LaunchTrace trace("admit_count_kernel", st);
   admit_count_kernel<<<p.H, kSelThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_admit_select(const AdmitPlan& p, cudaStream_t st) {
-  note_launch();
+  LaunchTrace trace("admit_select_kernel", st);
   admit_select_kernel<<<p.H, kSelThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_gather_admitted(const AdmitPlan& p, int maxP, cudaStream_t st) {
   if (maxP <= 0) return cudaSuccess;
-  note_launch();
+  LaunchTrace trace("gather_admitted_kernel", st);
   gather_admitted_kernel<<<dim3((maxP + 7) / 8, p.H), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_evict_select(const AdmitPlan& p, cudaStream_t st) {
-  note_launch();
+  LaunchTrace trace("evict_select_kernel", st);
   evict_select_kernel<<<p.H, kSelThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_gather_evicted(const AdmitPlan& p, cudaStream_t st) {
-  note_launch();
+  LaunchTrace trace("gather_evicted_kernel", st);
   gather_evicted_kernel<<<dim3((p.M + 7) / 8, p.H), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_compact(const AdmitPlan& p, cudaStream_t st) {
-  note_launch();
+  LaunchTrace trace("compact_kernel", st);
   compact_kernel<<<dim3((p.N + p.M + 7) / 8, p.H), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_finalize(const AdmitPlan& p, cudaStream_t st) {
-  note_launch();
+  LaunchTrace trace("finalize_kernel", st);
   finalize_kernel<<<dim3((p.M + 255) / 256, p.H), 256, 0, st>>>(p);
   return cudaGetLastError();
 }

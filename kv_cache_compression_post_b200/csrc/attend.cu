@@ -428,7 +428,7 @@ cudaError_t launch_attend_bf16(const AttnArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(attend_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = a.H * ((a.Nq + kTile - 1) / kTile);
-  note_launch();
+  LaunchTrace trace("attend_bf16_kernel", st);
   attend_bf16_kernel<<<grid, kThreads, smem, st>>>(maps, a);
   return cudaGetLastError();
 }
@@ -437,7 +437,7 @@ cudaError_t launch_attend_f32(const AttnArgs& a, cudaStream_t st) {
   if (a.Nq <= 0) return cudaSuccess;
   if (a.d > kF32MaxD) return cudaErrorInvalidValue;
   dim3 grid((a.Nq + 3) / 4, a.H);
-  note_launch();
+  LaunchTrace trace("attend_f32_kernel", st);
   attend_f32_kernel<<<grid, 128, 0, st>>>(a);
   return cudaGetLastError();
 }

@@ -230,7 +230,7 @@ cudaError_t launch_seg_cosine_ld(const void* K, const void* nextK, kvb_dtype dty
   if (H <= 0 || n_frames <= 0) return cudaSuccess;
   dim3 grid(g.seg_rows, n_frames, H);
   const size_t smem = sizeof(float) * g.seg_h * g.frame_w;
-  note_launch();
+  LaunchTrace trace("seg_cosine_kernel", st);
   if (dtype == KVB_BF16)
     seg_cosine_kernel<<<grid, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(K),
                                                static_cast<const __nv_bfloat16*>(nextK), n_frames, d, g, skip_mask,
@@ -242,19 +242,19 @@ cudaError_t launch_seg_cosine_ld(const void* K, const void* nextK, kvb_dtype dty
 }
 
 cudaError_t launch_prune_plan(const PrunePlan& p, cudaStream_t st) {
-  note_launch();
+  LaunchTrace trace("prune_plan_kernel", st);
   prune_plan_kernel<<<p.H, kPlanThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prune_gather(const PrunePlan& p, cudaStream_t st) {
-  note_launch();
+  LaunchTrace trace("prune_gather_kernel", st);
   prune_gather_kernel<<<dim3((p.ld_plan + 7) / 8, p.H), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_static_copy(const PrunePlan& p, cudaStream_t st) {
-  note_launch();
+  LaunchTrace trace("static_copy_kernel", st);
   static_copy_kernel<<<dim3((p.g.F + 7) / 8, p.H), 256, 0, st>>>(p);
   return cudaGetLastError();
 }

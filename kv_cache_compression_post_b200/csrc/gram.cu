@@ -515,17 +515,17 @@ cudaError_t launch_gram_bf16(const GramArgs& a, const CUtensorMap& tmR, const CU
   if (a.s == 2.f) {
     e = cudaFuncSetAttribute(gram_bf16_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    note_launch();
+    LaunchTrace trace("gram_bf16_kernel", st);
     gram_bf16_kernel<2><<<grid, kGramThreads, smem, st>>>(tmR, tmC, tmRa, tmCa, a);
   } else if (a.s == 1.f) {
     e = cudaFuncSetAttribute(gram_bf16_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    note_launch();
+    LaunchTrace trace("gram_bf16_kernel", st);
     gram_bf16_kernel<1><<<grid, kGramThreads, smem, st>>>(tmR, tmC, tmRa, tmCa, a);
   } else {
     e = cudaFuncSetAttribute(gram_bf16_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    note_launch();
+    LaunchTrace trace("gram_bf16_kernel", st);
     gram_bf16_kernel<0><<<grid, kGramThreads, smem, st>>>(tmR, tmC, tmRa, tmCa, a);
   }
   return cudaGetLastError();
@@ -535,7 +535,7 @@ cudaError_t launch_gram_f32(const GramArgs& a, cudaStream_t st) {
   const int maxR = a.max_rows;
   dim3 grid((maxR + kF32Warps - 1) / kF32Warps, a.H);
   const size_t smem = sizeof(float) * (kF32Warps * a.d + kF32Cols * (a.d + 1));
-  note_launch();
+  LaunchTrace trace("gram_f32_kernel", st);
   gram_f32_kernel<<<grid, kF32Warps * 32, smem, st>>>(a);
   return cudaGetLastError();
 }
@@ -543,7 +543,7 @@ cudaError_t launch_gram_f32(const GramArgs& a, cudaStream_t st) {
 cudaError_t launch_gram_reduce(const GramArgs& a, float* out, int ldOut, cudaStream_t st) {
   const int maxR = a.max_rows;
   dim3 grid((maxR + 255) / 256, a.H);
-  note_launch();
+  LaunchTrace trace("gram_reduce_kernel", st);
   gram_reduce_kernel<<<grid, 256, 0, st>>>(a, out, ldOut);
   return cudaGetLastError();
 }

@@ -28,8 +28,22 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, int d, long long rows, int
 // box 16 x box_rows x 1, 32-byte swizzle (one K=16 slice of an MMA operand).
 bool make_tmap_aug(CUtensorMap* m, const void* base, long long rows, int heads, int box_rows);
 
-// Count of kernel launches issued by the library in this process.
-void note_launch();
+// Every kernel launch of the library goes through one of these, constructed just
+// before the launch in the same scope: it counts the launch and, while tracing is
+// on, records a CUDA event pair around it on the launch stream (the destructor,
+// run after the launch statement, records the second event).
+class LaunchTrace {
+ public:
+  LaunchTrace(const char* kernel, cudaStream_t st);
+  ~LaunchTrace();
+  LaunchTrace(const LaunchTrace&) = delete;
+  LaunchTrace& operator=(const LaunchTrace&) = delete;
+
+ private:
+  const char* kernel_;
+  cudaStream_t st_;
+  int slot_ = -1;
+};
 
 inline kvb_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVB_OK : KVB_E_CUDA; }
 

@@ -60,7 +60,7 @@ cudaError_t launch_aug_rows(const void* X, kvb_dtype dtype, int H, long long ldX
                             int max_n, uint16_t* out, long long ldOut, float* norm_max, cudaStream_t st) {
   if (max_n <= 0 || H <= 0) return cudaSuccess;
   dim3 grid((max_n + 7) / 8, H);
-  note_launch();
+  LaunchTrace trace("aug_rows_kernel", st);
   if (dtype == KVB_BF16)
     aug_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), ldX, d, n_uni, n_dev, out, ldOut,
                                           norm_max);
@@ -74,7 +74,7 @@ cudaError_t launch_row_terms(const void* X, kvb_dtype dtype, int H, long long ld
                              cudaStream_t st) {
   if (max_n <= 0 || H <= 0) return cudaSuccess;
   dim3 grid((max_n + 7) / 8, H);
-  note_launch();
+  LaunchTrace trace("row_terms_kernel", st);
   if (dtype == KVB_BF16)
     row_terms_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), ldX, d, n_uni, n_dev, inv_h, add,
                                            out, ldOut);

@@ -17,7 +17,7 @@ __all__ = [
     "KVB_BF16", "KVB_F32", "KVB_DENSITYKV", "KVB_FORCINGKV",
     "kvb_workspace_size", "kvb_bank_create", "kvb_bank_destroy", "kvb_admit", "kvb_prune_hybrid",
     "kvb_attend", "kvb_read_stats", "kvb_bank_export", "kvb_bank_import", "kvb_device_status",
-    "kvb_status_string", "kvb_launch_count", "kvb_density_workspace_size", "kvb_density", "kvb_density_noalloc", "kvb_segment_cosine",
+    "kvb_status_string", "kvb_launch_count", "kvb_trace_enable", "kvb_trace_read", "kvb_density_workspace_size", "kvb_density", "kvb_density_noalloc", "kvb_segment_cosine",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvb.so")
@@ -50,7 +50,8 @@ class kvb_config(ctypes.Structure):
 
 class kvb_admit_stats(ctypes.Structure):
     _fields_ = [("admitted", ctypes.c_int32), ("feasible", ctypes.c_int32), ("mandatory", ctypes.c_int32),
-                ("capacity_evicted", ctypes.c_int32), ("size", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+                ("capacity_evicted", ctypes.c_int32), ("size", ctypes.c_int32), ("moved", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 2)]
 
 
 def make_config(**kw) -> kvb_config:
@@ -64,6 +65,10 @@ def make_config(**kw) -> kvb_config:
     for k, v in defaults.items():
         setattr(c, k, v)
     return c
+
+
+class kvb_trace_record(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_char_p), ("ms", ctypes.c_float), ("device", ctypes.c_int32)]
 
 
 if not os.path.exists(LIB_PATH):
@@ -85,6 +90,8 @@ _SIGS = {
     "kvb_device_status": (ctypes.c_int, [_vp, _vp]),
     "kvb_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "kvb_launch_count": (ctypes.c_ulonglong, []),
+    "kvb_trace_enable": (ctypes.c_int, [_i32]),
+    "kvb_trace_read": (ctypes.c_int, [ctypes.POINTER(kvb_trace_record), _i32, ctypes.POINTER(_i32)]),
     "kvb_density_workspace_size": (_sz, [_i32, _i32, _i32, _i32, ctypes.c_int]),
     "kvb_density": (ctypes.c_int, [_vp, _i32, _vp, _i32, _i32, _i32, ctypes.c_int, _f, _f, _f, _i32, _vp, _vp,
                                    _sz, _vp]),
@@ -123,6 +130,19 @@ def _check(st: int, where: str) -> None:
 
 def kvb_launch_count() -> int:
     return int(lib.kvb_launch_count())
+
+
+def kvb_trace_enable(enable: bool) -> None:
+    _check(lib.kvb_trace_enable(1 if enable else 0), "kvb_trace_enable")
+
+
+def kvb_trace_read(max_records: int = 65536) -> list:
+    """[(kernel name, device ms), ...] of the launches traced since the last read,
+    in launch order (waits for their events)."""
+    buf = (kvb_trace_record * max_records)()
+    n = _i32(0)
+    _check(lib.kvb_trace_read(buf, max_records, ctypes.byref(n)), "kvb_trace_read")
+    return [(buf[i].kernel.decode(), float(buf[i].ms)) for i in range(min(n.value, max_records))]
 
 
 def kvb_status_string(status: int) -> str:
@@ -170,7 +190,7 @@ def kvb_read_stats(bank: int, layer: int, heads: int, stream=None):
     arr = (kvb_admit_stats * heads)()
     _check(lib.kvb_read_stats(bank, layer, arr, _stream(stream)), "kvb_read_stats")
     return [dict(admitted=a.admitted, feasible=a.feasible, mandatory=a.mandatory,
-                 capacity_evicted=a.capacity_evicted, size=a.size) for a in arr]
+                 capacity_evicted=a.capacity_evicted, size=a.size, moved=a.moved) for a in arr]
 
 
 def kvb_bank_export(bank: int, layer: int, head: int, ids, rho, rho0, K, V, stream=None) -> int:

@@ -70,6 +70,8 @@ class Workload:
     hist_frames: int = 21
     # default seed namespace offset (see WORKLOADS["tiny"])
     seed_offset: int = 0
+    # history policy the workload exercises: "densitykv" or "forcingkv"
+    method: str = "densitykv"
 
     @property
     def F(self) -> int:
@@ -78,6 +80,15 @@ class Workload:
     @property
     def chunk_tokens(self) -> int:
         return self.chunk_frames * self.F
+
+    @property
+    def forcing(self) -> bool:
+        return self.method == "forcingkv"
+
+    @property
+    def n_segments(self) -> int:
+        """Forcing-KV segments per frame (partial edge segments included)."""
+        return -(-self.frame_h // self.seg_h) * -(-self.frame_w // self.seg_w)
 
 
 def _w(**kw) -> Workload:
@@ -101,7 +112,7 @@ WORKLOADS: Dict[str, Workload] = {
     # Forcing-KV hybrid prune at 480P
     "forcing480": _w(name="forcing480", wid=3, layers=30, heads=12, head_dim=128, dtype="bf16",
                      frame_h=30, frame_w=52, chunk_frames=3, n_chunks=9, capacity=9360,
-                     seg_h=4, seg_w=4, retention=0.7, hist_frames=21),
+                     seg_h=4, seg_w=4, retention=0.7, hist_frames=21, method="forcingkv"),
     # 1080P scale-up: 68x120 frames, M=32640, 10 chunks
     "wan1080": _w(name="wan1080", wid=4, layers=1, heads=12, head_dim=128, dtype="bf16",
                   frame_h=68, frame_w=120, chunk_frames=3, n_chunks=10, capacity=32640),
@@ -111,7 +122,7 @@ WORKLOADS: Dict[str, Workload] = {
     # mid-size Forcing-KV parity case
     "forcing_mid": _w(name="forcing_mid", wid=6, layers=1, heads=4, head_dim=128, dtype="bf16",
                       frame_h=10, frame_w=18, chunk_frames=3, n_chunks=6, capacity=900,
-                      seg_h=4, seg_w=4, retention=0.7, hist_frames=7),
+                      seg_h=4, seg_w=4, retention=0.7, hist_frames=7, method="forcingkv"),
 }
 
 

@@ -50,3 +50,15 @@ def test_density_argument_errors_without_gpu():
     with pytest.raises(kvb.KvbError) as e:   # misaligned workspace
         kvb.kvb_density(1, 10, 1, 10, 2, 128, 0, 0.0, 1e-3, 2.0, 0, 1, 257, 1 << 20, stream=0)
     assert e.value.status == 2
+
+
+def test_launch_trace_host_side():
+    import ctypes
+    import kv_cache_compression_post_b200 as kvb
+    kvb.kvb_trace_enable(True)
+    assert kvb.kvb_trace_read() == []          # nothing launched
+    kvb.kvb_trace_enable(False)
+    n = ctypes.c_int32(0)
+    assert kvb.lib.kvb_trace_read(None, 0, ctypes.byref(n)) == 0 and n.value == 0
+    assert kvb.lib.kvb_trace_read(None, 4, ctypes.byref(n)) == 1   # out NULL with max_records > 0
+    assert kvb.lib.kvb_trace_read(None, 0, None) == 1              # n_out NULL

@@ -107,7 +107,12 @@ def test_attend_full_size_sampled_rows():
                           capacity=w.capacity, max_candidates=w.chunk_tokens, max_queries=w.chunk_tokens)
     bank = kvb.Bank(cfg)
     import_oracle_banks(bank, banks, dkv.Params(capacity=w.capacity), w)
+    kvb.kvb_trace_enable(True)
     O, lse = _attend(bank, w, x)
+    trace = kvb.kvb_trace_read()
+    kvb.kvb_trace_enable(False)
+    # the launch trace saw exactly the one attention launch, with a device time
+    assert [n for n, _ in trace] == ["attend_bf16_kernel"] and trace[0][1] > 0
     for hh in range(H):
         idx = np.sort(rng.choice(w.chunk_tokens, 16, replace=False))
         K, V = dkv.attention_set(banks[hh], x["sinkK"][hh], x["sinkV"][hh], x["winK"][hh], x["winV"][hh])
