@@ -25,6 +25,10 @@ extern "C" kvb_status kvb_attend(kvb_bank* b, int32_t layer, const void* Q, int3
   a.O = O;
   a.lse = lse;
   a.status = b->status;
+  a.part = b->attn_part;
+  a.cnt = b->attn_cnt;
+  if (++b->attn_epoch == 0) ++b->attn_epoch;
+  a.epoch = b->attn_epoch;
   int n = 0;
   if (Ls > 0) {
     a.seg[n].K = sinkK;

@@ -8,6 +8,7 @@
 #include <new>
 
 #include "admit.cuh"
+#include "attend.cuh"
 #include "bank.h"
 #include "gram.cuh"
 #include "small_kernels.cuh"
@@ -42,6 +43,8 @@ size_t kvb_bank::layout(void* base) {
   const kvb_config& g = cfg;
   const size_t L = g.layers, H = g.heads, d = g.head_dim;
   status = c.take<int>(64);
+  attn_cnt = c.take<unsigned long long>(attend_counter_count(g.heads, g.max_queries));
+  attn_part = g.dtype == KVB_BF16 ? c.take<float>(attend_partial_floats(g.head_dim)) : nullptr;
   if (g.method == KVB_DENSITYKV) {
     const size_t M = g.capacity, N = g.max_candidates;
     ldN = static_cast<int>(N);
@@ -144,6 +147,9 @@ kvb_status kvb_bank_create(const kvb_config* cfg, void* workspace, size_t worksp
   // status word, and status[1] = the largest ||k||^2 ever stored (density clamp guard)
   cudaError_t e = cudaMemsetAsync(b->status, 0, 2 * sizeof(int), st);
   if (e == cudaSuccess) e = cudaMemsetAsync(b->stats, 0, LH * sizeof(kvb_admit_stats), st);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(b->attn_cnt, 0, attend_counter_count(cfg->heads, cfg->max_queries) * sizeof(unsigned long long),
+                        st);
   if (cfg->method == KVB_DENSITYKV) {
     // rows past a bank's size are read by full attention tiles (and masked): keep
     // them finite by starting from zeros

@@ -10,6 +10,17 @@
 namespace kvb {
 
 constexpr int kAttnMaxSeg = 5;
+// Persistent grid cap of the bf16 kernel (>= the SM count of a B200); the scratch
+// below is sized for it.
+constexpr int kAttnMaxCtas = 160;
+
+// Scratch of the bf16 kernel: partial results of query tiles whose key range is
+// split between CTAs, and one arrival counter per (query-tile pair, tile).
+inline size_t attend_partial_floats(int d) { return static_cast<size_t>(4) * kAttnMaxCtas * (128 * d + 256); }
+inline size_t attend_counter_count(int heads, int max_queries) {
+  const int nqt = (max_queries + 127) / 128;
+  return static_cast<size_t>(heads) * ((nqt + 1) / 2) * 2;
+}
 
 // One K/V source: [H][ld][d] buffers; per head a start row and a length, each
 // uniform or from a device array indexed by head.
@@ -32,6 +43,10 @@ struct AttnArgs {
   void* O = nullptr;            // [H][Nq][d]
   float* lse = nullptr;         // [H][Nq] or null
   int* status = nullptr;
+  // bf16 path scratch (attend_partial_floats / attend_counter_count entries)
+  float* part = nullptr;
+  unsigned long long* cnt = nullptr;
+  unsigned int epoch = 1;       // nonzero, different on consecutive launches
 };
 
 struct AttnMaps {

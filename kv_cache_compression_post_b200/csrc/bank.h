@@ -19,6 +19,10 @@ struct kvb_bank {
   int n_seg = 0;            // segments per frame (Forcing-KV)
   int ring_cap = 0;         // tokens a dynamic head's FIFO can hold
   int* status = nullptr;
+  // attention scratch (bf16 path): split-unit partials and arrival counters
+  float* attn_part = nullptr;
+  unsigned long long* attn_cnt = nullptr;
+  unsigned int attn_epoch = 0;  // launches so far (the kernel's epoch tag, never 0)
 
   // ---- DensityKV, per layer: base pointers of layer 0 and strides
   char* K = nullptr;        // [L][H][M][d]
