@@ -143,7 +143,8 @@ KVB_API kvb_status kvb_admit(kvb_bank* bank, int32_t layer, const void* candK, c
  * nextK: device [H][F][d], the first frame of the next chunk (successor of the
  * last new frame); new_ids: device [n_frames*F] int32.  Static heads take the
  * last new frame as their transition frame; dynamic heads push each new frame's
- * BottomK segments into their FIFO of hist_frames frames. */
+ * BottomK segments into their FIFO of hist_frames frames.  newK, newV and nextK
+ * must be 16-byte aligned (KVB_E_INVAL otherwise). */
 KVB_API kvb_status kvb_prune_hybrid(kvb_bank* bank, int32_t layer, const uint8_t* head_is_static,
                             const void* newK, const void* newV, const void* nextK,
                             const int32_t* new_ids, int32_t n_frames, void* stream);
@@ -258,7 +259,9 @@ KVB_API kvb_status kvb_density_noalloc(const void* rows, int32_t n_rows, const v
  * cos(K[h][t][p], succ[h][t][p]) with succ = frame t+1 of K, or `nextK` for the
  * last frame.  K [H][n_frames*F][d], nextK [H][F][d]; sim [H][n_frames][n_seg]
  * f32 with n_seg = ceil(frame_h/seg_h)*ceil(frame_w/seg_w), segments row-major.
- * cos(a, b) = a.b / max(|a| |b|, 1e-8). */
+ * cos(a, b) = a.b / max(|a| |b|, 1e-8).  K and nextK must be 16-byte aligned
+ * (KVB_E_INVAL) and head_dim * element size a multiple of 16 bytes
+ * (KVB_E_UNSUPPORTED). */
 KVB_API kvb_status kvb_segment_cosine(const void* K, const void* nextK, int32_t heads, int32_t n_frames,
                               int32_t frame_h, int32_t frame_w, int32_t seg_h, int32_t seg_w,
                               int32_t head_dim, kvb_dtype dtype, float* sim, void* stream);

@@ -17,7 +17,8 @@
 //             baselines rho0 = rho (co-admitted entries set them together)
 //
 // The selection kernels run one 1024-thread CTA per head (latency-bound, a few
-// microseconds); the row movers use one warp per 256-byte K/V row.
+// microseconds); the row movers move each K/V row with a group of lanes, one
+// 16-byte word per lane, over a grid of about one wave.
 #include <climits>
 
 #include "admit.cuh"
@@ -222,27 +223,22 @@ __global__ void __launch_bounds__(kSelThreads) admit_select_kernel(const AdmitPl
   }
 }
 
-// one warp per 16-byte-chunked row copy
-__device__ __forceinline__ void copy_row(void* dst, const void* src, int row_bytes, int lane) {
-  const uint4* s = static_cast<const uint4*>(src);
-  uint4* d = static_cast<uint4*>(dst);
-  for (int o = lane; o < row_bytes / 16; o += 32) d[o] = s[o];
-}
-// 64-byte augmented row, lanes 0..3
-__device__ __forceinline__ void copy_aug(uint16_t* dst, const uint16_t* src, int lane) {
-  if (lane < 4) reinterpret_cast<uint4*>(dst)[lane] = reinterpret_cast<const uint4*>(src)[lane];
+// 64-byte augmented row, the group's lanes 0..3
+__device__ __forceinline__ void copy_aug(uint16_t* dst, const uint16_t* src, const RowGroup& g) {
+  if (g.sub < 4) reinterpret_cast<uint4*>(dst)[g.sub] = reinterpret_cast<const uint4*>(src)[g.sub];
 }
 
 __global__ void gather_admitted_kernel(const AdmitPlan p) {
   const int h = blockIdx.y;
-  const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (w >= p.P[h]) return;
-  const int c = p.adm_idx[static_cast<size_t>(h) * p.ldN + w];
-  const size_t dst = static_cast<size_t>(h) * p.ldEA + p.M + w;
-  copy_row(static_cast<char*>(p.EA) + dst * p.row_bytes,
-           static_cast<const char*>(p.candK) + (static_cast<size_t>(h) * p.N + c) * p.row_bytes, p.row_bytes, lane);
-  copy_aug(p.EAaug + dst * 32, p.caug + (static_cast<size_t>(h) * p.ldN + c) * 32, lane);
+  const RowGroup g = row_group(p.row_bytes);
+  const int P = p.P[h];
+  for (int w = g.first; w < P; w += g.stride) {
+    const int c = p.adm_idx[static_cast<size_t>(h) * p.ldN + w];
+    const size_t dst = static_cast<size_t>(h) * p.ldEA + p.M + w;
+    copy_row(static_cast<char*>(p.EA) + dst * p.row_bytes,
+             static_cast<const char*>(p.candK) + (static_cast<size_t>(h) * p.N + c) * p.row_bytes, p.row_bytes, g);
+    copy_aug(p.EAaug + dst * 32, p.caug + (static_cast<size_t>(h) * p.ldN + c) * 32, g);
+  }
 }
 
 __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPlan p) {
@@ -321,62 +317,63 @@ __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPl
 
 __global__ void gather_evicted_kernel(const AdmitPlan p) {
   const int h = blockIdx.y;
-  const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+  const RowGroup g = row_group(p.row_bytes);
   const int E = p.E[h];
-  if (w >= E) return;
-  const int slot = p.ev_slot[static_cast<size_t>(h) * p.M + w];
-  const size_t src = static_cast<size_t>(h) * p.M + slot;
-  const size_t dst = static_cast<size_t>(h) * p.ldEA + (p.M - E) + w;
-  copy_row(static_cast<char*>(p.EA) + dst * p.row_bytes, static_cast<const char*>(p.K) + src * p.row_bytes,
-           p.row_bytes, lane);
-  copy_aug(p.EAaug + dst * 32, p.aug + src * 32, lane);
+  for (int w = g.first; w < E; w += g.stride) {
+    const int slot = p.ev_slot[static_cast<size_t>(h) * p.M + w];
+    const size_t src = static_cast<size_t>(h) * p.M + slot;
+    const size_t dst = static_cast<size_t>(h) * p.ldEA + (p.M - E) + w;
+    copy_row(static_cast<char*>(p.EA) + dst * p.row_bytes, static_cast<const char*>(p.K) + src * p.row_bytes,
+             p.row_bytes, g);
+    copy_aug(p.EAaug + dst * 32, p.aug + src * 32, g);
+  }
 }
 
 // moves: [0, P) admitted candidates, [P, P + ntail) surviving tail entries
 __global__ void compact_kernel(const AdmitPlan p) {
   const int h = blockIdx.y;
-  const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+  const RowGroup g = row_group(p.row_bytes);
   const int P = p.P[h], nt = p.ntail[h], nh = p.nhole[h], n_old = p.n_old[h];
   const size_t base = static_cast<size_t>(h) * p.M;
   const int* hole = p.ev_slot + base;  // evicted slots ascending: the first nh are holes
-  if (w < P) {
-    const int dst = (w < nh) ? hole[w] : n_old + (w - nh);
-    if (dst < 0 || dst >= p.M) {
-      if (lane == 0) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
-      return;
-    }
-    const int c = p.adm_idx[static_cast<size_t>(h) * p.ldN + w];
-    const size_t srow = static_cast<size_t>(h) * p.N + c;
-    copy_row(static_cast<char*>(p.K) + (base + dst) * p.row_bytes,
-             static_cast<const char*>(p.candK) + srow * p.row_bytes, p.row_bytes, lane);
-    copy_row(static_cast<char*>(p.V) + (base + dst) * p.row_bytes,
-             static_cast<const char*>(p.candV) + srow * p.row_bytes, p.row_bytes, lane);
-    copy_aug(p.aug + (base + dst) * 32, p.caug + (static_cast<size_t>(h) * p.ldN + c) * 32, lane);
-    if (lane == 0) {
-      p.ids[base + dst] = p.cand_ids[c];
-      p.rho[base + dst] = p.rhoB[static_cast<size_t>(h) * p.ldN + c];
-      p.newp[base + dst] = w;
-    }
-  } else if (w < P + nt) {
-    const int k = w - P;
-    const int src = p.tail[base + k];
-    const int dst = hole[P + k];
-    if (src < 0 || src >= p.M || dst < 0 || dst >= p.M) {
-      if (lane == 0) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
-      return;
-    }
-    copy_row(static_cast<char*>(p.K) + (base + dst) * p.row_bytes,
-             static_cast<const char*>(p.K) + (base + src) * p.row_bytes, p.row_bytes, lane);
-    copy_row(static_cast<char*>(p.V) + (base + dst) * p.row_bytes,
-             static_cast<const char*>(p.V) + (base + src) * p.row_bytes, p.row_bytes, lane);
-    copy_aug(p.aug + (base + dst) * 32, p.aug + (base + src) * 32, lane);
-    if (lane == 0) {
-      p.ids[base + dst] = p.ids[base + src];
-      p.rho0[base + dst] = p.rho0[base + src];
-      p.rho[base + dst] = p.rho[base + src] + p.proj[base + src];
-      p.newp[base + dst] = -2;
+  for (int w = g.first; w < P + nt; w += g.stride) {
+    if (w < P) {
+      const int dst = (w < nh) ? hole[w] : n_old + (w - nh);
+      if (dst < 0 || dst >= p.M) {
+        if (g.sub == 0) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
+        continue;
+      }
+      const int c = p.adm_idx[static_cast<size_t>(h) * p.ldN + w];
+      const size_t srow = static_cast<size_t>(h) * p.N + c;
+      copy_row(static_cast<char*>(p.K) + (base + dst) * p.row_bytes,
+               static_cast<const char*>(p.candK) + srow * p.row_bytes, p.row_bytes, g);
+      copy_row(static_cast<char*>(p.V) + (base + dst) * p.row_bytes,
+               static_cast<const char*>(p.candV) + srow * p.row_bytes, p.row_bytes, g);
+      copy_aug(p.aug + (base + dst) * 32, p.caug + (static_cast<size_t>(h) * p.ldN + c) * 32, g);
+      if (g.sub == 0) {
+        p.ids[base + dst] = p.cand_ids[c];
+        p.rho[base + dst] = p.rhoB[static_cast<size_t>(h) * p.ldN + c];
+        p.newp[base + dst] = w;
+      }
+    } else {
+      const int k = w - P;
+      const int src = p.tail[base + k];
+      const int dst = hole[P + k];
+      if (src < 0 || src >= p.M || dst < 0 || dst >= p.M) {
+        if (g.sub == 0) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
+        continue;
+      }
+      copy_row(static_cast<char*>(p.K) + (base + dst) * p.row_bytes,
+               static_cast<const char*>(p.K) + (base + src) * p.row_bytes, p.row_bytes, g);
+      copy_row(static_cast<char*>(p.V) + (base + dst) * p.row_bytes,
+               static_cast<const char*>(p.V) + (base + src) * p.row_bytes, p.row_bytes, g);
+      copy_aug(p.aug + (base + dst) * 32, p.aug + (base + src) * 32, g);
+      if (g.sub == 0) {
+        p.ids[base + dst] = p.ids[base + src];
+        p.rho0[base + dst] = p.rho0[base + src];
+        p.rho[base + dst] = p.rho[base + src] + p.proj[base + src];
+        p.newp[base + dst] = -2;
+      }
     }
   }
 }
@@ -413,7 +410,7 @@ cudaError_t launch_admit_select(const AdmitPlan& p, cudaStream_t st) {
 cudaError_t launch_gather_admitted(const AdmitPlan& p, int maxP, cudaStream_t st) {
   if (maxP <= 0) return cudaSuccess;
   LaunchTrace trace("gather_admitted_kernel", st);
-  gather_admitted_kernel<<<dim3((maxP + 7) / 8, p.H), 256, 0, st>>>(p);
+  gather_admitted_kernel<<<dim3(mover_blocks(maxP, p.row_bytes, p.H), p.H), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_evict_select(const AdmitPlan& p, cudaStream_t st) {
@@ -423,12 +420,12 @@ cudaError_t launch_evict_select(const AdmitPlan& p, cudaStream_t st) {
 }
 cudaError_t launch_gather_evicted(const AdmitPlan& p, cudaStream_t st) {
   LaunchTrace trace("gather_evicted_kernel", st);
-  gather_evicted_kernel<<<dim3((p.M + 7) / 8, p.H), 256, 0, st>>>(p);
+  gather_evicted_kernel<<<dim3(mover_blocks(p.M, p.row_bytes, p.H), p.H), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_compact(const AdmitPlan& p, cudaStream_t st) {
   LaunchTrace trace("compact_kernel", st);
-  compact_kernel<<<dim3((p.N + p.M + 7) / 8, p.H), 256, 0, st>>>(p);
+  compact_kernel<<<dim3(mover_blocks(p.N + p.M, p.row_bytes, p.H), p.H), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_finalize(const AdmitPlan& p, cudaStream_t st) {

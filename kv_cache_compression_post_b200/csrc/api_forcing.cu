@@ -72,6 +72,10 @@ extern "C" kvb_status kvb_prune_hybrid(kvb_bank* b, int32_t layer, const uint8_t
   if (g.method != KVB_FORCINGKV) return KVB_E_STATE;
   if (layer < 0 || layer >= g.layers || n_frames < 1 || n_frames > g.max_new_frames) return KVB_E_INVAL;
   if (!head_is_static || !newK || !newV || !nextK || !new_ids) return KVB_E_INVAL;
+  // rows are moved and read in 16-byte chunks
+  if (((reinterpret_cast<uintptr_t>(newK) | reinterpret_cast<uintptr_t>(newV) | reinterpret_cast<uintptr_t>(nextK)) &
+       15) != 0)
+    return KVB_E_INVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int H = g.heads;
   unsigned long long mask = 0;
@@ -177,6 +181,9 @@ extern "C" kvb_status kvb_segment_cosine(const void* K, const void* nextK, int32
   if (frame_h < 1 || frame_w < 1 || seg_h < 1 || seg_w < 1 || head_dim < 1 || head_dim > 1024) return KVB_E_INVAL;
   if (dtype != KVB_BF16 && dtype != KVB_F32) return KVB_E_INVAL;
   if (static_cast<size_t>(seg_h) * frame_w * sizeof(float) > 48 * 1024) return KVB_E_UNSUPPORTED;
+  const int esize = dtype == KVB_BF16 ? 2 : 4;
+  if ((head_dim * esize) % 16 != 0) return KVB_E_UNSUPPORTED;  // rows are read in 16-byte chunks
+  if (((reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(nextK)) & 15) != 0) return KVB_E_INVAL;
   const SegGeom sg = geom(frame_h, frame_w, seg_h, seg_w);
   return cuda_status(launch_seg_cosine(K, nextK, dtype, heads, n_frames, head_dim, sg, 0ull, sim,
                                        static_cast<cudaStream_t>(stream)));

@@ -22,8 +22,8 @@
 // instructions of one thread execute in issue order, so S_t(j) overwriting P_t
 // once PV_t(j-1) has been issued is safe.  The running max only moves when it
 // grows by more than 8 (log2 units); the O rescale (a TMEM read-modify-write) is
-// then rare and P stays below 2^8.  K and V stream through separate 2-stage TMA
-// rings, each fed by its own producer thread.
+// then rare and P stays below 2^8.  K and V stream through separate TMA
+// rings (2 stages each), each fed by its own producer thread.
 //
 // Warp roles: 0 Q/K producer, 1 MMA issuer, 2 TMEM owner, 3 V producer,
 // 4-7 softmax/epilogue of query tile A, 8-11 of query tile B.
@@ -51,10 +51,14 @@ constexpr int kW2 = 8;
 constexpr int kW1 = 7;
 // a CTA's share is at least this many key tiles of a two-tile unit
 constexpr int kMinTilesPerCta = 8;
+// K and V ring depths (a third K stage measured no faster: the loop is bound by
+// the tensor-core issue of its 128x128x16 MMAs, not by key-tile arrival)
+constexpr int kKStages = 2;
+constexpr int kVStages = 2;
 
 struct alignas(8) AttnBars {
   uint64_t q_full, q_empty;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2], o_full[2];  // per query tile
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -196,10 +200,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int d = a.d;
   const int nbox = d / 64;
   const uint32_t tileBytes = static_cast<uint32_t>(kTile) * d * 2;  // Q, K or V tile
-  uint8_t* sQ = smem;                // Q_A, Q_B
-  uint8_t* sK = sQ + 2 * tileBytes;  // 2 stages
-  uint8_t* sV = sK + 2 * tileBytes;  // 2 stages
-  AttnBars* bars = reinterpret_cast<AttnBars*>(sV + 2 * tileBytes);
+  uint8_t* sQ = smem;                        // Q_A, Q_B
+  uint8_t* sK = sQ + 2 * tileBytes;          // kKStages stages
+  uint8_t* sV = sK + kKStages * tileBytes;   // kVStages stages
+  AttnBars* bars = reinterpret_cast<AttnBars*>(sV + kVStages * tileBytes);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -232,11 +236,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kKStages; ++i) {
       mbar_init(&bars->k_full[i], 1);
       mbar_init(&bars->k_empty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
       mbar_init(&bars->v_full[i], 1);
       mbar_init(&bars->v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
       mbar_init(&bars->p_full[i], 4);
       mbar_init(&bars->o_full[i], 1);
@@ -268,8 +276,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = pc.j0; j < pc.j1; ++j) {
           int s, row, nv;
           tile_info(a, pc.h, j, s, row, nv);
-          const int st = g & 1;
-          if (!(ok = mbar_wait(&bars->k_empty[st], ((g >> 1) & 1) ^ 1, abort, a.status))) break;
+          const int st = g % kKStages;
+          if (!(ok = mbar_wait(&bars->k_empty[st], ((g / kKStages) & 1) ^ 1, abort, a.status))) break;
           mbar_arrive_expect_tx(&bars->k_full[st], tileBytes);
           for (int b = 0; b < nbox; ++b)
             tma_load_3d(sK + st * tileBytes + b * 16384, &maps.k[s], &bars->k_full[st], b * 64, row, pc.h);
@@ -289,7 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) {
         // let loads in flight land before the CTA exits
         if (np > 0) mbar_wait_drain(&bars->q_full, (np - 1) & 1, 200000000ull);
-        for (int i = max(0, g - 2); i < g; ++i) mbar_wait_drain(&bars->k_full[i & 1], (i >> 1) & 1, 200000000ull);
+        for (int i = max(0, g - kKStages); i < g; ++i)
+          mbar_wait_drain(&bars->k_full[i % kKStages], (i / kKStages) & 1, 200000000ull);
       }
     }
   } else if (warp == 3) {
@@ -304,8 +313,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = pc.j0; j < pc.j1; ++j) {
           int s, row, nv;
           tile_info(a, pc.h, j, s, row, nv);
-          const int st = g & 1;
-          if (!(ok = mbar_wait(&bars->v_empty[st], ((g >> 1) & 1) ^ 1, abort, a.status))) break;
+          const int st = g % kVStages;
+          if (!(ok = mbar_wait(&bars->v_empty[st], ((g / kVStages) & 1) ^ 1, abort, a.status))) break;
           mbar_arrive_expect_tx(&bars->v_full[st], tileBytes);
           for (int b = 0; b < nbox; ++b)
             tma_load_3d(sV + st * tileBytes + b * 16384, &maps.v[s], &bars->v_full[st], b * 64, row, pc.h);
@@ -313,7 +322,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok)
-        for (int i = max(0, g - 2); i < g; ++i) mbar_wait_drain(&bars->v_full[i & 1], (i >> 1) & 1, 200000000ull);
+        for (int i = max(0, g - kVStages); i < g; ++i)
+          mbar_wait_drain(&bars->v_full[i % kVStages], (i / kVStages) & 1, 200000000ull);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -341,16 +351,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = mbar_wait(&bars->q_full, np & 1, abort, a.status))) break;
         tc_fence_after();
         for (int j = pc.j0; j < pc.j1 && ok; ++j) {
-          const int kst = g & 1;
-          if (!(ok = mbar_wait(&bars->k_full[kst], (g >> 1) & 1, abort, a.status))) break;
-          if (j > pc.j0 && !(ok = mbar_wait(&bars->v_full[(g - 1) & 1], ((g - 1) >> 1) & 1, abort, a.status)))
+          const int kst = g % kKStages;
+          const int vprev = (g + kVStages - 1) % kVStages;  // V stage of tile g-1
+          if (!(ok = mbar_wait(&bars->k_full[kst], (g / kKStages) & 1, abort, a.status))) break;
+          if (j > pc.j0 && !(ok = mbar_wait(&bars->v_full[vprev], ((g - 1) / kVStages) & 1, abort, a.status)))
             break;
           tc_fence_after();
           for (int t = 0; t < pc.ntq; ++t) {
             if (j > pc.j0) {
               if (!(ok = mbar_wait(&bars->p_full[t], (ns[t] - 1) & 1, abort, a.status))) break;
               tc_fence_after();
-              pv(t, (g - 1) & 1, j - 1 == pc.j0);
+              pv(t, vprev, j - 1 == pc.j0);
             }
             for (int kk = 0; kk < d / 16; ++kk) {
               const uint32_t koff = static_cast<uint32_t>((kk >> 2) * 16384 + (kk & 3) * 32);
@@ -363,14 +374,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!ok) break;
           mma_commit(&bars->k_empty[kst]);
-          if (j > pc.j0) mma_commit(&bars->v_empty[(g - 1) & 1]);
+          if (j > pc.j0) mma_commit(&bars->v_empty[vprev]);
           if (j == pc.j1 - 1) mma_commit(&bars->q_empty);
           ++g;
         }
         if (!ok) break;
         // the last key tile's PV; then O of the piece is complete
-        const int vst = (g - 1) & 1;
-        if (!(ok = mbar_wait(&bars->v_full[vst], ((g - 1) >> 1) & 1, abort, a.status))) break;
+        const int vst = (g - 1) % kVStages;
+        if (!(ok = mbar_wait(&bars->v_full[vst], ((g - 1) / kVStages) & 1, abort, a.status))) break;
         for (int t = 0; t < pc.ntq && ok; ++t) {
           if (!(ok = mbar_wait(&bars->p_full[t], (ns[t] - 1) & 1, abort, a.status))) break;
           tc_fence_after();
@@ -682,7 +693,7 @@ __global__ void attend_f32_kernel(const AttnArgs a) {
 
 size_t attend_smem_bytes(int d) {
   const size_t tile = static_cast<size_t>(kTile) * d * 2;
-  return 1024 + 6 * tile + kBarBytes;  // Q_A, Q_B, 2 K stages, 2 V stages, barriers
+  return 1024 + (2 + kKStages + kVStages) * tile + kBarBytes;  // Q_A, Q_B, K and V rings, barriers
 }
 
 cudaError_t launch_attend_bf16(const AttnArgs& a, cudaStream_t st) {

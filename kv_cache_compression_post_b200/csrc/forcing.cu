@@ -10,7 +10,8 @@
 //                tokens row-major inside each; the frame is pushed into a FIFO of
 //                hist_frames frames stored as a token ring (the oldest frame is
 //                dropped when the FIFO is full); emits (source row, ring slot)
-//   prune_gather one warp per kept token: K, V rows and the id into the ring
+//   prune_gather kept tokens' K, V rows and ids into the ring (lane groups of 16
+//                bytes per lane, grid-strided)
 //   static_copy  static heads: the last new frame becomes the transition frame
 #include <cuda_bf16.h>
 
@@ -21,6 +22,36 @@
 namespace kvb {
 namespace {
 
+// Sum over the `width` lanes of an aligned lane group (width a power of two <= 32).
+__device__ __forceinline__ float group_sum(float v, int width) {
+  for (int o = width >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ void acc_words(uint4 a, uint4 b, float& dot, float& na, float& nb, __nv_bfloat16) {
+  const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float xl = __uint_as_float(wa[k] << 16), xh = __uint_as_float(wa[k] & 0xFFFF0000u);
+    const float yl = __uint_as_float(wb[k] << 16), yh = __uint_as_float(wb[k] & 0xFFFF0000u);
+    dot = fmaf(xl, yl, fmaf(xh, yh, dot));
+    na = fmaf(xl, xl, fmaf(xh, xh, na));
+    nb = fmaf(yl, yl, fmaf(yh, yh, nb));
+  }
+}
+__device__ __forceinline__ void acc_words(uint4 a, uint4 b, float& dot, float& na, float& nb, float) {
+  const float xa[4] = {__uint_as_float(a.x), __uint_as_float(a.y), __uint_as_float(a.z), __uint_as_float(a.w)};
+  const float xb[4] = {__uint_as_float(b.x), __uint_as_float(b.y), __uint_as_float(b.z), __uint_as_float(b.w)};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    dot = fmaf(xa[k], xb[k], dot);
+    na = fmaf(xa[k], xa[k], na);
+    nb = fmaf(xb[k], xb[k], nb);
+  }
+}
+
+// One CTA per (row of segments, frame, head).  A token's two rows are read by a
+// group of L lanes with 16-byte loads (L = row bytes / 16, at most 32), so a warp
+// covers 32/L tokens at once, two rounds in flight per iteration.
 template <typename T>
 __global__ void seg_cosine_kernel(const T* __restrict__ K, const T* __restrict__ nextK, int n_frames, int d,
                                   SegGeom g, unsigned long long skip_mask, float* __restrict__ sim, int ld_sim) {
@@ -30,25 +61,31 @@ __global__ void seg_cosine_kernel(const T* __restrict__ K, const T* __restrict__
   const int r0 = sr * g.seg_h;
   const int nrows = min(g.seg_h, g.frame_h - r0);
   const int ntok = nrows * g.frame_w;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int chunks = d * static_cast<int>(sizeof(T)) / 16;  // 16-byte chunks per row
+  const int L = chunks < 32 ? chunks : 32;                  // lanes per token
+  const int per_pass = blockDim.x / L;                       // tokens per pass of the CTA
+  const int slot = threadIdx.x / L, sub = threadIdx.x % L;
   const size_t Fd = static_cast<size_t>(g.F) * d;
   const T* base = K + static_cast<size_t>(h) * n_frames * Fd + static_cast<size_t>(t) * Fd;
   const T* succ = (t + 1 < n_frames) ? base + Fd : nextK + static_cast<size_t>(h) * Fd;
-  for (int i = warp; i < ntok; i += nw) {
-    const size_t p = static_cast<size_t>(r0 + i / g.frame_w) * g.frame_w + (i % g.frame_w);
-    const T* a = base + p * d;
-    const T* b = succ + p * d;
-    float dot = 0.f, na = 0.f, nb = 0.f;
-    for (int k = lane; k < d; k += 32) {
-      const float x = load_elem(a, k), y = load_elem(b, k);
-      dot = fmaf(x, y, dot);
-      na = fmaf(x, x, na);
-      nb = fmaf(y, y, nb);
+  const size_t first = static_cast<size_t>(r0) * g.frame_w;  // segment rows are contiguous tokens
+  for (int i0 = 0; i0 < ntok; i0 += 2 * per_pass) {
+    float dot[2] = {0.f, 0.f}, na[2] = {0.f, 0.f}, nb[2] = {0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = i0 + u * per_pass + slot;
+      if (i < ntok) {
+        const uint4* a = reinterpret_cast<const uint4*>(base + (first + i) * d);
+        const uint4* b = reinterpret_cast<const uint4*>(succ + (first + i) * d);
+        for (int c = sub; c < chunks; c += L) acc_words(__ldg(a + c), __ldg(b + c), dot[u], na[u], nb[u], T());
+      }
     }
-    dot = warp_sum(dot);
-    na = warp_sum(na);
-    nb = warp_sum(nb);
-    if (lane == 0) cosv[i] = dot / fmaxf(sqrtf(na) * sqrtf(nb), 1e-8f);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float dd = group_sum(dot[u], L), aa = group_sum(na[u], L), bb = group_sum(nb[u], L);
+      const int i = i0 + u * per_pass + slot;
+      if (sub == 0 && i < ntok) cosv[i] = dd / fmaxf(sqrtf(aa) * sqrtf(bb), 1e-8f);
+    }
   }
   __syncthreads();
   for (int sc = threadIdx.x; sc < g.seg_cols; sc += blockDim.x) {
@@ -62,13 +99,47 @@ __global__ void seg_cosine_kernel(const T* __restrict__ K, const T* __restrict__
 }
 
 constexpr int kPlanThreads = 256;
+constexpr int kPlanMaxSeg = 1024;
+
+// Exclusive scan of two ints over the CTA (kPlanThreads threads); returns the
+// totals through *ta / *tb.
+__device__ __forceinline__ int2 plan_scan2(int a, int b, int2* warp_tot, int* ta, int* tb) {
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  int ia = a, ib = b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int xa = __shfl_up_sync(0xffffffffu, ia, o), xb = __shfl_up_sync(0xffffffffu, ib, o);
+    if (l >= o) {
+      ia += xa;
+      ib += xb;
+    }
+  }
+  if (l == 31) warp_tot[w] = make_int2(ia, ib);
+  __syncthreads();
+  int oa = 0, ob = 0, sa = 0, sb = 0;
+  for (int k = 0; k < kPlanThreads / 32; ++k) {
+    const int2 v = warp_tot[k];
+    if (k < w) {
+      oa += v.x;
+      ob += v.y;
+    }
+    sa += v.x;
+    sb += v.y;
+  }
+  *ta = sa;
+  *tb = sb;
+  __syncthreads();  // warp_tot may be reused right after
+  return make_int2(oa + ia - a, ob + ib - b);
+}
 
 __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePlan p) {
-  __shared__ int s_kept[1024];   // kept segments of the current frame, ascending
-  __shared__ int s_off[1025];    // token offset of each kept segment
-  __shared__ int s_flag[1024];
+  __shared__ float s_sim[kPlanMaxSeg];
+  __shared__ int s_tok[kPlanMaxSeg + 1];  // token offset of each segment (segment-major list)
+  __shared__ int s_kept[kPlanMaxSeg];     // kept segments of the current frame, ascending
+  __shared__ int s_off[kPlanMaxSeg + 1];  // token offset of each kept segment in the frame
+  __shared__ int2 s_wtot[kPlanThreads / 32];
   __shared__ int s_state[4];
-  __shared__ int s_fs, s_cnt, s_total;
+  __shared__ int s_fs, s_total;
   const int h = blockIdx.x;
   const bool is_static = (p.static_mask >> h) & 1ull;
   const int n_seg = p.g.n_seg;
@@ -85,39 +156,52 @@ __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePla
     }
     return;
   }
-  if (n_seg > 1024) {
+  if (n_seg > kPlanMaxSeg) {
     if (threadIdx.x == 0) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
     return;
   }
   if (threadIdx.x < 4) s_state[threadIdx.x] = rs[threadIdx.x];
   if (threadIdx.x == 0) s_total = 0;
-  __syncthreads();
+  for (int j = threadIdx.x; j <= n_seg; j += blockDim.x) s_tok[j] = p.seg_tok[j];
   int* plan = p.plan + static_cast<size_t>(h) * p.ld_plan * 2;
+  // each thread owns a run of consecutive segments (for the ordered scans)
+  const int per = (n_seg + kPlanThreads - 1) / kPlanThreads;
+  const int j0 = threadIdx.x * per, j1 = min(n_seg, j0 + per);
   for (int t = 0; t < p.n_frames; ++t) {
-    const float* s = p.sims + static_cast<size_t>(h) * p.ld_sims + static_cast<size_t>(t) * n_seg;
+    const float* sg = p.sims + static_cast<size_t>(h) * p.ld_sims + static_cast<size_t>(t) * n_seg;
+    for (int j = threadIdx.x; j < n_seg; j += blockDim.x) s_sim[j] = sg[j];
+    __syncthreads();
     // BottomK: segment j is kept iff fewer than `keep` segments precede it in
     // (similarity ascending, index ascending) order
-    for (int j = threadIdx.x; j < n_seg; j += blockDim.x) {
-      const float sj = s[j];
+    int nk = 0, ntok = 0;
+    unsigned int kept_bits = 0;  // per <= 32 segments per thread
+    for (int j = j0; j < j1; ++j) {
+      const float sj = s_sim[j];
       int rank = 0;
       for (int i = 0; i < n_seg; ++i) {
-        const float si = s[i];
+        const float si = s_sim[i];
         rank += (si < sj) || (si == sj && i < j);
       }
-      s_flag[j] = rank < p.keep ? 1 : 0;
+      if (rank < p.keep) {
+        kept_bits |= 1u << (j - j0);
+        ++nk;
+        ntok += s_tok[j + 1] - s_tok[j];
+      }
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int q = 0, off = 0;
-      for (int j = 0; j < n_seg; ++j) {
-        if (!s_flag[j]) continue;
+    int tot_k, tot_tok;
+    const int2 pos = plan_scan2(nk, ntok, s_wtot, &tot_k, &tot_tok);
+    {
+      int q = pos.x, off = pos.y;
+      for (int j = j0; j < j1; ++j) {
+        if (!((kept_bits >> (j - j0)) & 1u)) continue;
         s_kept[q] = j;
         s_off[q] = off;
-        off += p.seg_tok[j + 1] - p.seg_tok[j];
+        off += s_tok[j + 1] - s_tok[j];
         ++q;
       }
-      s_off[q] = off;
-      s_cnt = off;
+    }
+    if (threadIdx.x == 0) {
+      s_off[tot_k] = tot_tok;
       // FIFO: drop the oldest frame when full, then append this one
       int first = s_state[0], held = s_state[1], tstart = s_state[2], theld = s_state[3];
       if (held == p.hist_frames) {
@@ -130,30 +214,35 @@ __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePla
       const int slot = (first + held) % p.hist_frames;
       s_fs = (tstart + theld) % p.ring_cap;
       p.fstart[h * p.hist_frames + slot] = s_fs;
-      p.fcount[h * p.hist_frames + slot] = off;
+      p.fcount[h * p.hist_frames + slot] = tot_tok;
       s_state[0] = first;
       s_state[1] = held + 1;
       s_state[2] = tstart;
-      s_state[3] = theld + off;
-      for (int k = 0; k < q; ++k) p.keep_list[static_cast<size_t>(h) * p.ld_sims + t * n_seg + k] = s_kept[k];
+      s_state[3] = theld + tot_tok;
     }
     __syncthreads();
-    // plan entries of this frame: kept segment q, token m of it
-    const int nk = p.keep;
+    for (int k = threadIdx.x; k < tot_k; k += blockDim.x)
+      p.keep_list[static_cast<size_t>(h) * p.ld_sims + t * n_seg + k] = s_kept[k];
+    // plan entries of this frame: entry e lies in kept segment q with
+    // s_off[q] <= e < s_off[q + 1] (binary search)
     const int base = s_total;
-    for (int q = 0; q < nk; ++q) {
-      const int j = s_kept[q];
-      const int t0 = p.seg_tok[j], t1 = p.seg_tok[j + 1];
-      for (int m = threadIdx.x; m < t1 - t0; m += blockDim.x) {
-        const int e = base + s_off[q] + m;
-        if (e < p.ld_plan) {
-          plan[2 * e] = t * p.g.F + p.seg_list[t0 + m];
-          plan[2 * e + 1] = (s_fs + s_off[q] + m) % p.ring_cap;
-        }
+    for (int e = threadIdx.x; e < tot_tok; e += blockDim.x) {
+      int lo = 0, hi = tot_k - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_off[mid] <= e) lo = mid;
+        else hi = mid - 1;
+      }
+      const int j = s_kept[lo];
+      const int m = e - s_off[lo];
+      const int g = base + e;
+      if (g < p.ld_plan) {
+        plan[2 * g] = t * p.g.F + p.seg_list[s_tok[j] + m];
+        plan[2 * g + 1] = (s_fs + e) % p.ring_cap;
       }
     }
     __syncthreads();
-    if (threadIdx.x == 0) s_total += s_cnt;
+    if (threadIdx.x == 0) s_total += tot_tok;
     __syncthreads();
   }
   if (threadIdx.x == 0) {
@@ -172,48 +261,44 @@ __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePla
   }
 }
 
-__device__ __forceinline__ void copy_row16(void* dst, const void* src, int row_bytes, int lane) {
-  const uint4* s = static_cast<const uint4*>(src);
-  uint4* d = static_cast<uint4*>(dst);
-  for (int o = lane; o < row_bytes / 16; o += 32) d[o] = s[o];
-}
-
 __global__ void prune_gather_kernel(const PrunePlan p) {
   const int h = blockIdx.y;
-  const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
   if ((p.static_mask >> h) & 1ull) return;
-  if (e >= min(p.plan_n[h], p.ld_plan)) return;
+  const RowGroup g = row_group(p.row_bytes);
+  const int n = min(p.plan_n[h], p.ld_plan);
   const int* plan = p.plan + static_cast<size_t>(h) * p.ld_plan * 2;
-  const int src = plan[2 * e], dst = plan[2 * e + 1];
-  if (src < 0 || src >= p.n_frames * p.g.F || dst < 0 || dst >= p.ring_cap) {
-    if (lane == 0) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
-    return;
+  for (int e = g.first; e < n; e += g.stride) {
+    const int src = plan[2 * e], dst = plan[2 * e + 1];
+    if (src < 0 || src >= p.n_frames * p.g.F || dst < 0 || dst >= p.ring_cap) {
+      if (g.sub == 0) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
+      continue;
+    }
+    const size_t s = static_cast<size_t>(h) * p.n_frames * p.g.F + src;
+    const size_t t = static_cast<size_t>(h) * p.ring_cap + dst;
+    copy_row(static_cast<char*>(p.rK) + t * p.row_bytes, static_cast<const char*>(p.newK) + s * p.row_bytes,
+             p.row_bytes, g);
+    copy_row(static_cast<char*>(p.rV) + t * p.row_bytes, static_cast<const char*>(p.newV) + s * p.row_bytes,
+             p.row_bytes, g);
+    if (g.sub == 0) p.rids[t] = p.new_ids[src];
   }
-  const size_t s = static_cast<size_t>(h) * p.n_frames * p.g.F + src;
-  const size_t t = static_cast<size_t>(h) * p.ring_cap + dst;
-  copy_row16(static_cast<char*>(p.rK) + t * p.row_bytes, static_cast<const char*>(p.newK) + s * p.row_bytes,
-             p.row_bytes, lane);
-  copy_row16(static_cast<char*>(p.rV) + t * p.row_bytes, static_cast<const char*>(p.newV) + s * p.row_bytes,
-             p.row_bytes, lane);
-  if (lane == 0) p.rids[t] = p.new_ids[src];
 }
 
 __global__ void static_copy_kernel(const PrunePlan p) {
   const int h = blockIdx.y;
-  const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (!((p.static_mask >> h) & 1ull) || i >= p.g.F) return;
-  const int src = (p.n_frames - 1) * p.g.F + i;
-  const size_t s = static_cast<size_t>(h) * p.n_frames * p.g.F + src;
-  const size_t t = static_cast<size_t>(h) * p.g.F + i;
-  copy_row16(static_cast<char*>(p.tK) + t * p.row_bytes, static_cast<const char*>(p.newK) + s * p.row_bytes,
-             p.row_bytes, lane);
-  copy_row16(static_cast<char*>(p.tV) + t * p.row_bytes, static_cast<const char*>(p.newV) + s * p.row_bytes,
-             p.row_bytes, lane);
-  if (lane == 0) {
-    p.tids[t] = p.new_ids[src];
-    if (i == 0) p.tlen[h] = p.g.F;
+  if (!((p.static_mask >> h) & 1ull)) return;
+  const RowGroup g = row_group(p.row_bytes);
+  for (int i = g.first; i < p.g.F; i += g.stride) {
+    const int src = (p.n_frames - 1) * p.g.F + i;
+    const size_t s = static_cast<size_t>(h) * p.n_frames * p.g.F + src;
+    const size_t t = static_cast<size_t>(h) * p.g.F + i;
+    copy_row(static_cast<char*>(p.tK) + t * p.row_bytes, static_cast<const char*>(p.newK) + s * p.row_bytes,
+             p.row_bytes, g);
+    copy_row(static_cast<char*>(p.tV) + t * p.row_bytes, static_cast<const char*>(p.newV) + s * p.row_bytes,
+             p.row_bytes, g);
+    if (g.sub == 0) {
+      p.tids[t] = p.new_ids[src];
+      if (i == 0) p.tlen[h] = p.g.F;
+    }
   }
 }
 
@@ -249,13 +334,13 @@ cudaError_t launch_prune_plan(const PrunePlan& p, cudaStream_t st) {
 
 cudaError_t launch_prune_gather(const PrunePlan& p, cudaStream_t st) {
   LaunchTrace trace("prune_gather_kernel", st);
-  prune_gather_kernel<<<dim3((p.ld_plan + 7) / 8, p.H), 256, 0, st>>>(p);
+  prune_gather_kernel<<<dim3(mover_blocks(p.ld_plan, p.row_bytes, p.H), p.H), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_static_copy(const PrunePlan& p, cudaStream_t st) {
   LaunchTrace trace("static_copy_kernel", st);
-  static_copy_kernel<<<dim3((p.g.F + 7) / 8, p.H), 256, 0, st>>>(p);
+  static_copy_kernel<<<dim3(mover_blocks(p.g.F, p.row_bytes, p.H), p.H), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -45,6 +45,17 @@ class LaunchTrace {
   int slot_ = -1;
 };
 
+// CTAs per head of a row-moving kernel (256 threads, row_group lanes per row):
+// enough for `rows` rows, capped so that the grid stays near one wave (about
+// 1024 CTAs over all heads).
+inline int mover_blocks(int rows, int row_bytes, int H) {
+  const int words = row_bytes / 16;
+  const int per_cta = 256 / (words < 32 ? words : 32);
+  const int need = (rows + per_cta - 1) / per_cta;
+  const int cap = 1024 / (H > 0 ? H : 1);
+  return need < 1 ? 1 : (need < cap ? need : (cap < 1 ? 1 : cap));
+}
+
 inline kvb_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVB_OK : KVB_E_CUDA; }
 
 // Bump allocation inside a caller workspace, 256-byte aligned pieces.

@@ -33,4 +33,27 @@ __device__ __forceinline__ int warp_sum_int(int v) {
   return v;
 }
 
+// Rows are moved by groups of L = min(32, row_bytes / 16) lanes, one 16-byte
+// word per lane per step: a warp moves 32/L rows at once, and each group strides
+// over the rows of its head (row_bytes a multiple of 16 and L a power of two:
+// 128, 256 or 512-byte rows).
+struct RowGroup {
+  int L, sub, first, stride;
+};
+__device__ __forceinline__ RowGroup row_group(int row_bytes) {
+  RowGroup g;
+  const int words = row_bytes / 16;
+  g.L = words < 32 ? words : 32;
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  g.sub = t % g.L;
+  g.first = t / g.L;
+  g.stride = gridDim.x * blockDim.x / g.L;
+  return g;
+}
+__device__ __forceinline__ void copy_row(void* dst, const void* src, int row_bytes, const RowGroup& g) {
+  const uint4* s = static_cast<const uint4*>(src);
+  uint4* d = static_cast<uint4*>(dst);
+  for (int o = g.sub; o < row_bytes / 16; o += g.L) d[o] = s[o];
+}
+
 }  // namespace kvb
