@@ -188,6 +188,14 @@ def _cfg(w, kvb):
                            sync_heads=1, max_queries=w.chunk_tokens)
 
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
+# ncu captures summarised under profiles/, by (workload, kernel); valid only for
+# the kernel versions those files name.
+DRAM_TRAFFIC = {
+    # the four density passes of one 480P admit: 54.12 + 54.13 + 54.71 + 18.16 MB
+    ("wan480", "gram_bf16_kernel"): (181.12e6 / 4, "profiles/gram_bf16_kernel_wan480.md"),
+}
+
 # first timed chunk: steady state (DensityKV bank full; Forcing-KV ring of 21 frames full)
 FIRST_TIMED = {"wan480": 19, "wan1080": 9, "mid": 4, "tiny": 4, "forcing480": 8, "forcing_mid": 4}
 
@@ -424,8 +432,10 @@ def run_workload(args, w, rank, world):
     bf16_peak = peaks["bf16_tflops"]
 
     def roof_of(k):
+        tr = DRAM_TRAFFIC.get((w.name, k["kernel"]))
         r = {"bound": k["bound"], "achieved": k.get("achieved"), "peak": k.get("peak"), "unit": k.get("unit"),
-             "frac": k.get("frac"), "traffic": None, "kernel": k["kernel"],
+             "frac": k.get("frac"), "traffic": round(tr[0]) if tr else None,
+             "traffic_source": tr[1] if tr else None, "kernel": k["kernel"],
              "launches_per_step": k["launches_per_step"], "ms_per_launch": k["ms_per_launch"],
              "peak_source": f"{peak_src} " + ("bf16 burst" if k["bound"] == "tensor" else "HBM copy"),
              "algorithmic": k["algorithmic"]}
