@@ -2,7 +2,7 @@
 """Benchmark of the KV-bank hot path: ms per chunk-layer (bank update + history
 attention) on synthetic Wan2.1-1.3B-shaped data.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan480|wan1080|forcing480|mid|tiny]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan480|wan1080|forcing480|rollout|mid|tiny]
                     [--impl kvb|reference]
 
 A step is one chunk-layer of the streaming rollout: one DensityKV kvb_admit of
@@ -477,6 +477,68 @@ def run_workload(args, w, rank, world):
     }
 
 
+def run_rollout(args, w, rank, world):
+    """The full streaming rollout: every chunk i = 1..n_chunks-1 runs kvb_admit +
+    kvb_attend at each of the workload's layers (one bank holds all layers), with
+    inputs drawn on the GPU (kvgen.gpu) between the timed calls.  Each chunk-layer
+    is timed with CUDA events around its two calls; the banks of 30 layers (2 GB)
+    are far larger than L2, so every chunk-layer starts cold on its own bank."""
+    import torch
+    import kv_cache_compression_post_b200 as kvb
+    from kvgen.gpu import GpuLayerStream
+    dev = torch.cuda.current_device()
+    cfg = _cfg(w, kvb)
+    cfg.layers = w.layers
+    bank = kvb.Bank(cfg)
+    streams = [GpuLayerStream(w, l, seed=rank) for l in range(w.layers)]
+    stream = torch.cuda.current_stream()
+    O = torch.empty(w.heads, w.chunk_tokens, w.head_dim, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(w.heads, w.chunk_tokens, device="cuda")
+    sampler = ClockSampler(dev)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    rows = []   # (chunk, layer, admit ms, attend ms, attention flops)
+    launches0 = kvb.kvb_launch_count()
+    for i in range(1, w.n_chunks):
+        ev = []
+        for l in range(w.layers):
+            x = streams[l].step(i)
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            e[0].record(stream)
+            bank.admit(l, x["candK"], x["candV"], x["cand_ids"], stream)
+            e[1].record(stream)
+            bank.attend(l, x["Q"], x["sinkK"], x["sinkV"], x["winK"], x["winV"], O, lse, stream)
+            e[2].record(stream)
+            ev.append(e)
+        torch.cuda.synchronize()
+        for l, e in enumerate(ev):
+            sizes = [st["size"] for st in bank.stats(l)] if i % 10 == 0 or i < 5 else None
+            rows.append((i, l, e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]),
+                         attention_flops(w, sizes) if sizes else None))
+    launches = kvb.kvb_launch_count() - launches0
+    clocks = sampler.stop()
+    status = bank.status()
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+    per = np.array([a + b for _, _, a, b, _ in rows])
+    steady = [(a, b, f) for i, _, a, b, f in rows if i >= 4]
+    att_fl = [(b, f) for a, b, f in steady if f]
+    total_ms = max_over_ranks(float(per.sum()), world)
+    return {
+        "ms_per_step": float(per.mean()),
+        "dist": {"chunk_layers": int(per.size), "total_ms": round(total_ms, 2), "mean_ms": round(float(per.mean()), 4),
+                 "p50_ms": round(float(np.percentile(per, 50)), 4), "p90_ms": round(float(np.percentile(per, 90)), 4),
+                 "max_ms": round(float(per.max()), 4),
+                 "steady_mean_ms (chunks >= 4)": round(float(np.mean([a + b for a, b, _ in steady])), 4)},
+        "breakdown": {"admit_ms": round(float(np.mean([a for a, _, _ in steady])), 4),
+                      "attend_ms": round(float(np.mean([b for _, b, _ in steady])), 4),
+                      "attend_tflops": round(float(np.mean([f / (b * 1e-3) for b, f in att_fl])) / 1e12, 1)
+                      if att_fl else None},
+        "clocks": clocks, "launches": launches,
+    }
+
+
 # ------------------------------------------------------------------ oracle (CPU) leg
 def oracle_sample(w, reps: int = 1):
     """Time the fp64 oracle on a bounded, stated sample of one 480P chunk-layer and
@@ -599,6 +661,31 @@ def run_reference(args, w, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def print_rollout(args, w, r, world):
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        ms, sample, (cores, blas) = cpu_sample(w, reps=1)
+        cpu = {"value": round(ms, 3), "unit": UNIT, "cores": cores, "blas_threads": blas, "kind": "oracle",
+               "sample": sample}
+    line = {
+        "metric": METRIC, "value": round(r["ms_per_step"], 4), "unit": UNIT, "n_gpus": world,
+        "steps": r["dist"]["chunk_layers"], "warmup": 0, "ms_per_step": round(r["ms_per_step"], 4),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (GPU generator)",
+        "config": {"workload": (f"rollout: {w.layers} layers x {w.n_chunks} chunks (every chunk-layer from chunk 1), "
+                                f"DensityKV admit + attention, {w.heads} heads, d={w.head_dim}, F={w.F}, "
+                                f"M={w.capacity}, background rows 0..{w.background_rows - 1} at a={w.ar_a_bg}, "
+                                f"others at a={w.ar_a_fg}"),
+                   "heads": w.heads, "head_dim": w.head_dim, "F": w.F, "N": w.chunk_tokens, "M": w.capacity,
+                   "layers": w.layers, "chunks": w.n_chunks, "parallelism": f"replicas x{world}",
+                   "l2": "not flushed: 30 layers' banks (2 GB) exceed L2; inputs are generated on the GPU between "
+                         "chunk-layers"},
+        "distribution": r["dist"], "breakdown": r["breakdown"], "gpu_launches": r["launches"],
+        "e2e": None, "roofline": None, "clocks": r["clocks"], "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def workload_config(w, args, world):
     first = FIRST_TIMED.get(w.name, 4) + args.warmup
     chunks = f"chunks {first}..{first + args.steps - 1}"
@@ -637,6 +724,11 @@ def main():
         return
     import torch
     torch.cuda.set_device(local)
+    if w.name == "rollout":
+        r = run_rollout(args, w, rank, world)
+        if rank == 0:
+            print_rollout(args, w, r, world)
+        return
     r = run_workload(args, w, rank, world)
     if rank != 0:
         return

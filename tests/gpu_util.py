@@ -29,14 +29,98 @@ def aligned_ptr(buf):
     return (p + 255) & ~255
 
 
-def import_oracle_banks(bank, banks, params, w, layer=0):
-    """Load oracle HeadBanks (with from-scratch densities) into a GPU bank."""
+def import_oracle_banks(bank, banks, params, w, layer=0, densities=True):
+    """Load oracle HeadBanks into a GPU bank, with from-scratch densities (or, for
+    callers that only attend over the bank, with rho = rho0)."""
     import torch
     from oracle import densitykv as dkv
     for hh, b in enumerate(banks):
         if b.size == 0:
             bank.import_(layer, hh, torch.zeros(0, dtype=torch.int32, device="cuda"), None, None, None, None)
             continue
-        rho = dkv.densities_from_scratch(b, params)
+        rho = dkv.densities_from_scratch(b, params) if densities else b.rho0
         bank.import_(layer, hh, dev_ids(b.ids), dev_tensor(rho, "f32"), dev_tensor(b.rho0, "f32"),
                      dev_tensor(b.K, w.dtype), dev_tensor(b.V, w.dtype))
+
+
+def export_banks(bank, layer, H):
+    """Host copies (ids, rho, rho0, K, V as numpy) of every head's bank of a layer."""
+    out = []
+    for hh in range(H):
+        ids, rho, rho0, K, V = bank.export(layer, hh)
+        out.append(dict(ids=host(ids).astype(np.int64), rho=host(rho).astype(np.float64),
+                        rho0=host(rho0).astype(np.float64), K=host(K), V=host(V)))
+    return out
+
+
+def check_admit_sampled(w, pre, post, stats, cand_ids, candK, rng, rtol=1e-4, n=12):
+    """One GPU admit step at any size, checked on sampled outputs the oracle
+    computes one by one and on the rule's invariants (DensityKV §3, App. B.1):
+    * sizes <= M, the same admitted count P on every head, K/V pairing by id;
+    * rho of sampled entries of the new bank = from-scratch oracle density within
+      rtol; new entries have rho0 = rho, survivors keep their rho0;
+    * admitted candidates precede rejected ones in (score, id) order, and are all
+      feasible when every candidate is admitted;
+    * survivors have projected ratio <= tau, and every evicted entry has a ratio
+      at least every survivor's (mandatory ones above tau, capacity ones next).
+    pre / post: export_banks before / after the step; candK [H][N][d] (host or
+    torch); cand_ids [N]."""
+    import kvgen
+    from oracle.density import density
+    H = len(post)
+    kw = dict(h=float(w.head_dim), eps=w.eps, s=w.s)
+    cand_ids = np.asarray(host(cand_ids) if hasattr(cand_ids, "cpu") else cand_ids, np.int64)
+    cK = np.asarray(host(candK) if hasattr(candK, "cpu") else candK, np.float64)
+    cid_pos = {int(c): k for k, c in enumerate(cand_ids)}
+    assert len({s["admitted"] for s in stats}) == 1
+    for hh in range(H):
+        b0, b1 = pre[hh], post[hh]
+        assert b0["ids"].size <= w.capacity and b1["ids"].size <= w.capacity
+        assert (kvgen.untag_ids(b1["V"]) == b1["ids"]).all()
+        pre_pos = {int(v): k for k, v in enumerate(b0["ids"])}
+        adm = np.array([k for k, v in enumerate(b1["ids"]) if int(v) in cid_pos], np.int64)
+        surv = np.array([k for k, v in enumerate(b1["ids"]) if int(v) in pre_pos], np.int64)
+        assert adm.size == stats[hh]["admitted"] and adm.size + surv.size == b1["ids"].size
+        evicted = np.array(sorted(set(pre_pos) - set(b1["ids"].tolist())), np.int64)
+        # densities of sampled new-bank entries, from scratch
+        smp = np.sort(rng.choice(b1["ids"].size, min(n, b1["ids"].size), replace=False))
+        ref = density(b1["K"][smp], b1["K"], row_ids=b1["ids"][smp], col_ids=b1["ids"], **kw)
+        np.testing.assert_allclose(b1["rho"][smp], ref, rtol=rtol)
+        np.testing.assert_array_equal(b1["rho0"][adm], b1["rho"][adm])
+        np.testing.assert_array_equal(b1["rho0"][surv], b0["rho0"][[pre_pos[int(v)] for v in b1["ids"][surv]]])
+        if b0["ids"].size == 0:
+            continue
+        # admission order on sampled candidates (scores against the pre-step bank)
+        mean0 = float(np.mean(b0["rho0"]))
+        a_ids = sorted(set(b1["ids"][adm].tolist()))
+        r_all = sorted(set(cand_ids.tolist()) - set(a_ids))
+
+        def score(ids_):
+            rows = cK[hh][[cid_pos[int(c)] for c in ids_]]
+            return density(rows, b0["K"], row_ids=np.asarray(ids_), col_ids=b0["ids"], **kw) / mean0
+
+        if a_ids:
+            sa = score(rng.choice(a_ids, min(n, len(a_ids)), replace=False))
+            if r_all:
+                sr = score(rng.choice(r_all, min(n, len(r_all)), replace=False))
+                assert sa.max() <= sr.min() * (1 + rtol)
+            else:
+                assert sa.max() <= w.tau * (1 + rtol)   # every candidate of every head was feasible
+        # eviction rule on sampled survivors and evicted entries
+        A_rows = cK[hh][[cid_pos[int(c)] for c in a_ids]]
+        A_ids = np.asarray(a_ids, np.int64)
+
+        def ratio(ids_):
+            k = [pre_pos[int(v)] for v in ids_]
+            rows = b0["K"][k]
+            rh = density(rows, b0["K"], row_ids=np.asarray(ids_), col_ids=b0["ids"], **kw)
+            if A_ids.size:
+                rh = rh + density(rows, A_rows, row_ids=np.asarray(ids_), col_ids=A_ids, **kw)
+            return rh / b0["rho0"][k]
+
+        if surv.size:
+            rs = ratio(rng.choice(b1["ids"][surv], min(n, surv.size), replace=False))
+            assert rs.max() <= w.tau * (1 + rtol)
+            if evicted.size:
+                re_ = ratio(rng.choice(evicted, min(n, evicted.size), replace=False))
+                assert re_.min() >= rs.max() * (1 - rtol)

@@ -88,11 +88,13 @@ def test_attend_ragged_bank_sizes_and_no_sink(bank_size):
     bank.close()
 
 
-def test_attend_full_size_sampled_rows():
-    """480P shapes: 4680 queries over 1560 sink + 9360 bank + 4680 window keys."""
+@pytest.mark.parametrize("name,H", [("wan480", 4), ("wan1080", 1)])
+def test_attend_full_size_sampled_rows(name, H):
+    """480P shapes: 4680 queries over 1560 sink + 9360 bank + 4680 window keys;
+    1080P: 24480 queries over 8160 + 32640 + 24480 keys.  Fewer heads keep the
+    host-side generation short; the shapes per head are full size."""
     import kv_cache_compression_post_b200 as kvb
-    w = kvgen.WORKLOADS["wan480"]
-    H = 4  # four heads keep the host-side generation short; shapes per head are full size
+    w = kvgen.WORKLOADS[name]
     L = kvgen.LayerInputs(w, 0, n_chunks=5, heads=range(H))
     x = L.step(4)
     rng = np.random.default_rng(1)
@@ -106,7 +108,7 @@ def test_attend_full_size_sampled_rows():
     cfg = kvb.make_config(method=kvb.KVB_DENSITYKV, dtype=kvb.KVB_BF16, heads=H, head_dim=w.head_dim,
                           capacity=w.capacity, max_candidates=w.chunk_tokens, max_queries=w.chunk_tokens)
     bank = kvb.Bank(cfg)
-    import_oracle_banks(bank, banks, dkv.Params(capacity=w.capacity), w)
+    import_oracle_banks(bank, banks, dkv.Params(capacity=w.capacity), w, densities=False)  # attention reads K, V only
     kvb.kvb_trace_enable(True)
     O, lse = _attend(bank, w, x)
     trace = kvb.kvb_trace_read()

@@ -14,7 +14,7 @@ import pytest
 
 import kvgen
 from oracle import densitykv as dkv
-from tests.gpu_util import dev_ids, dev_tensor, host
+from tests.gpu_util import check_admit_sampled, dev_ids, dev_tensor, export_banks, host
 
 pytestmark = pytest.mark.gpu
 
@@ -30,12 +30,7 @@ def _cfg(w, tau=None, sync=1, layers=1):
 
 
 def _export(bank, layer, H):
-    out = []
-    for hh in range(H):
-        ids, rho, rho0, K, V = bank.export(layer, hh)
-        out.append(dict(ids=host(ids).astype(np.int64), rho=host(rho).astype(np.float64),
-                        rho0=host(rho0).astype(np.float64), K=host(K), V=host(V)))
-    return out
+    return export_banks(bank, layer, H)
 
 
 def _compare(g, r, hh, exact=True, tie_ids=frozenset()):
@@ -142,4 +137,30 @@ def test_admit_argument_errors():
     with pytest.raises(kvb.KvbError) as e:
         kvb.kvb_prune_hybrid(bank.handle, 0, bytes(w.heads), K, K, K, ids, 1)  # wrong method
     assert e.value.status in (6, 7)
+    bank.close()
+
+
+@pytest.mark.parametrize("name,H,steps", [("wan480", 2, 4), ("wan1080", 1, 3)])
+def test_full_size_step_sampled(name, H, steps):
+    """Full 480P / 1080P sizes (fewer heads): the GPU runs the rollout from an empty
+    bank; the last step (bank full, evictions) is checked on sampled outputs the
+    oracle computes one by one and on the rule's invariants (check_admit_sampled)."""
+    import dataclasses
+    import torch
+    import kv_cache_compression_post_b200 as kvb
+    w = kvgen.WORKLOADS[name]
+    L = kvgen.LayerInputs(w, 0, n_chunks=steps + 2, tagged=True, heads=range(H))
+    bank = kvb.Bank(_cfg(dataclasses.replace(w, heads=H)))
+    for i in range(1, steps):
+        x = L.step(i)
+        bank.admit(0, dev_tensor(x["candK"], w.dtype), dev_tensor(x["candV"], w.dtype), dev_ids(x["cand_ids"]))
+    torch.cuda.synchronize()
+    assert bank.status() == 0
+    pre = export_banks(bank, 0, H)
+    x = L.step(steps)
+    bank.admit(0, dev_tensor(x["candK"], w.dtype), dev_tensor(x["candV"], w.dtype), dev_ids(x["cand_ids"]))
+    torch.cuda.synchronize()
+    assert bank.status() == 0
+    check_admit_sampled(w, pre, export_banks(bank, 0, H), bank.stats(0), x["cand_ids"], x["candK"],
+                        np.random.default_rng(7))
     bank.close()
