@@ -120,6 +120,13 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ distributed
+def dist_backend() -> str:
+    """NCCL on GPUs; gloo where CUDA is absent (CPU tests of the multi-rank path) or
+    when KVB_DIST_BACKEND says so."""
+    import torch
+    return os.environ.get("KVB_DIST_BACKEND") or ("nccl" if torch.cuda.is_available() else "gloo")
+
+
 def dist_init():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -128,8 +135,10 @@ def dist_init():
         import datetime
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+        backend = dist_backend()
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
     return rank, world, local
 
 
@@ -140,11 +149,13 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of every rank's x (device times: the job ends with its slowest rank)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 

@@ -29,6 +29,8 @@ namespace kvb {
 namespace {
 
 constexpr int kSelThreads = 1024;
+// banks up to this many bytes of 64-bit keys keep them in shared memory
+constexpr size_t kEvictKeyBytes = 200 * 1024;
 
 struct SelShared {
   unsigned int hist[256];
@@ -241,8 +243,13 @@ __global__ void gather_admitted_kernel(const AdmitPlan p) {
   }
 }
 
+// SKEYS: every entry's 64-bit key is computed once into shared memory (the radix
+// passes then read 8 bytes of shared memory instead of recomputing the ratio);
+// mandatory evictions get the largest key, so the selection needs no flags.
+template <bool SKEYS>
 __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPlan p) {
   __shared__ SelShared S;
+  extern __shared__ unsigned long long s_key[];  // [n] (SKEYS)
   const int h = blockIdx.x;
   const int n = p.n_old[h];
   const int Ph = p.P[h];
@@ -256,19 +263,26 @@ __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPl
   // mandatory evictions: projected growth above tau
   int cnt = 0;
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const bool m = ratio(i) > p.tau;
+    const float r = ratio(i);
+    const bool m = r > p.tau;
     evflag[i] = m ? 1 : 0;
     cnt += m ? 1 : 0;
+    if (SKEYS)
+      s_key[i] = m ? ~0ull
+                   : (static_cast<unsigned long long>(~float_key(r)) << 32) | static_cast<unsigned int>(ids[i]);
   }
   int n_mand;
   block_excl_scan(cnt, &S, &n_mand);
   const int ecap = max(0, n - n_mand + Ph - p.M);
   const int n_free = n - n_mand;
   if (ecap > 0) {
+    // the key of an entry: ratio descending, then id ascending (ratios are >= 0, so
+    // no such key has the top byte 0xFF of the mandatory entries' key)
     auto key = [&](int i) -> unsigned long long {
+      if (SKEYS) return s_key[i];
       return (static_cast<unsigned long long>(~float_key(ratio(i))) << 32) | static_cast<unsigned int>(ids[i]);
     };
-    auto keep = [&](int i) { return evflag[i] == 0; };
+    auto keep = [&](int i) { return SKEYS || evflag[i] == 0; };
     if (ecap >= n_free) {
       for (int i = threadIdx.x; i < n; i += blockDim.x) evflag[i] = 1;
     } else {
@@ -414,8 +428,17 @@ cudaError_t launch_gather_admitted(const AdmitPlan& p, int maxP, cudaStream_t st
   return cudaGetLastError();
 }
 cudaError_t launch_evict_select(const AdmitPlan& p, cudaStream_t st) {
-  LaunchTrace trace("evict_select_kernel", st);
-  evict_select_kernel<<<p.H, kSelThreads, 0, st>>>(p);
+  const size_t keys = sizeof(unsigned long long) * static_cast<size_t>(p.M);
+  if (keys <= kEvictKeyBytes) {
+    cudaError_t e = cudaFuncSetAttribute(evict_select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(keys));
+    if (e != cudaSuccess) return e;
+    LaunchTrace trace("evict_select_kernel", st);
+    evict_select_kernel<true><<<p.H, kSelThreads, keys, st>>>(p);
+  } else {
+    LaunchTrace trace("evict_select_kernel", st);
+    evict_select_kernel<false><<<p.H, kSelThreads, 0, st>>>(p);
+  }
   return cudaGetLastError();
 }
 cudaError_t launch_gather_evicted(const AdmitPlan& p, cudaStream_t st) {

@@ -1,0 +1,48 @@
+"""The multi-rank plumbing of bench.py on CPU (gloo, world size 2): rendezvous on
+127.0.0.1, the barrier, and the max-over-ranks reduction that turns per-rank
+device times into the job's time.  Each rank runs an independent replica (the
+path shards by layer and head; there is no data exchange)."""
+import os
+import socket
+
+import pytest
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank), KVB_DIST_BACKEND="gloo")
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    import torch.distributed as dist
+    r, w, _ = bench.dist_init()
+    bench.barrier(w)
+    m = bench.max_over_ranks(1.5 * (r + 1), w)
+    bench.barrier(w)
+    out.put((r, w, m, dist.get_backend()))
+    dist.destroy_process_group()
+
+
+def test_two_rank_barrier_and_max_over_ranks():
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[0] for r in res] == [0, 1]
+    assert all(r[1] == 2 and r[3] == "gloo" for r in res)
+    assert all(r[2] == pytest.approx(3.0) for r in res)   # every rank sees the slowest rank's time
