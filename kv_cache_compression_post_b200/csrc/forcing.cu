@@ -3,8 +3,8 @@
 //
 //   seg_cosine   per dynamic head and new frame t: token-wise cosine between frame
 //                t and its successor at the same spatial position, averaged over
-//                each seg_h x seg_w segment (one CTA per row of segments, one
-//                warp per token, fixed-order segment sums)
+//                each seg_h x seg_w segment (one CTA per row of segments, a
+//                lane group of 16-byte loads per token, fixed-order segment sums)
 //   prune_plan   per dynamic head: per frame the BottomK(floor(r n)) least
 //                similar segments (ties: lower index), kept segments ascending,
 //                tokens row-major inside each; the frame is pushed into a FIFO of
