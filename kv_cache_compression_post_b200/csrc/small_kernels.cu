@@ -7,24 +7,6 @@
 namespace kvb {
 namespace {
 
-template <typename T>
-__global__ void row_terms_kernel(const T* __restrict__ X, long long ldX, int d, int n_uni, const int* n_dev,
-                                 float inv_h, float add, float* __restrict__ out, long long ldOut) {
-  const int h = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x * (blockDim.x >> 5) + warp;
-  const int n = n_dev ? n_dev[h] : n_uni;
-  if (r >= n) return;
-  const T* x = X + (static_cast<long long>(h) * ldX + r) * d;
-  float acc = 0.f;
-  for (int k = lane; k < d; k += 32) {
-    const float v = load_elem(x, k);
-    acc = fmaf(v, v, acc);
-  }
-  acc = warp_sum(acc);
-  if (lane == 0) out[static_cast<long long>(h) * ldOut + r] = fmaf(acc, inv_h, add);
-}
-
 // Rows are read by lane groups (row_group: 16-byte words, several rows per warp,
 // rows strided over the grid); the largest ||x||^2 seen by the CTA goes to
 // norm_max with a single atomic (per-row atomics on one word serialise).
@@ -106,19 +88,5 @@ cudaError_t launch_aug_rows(const void* X, kvb_dtype dtype, int H, long long ldX
   return cudaGetLastError();
 }
 
-cudaError_t launch_row_terms(const void* X, kvb_dtype dtype, int H, long long ldX, int d, int n_uni,
-                             const int* n_dev, int max_n, float inv_h, float add, float* out, long long ldOut,
-                             cudaStream_t st) {
-  if (max_n <= 0 || H <= 0) return cudaSuccess;
-  dim3 grid((max_n + 7) / 8, H);
-  LaunchTrace trace("row_terms_kernel", st);
-  if (dtype == KVB_BF16)
-    row_terms_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), ldX, d, n_uni, n_dev, inv_h, add,
-                                           out, ldOut);
-  else
-    row_terms_kernel<<<grid, 256, 0, st>>>(static_cast<const float*>(X), ldX, d, n_uni, n_dev, inv_h, add, out,
-                                           ldOut);
-  return cudaGetLastError();
-}
 
 }  // namespace kvb

@@ -1,4 +1,4 @@
-// Small HBM-bound kernels shared by the entry points.
+// The augmented-row kernel shared by the entry points (HBM-bound).
 #pragma once
 
 #include <cstdint>
@@ -7,12 +7,6 @@
 #include "kvb.h"
 
 namespace kvb {
-
-// out[h][ldOut*h + off + r] = ||X[h][xoff + r]||^2 * inv_h + add, r < n (uniform or per-head n_dev),
-// X [H][ldX][d] of `dtype`.  One warp per row.
-cudaError_t launch_row_terms(const void* X, kvb_dtype dtype, int H, long long ldX, int d, int n_uni,
-                             const int* n_dev, int max_n, float inv_h, float add, float* out, long long ldOut,
-                             cudaStream_t st);
 
 // Augmented rows for the density MMA: for x = X[h][r] (r < n), with
 // nrm = -||x||^2 / 2 split exactly into three bf16 parts (hi, mid, lo):
