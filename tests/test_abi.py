@@ -62,3 +62,55 @@ def test_launch_trace_host_side():
     assert kvb.lib.kvb_trace_read(None, 0, ctypes.byref(n)) == 0 and n.value == 0
     assert kvb.lib.kvb_trace_read(None, 4, ctypes.byref(n)) == 1   # out NULL with max_records > 0
     assert kvb.lib.kvb_trace_read(None, 0, None) == 1              # n_out NULL
+
+
+def test_config_validation_and_workspace_sizes():
+    """kvb_workspace_size: 0 for every invalid configuration; for valid ones it
+    grows with the number of layers (per-layer banks) and with max_queries
+    (attention scratch), and bf16 banks are smaller than f32 ones."""
+    import kv_cache_compression_post_b200 as kvb
+    ok = kvb.make_config()
+    base = kvb.kvb_workspace_size(ok)
+    assert base > 0
+    bad = [dict(heads=65), dict(heads=0), dict(head_dim=96), dict(capacity=0), dict(max_candidates=0),
+           dict(max_queries=0), dict(eps=0.0), dict(tau=0.0), dict(dist_scale=-1.0), dict(layers=0)]
+    for kw in bad:
+        assert kvb.kvb_workspace_size(kvb.make_config(**kw)) == 0, kw
+    two = kvb.kvb_workspace_size(kvb.make_config(layers=2))
+    three = kvb.kvb_workspace_size(kvb.make_config(layers=3))
+    assert two > base and abs((three - two) - (two - base)) <= 4096   # one bank per layer (+ 256-byte alignment)
+    assert kvb.kvb_workspace_size(kvb.make_config(max_queries=2 * 4680)) > base
+    assert kvb.kvb_workspace_size(kvb.make_config(dtype=kvb.KVB_F32)) > base
+    f = kvb.make_config(method=kvb.KVB_FORCINGKV, frame_h=30, frame_w=52)
+    assert kvb.kvb_workspace_size(f) > 0
+    for kw in [dict(frame_h=0), dict(seg_w=0), dict(hist_frames=0), dict(retention=1.5), dict(max_new_frames=0)]:
+        c = kvb.make_config(method=kvb.KVB_FORCINGKV, frame_h=30, frame_w=52)
+        for k, v in kw.items():
+            setattr(c, k, v)
+        assert kvb.kvb_workspace_size(c) == 0, kw
+
+
+def test_entry_points_reject_bad_arguments_before_any_launch():
+    """Null handles and malformed operation-level arguments return KVB_E_INVAL /
+    KVB_E_UNSUPPORTED without touching the device."""
+    import ctypes
+    import kv_cache_compression_post_b200 as kvb
+    lib = kvb.lib
+    assert lib.kvb_admit(None, 0, None, None, None, 1, None) == 1
+    assert lib.kvb_prune_hybrid(None, 0, None, None, None, None, None, 1, None) == 1
+    assert lib.kvb_attend(None, 0, None, 1, None, None, 0, None, None, 0, None, None, None) == 1
+    assert lib.kvb_bank_destroy(None) == 1
+    n = ctypes.c_int32(0)
+    assert lib.kvb_bank_export(None, 0, 0, None, None, None, None, None, ctypes.byref(n), None) == 1
+    out = ctypes.c_void_p()
+    assert lib.kvb_bank_create(None, None, 0, None, ctypes.byref(out)) == 1
+    assert lib.kvb_bank_create(ctypes.byref(kvb.make_config()), ctypes.c_void_p(0x1001), 1 << 40, None,
+                               ctypes.byref(out)) == 2                       # misaligned workspace
+    # segment cosine: 16-byte rows and aligned pointers only
+    sim = ctypes.c_void_p(0x2000)
+    assert lib.kvb_segment_cosine(ctypes.c_void_p(0x1008), ctypes.c_void_p(0x3000), 1, 1, 4, 4, 4, 4, 128,
+                                  kvb.KVB_BF16, sim, None) == 1              # K not 16-byte aligned
+    assert lib.kvb_segment_cosine(ctypes.c_void_p(0x1000), ctypes.c_void_p(0x3000), 1, 1, 4, 4, 4, 4, 4,
+                                  kvb.KVB_BF16, sim, None) == 7              # 8-byte rows
+    assert lib.kvb_segment_cosine(None, ctypes.c_void_p(0x3000), 1, 1, 4, 4, 4, 4, 128, kvb.KVB_BF16, sim,
+                                  None) == 1
