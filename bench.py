@@ -568,7 +568,7 @@ def oracle_sample(w, reps: int = 1):
     Mb = Kb.shape[0]
     cand = x["candK"][0]
     N = cand.shape[0]
-    rr, qr = 512, 256
+    rr, qr = min(512, Mb, N), min(256, w.chunk_tokens)
     kw = dict(h=float(w.head_dim), eps=w.eps, s=w.s)
     times = []
     for _ in range(reps):
@@ -730,9 +730,18 @@ def main():
         args.warmup = 3
     w = kvgen.WORKLOADS[args.workload]
     rank, world, local = dist_init()
-    if args.impl == "reference":
-        run_reference(args, w, rank, world)
-        return
+    try:
+        if args.impl == "reference":
+            run_reference(args, w, rank, world)
+        else:
+            run_kvb(args, w, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+def run_kvb(args, w, rank, world, local):
     import torch
     torch.cuda.set_device(local)
     if w.name == "rollout":
@@ -765,9 +774,6 @@ def main():
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
 
 
 if __name__ == "__main__":
