@@ -38,6 +38,21 @@ Readings taken where the pages are silent (each is a parameter or a plain choice
 * after the update every density is recomputed from scratch over the new bank;
   new entries take rho0 = that density.
 
+Ablation switches of App. E (off by default; each replaces one default above):
+
+* ``cand_order="source"``: candidates in spatiotemporal source order (id
+  ascending) instead of by score; a head's feasible prefix is the run of
+  candidates from the lowest id up to, not including, its lowest-id infeasible
+  one, and a head admits its P lowest ids;
+* ``baselines="refresh"``: after every update every entry's rho0 becomes its
+  density within the new bank (App. E "refresh baselines"), not only the new
+  entries';
+* ``eviction="densest"``: no ratio threshold; the bank sheds
+  max(0, |B| + P - M) entries by (projected density rho_i + sum_A phi descending,
+  id ascending) -- the reading of App. E "densest-only eviction";
+* ``eviction="source"``: mandatory evictions as by default, then the capacity
+  evictions by id ascending (oldest first) -- App. E "source-order completion".
+
 Nothing here is incremental: the CUDA path's incremental maintenance (App. B.1:
 "exact update in O(N M d_k)") is checked against these from-scratch values.
 """
@@ -59,6 +74,9 @@ class Params:
     s: float = 2.0
     h: float = 0.0           # distance scale; 0 => head_dim
     sync_heads: bool = True
+    cand_order: str = "score"    # "score" | "source"
+    baselines: str = "fixed"     # "fixed" | "refresh"
+    eviction: str = "ratio"      # "ratio" | "densest" | "source"
 
     def scale(self, d: int) -> float:
         return float(self.h) if self.h > 0 else float(d)
@@ -127,7 +145,7 @@ def admit(banks: List[HeadBank], cand_ids: np.ndarray, candK: np.ndarray, candV:
         rho_cand.append(rc)
         score.append(sc)
         feas.append(sc <= p.tau)
-    P_h = np.array([int(f.sum()) for f in feas])
+    P_h = np.array([_feasible_prefix(p, f, cand_ids) for f in feas])
 
     # -- step 3: largest feasible prefix, synchronised across heads --------------------
     if p.sync_heads:
@@ -136,11 +154,11 @@ def admit(banks: List[HeadBank], cand_ids: np.ndarray, candK: np.ndarray, candV:
         P_all = [int(min(P_h[hh], M, N)) for hh in range(H)]
     admitted = []
     for hh in range(H):
-        order = _lex_order(score[hh], cand_ids)
+        order = _lex_order(_cand_key(p, score[hh]), cand_ids)
         admitted.append(order[:P_all[hh]])
 
     # -- step 4: projected growth, threshold-first and capacity eviction ---------------
-    rho_cur, proj, ratio, mand, evicted, n_cap = [], [], [], [], [], []
+    rho_cur, proj, ratio, mand, evicted, n_cap, cutv = [], [], [], [], [], [], []
     for hh in range(H):
         b = banks[hh]
         A = admitted[hh]
@@ -149,16 +167,17 @@ def admit(banks: List[HeadBank], cand_ids: np.ndarray, candK: np.ndarray, candV:
         rhat = rcur + pj
         with np.errstate(divide="ignore", invalid="ignore"):
             rt = np.where(b.rho0 > 0, rhat / np.where(b.rho0 > 0, b.rho0, 1.0), 0.0)
-        md = rt > p.tau
+        md = _mandatory(p, rt)
         ecap = max(0, b.size - int(md.sum()) + len(A) - M)
         ev = md.copy()
         if ecap:
             rest = np.nonzero(~md)[0]
-            order = _lex_order(-rt[rest], b.ids[rest])
+            order = _lex_order(-_cut_value(p, rt, rhat, b.ids)[rest], b.ids[rest])
             ev[rest[order[:ecap]]] = True
         rho_cur.append(rcur)
         proj.append(pj)
         ratio.append(rt)
+        cutv.append(_cut_value(p, rt, rhat, b.ids))
         mand.append(md)
         evicted.append(ev)
         n_cap.append(ecap)
@@ -174,15 +193,49 @@ def admit(banks: List[HeadBank], cand_ids: np.ndarray, candK: np.ndarray, candV:
         V = np.concatenate([b.V[keep], np.asarray(candV[hh][A], np.float64)])
         rn = density(K, K, row_ids=ids, col_ids=ids, **kw)
         n_old = int(keep.sum())
-        rho0 = np.concatenate([b.rho0[keep], rn[n_old:]])
+        rho0 = rn.copy() if p.baselines == "refresh" else np.concatenate([b.rho0[keep], rn[n_old:]])
         new_banks.append(HeadBank(ids, K, V, rho0))
         rho_new.append(rn)
 
-    margins = _margins(p, score, P_h, P_all, admitted, ratio, mand, evicted, n_cap, banks, cand_ids)
+    margins = _margins(p, score, P_h, P_all, admitted, ratio, mand, evicted, n_cap, banks, cand_ids, cutv)
     near = sum(int((m < tie_margin).sum()) for m in margins.values())
-    tc, tb = _tie_ids(p, score, P_h, P_all, ratio, mand, n_cap, banks, cand_ids, tie_margin)
+    tc, tb = _tie_ids(p, score, P_h, P_all, ratio, mand, n_cap, banks, cand_ids, tie_margin, cutv)
     return AdmitResult(new_banks, P_all[0] if p.sync_heads else -1, P_h, rho_cand, score, admitted,
                        rho_cur, proj, ratio, mand, evicted, np.array(n_cap), rho_new, near, margins, tc, tb)
+
+
+def _feasible_prefix(p: Params, feasible: np.ndarray, cand_ids: np.ndarray) -> int:
+    """Length of a head's largest feasible prefix of the candidate order: every
+    feasible candidate (disturbance order puts them first), or, in source order,
+    the leading run of feasible candidates by id."""
+    if p.cand_order == "source":
+        f = feasible[np.argsort(cand_ids, kind="stable")]
+        return int(f.size if f.all() else np.argmin(f))
+    return int(feasible.sum())
+
+
+def _cand_key(p: Params, score: np.ndarray) -> np.ndarray:
+    """Primary key of the candidate order (ties: id ascending): the disturbance
+    score, or nothing (source order, i.e. by id alone)."""
+    return np.zeros_like(score) if p.cand_order == "source" else score
+
+
+def _mandatory(p: Params, ratio: np.ndarray) -> np.ndarray:
+    """Threshold-first evictions: projected ratio above tau (none when densest-only)."""
+    if p.eviction == "densest":
+        return np.zeros(ratio.shape, bool)
+    return ratio > p.tau
+
+
+def _cut_value(p: Params, ratio: np.ndarray, rhat: np.ndarray, ids: np.ndarray) -> np.ndarray:
+    """The value whose descending order (ties: id ascending) picks the capacity
+    evictions: the projected ratio (default), the projected density (densest-only),
+    or minus the id (source order: oldest first)."""
+    if p.eviction == "densest":
+        return rhat
+    if p.eviction == "source":
+        return -np.asarray(ids, np.float64)
+    return ratio
 
 
 def _rel(a, b):
@@ -192,7 +245,7 @@ def _rel(a, b):
     return np.where(np.isnan(r), np.inf, r)
 
 
-def _margins(p, score, P_h, P_all, admitted, ratio, mand, evicted, n_cap, banks, cand_ids):
+def _margins(p, score, P_h, P_all, admitted, ratio, mand, evicted, n_cap, banks, cand_ids, cutv):
     """Relative margins of every decision that a rounding difference could flip.
 
     * admission threshold: |score - tau| / tau for each candidate;
@@ -206,23 +259,24 @@ def _margins(p, score, P_h, P_all, admitted, ratio, mand, evicted, n_cap, banks,
         if banks[hh].size and banks[hh].rho0.mean() > 0:
             out["adm_thr"].append(_rel(score[hh], p.tau))
         P = P_all[hh]
-        if 0 < P < int(P_h[hh]):
+        if 0 < P < int(P_h[hh]) and p.cand_order != "source":   # ids never tie
             order = _lex_order(score[hh], cand_ids)
             a, b = score[hh][order[P - 1]], score[hh][order[P]]
             out["adm_cut"].append(np.array([_rel(b, a) if a != 0 else 1.0]))
-        if banks[hh].size:
+        if banks[hh].size and p.eviction != "densest":
             out["ev_thr"].append(_rel(ratio[hh], p.tau))
-        if n_cap[hh] > 0:
+        if n_cap[hh] > 0 and p.eviction != "source":   # ids never tie
+            cv = cutv[hh]
             rest = np.nonzero(~mand[hh])[0]
-            order = _lex_order(-ratio[hh][rest], banks[hh].ids[rest])
+            order = _lex_order(-cv[rest], banks[hh].ids[rest])
             if n_cap[hh] < rest.size:
-                a = ratio[hh][rest[order[n_cap[hh] - 1]]]
-                b = ratio[hh][rest[order[n_cap[hh]]]]
+                a = cv[rest[order[n_cap[hh] - 1]]]
+                b = cv[rest[order[n_cap[hh]]]]
                 out["ev_cut"].append(np.array([_rel(b, a) if a != 0 else 1.0]))
     return {k: (np.concatenate(v) if v else np.zeros(0)) for k, v in out.items()}
 
 
-def _tie_ids(p, score, P_h, P_all, ratio, mand, n_cap, banks, cand_ids, m):
+def _tie_ids(p, score, P_h, P_all, ratio, mand, n_cap, banks, cand_ids, m, cutv):
     """Ids whose admit/evict decision could flip under a relative perturbation < m."""
     tc, tb = [], []
     for hh in range(len(score)):
@@ -230,24 +284,32 @@ def _tie_ids(p, score, P_h, P_all, ratio, mand, n_cap, banks, cand_ids, m):
         if banks[hh].size and banks[hh].rho0.mean() > 0:
             c |= set(cand_ids[_rel(score[hh], p.tau) < m].tolist())
         P = P_all[hh]
-        if 0 < P < int(P_h[hh]):
+        if 0 < P < int(P_h[hh]) and p.cand_order != "source":
             order = _lex_order(score[hh], cand_ids)
             lo, hi = score[hh][order[P - 1]], score[hh][order[P]]
             close = np.abs(score[hh] - lo) <= m * max(abs(lo), 1e-300)
             if _rel(hi, lo) < m:
                 c |= set(cand_ids[close | (np.abs(score[hh] - hi) <= m * max(abs(hi), 1e-300))].tolist())
         ids = banks[hh].ids
-        if banks[hh].size:
-            b |= set(ids[_rel(ratio[hh], p.tau) < m].tolist())
-        if n_cap[hh] > 0:
+        if banks[hh].size and p.eviction != "densest":
+            near = _rel(ratio[hh], p.tau) < m
+            b |= set(ids[near].tolist())
+            k = int(near.sum())
+            if k and p.eviction == "source":
+                # each flipped threshold decision moves the capacity cut by one in
+                # id order, onto entries whose own decision is not close
+                raw = banks[hh].size - int(mand[hh].sum()) + P - p.capacity
+                rest = np.sort(ids[~mand[hh]])
+                b |= set(rest[max(0, raw - k):max(0, raw + k)].tolist())
+        if n_cap[hh] > 0 and p.eviction != "source":
+            cv = cutv[hh]
             rest = np.nonzero(~mand[hh])[0]
-            order = _lex_order(-ratio[hh][rest], ids[rest])
+            order = _lex_order(-cv[rest], ids[rest])
             if n_cap[hh] < rest.size:
-                lo = ratio[hh][rest[order[n_cap[hh] - 1]]]
-                hi = ratio[hh][rest[order[n_cap[hh]]]]
+                lo = cv[rest[order[n_cap[hh] - 1]]]
+                hi = cv[rest[order[n_cap[hh]]]]
                 if _rel(hi, lo) < m:
-                    r = ratio[hh]
-                    b |= set(ids[(np.abs(r - lo) <= m * abs(lo)) | (np.abs(r - hi) <= m * abs(hi))].tolist())
+                    b |= set(ids[(np.abs(cv - lo) <= m * abs(lo)) | (np.abs(cv - hi) <= m * abs(hi))].tolist())
         tc.append(c)
         tb.append(b)
     return tc, tb

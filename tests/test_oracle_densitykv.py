@@ -7,8 +7,11 @@
 * tau = inf with M >= history: the bank is the whole non-sink history and the
   attention equals full chunk-causal attention over every generated token;
 * the incremental algebra the CUDA path uses equals the from-scratch densities;
+* the App. E ablation switches (refresh baselines, densest-only eviction,
+  source-order completion, source candidate order) on hand scenarios G5-G11;
 * planted mistakes (strict vs non-strict bounds, tie directions, the self term,
-  refreshed baselines) each break at least one pin.
+  refreshed baselines, each ablation switch ignored or misread) each break at
+  least one pin.
 """
 import json
 import os
@@ -31,7 +34,9 @@ def _val(s):
 
 def _run_scenario(sc):
     prm = sc["params"]
-    p = dkv.Params(capacity=prm["capacity"], tau=prm["tau"], eps=prm["eps"], s=prm["s"], h=prm["h"])
+    p = dkv.Params(capacity=prm["capacity"], tau=prm["tau"], eps=prm["eps"], s=prm["s"], h=prm["h"],
+                   sync_heads=prm.get("sync_heads", True), cand_order=prm.get("cand_order", "score"),
+                   baselines=prm.get("baselines", "fixed"), eviction=prm.get("eviction", "ratio"))
     H = prm["heads"]
     banks = [dkv.HeadBank.empty(1) for _ in range(H)]
     for st in sc["steps"]:
@@ -225,6 +230,14 @@ class _NonStrict(dkv.Params):
         self.tau = float(np.nextafter(self.tau, -np.inf))
 
 
+class _NoRefresh(dkv.Params):
+    """Params that ignore the refresh-baselines switch."""
+
+    def __init__(self, *a, **k):
+        super().__init__(*a, **k)
+        self.baselines = "fixed"
+
+
 def _refresh_admit(real_admit):
     def admit(banks, *a, **k):
         r = real_admit(banks, *a, **k)
@@ -244,6 +257,11 @@ def test_pins_catch_planted_mistakes():
         "non_strict_evict": ("Params", _NonStrict),
         "refresh_baselines": ("admit", _refresh_admit(dkv.admit)),
         "capacity_lowest_ratio": ("_lex_order", lambda prim, ids: np.lexsort((np.asarray(ids), -np.asarray(prim)))),
+        "refresh_ignored": ("Params", _NoRefresh),
+        "source_order_by_score": ("_cand_key", lambda p, score: score),
+        "source_prefix_counts_all_feasible": ("_feasible_prefix", lambda p, f, ids: int(f.sum())),
+        "eviction_switch_ignored": ("_cut_value", lambda p, ratio, rhat, ids: ratio),
+        "densest_keeps_threshold": ("_mandatory", lambda p, ratio: ratio > p.tau),
     }
     for name, (attr, repl) in mutations.items():
         real = getattr(dkv, attr)
