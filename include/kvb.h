@@ -46,7 +46,9 @@
  *  - Argument errors return before anything is launched.  Device-side failures
  *    (a bounded wait that gave up, an index a kernel refused) are latched into
  *    the status word and reported by kvb_device_status; kernels never trap.
- *  - Token ids must be unique across a layer's bank and the candidate block.
+ *  - Token ids must be unique across a layer's bank and the candidate block, and
+ *    non-negative: every ordering by id (tie-breaks, source order) compares them
+ *    as unsigned 32-bit values.
  */
 #ifndef KVB_H
 #define KVB_H
@@ -101,12 +103,43 @@ typedef struct {
   float retention;          /* r: each frame keeps floor(r * n_segments) segments */
   /* attention */
   int32_t max_queries;      /* upper bound on Nq of kvb_attend */
+  /* DensityKV ablation switches (DensityKV App. E "Ablation Details"); 0 is the
+   * default policy everywhere, so a zero-filled tail keeps it. */
+  int32_t cand_order;       /* kvb_cand_order */
+  int32_t baselines;        /* kvb_baselines */
+  int32_t evict_order;      /* kvb_evict_order */
 } kvb_config;
+
+/* Candidate ordering (App. E "candidate-ordering ablations").
+ *  KVB_ORDER_DISTURBANCE: candidates by (score ascending, id ascending); the
+ *    feasible prefix is every candidate with score <= tau.
+ *  KVB_ORDER_SOURCE: candidates in spatiotemporal source order, i.e. by id
+ *    ascending; a head's feasible prefix is the run of candidates, from the
+ *    lowest id, that ends before its lowest-id infeasible candidate. */
+typedef enum { KVB_ORDER_DISTURBANCE = 0, KVB_ORDER_SOURCE = 1 } kvb_cand_order;
+
+/* Density baselines (App. E "baseline ablations").
+ *  KVB_BASELINES_FIXED: rho0 is frozen at insertion (co-admitted entries set it
+ *    together, after the update).
+ *  KVB_BASELINES_REFRESH: after every update every entry's rho0 becomes its
+ *    density within the updated bank. */
+typedef enum { KVB_BASELINES_FIXED = 0, KVB_BASELINES_REFRESH = 1 } kvb_baselines;
+
+/* Eviction set (App. E "eviction ablations").
+ *  KVB_EVICT_THRESHOLD_RATIO: every ratio_i > tau, then the capacity evictions by
+ *    (ratio descending, id ascending).
+ *  KVB_EVICT_DENSEST: no threshold step; max(0, |B| + P - M) entries by
+ *    (projected density rho_i + sum_A phi descending, id ascending).
+ *  KVB_EVICT_THRESHOLD_SOURCE: every ratio_i > tau, then the capacity evictions
+ *    by id ascending (oldest source position first). */
+typedef enum { KVB_EVICT_THRESHOLD_RATIO = 0, KVB_EVICT_DENSEST = 1, KVB_EVICT_THRESHOLD_SOURCE = 2 } kvb_evict_order;
 
 /* Per-(layer, head) counters of the last kvb_admit / kvb_prune_hybrid. */
 typedef struct {
   int32_t admitted;      /* P (DensityKV) or kept tokens pushed (Forcing-KV) */
-  int32_t feasible;      /* candidates with score <= tau (DensityKV) */
+  int32_t feasible;      /* DensityKV: length of the head's feasible prefix (the
+                            candidates with score <= tau; KVB_ORDER_SOURCE: the
+                            leading run of them in id order) */
   int32_t mandatory;     /* evictions with ratio > tau */
   int32_t capacity_evicted;
   int32_t size;          /* bank size after the update (ring size for Forcing-KV) */

@@ -9,6 +9,12 @@
 //   evict     projected ratio (rho_i + sum_A phi) / rho0_i; every entry above tau
 //             is evicted, then max(0, |B| - mandatory + P - M) more by (ratio
 //             descending, id ascending) -- another radix select
+//
+// App. E's ablation switches change only keys and flags of these kernels: source
+// candidate order (the feasible prefix is the leading run in id order, admitted
+// by id), densest-only eviction (no threshold step, capacity cut by projected
+// density), source-order completion (capacity cut by id), refreshed baselines
+// (finalize writes rho0 = rho for every entry).
 //   compact   admitted entries fill the evicted slots below the new size, then
 //             append; surviving entries beyond the new size move into the
 //             remaining holes, so every bank stays dense in [0, size)
@@ -185,7 +191,19 @@ __global__ void __launch_bounds__(kSelThreads) admit_count_kernel(const AdmitPla
   const float mean0 = n > 0 ? sum / static_cast<float>(n) : 0.f;
   const float* rb = p.rhoB + static_cast<size_t>(h) * p.ldN;
   int cnt = 0;
-  for (int c = threadIdx.x; c < p.N; c += blockDim.x) cnt += (score_of(rb[c], mean0) <= p.tau) ? 1 : 0;
+  if (p.cand_order == KVB_ORDER_SOURCE) {
+    // the leading run in id order: every candidate below the lowest infeasible id
+    __shared__ unsigned int s_first_bad;
+    if (threadIdx.x == 0) s_first_bad = UINT_MAX;
+    __syncthreads();
+    for (int c = threadIdx.x; c < p.N; c += blockDim.x)
+      if (!(score_of(rb[c], mean0) <= p.tau)) atomicMin(&s_first_bad, static_cast<unsigned int>(p.cand_ids[c]));
+    __syncthreads();
+    const unsigned int bad = s_first_bad;
+    for (int c = threadIdx.x; c < p.N; c += blockDim.x) cnt += (static_cast<unsigned int>(p.cand_ids[c]) < bad) ? 1 : 0;
+  } else {
+    for (int c = threadIdx.x; c < p.N; c += blockDim.x) cnt += (score_of(rb[c], mean0) <= p.tau) ? 1 : 0;
+  }
   int total;
   block_excl_scan(cnt, &S, &total);
   if (threadIdx.x == 0) {
@@ -205,9 +223,10 @@ __global__ void __launch_bounds__(kSelThreads) admit_select_kernel(const AdmitPl
   const float mean0 = p.mean0[h];
   const float* rb = p.rhoB + static_cast<size_t>(h) * p.ldN;
   int* out = p.adm_idx + static_cast<size_t>(h) * p.ldN;
+  const bool by_source = p.cand_order == KVB_ORDER_SOURCE;
   auto key = [&](int c) -> unsigned long long {
-    return (static_cast<unsigned long long>(float_key(score_of(rb[c], mean0))) << 32) |
-           static_cast<unsigned int>(p.cand_ids[c]);
+    const unsigned long long hi = by_source ? 0ull : static_cast<unsigned long long>(float_key(score_of(rb[c], mean0)));
+    return (hi << 32) | static_cast<unsigned int>(p.cand_ids[c]);
   };
   auto all = [](int) { return true; };
   if (P >= p.N) {
@@ -260,27 +279,34 @@ __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPl
   const int* ids = p.ids + base;
   int* evflag = p.tail + base;  // per-slot flags live in the tail array until the tail list is built
   auto ratio = [&](int i) { return ratio_of(rho[i], proj[i], rho0[i]); };
-  // mandatory evictions: projected growth above tau
+  const int mode = p.evict_order;
+  // the capacity-cut key of a non-mandatory entry (ascending = evicted first):
+  // ratio descending (default), projected density descending (densest-only), or
+  // nothing (source order); id ascending breaks ties.  Ratios and densities are
+  // >= 0, so no such key has the top byte 0xFF of the mandatory entries' key.
+  auto cut_key = [&](int i, float r) -> unsigned long long {
+    unsigned long long hi = 0ull;
+    if (mode == KVB_EVICT_THRESHOLD_RATIO) hi = ~float_key(r);
+    else if (mode == KVB_EVICT_DENSEST) hi = ~float_key(rho[i] + proj[i]);
+    return (hi << 32) | static_cast<unsigned int>(ids[i]);
+  };
+  // mandatory evictions: projected growth above tau (none when densest-only)
   int cnt = 0;
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     const float r = ratio(i);
-    const bool m = r > p.tau;
+    const bool m = mode != KVB_EVICT_DENSEST && r > p.tau;
     evflag[i] = m ? 1 : 0;
     cnt += m ? 1 : 0;
-    if (SKEYS)
-      s_key[i] = m ? ~0ull
-                   : (static_cast<unsigned long long>(~float_key(r)) << 32) | static_cast<unsigned int>(ids[i]);
+    if (SKEYS) s_key[i] = m ? ~0ull : cut_key(i, r);
   }
   int n_mand;
   block_excl_scan(cnt, &S, &n_mand);
   const int ecap = max(0, n - n_mand + Ph - p.M);
   const int n_free = n - n_mand;
   if (ecap > 0) {
-    // the key of an entry: ratio descending, then id ascending (ratios are >= 0, so
-    // no such key has the top byte 0xFF of the mandatory entries' key)
     auto key = [&](int i) -> unsigned long long {
       if (SKEYS) return s_key[i];
-      return (static_cast<unsigned long long>(~float_key(ratio(i))) << 32) | static_cast<unsigned int>(ids[i]);
+      return cut_key(i, ratio(i));
     };
     auto keep = [&](int i) { return SKEYS || evflag[i] == 0; };
     if (ecap >= n_free) {
@@ -404,8 +430,10 @@ __global__ void finalize_kernel(const AdmitPlan p) {
     v += p.proj[i];
   } else if (tag >= 0) {
     v += p.coadm[static_cast<size_t>(h) * p.ldN + tag];
-    p.rho0[i] = v;
   }
+  // new entries set their baselines after the update; refreshed baselines follow
+  // every entry's density in the updated bank
+  if (tag >= 0 || p.baselines == KVB_BASELINES_REFRESH) p.rho0[i] = v;
   p.rho[i] = v;
 }
 

@@ -17,6 +17,9 @@ struct AdmitPlan {
   int row_bytes = 0;        // d * element size
   float tau = 2.f;
   int sync_heads = 1;
+  int cand_order = KVB_ORDER_DISTURBANCE;
+  int baselines = KVB_BASELINES_FIXED;
+  int evict_order = KVB_EVICT_THRESHOLD_RATIO;
   // bank (this layer)
   void* K = nullptr;
   void* V = nullptr;

@@ -28,6 +28,11 @@ bool config_ok(const kvb_config* c) {
     if (c->capacity < 1 || c->max_candidates < 1) return false;
     if (!(c->eps > 0.f) || !std::isfinite(c->eps) || !(c->s >= 0.f) || !std::isfinite(c->s)) return false;
     if (!(c->tau > 0.f) || !(c->dist_scale >= 0.f)) return false;
+    if (c->cand_order != KVB_ORDER_DISTURBANCE && c->cand_order != KVB_ORDER_SOURCE) return false;
+    if (c->baselines != KVB_BASELINES_FIXED && c->baselines != KVB_BASELINES_REFRESH) return false;
+    if (c->evict_order != KVB_EVICT_THRESHOLD_RATIO && c->evict_order != KVB_EVICT_DENSEST &&
+        c->evict_order != KVB_EVICT_THRESHOLD_SOURCE)
+      return false;
   } else {
     if (c->frame_h < 1 || c->frame_w < 1 || c->seg_h < 1 || c->seg_w < 1) return false;
     if (c->hist_frames < 1 || c->max_new_frames < 1) return false;
@@ -263,6 +268,9 @@ extern "C" kvb_status kvb_admit(kvb_bank* b, int32_t layer, const void* candK, c
   p.row_bytes = b->row_bytes;
   p.tau = g.tau;
   p.sync_heads = g.sync_heads;
+  p.cand_order = g.cand_order;
+  p.baselines = g.baselines;
+  p.evict_order = g.evict_order;
   p.K = b->K + lo * b->row_bytes;
   p.V = b->V + lo * b->row_bytes;
   p.ids = b->ids + lo;

@@ -15,6 +15,8 @@ from typing import Optional
 __all__ = [
     "KvbError", "kvb_config", "kvb_admit_stats", "make_config", "lib", "LIB_PATH", "Bank",
     "KVB_BF16", "KVB_F32", "KVB_DENSITYKV", "KVB_FORCINGKV",
+    "KVB_ORDER_DISTURBANCE", "KVB_ORDER_SOURCE", "KVB_BASELINES_FIXED", "KVB_BASELINES_REFRESH",
+    "KVB_EVICT_THRESHOLD_RATIO", "KVB_EVICT_DENSEST", "KVB_EVICT_THRESHOLD_SOURCE",
     "kvb_workspace_size", "kvb_bank_create", "kvb_bank_destroy", "kvb_admit", "kvb_prune_hybrid",
     "kvb_attend", "kvb_read_stats", "kvb_bank_export", "kvb_bank_import", "kvb_device_status",
     "kvb_status_string", "kvb_launch_count", "kvb_trace_enable", "kvb_trace_read", "kvb_density_workspace_size", "kvb_density", "kvb_density_noalloc", "kvb_segment_cosine",
@@ -24,6 +26,9 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvb.so")
 
 KVB_BF16, KVB_F32 = 0, 1
 KVB_DENSITYKV, KVB_FORCINGKV = 0, 1
+KVB_ORDER_DISTURBANCE, KVB_ORDER_SOURCE = 0, 1
+KVB_BASELINES_FIXED, KVB_BASELINES_REFRESH = 0, 1
+KVB_EVICT_THRESHOLD_RATIO, KVB_EVICT_DENSEST, KVB_EVICT_THRESHOLD_SOURCE = 0, 1, 2
 
 STATUS = {0: "KVB_OK", 1: "KVB_E_INVAL", 2: "KVB_E_WORKSPACE", 3: "KVB_E_CUDA", 4: "KVB_E_DEVICE_TIMEOUT",
           5: "KVB_E_DEVICE_BOUNDS", 6: "KVB_E_STATE", 7: "KVB_E_UNSUPPORTED"}
@@ -45,6 +50,7 @@ class kvb_config(ctypes.Structure):
         ("frame_h", ctypes.c_int32), ("frame_w", ctypes.c_int32), ("seg_h", ctypes.c_int32),
         ("seg_w", ctypes.c_int32), ("hist_frames", ctypes.c_int32), ("max_new_frames", ctypes.c_int32),
         ("retention", ctypes.c_float), ("max_queries", ctypes.c_int32),
+        ("cand_order", ctypes.c_int32), ("baselines", ctypes.c_int32), ("evict_order", ctypes.c_int32),
     ]
 
 
@@ -60,7 +66,8 @@ def make_config(**kw) -> kvb_config:
     defaults = dict(method=KVB_DENSITYKV, dtype=KVB_BF16, layers=1, heads=12, head_dim=128, capacity=9360,
                     max_candidates=4680, tau=2.0, eps=1e-3, s=2.0, dist_scale=0.0, sync_heads=1,
                     frame_h=0, frame_w=0, seg_h=4, seg_w=4, hist_frames=21, max_new_frames=3,
-                    retention=0.7, max_queries=4680)
+                    retention=0.7, max_queries=4680, cand_order=KVB_ORDER_DISTURBANCE,
+                    baselines=KVB_BASELINES_FIXED, evict_order=KVB_EVICT_THRESHOLD_RATIO)
     defaults.update(kw)
     for k, v in defaults.items():
         setattr(c, k, v)

@@ -73,9 +73,14 @@ def test_config_validation_and_workspace_sizes():
     base = kvb.kvb_workspace_size(ok)
     assert base > 0
     bad = [dict(heads=65), dict(heads=0), dict(head_dim=96), dict(capacity=0), dict(max_candidates=0),
-           dict(max_queries=0), dict(eps=0.0), dict(tau=0.0), dict(dist_scale=-1.0), dict(layers=0)]
+           dict(max_queries=0), dict(eps=0.0), dict(tau=0.0), dict(dist_scale=-1.0), dict(layers=0),
+           dict(cand_order=2), dict(cand_order=-1), dict(baselines=2), dict(evict_order=3), dict(evict_order=-1)]
     for kw in bad:
         assert kvb.kvb_workspace_size(kvb.make_config(**kw)) == 0, kw
+    # the ablation switches change no buffer
+    for kw in [dict(cand_order=kvb.KVB_ORDER_SOURCE), dict(baselines=kvb.KVB_BASELINES_REFRESH),
+               dict(evict_order=kvb.KVB_EVICT_DENSEST), dict(evict_order=kvb.KVB_EVICT_THRESHOLD_SOURCE)]:
+        assert kvb.kvb_workspace_size(kvb.make_config(**kw)) == base, kw
     two = kvb.kvb_workspace_size(kvb.make_config(layers=2))
     three = kvb.kvb_workspace_size(kvb.make_config(layers=3))
     assert two > base and abs((three - two) - (two - base)) <= 4096   # one bank per layer (+ 256-byte alignment)

@@ -7,7 +7,9 @@
 * mid bf16 workload (4 heads, d 128, 170-token frames, M 900: several 128-row
   tiles with ragged tails): stepwise -- the oracle's bank before step i is
   imported, one GPU step runs, and its bank is compared with the oracle's step
-  i; id sets may differ only on decisions within 1e-4 of their threshold or cut.
+  i; id sets may differ only on decisions within 1e-4 of their threshold or cut;
+* the same stepwise check for each App. E ablation switch (source candidate
+  order, refreshed baselines, densest-only eviction, source-order completion).
 """
 import numpy as np
 import pytest
@@ -21,12 +23,12 @@ pytestmark = pytest.mark.gpu
 RTOL = 1e-4
 
 
-def _cfg(w, tau=None, sync=1, layers=1):
+def _cfg(w, tau=None, sync=1, layers=1, **switches):
     import kv_cache_compression_post_b200 as kvb
     return kvb.make_config(method=kvb.KVB_DENSITYKV, dtype=kvb.KVB_BF16 if w.dtype == "bf16" else kvb.KVB_F32,
                            layers=layers, heads=w.heads, head_dim=w.head_dim, capacity=w.capacity,
                            max_candidates=w.chunk_tokens, tau=w.tau if tau is None else tau, eps=w.eps, s=w.s,
-                           sync_heads=sync, max_queries=w.chunk_tokens)
+                           sync_heads=sync, max_queries=w.chunk_tokens, **switches)
 
 
 def _export(bank, layer, H):
@@ -117,6 +119,66 @@ def test_mid_stepwise_matches_oracle(tau, sync):
             all_exact &= _compare(g[hh], r, hh, exact=False, tie_ids=ties)
         exact_steps += int(all_exact)
         banks = r.banks
+    assert exact_steps >= (w.n_chunks - 1) // 2
+    bank.close()
+
+
+# App. E ablation switches: (tau, oracle Params fields).  tau 1.2 with source
+# candidate order gives feasible runs from 0 to N over the steps; the tau 2 cases
+# reach capacity evictions; tau 1 with refresh + densest changes admission too.
+ABLATIONS = [
+    (1.2, dict(cand_order="source")),
+    (2.0, dict(baselines="refresh")),
+    (2.0, dict(eviction="densest")),
+    (2.0, dict(eviction="source")),
+    (1.0, dict(baselines="refresh", eviction="densest")),
+]
+
+
+def _switches(kvb, kw):
+    return dict(cand_order=kvb.KVB_ORDER_SOURCE if kw.get("cand_order") == "source" else kvb.KVB_ORDER_DISTURBANCE,
+                baselines=kvb.KVB_BASELINES_REFRESH if kw.get("baselines") == "refresh" else kvb.KVB_BASELINES_FIXED,
+                evict_order={"ratio": kvb.KVB_EVICT_THRESHOLD_RATIO, "densest": kvb.KVB_EVICT_DENSEST,
+                             "source": kvb.KVB_EVICT_THRESHOLD_SOURCE}[kw.get("eviction", "ratio")])
+
+
+@pytest.mark.parametrize("tau,kw", ABLATIONS, ids=lambda v: str(v))
+def test_mid_stepwise_ablation_switches(tau, kw):
+    """The App. E switches, stepwise against the oracle as above.  A step whose
+    source-order prefix has a near-tie candidate is not compared (one flip there
+    moves the whole run); every other step may differ only on near ties, and
+    exact steps also match the per-head counters."""
+    import torch
+    import kv_cache_compression_post_b200 as kvb
+    w = kvgen.WORKLOADS["mid"]
+    L = kvgen.LayerInputs(w, 0, tagged=True)
+    p = dkv.Params(capacity=w.capacity, tau=tau, eps=w.eps, s=w.s, **kw)
+    bank = kvb.Bank(_cfg(w, tau=tau, **_switches(kvb, kw)))
+    banks = [dkv.HeadBank.empty(w.head_dim) for _ in range(w.heads)]
+    exact_steps = 0
+    for i in range(1, w.n_chunks):
+        x = L.step(i)
+        r = dkv.admit(banks, x["cand_ids"], x["candK"], x["candV"], p)
+        _import(bank, banks, p, w)
+        bank.admit(0, dev_tensor(x["candK"], w.dtype), dev_tensor(x["candV"], w.dtype), dev_ids(x["cand_ids"]))
+        torch.cuda.synchronize()
+        assert bank.status() == 0
+        banks = r.banks
+        if kw.get("cand_order") == "source" and any(r.tie_cand_ids):
+            continue
+        g = _export(bank, 0, w.heads)
+        st = bank.stats(0)
+        all_exact = True
+        for hh in range(w.heads):
+            ties = r.tie_cand_ids[hh] | r.tie_bank_ids[hh]
+            all_exact &= _compare(g[hh], r, hh, exact=False, tie_ids=ties)
+        if all_exact:
+            for hh in range(w.heads):
+                assert st[hh]["feasible"] == int(r.P_h[hh])
+                assert st[hh]["admitted"] == len(r.admitted[hh])
+                assert st[hh]["mandatory"] == int(r.mandatory[hh].sum())
+                assert st[hh]["capacity_evicted"] == int(r.n_capacity[hh])
+        exact_steps += int(all_exact)
     assert exact_steps >= (w.n_chunks - 1) // 2
     bank.close()
 
