@@ -54,16 +54,20 @@ def _kept_near_tie(sim, k, margin=1e-4):
     return abs(b - a) <= margin * max(abs(a), 1e-3)
 
 
-def _rollout(name, steps, labels, sample_rows=None):
+def _rollout(name, steps, labels, sample_rows=None, **geometry):
+    """``geometry`` overrides the segmentation (frame_h, frame_w, seg_h, seg_w,
+    retention) of both the library and the oracle; the inputs keep the workload's
+    own frames."""
+    import dataclasses
     import torch
     import kv_cache_compression_post_b200 as kvb
     w = kvgen.WORKLOADS[name]
     H = len(labels)
     L = kvgen.LayerInputs(w, 0, n_chunks=steps + 2, heads=range(H))
-    p = fkv.Params(w.frame_h, w.frame_w, w.seg_h, w.seg_w, w.retention, w.hist_frames)
+    ws = dataclasses.replace(w, heads=H, **geometry)
+    p = fkv.Params(ws.frame_h, ws.frame_w, ws.seg_h, ws.seg_w, ws.retention, ws.hist_frames)
     states = [fkv.HeadState(bool(s)) for s in labels]
-    import dataclasses
-    bank = kvb.Bank(_cfg(dataclasses.replace(w, heads=H)))
+    bank = kvb.Bank(_cfg(ws))
     rng = np.random.default_rng(0)
     tie_frames = [set() for _ in range(H)]   # frames pushed with a near-tie BottomK decision
     for i in range(1, steps + 1):
@@ -74,7 +78,7 @@ def _rollout(name, steps, labels, sample_rows=None):
         for hh in range(H):
             if not states[hh].static:
                 for f, s in zip(new_frames, states[hh].sims):
-                    if _kept_near_tie(s, fkv.keep_count(s.size, w.retention)):
+                    if _kept_near_tie(s, fkv.keep_count(s.size, ws.retention)):
                         tie_frames[hh].add(f)
         bank.prune_hybrid(0, np.array(labels, np.uint8), dev_tensor(x["newK"], "bf16"), dev_tensor(x["newV"], "bf16"),
                           dev_tensor(x["nextK"], "bf16"), dev_ids(x["new_ids"]), nf)
@@ -115,6 +119,13 @@ def _rollout(name, steps, labels, sample_rows=None):
 def test_forcing_mid_rollout_matches_oracle():
     # hist_frames 7 < frames pushed: the FIFO wraps and drops old frames
     _rollout("forcing_mid", 4, [1, 0, 1, 0])
+
+
+def test_forcing_mid_contiguous_segments():
+    # the pages' own segmentation: n = 6 contiguous runs of the row-major frame,
+    # r = 0.3 (one run kept per frame)
+    F = kvgen.WORKLOADS["forcing_mid"].F
+    _rollout("forcing_mid", 4, [0, 1, 0, 0], frame_h=1, frame_w=F, seg_h=1, seg_w=F // 6, retention=0.3)
 
 
 def test_forcing480_full_size_sampled():

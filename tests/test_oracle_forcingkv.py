@@ -26,6 +26,21 @@ def test_segment_partition_480p():
     assert fkv.keep_count(104, 1.0) == 104
 
 
+def test_contiguous_segments_as_a_one_row_frame():
+    """The pages' n = 6 contiguous segments of a frame (Forcing-KV §3.4 and its
+    implementation notes: the frame's tokens reshaped into n runs) are the 1 x F
+    view of the row-major frame cut into 1 x F/n tiles."""
+    F = 30 * 52
+    segs = fkv.segments(1, F, 1, F // 6)
+    assert len(segs) == 6
+    for j, sg in enumerate(segs):
+        np.testing.assert_array_equal(sg, np.arange(j * 260, (j + 1) * 260))
+    # a length that does not divide: the last run is partial
+    segs = fkv.segments(1, 10, 1, 4)
+    assert [sg.tolist() for sg in segs] == [[0, 1, 2, 3], [4, 5, 6, 7], [8, 9]]
+    assert fkv.keep_count(6, 0.33) == 1
+
+
 def test_hand_built_cosines_and_bottom_k():
     # frame 2 x 4 tokens, 2 x 2 segments -> segment 0 = tokens {0,1,4,5}, segment 1 = {2,3,6,7}
     Kt = np.array([[1, 0]] * 8, dtype=np.float64)
