@@ -119,3 +119,34 @@ def test_entry_points_reject_bad_arguments_before_any_launch():
                                   kvb.KVB_BF16, sim, None) == 7              # 8-byte rows
     assert lib.kvb_segment_cosine(None, ctypes.c_void_p(0x3000), 1, 1, 4, 4, 4, 4, 128, kvb.KVB_BF16, sim,
                                   None) == 1
+
+
+def test_plain_c_program_agrees_with_the_binding(tmp_path):
+    """include/kvb.h compiles as strict C99 in a plain C program linked against
+    libkvb.so; the struct layouts it sees equal the ctypes mirror's, and the
+    host-only entry points return the same values through both."""
+    import ctypes
+    import shutil
+    import subprocess
+    import kv_cache_compression_post_b200 as kvb
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(kvb.LIB_PATH)
+    exe = str(tmp_path / "abi_layout")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c", "abi_layout.c"), "-L", libdir, "-lkvb",
+                    "-Wl,-rpath," + libdir, "-o", exe], check=True)
+    out = subprocess.run([exe], check=True, capture_output=True, text=True).stdout
+    got = dict(line.split(" ", 1) for line in out.strip().splitlines())
+    for T in (kvb.kvb_config, kvb.kvb_admit_stats, kvb.kvb_trace_record):
+        assert int(got["sizeof." + T.__name__]) == ctypes.sizeof(T), T.__name__
+        for name, _ in T._fields_:
+            assert int(got[f"{T.__name__}.{name}"]) == getattr(T, name).offset, (T.__name__, name)
+    # every field the C program prints exists in the mirror
+    mirrored = {f"{T.__name__}.{n}" for T in (kvb.kvb_config, kvb.kvb_admit_stats, kvb.kvb_trace_record)
+                for n, _ in T._fields_}
+    assert {k for k in got if "." in k and not k.startswith(("sizeof", "workspace", "status"))} == mirrored
+    ref = kvb.make_config(heads=12, head_dim=128, capacity=9360, max_candidates=4680, max_queries=4680)
+    assert int(got["workspace.wan480"]) == kvb.kvb_workspace_size(ref) > 0
+    assert int(got["workspace.invalid"]) == 0
+    assert got["status.0"] == kvb.kvb_status_string(0)
