@@ -586,16 +586,11 @@ def oracle_sample(w, reps: int = 1):
         per_head = ((t1 - t) * N / rr + (t2 - t1) * 2 * Mb / rr + (t3 - t2) * Mb / rr
                     + (t4 - t3) * w.chunk_tokens / qr)
         times.append(per_head * w.heads * 1e3)
-    try:
-        from threadpoolctl import threadpool_info
-        blas_threads = max((p.get("num_threads", 1) for p in threadpool_info()), default=1)
-    except Exception:
-        blas_threads = None
-    sample = (f"one head of a 480P chunk-layer (step {i}): density of {rr} of {N} candidates vs {Mb} bank keys, "
+    sample = (f"one head of a {w.name} chunk-layer (step {i}): density of {rr} of {N} candidates vs {Mb} bank keys, "
               f"from-scratch density of {rr} of {Mb} bank keys (x2: before and after the update), projected "
               f"growth of {rr} bank keys vs {N} candidates, attention of {qr} of {w.chunk_tokens} queries over "
               f"{Kall.shape[0]} keys; scaled by rows and by {w.heads} heads")
-    return statistics.mean(times), sample, (os.cpu_count(), blas_threads)
+    return statistics.mean(times), sample
 
 
 def oracle_sample_forcing(w, reps: int = 1):
@@ -644,29 +639,36 @@ def oracle_sample_forcing(w, reps: int = 1):
 
 
 def cpu_sample(w, reps: int = 1):
+    """(ms, cpu_baseline dict) of the oracle on a bounded sample of workload w.
+
+    The oracle's differences, einsum reductions and elementwise kernels run on one
+    thread; only its matrix products (attention) use the BLAS pool, so the threads
+    it actually uses are max(1, BLAS pool size)."""
     if w.forcing:
         ms, sample = oracle_sample_forcing(w, reps)
     else:
-        ms, sample, _ = oracle_sample(w, reps)
+        ms, sample = oracle_sample(w, reps)
     try:
         from threadpoolctl import threadpool_info
         blas_threads = max((p.get("num_threads", 1) for p in threadpool_info()), default=1)
     except Exception:
         blas_threads = None
-    return ms, sample, (os.cpu_count(), blas_threads)
+    cpu = {"value": round(ms, 3), "unit": UNIT, "cores": max(1, blas_threads or 1), "host_cpus": os.cpu_count(),
+           "blas_threads": blas_threads, "kind": "oracle",
+           "sample": sample + "; NumPy differences and reductions on one thread, matrix products on the BLAS pool"}
+    return ms, cpu
 
 
 def run_reference(args, w, rank, world):
     if rank != 0:
         return
     t0 = time.time()
-    ms, sample, (cores, blas) = cpu_sample(w, reps=max(1, args.steps))
+    ms, cpu = cpu_sample(w, reps=max(1, args.steps))
     line = {"impl": "reference", "metric": METRIC, "value": round(ms, 3), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(w, args, world),
-            "cpu_baseline": {"value": round(ms, 3), "unit": UNIT, "cores": cores, "blas_threads": blas,
-                             "kind": "oracle", "sample": sample},
+            "cpu_baseline": cpu,
             "e2e": {"value": round(ms, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "wall_s": round(time.time() - t0, 1)}
     print(json.dumps(line), flush=True)
@@ -675,9 +677,7 @@ def run_reference(args, w, rank, world):
 def print_rollout(args, w, r, world):
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        ms, sample, (cores, blas) = cpu_sample(w, reps=1)
-        cpu = {"value": round(ms, 3), "unit": UNIT, "cores": cores, "blas_threads": blas, "kind": "oracle",
-               "sample": sample}
+        _, cpu = cpu_sample(w, reps=1)
     line = {
         "metric": METRIC, "value": round(r["ms_per_step"], 4), "unit": UNIT, "n_gpus": world,
         "steps": r["dist"]["chunk_layers"], "warmup": 0, "ms_per_step": round(r["ms_per_step"], 4),
@@ -754,9 +754,7 @@ def run_kvb(args, w, rank, world, local):
         return
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        ms, sample, (cores, blas) = cpu_sample(w, reps=1)
-        cpu = {"value": round(ms, 3), "unit": UNIT, "cores": cores, "blas_threads": blas, "kind": "oracle",
-               "sample": sample}
+        _, cpu = cpu_sample(w, reps=1)
     line = {
         "metric": METRIC, "value": round(r["ms_per_step"], 4), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["ms_per_step"], 4),

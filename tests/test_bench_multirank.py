@@ -46,3 +46,18 @@ def test_two_rank_barrier_and_max_over_ranks():
     assert [r[0] for r in res] == [0, 1]
     assert all(r[1] == 2 and r[3] == "gloo" for r in res)
     assert all(r[2] == pytest.approx(3.0) for r in res)   # every rank sees the slowest rank's time
+
+
+@pytest.mark.parametrize("name", ["tiny", "forcing_mid"])
+def test_cpu_baseline_record(name):
+    """The oracle leg that every bench line carries: a positive time and the keys
+    the line needs (threads actually used, host CPUs, the stated sample)."""
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    import kvgen
+    ms, cpu = bench.cpu_sample(kvgen.WORKLOADS[name], reps=1)
+    assert ms > 0 and cpu["value"] == round(ms, 3)
+    assert cpu["kind"] == "oracle" and cpu["unit"] == bench.UNIT
+    assert 1 <= cpu["cores"] <= (cpu["host_cpus"] or cpu["cores"])
+    assert name.split("_")[0] in cpu["sample"] or "Forcing-KV" in cpu["sample"]
