@@ -243,6 +243,23 @@ KVB_API kvb_status kvb_trace_read(kvb_trace_record* out, int32_t max_records, in
 /* Static string for a status code. */
 KVB_API const char* kvb_status_string(kvb_status st);
 
+/* Self-test of the device-side failure detection (no counterpart on the pages).
+ * Every mbarrier wait of the tensor-core kernels is bounded; on expiry it
+ * latches KVB_E_DEVICE_TIMEOUT into the status word and raises its CTA's abort
+ * flag, on which every other role of the CTA gives up its own wait.  This call
+ * runs that wait, asynchronously on `stream`, in one CTA with two roles, each on
+ * an mbarrier that nothing ever arrives on: role 0 with the limit `timeout_ns`,
+ * role 1 with 50 x `timeout_ns`, so that role 1 returns early only through the
+ * abort flag.  No fault, trap or unbounded wait is involved.
+ *   status: device int32, the word the timeout is latched into (the first
+ *           nonzero code stays; clear it to 0 before the call to observe it).
+ *   out:    device int64[4]: out[0] = 1 if role 0's wait completed (never),
+ *           out[1] = role 0's wait in ns, out[2], out[3] the same for role 1.
+ *   timeout_ns: 1e3 .. 1e8 (1 us .. 100 ms; the kernels' own limit is 2 s).
+ * KVB_E_INVAL on a NULL pointer or a limit out of range (nothing launched);
+ * KVB_E_CUDA if the launch fails. */
+KVB_API kvb_status kvb_selftest_timeout(int32_t* status, int64_t* out, int64_t timeout_ns, void* stream);
+
 /* ------------------------------------------------------------------------------
  * Operation-level entry points: the same kernels on caller buffers, for callers
  * that manage their own caches.  They use the scratch of a caller workspace.

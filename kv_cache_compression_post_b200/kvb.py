@@ -20,6 +20,7 @@ __all__ = [
     "kvb_workspace_size", "kvb_bank_create", "kvb_bank_destroy", "kvb_admit", "kvb_prune_hybrid",
     "kvb_attend", "kvb_read_stats", "kvb_bank_export", "kvb_bank_import", "kvb_device_status",
     "kvb_status_string", "kvb_launch_count", "kvb_trace_enable", "kvb_trace_read", "kvb_density_workspace_size", "kvb_density", "kvb_density_noalloc", "kvb_segment_cosine",
+    "kvb_selftest_timeout",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvb.so")
@@ -106,6 +107,7 @@ _SIGS = {
                                            _vp, _vp]),
     "kvb_segment_cosine": (ctypes.c_int, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_int, _vp,
                                           _vp]),
+    "kvb_selftest_timeout": (ctypes.c_int, [_vp, _vp, ctypes.c_int64, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -226,6 +228,12 @@ def kvb_density(rows, n_rows: int, cols, n_cols: int, heads: int, head_dim: int,
     _check(lib.kvb_density(_ptr(rows), n_rows, _ptr(cols), n_cols, heads, head_dim, dtype, dist_scale, eps, s,
                            exclude_diagonal, _ptr(out), _ptr(workspace), workspace_bytes, _stream(stream)),
            "kvb_density")
+
+
+def kvb_selftest_timeout(status, out, timeout_ns: int, stream=None) -> None:
+    """Run the library's bounded mbarrier wait to expiry (see kvb.h): status is a
+    device int32 word, out a device int64[4]."""
+    _check(lib.kvb_selftest_timeout(_ptr(status), _ptr(out), int(timeout_ns), _stream(stream)), "kvb_selftest_timeout")
 
 
 def kvb_density_noalloc(rows, n_rows: int, cols, n_cols: int, heads: int, head_dim: int, dtype: int,

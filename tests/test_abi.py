@@ -150,3 +150,13 @@ def test_plain_c_program_agrees_with_the_binding(tmp_path):
     assert int(got["workspace.wan480"]) == kvb.kvb_workspace_size(ref) > 0
     assert int(got["workspace.invalid"]) == 0
     assert got["status.0"] == kvb.kvb_status_string(0)
+
+
+def test_selftest_timeout_argument_errors_without_gpu():
+    import ctypes
+    import kv_cache_compression_post_b200 as kvb
+    fake = ctypes.c_void_p(256)   # never dereferenced: the checks return before any launch
+    assert kvb.lib.kvb_selftest_timeout(None, fake, 1000, None) == 1
+    assert kvb.lib.kvb_selftest_timeout(fake, None, 1000, None) == 1
+    assert kvb.lib.kvb_selftest_timeout(fake, fake, 999, None) == 1
+    assert kvb.lib.kvb_selftest_timeout(fake, fake, 100_000_001, None) == 1
