@@ -170,6 +170,26 @@ KVB_API kvb_status kvb_bank_destroy(kvb_bank* bank);
 KVB_API kvb_status kvb_admit(kvb_bank* bank, int32_t layer, const void* candK, const void* candV,
                      const int32_t* cand_ids, int32_t N, void* stream);
 
+/* kvb_admit in two halves, for banks whose heads are split across processes or
+ * GPUs (each holding some heads of a layer) under synchronised admission: the
+ * shared prefix P = min over ALL heads of the layer is the one value they must
+ * exchange (DensityKV App. E cross-head synchronisation).
+ *   kvb_admit_begin: the arguments of kvb_admit plus prefix_out (device int32):
+ *     launches the candidate densities and feasible counts, then writes
+ *     min(min_h #feasible_h over this bank's heads, M, N) to *prefix_out.
+ *   kvb_admit_finish: completes the begun step of `layer` with
+ *     P = min(this bank's prefix, max(0, *prefix_bound)); prefix_bound is a
+ *     device int32 (typically the MIN over every process's prefix_out) or NULL
+ *     (then the result equals kvb_admit's).  Requires sync_heads = 1 when
+ *     prefix_bound is not NULL (KVB_E_INVAL otherwise).
+ * Between the two calls the caller's candidate buffers must stay valid and
+ * nothing else may run on this bank; kvb_admit, kvb_admit_begin and
+ * kvb_bank_import cancel a begun step.  kvb_admit_finish without a begun step
+ * of that layer returns KVB_E_STATE.  Both are asynchronous on `stream`. */
+KVB_API kvb_status kvb_admit_begin(kvb_bank* bank, int32_t layer, const void* candK, const void* candV,
+                                   const int32_t* cand_ids, int32_t N, int32_t* prefix_out, void* stream);
+KVB_API kvb_status kvb_admit_finish(kvb_bank* bank, int32_t layer, const int32_t* prefix_bound, void* stream);
+
 /* Forcing-KV history update with the frames of a finalised chunk (§3.3-§3.5):
  * head_is_static: host [H] (1 static, 0 dynamic); newK/newV: device
  * [H][n_frames*F][d] (frames oldest first; the sink frame is never passed);

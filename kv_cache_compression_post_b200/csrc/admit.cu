@@ -219,6 +219,7 @@ __global__ void __launch_bounds__(kSelThreads) admit_select_kernel(const AdmitPl
   int Pt = p.feasible[h];
   if (p.sync_heads)
     for (int g = 0; g < p.H; ++g) Pt = min(Pt, p.feasible[g]);
+  if (p.p_bound) Pt = min(Pt, max(0, *p.p_bound));
   const int P = min(Pt, min(p.M, p.N));
   const float mean0 = p.mean0[h];
   const float* rb = p.rhoB + static_cast<size_t>(h) * p.ldN;
@@ -242,6 +243,13 @@ __global__ void __launch_bounds__(kSelThreads) admit_select_kernel(const AdmitPl
     p.stats[h].admitted = P;
     p.stats[h].feasible = p.feasible[h];
   }
+}
+
+__global__ void feasible_min_kernel(const AdmitPlan p, int* out) {
+  int v = min(p.M, p.N);
+  for (int h = threadIdx.x; h < p.H; h += 32) v = min(v, p.feasible[h]);
+  for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (threadIdx.x == 0) out[0] = v;
 }
 
 // 64-byte augmented row, the group's lanes 0..3
@@ -442,6 +450,11 @@ __global__ void finalize_kernel(const AdmitPlan p) {
 cudaError_t launch_admit_count(const AdmitPlan& p, cudaStream_t st) {
   LaunchTrace trace("admit_count_kernel", st);
   admit_count_kernel<<<p.H, kSelThreads, 0, st>>>(p);
+  return cudaGetLastError();
+}
+cudaError_t launch_feasible_min(const AdmitPlan& p, int* out, cudaStream_t st) {
+  LaunchTrace trace("feasible_min_kernel", st);
+  feasible_min_kernel<<<1, 32, 0, st>>>(p, out);
   return cudaGetLastError();
 }
 cudaError_t launch_admit_select(const AdmitPlan& p, cudaStream_t st) {

@@ -20,6 +20,7 @@ struct AdmitPlan {
   int cand_order = KVB_ORDER_DISTURBANCE;
   int baselines = KVB_BASELINES_FIXED;
   int evict_order = KVB_EVICT_THRESHOLD_RATIO;
+  const int* p_bound = nullptr;  // device: an outside bound on P (the other ranks' prefixes), or null
   // bank (this layer)
   void* K = nullptr;
   void* V = nullptr;
@@ -61,6 +62,8 @@ struct AdmitPlan {
 };
 
 cudaError_t launch_admit_count(const AdmitPlan& p, cudaStream_t st);
+// out[0] = min(min_h feasible_h, M, N): the prefix this bank's heads allow
+cudaError_t launch_feasible_min(const AdmitPlan& p, int* out, cudaStream_t st);
 cudaError_t launch_admit_select(const AdmitPlan& p, cudaStream_t st);
 cudaError_t launch_gather_admitted(const AdmitPlan& p, int maxP, cudaStream_t st);
 cudaError_t launch_evict_select(const AdmitPlan& p, cudaStream_t st);

@@ -244,22 +244,19 @@ cudaError_t run_pass(kvb_bank* b, const Pass& ps, const DeviceInfo& dev, cudaStr
   return e;
 }
 
-}  // namespace
-
-extern "C" kvb_status kvb_admit(kvb_bank* b, int32_t layer, const void* candK, const void* candV,
-                                const int32_t* cand_ids, int32_t N, void* stream) {
+// Checks the arguments of an admit step and fills its plan (no launch).
+kvb_status admit_plan(kvb_bank* b, int32_t layer, const void* candK, const void* candV, const int32_t* cand_ids,
+                      int32_t N, AdmitPlan* out) {
   if (!b) return KVB_E_INVAL;
   const kvb_config& g = b->cfg;
   if (g.method != KVB_DENSITYKV) return KVB_E_STATE;
   if (layer < 0 || layer >= g.layers || N < 1 || N > g.max_candidates) return KVB_E_INVAL;
   if (!candK || !candV || !cand_ids) return KVB_E_INVAL;
-  DeviceInfo dev;
-  if (!current_device(&dev)) return KVB_E_CUDA;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int H = g.heads, M = g.capacity, d = g.head_dim;
   const size_t lo = static_cast<size_t>(layer) * H * M;  // slot offset of this layer
 
-  AdmitPlan p;
+  AdmitPlan& p = *out;
+  p = AdmitPlan();
   p.H = H;
   p.M = M;
   p.N = N;
@@ -307,6 +304,14 @@ extern "C" kvb_status kvb_admit(kvb_bank* b, int32_t layer, const void* candK, c
   p.ldN = b->ldN;
   p.status = b->status;
 
+  return KVB_OK;
+}
+
+// Pass 1 and the feasible counts: everything before the prefix is fixed.
+cudaError_t admit_phase1(kvb_bank* b, const AdmitPlan& p, const DeviceInfo& dev, cudaStream_t st) {
+  const kvb_config& g = b->cfg;
+  const int H = p.H, M = p.M, N = p.N, d = p.d;
+  const void* candK = p.candK;
   cudaError_t e = cudaSuccess;
   if (g.dtype == KVB_BF16)
     e = launch_aug_rows(candK, g.dtype, H, N, d, N, nullptr, N, b->caug, b->ldN, reinterpret_cast<float*>(b->status + 1),
@@ -320,7 +325,14 @@ extern "C" kvb_status kvb_admit(kvb_bank* b, int32_t layer, const void* candK, c
     e = run_pass(b, ps, dev, st);
   }
   if (e == cudaSuccess) e = launch_admit_count(p, st);
-  if (e == cudaSuccess) e = launch_admit_select(p, st);
+  return e;
+}
+
+// Selection under the prefix, projected growth, eviction, compaction and the
+// incremental density update.
+cudaError_t admit_phase2(kvb_bank* b, const AdmitPlan& p, const DeviceInfo& dev, cudaStream_t st) {
+  const int M = p.M, N = p.N;
+  cudaError_t e = launch_admit_select(p, st);
   if (e == cudaSuccess) e = launch_gather_admitted(p, N < M ? N : M, st);
   // pass 2: projected growth of every bank entry from the admitted block
   if (e == cudaSuccess) {
@@ -351,7 +363,59 @@ extern "C" kvb_status kvb_admit(kvb_bank* b, int32_t layer, const void* candK, c
     e = run_pass(b, ps, dev, st);
   }
   if (e == cudaSuccess) e = launch_finalize(p, st);
+  return e;
+}
+
+}  // namespace
+
+extern "C" kvb_status kvb_admit(kvb_bank* b, int32_t layer, const void* candK, const void* candV,
+                                const int32_t* cand_ids, int32_t N, void* stream) {
+  AdmitPlan p;
+  const kvb_status s = admit_plan(b, layer, candK, candV, cand_ids, N, &p);
+  if (s != KVB_OK) return s;
+  DeviceInfo dev;
+  if (!current_device(&dev)) return KVB_E_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  b->pending.layer = -1;  // the scratch of a begun step is overwritten
+  cudaError_t e = admit_phase1(b, p, dev, st);
+  if (e == cudaSuccess) e = admit_phase2(b, p, dev, st);
   return cuda_status(e);
+}
+
+extern "C" kvb_status kvb_admit_begin(kvb_bank* b, int32_t layer, const void* candK, const void* candV,
+                                      const int32_t* cand_ids, int32_t N, int32_t* prefix_out, void* stream) {
+  if (!prefix_out) return KVB_E_INVAL;
+  AdmitPlan p;
+  const kvb_status s = admit_plan(b, layer, candK, candV, cand_ids, N, &p);
+  if (s != KVB_OK) return s;
+  DeviceInfo dev;
+  if (!current_device(&dev)) return KVB_E_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  b->pending.layer = -1;
+  cudaError_t e = admit_phase1(b, p, dev, st);
+  if (e == cudaSuccess) e = launch_feasible_min(p, prefix_out, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  b->pending.layer = layer;
+  b->pending.candK = candK;
+  b->pending.candV = candV;
+  b->pending.cand_ids = cand_ids;
+  b->pending.N = N;
+  return KVB_OK;
+}
+
+extern "C" kvb_status kvb_admit_finish(kvb_bank* b, int32_t layer, const int32_t* prefix_bound, void* stream) {
+  if (!b) return KVB_E_INVAL;
+  if (b->cfg.method != KVB_DENSITYKV || b->pending.layer < 0 || b->pending.layer != layer) return KVB_E_STATE;
+  if (prefix_bound && !b->cfg.sync_heads) return KVB_E_INVAL;
+  AdmitPlan p;
+  const kvb_status s = admit_plan(b, layer, b->pending.candK, b->pending.candV, b->pending.cand_ids, b->pending.N, &p);
+  if (s != KVB_OK) return s;
+  DeviceInfo dev;
+  if (!current_device(&dev)) return KVB_E_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  p.p_bound = prefix_bound;
+  b->pending.layer = -1;
+  return cuda_status(admit_phase2(b, p, dev, st));
 }
 
 extern "C" {
@@ -416,6 +480,7 @@ kvb_status kvb_bank_import(kvb_bank* b, int32_t layer, int32_t head, const int32
                            const float* rho0, const void* K, const void* V, int32_t size, void* stream) {
   if (!b || layer < 0 || layer >= b->cfg.layers || head < 0 || head >= b->cfg.heads) return KVB_E_INVAL;
   if (b->cfg.method != KVB_DENSITYKV) return KVB_E_STATE;
+  b->pending.layer = -1;  // a begun admit step was computed against the old bank
   const int M = b->cfg.capacity;
   if (size < 0 || size > M) return KVB_E_INVAL;
   if (size > 0 && (!ids || !rho || !rho0 || !K || !V)) return KVB_E_INVAL;

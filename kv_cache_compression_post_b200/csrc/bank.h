@@ -57,6 +57,14 @@ struct kvb_bank {
   float* sub = nullptr;
   float* coadm = nullptr;
   float* partial = nullptr;
+  // a kvb_admit_begin whose kvb_admit_finish is still due (host-side)
+  struct PendingAdmit {
+    int layer = -1;
+    const void* candK = nullptr;
+    const void* candV = nullptr;
+    const int32_t* cand_ids = nullptr;
+    int N = 0;
+  } pending;
 
   // ---- Forcing-KV, per layer
   char* tK = nullptr;       // [L][H][F][d] transition frame (static heads)

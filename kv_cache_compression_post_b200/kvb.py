@@ -20,7 +20,7 @@ __all__ = [
     "kvb_workspace_size", "kvb_bank_create", "kvb_bank_destroy", "kvb_admit", "kvb_prune_hybrid",
     "kvb_attend", "kvb_read_stats", "kvb_bank_export", "kvb_bank_import", "kvb_device_status",
     "kvb_status_string", "kvb_launch_count", "kvb_trace_enable", "kvb_trace_read", "kvb_density_workspace_size", "kvb_density", "kvb_density_noalloc", "kvb_segment_cosine",
-    "kvb_selftest_timeout",
+    "kvb_selftest_timeout", "kvb_admit_begin", "kvb_admit_finish",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvb.so")
@@ -108,6 +108,8 @@ _SIGS = {
     "kvb_segment_cosine": (ctypes.c_int, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_int, _vp,
                                           _vp]),
     "kvb_selftest_timeout": (ctypes.c_int, [_vp, _vp, ctypes.c_int64, _vp]),
+    "kvb_admit_begin": (ctypes.c_int, [_vp, _i32, _vp, _vp, _vp, _i32, _vp, _vp]),
+    "kvb_admit_finish": (ctypes.c_int, [_vp, _i32, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -175,6 +177,15 @@ def kvb_bank_destroy(bank: int) -> None:
 
 def kvb_admit(bank: int, layer: int, candK, candV, cand_ids, N: int, stream=None) -> None:
     _check(lib.kvb_admit(bank, layer, _ptr(candK), _ptr(candV), _ptr(cand_ids), N, _stream(stream)), "kvb_admit")
+
+
+def kvb_admit_begin(bank: int, layer: int, candK, candV, cand_ids, N: int, prefix_out, stream=None) -> None:
+    _check(lib.kvb_admit_begin(bank, layer, _ptr(candK), _ptr(candV), _ptr(cand_ids), N, _ptr(prefix_out),
+                               _stream(stream)), "kvb_admit_begin")
+
+
+def kvb_admit_finish(bank: int, layer: int, prefix_bound=None, stream=None) -> None:
+    _check(lib.kvb_admit_finish(bank, layer, _ptr(prefix_bound), _stream(stream)), "kvb_admit_finish")
 
 
 def kvb_prune_hybrid(bank: int, layer: int, head_is_static, newK, newV, nextK, new_ids, n_frames: int,
@@ -279,6 +290,12 @@ class Bank:
 
     def admit(self, layer, candK, candV, cand_ids, stream=None):
         kvb_admit(self.handle, layer, candK, candV, cand_ids, cand_ids.shape[0], stream)
+
+    def admit_begin(self, layer, candK, candV, cand_ids, prefix_out, stream=None):
+        kvb_admit_begin(self.handle, layer, candK, candV, cand_ids, cand_ids.shape[0], prefix_out, stream)
+
+    def admit_finish(self, layer, prefix_bound=None, stream=None):
+        kvb_admit_finish(self.handle, layer, prefix_bound, stream)
 
     def prune_hybrid(self, layer, head_is_static, newK, newV, nextK, new_ids, n_frames, stream=None):
         kvb_prune_hybrid(self.handle, layer, head_is_static, newK, newV, nextK, new_ids, n_frames, stream)
