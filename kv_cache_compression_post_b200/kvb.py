@@ -293,9 +293,12 @@ class Bank:
 
     def admit_begin(self, layer, candK, candV, cand_ids, prefix_out, stream=None):
         kvb_admit_begin(self.handle, layer, candK, candV, cand_ids, cand_ids.shape[0], prefix_out, stream)
+        # the library reads the candidates again in kvb_admit_finish: keep them alive
+        self._pending = (candK, candV, cand_ids)
 
     def admit_finish(self, layer, prefix_bound=None, stream=None):
         kvb_admit_finish(self.handle, layer, prefix_bound, stream)
+        self._pending = None
 
     def prune_hybrid(self, layer, head_is_static, newK, newV, nextK, new_ids, n_frames, stream=None):
         kvb_prune_hybrid(self.handle, layer, head_is_static, newK, newV, nextK, new_ids, n_frames, stream)

@@ -44,9 +44,11 @@ def test_two_bank_head_split_matches_oracle():
         x = L.step(i)
         r = dkv.admit(banks, x["cand_ids"], x["candK"], x["candV"], p)
         ids = dev_ids(x["cand_ids"])
-        for (h0, h1), bank, pre in zip(SPLIT, gb, prefix):
+        # each half's candidate buffers stay alive until its kvb_admit_finish has run
+        cand = [(dev_tensor(x["candK"][h0:h1]), dev_tensor(x["candV"][h0:h1])) for h0, h1 in SPLIT]
+        for (h0, h1), bank, pre, (cK, cV) in zip(SPLIT, gb, prefix, cand):
             import_oracle_banks(bank, banks[h0:h1], p, w)
-            bank.admit_begin(0, dev_tensor(x["candK"][h0:h1]), dev_tensor(x["candV"][h0:h1]), ids, pre)
+            bank.admit_begin(0, cK, cV, ids, pre)
         bound = torch.minimum(prefix[0], prefix[1])
         for bank in gb:
             bank.admit_finish(0, bound)
