@@ -160,3 +160,12 @@ def test_selftest_timeout_argument_errors_without_gpu():
     assert kvb.lib.kvb_selftest_timeout(fake, None, 1000, None) == 1
     assert kvb.lib.kvb_selftest_timeout(fake, fake, 999, None) == 1
     assert kvb.lib.kvb_selftest_timeout(fake, fake, 100_000_001, None) == 1
+
+
+def test_admit_halves_argument_errors_without_gpu():
+    import ctypes
+    import kv_cache_compression_post_b200 as kvb
+    fake = ctypes.c_void_p(256)   # never dereferenced: the checks return before any launch
+    assert kvb.lib.kvb_admit_begin(None, 0, fake, fake, fake, 10, fake, None) == 1    # no bank
+    assert kvb.lib.kvb_admit_begin(fake, 0, fake, fake, fake, 10, None, None) == 1    # no prefix_out
+    assert kvb.lib.kvb_admit_finish(None, 0, None, None) == 1
