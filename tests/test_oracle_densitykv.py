@@ -147,6 +147,74 @@ def test_rollout_invariants(tau):
         assert any(0 < len(rec["admit"].admitted[0]) < len(rec["inputs"]["cand_ids"]) for rec in res)
 
 
+def _switch_rollout(tau, **switches):
+    w = kvgen.WORKLOADS["tiny"]
+    L = kvgen.LayerInputs(w, 0, tagged=True)
+    p = dkv.Params(capacity=w.capacity, tau=tau, eps=w.eps, s=w.s, **switches)
+    return p, dkv.rollout(L, p, 7, attend=False)
+
+
+def _lead_run(score, ids, tau):
+    """Brute force: walk the candidates by id until the first one above tau."""
+    n = 0
+    for k in np.argsort(ids, kind="stable"):
+        if not score[k] <= tau:
+            break
+        n += 1
+    return n
+
+
+@pytest.mark.parametrize("tau,switches", [
+    (2.0, dict(baselines="refresh")),
+    (2.0, dict(eviction="densest")),
+    (2.0, dict(eviction="source")),
+    (1.0, dict(cand_order="source")),
+    (1.0, dict(cand_order="source", sync_heads=False)),
+])
+def test_ablation_switch_invariants(tau, switches):
+    """What each App. E switch implies, checked on the outputs of seeded tiny
+    rollouts by direct computation (sorts and loops over the step's results)."""
+    p, res = _switch_rollout(tau, **switches)
+    exercised = False
+    for rec in res:
+        r = rec["admit"]
+        ids_c = np.asarray(rec["inputs"]["cand_ids"])
+        N = ids_c.size
+        for hh, b in enumerate(r.banks):
+            old_ids = (res[rec["step"] - 2]["admit"].banks[hh].ids if rec["step"] > 1 else np.zeros(0, np.int64))
+            if switches.get("baselines") == "refresh":
+                np.testing.assert_allclose(b.rho0, r.rho_new[hh], rtol=1e-14)
+            if switches.get("eviction") == "densest":
+                assert not r.mandatory[hh].any()
+                ev = r.evicted[hh]
+                assert ev.sum() == max(0, old_ids.size + len(r.admitted[hh]) - p.capacity)
+                rhat = r.rho_cur[hh] + r.proj[hh]
+                if ev.any() and (~ev).any():
+                    assert rhat[ev].min() >= rhat[~ev].max()
+                    exercised = True
+            if switches.get("eviction") == "source":
+                np.testing.assert_array_equal(r.mandatory[hh], r.ratio[hh] > p.tau)
+                cap = r.evicted[hh] & ~r.mandatory[hh]
+                kept = ~r.evicted[hh]
+                if cap.any() and kept.any():
+                    assert old_ids[cap].max() < old_ids[kept].min()
+                    exercised = True
+            if switches.get("cand_order") == "source":
+                run = _lead_run(r.score[hh], ids_c, p.tau)
+                assert int(r.P_h[hh]) == run
+                adm = np.sort(ids_c[r.admitted[hh]])
+                np.testing.assert_array_equal(adm, np.sort(ids_c)[:adm.size])
+                assert np.all(r.score[hh][r.admitted[hh]] <= p.tau)
+                if 0 < run < N:
+                    exercised = True
+        if switches.get("cand_order") == "source":
+            P_expect = [min(int(r.P_h.min()), p.capacity, N)] * len(r.banks) if p.sync_heads else \
+                [min(int(v), p.capacity, N) for v in r.P_h]
+            assert [len(a) for a in r.admitted] == P_expect
+    if switches.get("baselines") != "refresh":
+        assert exercised, "the rollout never reached the case the switch changes"
+
+
 def test_incremental_update_equals_from_scratch():
     """The CUDA path keeps densities incrementally (App. B.1, O(N M d_k) exact update):
     survivors rho + sum_A phi - sum_E phi; new c: rho_B(c) - sum_E phi + sum_{A, c' != c} phi."""
