@@ -215,6 +215,79 @@ def test_ablation_switch_invariants(tau, switches):
         assert exercised, "the rollout never reached the case the switch changes"
 
 
+def _run_blocks(blocks, p, perm=None, scale=1.0):
+    """Admit a list of (ids, K, V) blocks from empty banks; returns the final banks.
+    ``perm`` permutes every block's candidates; ``scale`` multiplies every key."""
+    H, d = blocks[0][1].shape[0], blocks[0][1].shape[-1]
+    banks = [dkv.HeadBank.empty(d) for _ in range(H)]
+    for ids, K, V in blocks:
+        o = perm(ids.size) if perm is not None else np.arange(ids.size)
+        banks = dkv.admit(banks, ids[o], K[:, o] * scale, V[:, o], p).banks
+    return banks
+
+
+def _bank_map(banks):
+    return [{int(i): (tuple(k), r0) for i, k, r0 in zip(b.ids, b.K.round(12), b.rho0.round(12))} for b in banks]
+
+
+def _random_blocks(seed, H=2, d=4, n=12, steps=4):
+    rng = np.random.default_rng(seed)
+    out = []
+    for t in range(steps):
+        ids = np.arange(100 * t, 100 * t + n)
+        K = rng.standard_normal((H, n, d))
+        V = np.broadcast_to(ids[None, :, None].astype(np.float64), (H, n, d)).copy()
+        out.append((ids, K, V))
+    return out
+
+
+@pytest.mark.parametrize("tau", [2.0, 1.2])   # 2.0: mandatory and capacity evictions; 1.2: P < N
+@pytest.mark.parametrize("switches", [dict(), dict(eviction="densest"), dict(eviction="source"),
+                                      dict(cand_order="source"), dict(baselines="refresh")])
+def test_admit_ignores_candidate_array_order(switches, tau):
+    """Decisions depend on (score, id), never on where a candidate sits in the
+    block: any permutation of every block leaves the same banks."""
+    p = dkv.Params(capacity=20, tau=tau, eps=0.5, s=2.0, **switches)
+    blocks = _random_blocks(1)
+    ref = _bank_map(_run_blocks(blocks, p))
+    for k in range(3):
+        rng = np.random.default_rng(10 + k)
+        got = _bank_map(_run_blocks(blocks, p, perm=lambda n: rng.permutation(n)))
+        assert [set(g) for g in got] == [set(r) for r in ref]
+        for g, r in zip(got, ref):
+            for i in r:
+                assert g[i][0] == r[i][0]
+                assert g[i][1] == pytest.approx(r[i][1], rel=1e-12)
+
+
+def test_distance_scale_enters_only_through_the_scaled_distance():
+    """phi depends on ||a - b||^2 / h: scaling every key by c and h by c^2 leaves
+    every density, score and decision unchanged (a check that h is applied to
+    the squared distance, in every pass)."""
+    blocks = _random_blocks(2)
+    c = 3.0
+    base = dkv.Params(capacity=20, tau=2.0, eps=0.5, s=2.0, h=4.0)
+    scaled = dkv.Params(capacity=20, tau=2.0, eps=0.5, s=2.0, h=4.0 * c * c)
+    a, b = _run_blocks(blocks, base), _run_blocks(blocks, scaled, scale=c)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(np.sort(x.ids), np.sort(y.ids))
+        ox, oy = np.argsort(x.ids), np.argsort(y.ids)
+        np.testing.assert_allclose(x.rho0[ox], y.rho0[oy], rtol=1e-12)
+        np.testing.assert_allclose(x.K[ox] * c, y.K[oy], rtol=1e-15)
+
+
+def test_independent_heads_equal_one_head_banks():
+    """With sync_heads=False a head's bank is exactly what a one-head layer with
+    that head's inputs produces: no information crosses heads."""
+    blocks = _random_blocks(3, H=3)
+    p = dkv.Params(capacity=20, tau=1.2, eps=0.5, s=2.0, sync_heads=False)
+    together = _run_blocks(blocks, p)
+    for hh in range(3):
+        alone = _run_blocks([(ids, K[hh:hh + 1], V[hh:hh + 1]) for ids, K, V in blocks], p)[0]
+        np.testing.assert_array_equal(together[hh].ids, alone.ids)
+        np.testing.assert_array_equal(together[hh].rho0, alone.rho0)
+
+
 def test_incremental_update_equals_from_scratch():
     """The CUDA path keeps densities incrementally (App. B.1, O(N M d_k) exact update):
     survivors rho + sum_A phi - sum_E phi; new c: rho_B(c) - sum_E phi + sum_{A, c' != c} phi."""
