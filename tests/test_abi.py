@@ -169,3 +169,21 @@ def test_admit_halves_argument_errors_without_gpu():
     assert kvb.lib.kvb_admit_begin(None, 0, fake, fake, fake, 10, fake, None) == 1    # no bank
     assert kvb.lib.kvb_admit_begin(fake, 0, fake, fake, fake, 10, None, None) == 1    # no prefix_out
     assert kvb.lib.kvb_admit_finish(None, 0, None, None) == 1
+
+
+def test_plain_c_caller_of_the_whole_path_builds(tmp_path):
+    """tests/c/c_user.c drives create / admit / attend / stats / status through
+    the header alone; it compiles as strict C99 and links against libkvb.so and
+    the CUDA runtime (running it needs a B200)."""
+    import shutil
+    import subprocess
+    import kv_cache_compression_post_b200 as kvb
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    if shutil.which("gcc") is None or not os.path.exists(os.path.join(cuda, "include", "cuda_runtime.h")):
+        pytest.skip("no C compiler or CUDA headers")
+    libdir = os.path.dirname(kvb.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    "-I", os.path.join(cuda, "include"), os.path.join(ROOT, "tests", "c", "c_user.c"),
+                    "-L", libdir, "-lkvb", "-L", os.path.join(cuda, "lib64"), "-lcudart",
+                    "-Wl,-rpath," + libdir, "-o", str(tmp_path / "c_user")], check=True)
+    assert os.path.getsize(tmp_path / "c_user") > 0
