@@ -22,6 +22,13 @@ Readings taken:
 * the dynamic history is a FIFO of the last ``hist_frames`` pruned frames; the
   sink frame (frame 0) is kept whole and separately and never enters it;
 * head labels are inputs (the offline profiling step needs a trained model).
+
+Variant (off by default): ``bottomk_scope="global"`` follows the reading notes'
+§3.5 listing instead of the §3.4 formula: the similarities of all frames pushed
+by one call are ranked together and floor(r * n_frames * n) (frame, segment)
+pairs are kept, so a frame can keep more or fewer than floor(r n) segments; ties
+go to the lower (frame, segment) position.  The CUDA path implements only the
+per-frame scope.
 """
 from __future__ import annotations
 
@@ -41,6 +48,7 @@ class Params:
     seg_w: int
     retention: float
     hist_frames: int
+    bottomk_scope: str = "frame"     # "frame" (per-frame BottomK) | "global" (over the call's frames)
 
     @property
     def F(self) -> int:
@@ -116,16 +124,27 @@ def prune_hybrid(states: List[HeadState], p: Params, newK, newV, new_ids, nextK)
             st.transition = Frame(ids[-1], K[-1], V[-1])
             continue
         st.sims, st.kept = [], []
+        sims = [segment_similarity(K[t], K[t + 1] if t + 1 < n_frames else np.asarray(nextK[hh], np.float64), segs)
+                for t in range(n_frames)]
+        keeps = _keep_sets(p, sims, kkeep)
         for t in range(n_frames):
-            succ = K[t + 1] if t + 1 < n_frames else np.asarray(nextK[hh], np.float64)
-            sim = segment_similarity(K[t], succ, segs)
-            keep = bottom_k(sim, kkeep)
+            sim, keep = sims[t], keeps[t]
             tok = np.concatenate([segs[j] for j in keep]) if keep.size else np.zeros(0, np.int64)
             st.ring.append(Frame(ids[t][tok], K[t][tok], V[t][tok]))
             st.sims.append(sim)
             st.kept.append(keep)
             while len(st.ring) > p.hist_frames:
                 st.ring.popleft()
+
+
+def _keep_sets(p: Params, sims: List[np.ndarray], kkeep: int) -> List[np.ndarray]:
+    """Kept segment indices (ascending) of each frame: BottomK per frame, or one
+    BottomK over every (frame, segment) pair of the call (global scope)."""
+    if p.bottomk_scope != "global":
+        return [bottom_k(sim, kkeep) for sim in sims]
+    n = sims[0].size
+    flat = bottom_k(np.concatenate(sims), keep_count(n * len(sims), p.retention))
+    return [flat[flat // n == t] - t * n for t in range(len(sims))]
 
 
 def history(st: HeadState, d: int):

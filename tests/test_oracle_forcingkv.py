@@ -64,6 +64,54 @@ def test_hand_built_cosines_and_bottom_k():
     assert fkv.token_cosine(np.zeros((1, 2)), np.ones((1, 2)))[0] == 0.0
 
 
+def _two_frame_chunk(d=2):
+    """Frames 1 and 2 (2 x 4 tokens, 2 x 2 segments) and the next chunk's first
+    frame, built so that both of frame 1's segments change more than either of
+    frame 2's: cos(frame1 seg0 -> frame2) = 0, seg1 = 0.5; frame 2 -> next:
+    seg0 = 0.8, seg1 = 0.9 (every token of a segment turns by the same angle)."""
+    F = 8
+    segs = fkv.segments(2, 4, 2, 2)
+    base = np.zeros((F, d))
+    base[:, 0] = 1.0
+
+    def turned(cos_by_seg, ref):
+        out = ref.copy()
+        for j, c in enumerate(cos_by_seg):
+            for k in segs[j]:
+                a = np.arctan2(ref[k, 1], ref[k, 0]) + np.arccos(c)
+                out[k] = [np.cos(a), np.sin(a)]
+        return out
+    f1 = base
+    f2 = turned([0.0, 0.5], f1)
+    nxt = turned([0.8, 0.9], f2)
+    K = np.concatenate([f1, f2])[None]
+    return K, nxt[None], np.arange(8, 24)
+
+
+def test_global_bottom_k_ranks_all_frames_of_the_call_together():
+    """The listing's variant: 2 frames x 2 segments at r = 0.5 keep floor(0.5*4) = 2
+    (frame, segment) pairs overall -- both of frame 1's, none of frame 2's --
+    where the per-frame formula keeps one segment of each frame."""
+    K, nxt, ids = _two_frame_chunk()
+    V = K.copy()
+    per = fkv.Params(2, 4, 2, 2, 0.5, 8)
+    glob = fkv.Params(2, 4, 2, 2, 0.5, 8, bottomk_scope="global")
+    a, b = [fkv.HeadState(False)], [fkv.HeadState(False)]
+    fkv.prune_hybrid(a, per, K, V, ids, nxt)
+    fkv.prune_hybrid(b, glob, K, V, ids, nxt)
+    np.testing.assert_allclose(a[0].sims[0], [0.0, 0.5], atol=1e-12)
+    np.testing.assert_allclose(a[0].sims[1], [0.8, 0.9], atol=1e-12)
+    assert [k.tolist() for k in a[0].kept] == [[0], [0]]
+    assert [k.tolist() for k in b[0].kept] == [[0, 1], []]
+    gid, _, _ = fkv.history(b[0], 2)
+    np.testing.assert_array_equal(gid, ids[:8][np.concatenate(fkv.segments(2, 4, 2, 2))])
+    # one frame per call: both scopes agree
+    c, e = [fkv.HeadState(False)], [fkv.HeadState(False)]
+    fkv.prune_hybrid(c, per, K[:, :8], V[:, :8], ids[:8], K[:, 8:])
+    fkv.prune_hybrid(e, glob, K[:, :8], V[:, :8], ids[:8], K[:, 8:])
+    assert [k.tolist() for k in c[0].kept] == [k.tolist() for k in e[0].kept] == [[0]]
+
+
 def test_bottom_k_ties_take_lower_index_and_sorted_output():
     sim = np.array([0.5, 0.2, 0.5, 0.2, 0.9])
     np.testing.assert_array_equal(fkv.bottom_k(sim, 3), [0, 1, 3])
