@@ -32,6 +32,8 @@
  *       evicted: every ratio_i > tau, then max(0, |B|-|mandatory|+P-M) more by
  *       (ratio descending, id ascending)
  *   new entries: rho0 = rho = density within the updated bank.
+ *   (The App. E ablation switches of kvb_config -- cand_order, baselines,
+ *   evict_order -- each replace one of these rules; see their enums.)
  *
  * Conventions
  *  - All device pointers are caller-owned device memory, head-major and
