@@ -61,6 +61,25 @@ def test_self_exclusion_by_id_matches_pair_loop():
         assert rho[i] == pytest.approx(acc, rel=1e-12)
 
 
+def test_exclusion_follows_ids_not_positions():
+    # rows that are a reordered subset of the columns exclude the column with
+    # their own id; rows whose ids the columns do not hold exclude nothing
+    rng = np.random.default_rng(5)
+    K = rng.standard_normal((5, 4))
+    ids = np.array([10, 11, 12, 13, 14])
+    rows, rid = K[[3, 0]], ids[[3, 0]]
+    got = density(rows, K, h=4.0, eps=0.5, s=2.0, row_ids=rid, col_ids=ids)
+    for r in range(2):
+        acc = 0.0
+        for j in range(5):
+            if ids[j] == rid[r]:
+                continue
+            acc += 1.0 / (sum((rows[r, k] - K[j, k]) ** 2 for k in range(4)) / 4.0 + 0.5)
+        assert got[r] == pytest.approx(acc, rel=1e-12)
+    fresh = density(K, K, h=4.0, eps=0.5, s=2.0, row_ids=ids + 100, col_ids=ids)
+    np.testing.assert_allclose(fresh, density(K, K, h=4.0, eps=0.5, s=2.0), rtol=1e-15)
+
+
 def test_duplicate_raises_density_by_inverse_eps_power():
     # an exact duplicate with a new id adds eps^(-s/2) to its twin (1000 at eps=1e-3, s=2)
     rng = np.random.default_rng(3)
