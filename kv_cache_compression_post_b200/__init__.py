@@ -8,7 +8,8 @@ use: importing it fails loudly if ``libkvb.so`` has not been built with
 
 
 def __getattr__(name):
-    if name.startswith("kvb_") or name in ("KvbError", "make_config", "lib", "LIB_PATH", "Bank") or name.startswith("KVB_"):
+    if name.startswith("kvb_") or name in ("KvbError", "make_config", "lib", "LIB_PATH", "Bank", "PAGES_PRESET") \
+            or name.startswith("KVB_"):
         from . import kvb as _kvb
         return getattr(_kvb, name)
     raise AttributeError(name)

@@ -13,7 +13,7 @@ import os
 from typing import Optional
 
 __all__ = [
-    "KvbError", "kvb_config", "kvb_admit_stats", "make_config", "lib", "LIB_PATH", "Bank",
+    "KvbError", "kvb_config", "kvb_admit_stats", "make_config", "lib", "LIB_PATH", "Bank", "PAGES_PRESET",
     "KVB_BF16", "KVB_F32", "KVB_DENSITYKV", "KVB_FORCINGKV",
     "KVB_ORDER_DISTURBANCE", "KVB_ORDER_SOURCE", "KVB_BASELINES_FIXED", "KVB_BASELINES_REFRESH",
     "KVB_EVICT_THRESHOLD_RATIO", "KVB_EVICT_DENSEST", "KVB_EVICT_THRESHOLD_SOURCE",
@@ -30,6 +30,12 @@ KVB_DENSITYKV, KVB_FORCINGKV = 0, 1
 KVB_ORDER_DISTURBANCE, KVB_ORDER_SOURCE = 0, 1
 KVB_BASELINES_FIXED, KVB_BASELINES_REFRESH = 0, 1
 KVB_EVICT_THRESHOLD_RATIO, KVB_EVICT_DENSEST, KVB_EVICT_THRESHOLD_SOURCE = 0, 1, 2
+
+# The Soft-Riesz parameters the DensityKV pages select (§4 parameter sensitivity,
+# App. E parameter sweeps: width sigma = 8, decay p = 2, regulariser eps fixed
+# at 1) in this library's form phi = (||a - b||^2 / h + eps)^(-s/2): h = sigma^2.
+# make_config(**PAGES_PRESET) uses them instead of the defaults (h = d, eps 1e-3).
+PAGES_PRESET = dict(dist_scale=64.0, eps=1.0, s=2.0)
 
 STATUS = {0: "KVB_OK", 1: "KVB_E_INVAL", 2: "KVB_E_WORKSPACE", 3: "KVB_E_CUDA", 4: "KVB_E_DEVICE_TIMEOUT",
           5: "KVB_E_DEVICE_BOUNDS", 6: "KVB_E_STATE", 7: "KVB_E_UNSUPPORTED"}

@@ -187,3 +187,16 @@ def test_plain_c_caller_of_the_whole_path_builds(tmp_path):
                     "-L", libdir, "-lkvb", "-L", os.path.join(cuda, "lib64"), "-lcudart",
                     "-Wl,-rpath," + libdir, "-o", str(tmp_path / "c_user")], check=True)
     assert os.path.getsize(tmp_path / "c_user") > 0
+
+
+def test_pages_preset_is_a_valid_configuration():
+    """sigma = 8, p = 2, eps = 1 in the library's parameters: h = 64, s = 2, eps = 1;
+    phi of two keys at squared distance 64 is then exactly 1/2."""
+    import numpy as np
+    import kv_cache_compression_post_b200 as kvb
+    from oracle.density import density
+    pre = kvb.PAGES_PRESET
+    assert kvb.kvb_workspace_size(kvb.make_config(**pre)) == kvb.kvb_workspace_size(kvb.make_config()) > 0
+    a, b = np.zeros((1, 128)), np.zeros((1, 128))
+    b[0, 0] = 8.0
+    assert density(a, b, h=pre["dist_scale"], eps=pre["eps"], s=pre["s"])[0] == 0.5
