@@ -112,7 +112,7 @@ typedef struct {
   int32_t evict_order;      /* kvb_evict_order */
 } kvb_config;
 
-/* Candidate ordering (App. E "candidate-ordering ablations").
+/* Candidate ordering (App. E, candidate ordering).
  *  KVB_ORDER_DISTURBANCE: candidates by (score ascending, id ascending); the
  *    feasible prefix is every candidate with score <= tau.
  *  KVB_ORDER_SOURCE: candidates in spatiotemporal source order, i.e. by id
@@ -120,14 +120,14 @@ typedef struct {
  *    lowest id, that ends before its lowest-id infeasible candidate. */
 typedef enum { KVB_ORDER_DISTURBANCE = 0, KVB_ORDER_SOURCE = 1 } kvb_cand_order;
 
-/* Density baselines (App. E "baseline ablations").
+/* Density baselines (App. E, baselines).
  *  KVB_BASELINES_FIXED: rho0 is frozen at insertion (co-admitted entries set it
  *    together, after the update).
  *  KVB_BASELINES_REFRESH: after every update every entry's rho0 becomes its
  *    density within the updated bank. */
 typedef enum { KVB_BASELINES_FIXED = 0, KVB_BASELINES_REFRESH = 1 } kvb_baselines;
 
-/* Eviction set (App. E "eviction ablations").
+/* Eviction set (App. E, eviction).
  *  KVB_EVICT_THRESHOLD_RATIO: every ratio_i > tau, then the capacity evictions by
  *    (ratio descending, id ascending).
  *  KVB_EVICT_DENSEST: no threshold step; max(0, |B| + P - M) entries by

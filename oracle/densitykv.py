@@ -7,15 +7,15 @@ Bank Update" and App. E (default policy), in the pages' order:
    (App. B.1; App. D: independent layer-head banks, M = 9,360);
 2. the finalised block's tokens are candidates; each is scored by its density
    against the head's bank, normalised by the mean of the bank's frozen
-   insertion baselines ("mean-normalised insertion disturbance", lower first;
-   App. E candidate ordering);
+   insertion baselines (the mean-normalised disturbance order of App. E, smaller
+   first);
 3. the admitted count P is the largest prefix feasible for every head of the
    layer (synchronised admission, App. E cross-head synchronisation); each head
    admits its own P lowest-scoring candidates;
 4. bank entries whose projected density ratio crosses tau are evicted first
    (threshold-first eviction, App. E); capacity eviction then removes the
-   highest-ratio entries until the bank fits M (§3, "mandatory or highest-density
-   states until capacity is released");
+   highest-ratio entries until the bank fits M (§3: the states that must go,
+   then the densest, until there is room);
 5. co-admitted candidates set their insertion baselines together, after the
    update (App. B.1: mutual interactions among the admitted block do not reject
    one another; only growth from later blocks counts); baselines of older entries
@@ -53,8 +53,8 @@ Ablation switches of App. E (off by default; each replaces one default above):
 * ``eviction="source"``: mandatory evictions as by default, then the capacity
   evictions by id ascending (oldest first) -- App. E "source-order completion".
 
-Nothing here is incremental: the CUDA path's incremental maintenance (App. B.1:
-"exact update in O(N M d_k)") is checked against these from-scratch values.
+Nothing here is incremental: the CUDA path's incremental maintenance (the exact
+O(N M d_k) update of App. B.1) is checked against these from-scratch values.
 """
 from __future__ import annotations
 
