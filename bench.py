@@ -551,7 +551,7 @@ def run_rollout(args, w, rank, world):
 
 
 # ------------------------------------------------------------------ oracle (CPU) leg
-def oracle_sample(w, reps: int = 1):
+def oracle_sample(w, reps: int = 1, warmup: int = 0):
     """Time the fp64 oracle on a bounded, stated sample of one 480P chunk-layer and
     extrapolate linearly to the full chunk-layer (rows of every density / attention
     evaluation are independent, so time scales with rows)."""
@@ -571,7 +571,7 @@ def oracle_sample(w, reps: int = 1):
     rr, qr = min(512, Mb, N), min(256, w.chunk_tokens)
     kw = dict(h=float(w.head_dim), eps=w.eps, s=w.s)
     times = []
-    for _ in range(reps):
+    for rep in range(warmup + reps):     # the first `warmup` repetitions are not kept
         t = time.perf_counter()
         density(cand[:rr], Kb, **kw)                                   # rho_B of candidates
         t1 = time.perf_counter()
@@ -585,7 +585,8 @@ def oracle_sample(w, reps: int = 1):
         t4 = time.perf_counter()
         per_head = ((t1 - t) * N / rr + (t2 - t1) * 2 * Mb / rr + (t3 - t2) * Mb / rr
                     + (t4 - t3) * w.chunk_tokens / qr)
-        times.append(per_head * w.heads * 1e3)
+        if rep >= warmup:
+            times.append(per_head * w.heads * 1e3)
     sample = (f"one head of a {w.name} chunk-layer (step {i}): density of {rr} of {N} candidates vs {Mb} bank keys, "
               f"from-scratch density of {rr} of {Mb} bank keys (x2: before and after the update), projected "
               f"growth of {rr} bank keys vs {N} candidates, attention of {qr} of {w.chunk_tokens} queries over "
@@ -593,7 +594,7 @@ def oracle_sample(w, reps: int = 1):
     return statistics.mean(times), sample
 
 
-def oracle_sample_forcing(w, reps: int = 1):
+def oracle_sample_forcing(w, reps: int = 1, warmup: int = 0):
     """Time the fp64 Forcing-KV oracle on a bounded sample of one chunk-layer: the
     hybrid prune of one static and one dynamic head (full), and attention of a
     few queries over each head's history; scaled to the workload's head labels
@@ -613,7 +614,7 @@ def oracle_sample_forcing(w, reps: int = 1):
     qr = 2048
     n_static = int(labels.sum())
     times = []
-    for _ in range(reps):
+    for rep in range(warmup + reps):     # the first `warmup` repetitions are not kept
         st = [fkv.HeadState(True), fkv.HeadState(False)]
         st[0].transition = states[0].transition
         st[1].ring = type(states[1].ring)(states[1].ring)
@@ -631,23 +632,24 @@ def oracle_sample_forcing(w, reps: int = 1):
         scale = w.chunk_tokens / qr
         static_ms = (t1 - t) + (t3 - t2) * scale
         dyn_ms = (t2 - t1) + (t4 - t3) * scale
-        times.append((n_static * static_ms + (w.heads - n_static) * dyn_ms) * 1e3)
+        if rep >= warmup:
+            times.append((n_static * static_ms + (w.heads - n_static) * dyn_ms) * 1e3)
     sample = (f"chunk {first} of layer 0: Forcing-KV prune of one static and one dynamic head (full), attention of "
               f"{qr} of {w.chunk_tokens} queries over {Ks.shape[0]} (static) and {Kd.shape[0]} (dynamic) keys; "
               f"scaled by queries and by the layer's {n_static} static / {w.heads - n_static} dynamic heads")
     return statistics.mean(times), sample
 
 
-def cpu_sample(w, reps: int = 1):
+def cpu_sample(w, reps: int = 1, warmup: int = 0):
     """(ms, cpu_baseline dict) of the oracle on a bounded sample of workload w.
 
     The oracle's differences, einsum reductions and elementwise kernels run on one
     thread; only its matrix products (attention) use the BLAS pool, so the threads
     it actually uses are max(1, BLAS pool size)."""
     if w.forcing:
-        ms, sample = oracle_sample_forcing(w, reps)
+        ms, sample = oracle_sample_forcing(w, reps, warmup)
     else:
-        ms, sample = oracle_sample(w, reps)
+        ms, sample = oracle_sample(w, reps, warmup)
     try:
         from threadpoolctl import threadpool_info
         blas_threads = max((p.get("num_threads", 1) for p in threadpool_info()), default=1)
@@ -663,7 +665,7 @@ def run_reference(args, w, rank, world):
     if rank != 0:
         return
     t0 = time.time()
-    ms, cpu = cpu_sample(w, reps=max(1, args.steps))
+    ms, cpu = cpu_sample(w, reps=max(1, args.steps), warmup=args.warmup)
     line = {"impl": "reference", "metric": METRIC, "value": round(ms, 3), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
