@@ -125,8 +125,12 @@ def _lex_order(primary: np.ndarray, ids: np.ndarray) -> np.ndarray:
 
 
 def admit(banks: List[HeadBank], cand_ids: np.ndarray, candK: np.ndarray, candV: np.ndarray,
-          p: Params, tie_margin: float = 1e-4) -> AdmitResult:
-    """One admit step for one layer.  candK/candV [H][N][d] (storage precision)."""
+          p: Params, tie_margin: float = 1e-4, prefix_bound: Optional[int] = None) -> AdmitResult:
+    """One admit step for one layer.  candK/candV [H][N][d] (storage precision).
+
+    ``prefix_bound`` caps the synchronised P from outside: the prefix the other
+    heads of the layer allow when ``banks`` holds only some of them (heads split
+    across processes); the shared P is then min(own prefix, prefix_bound)."""
     H = len(banks)
     cand_ids = np.asarray(cand_ids, dtype=np.int64)
     N = cand_ids.shape[0]
@@ -149,8 +153,12 @@ def admit(banks: List[HeadBank], cand_ids: np.ndarray, candK: np.ndarray, candV:
 
     # -- step 3: largest feasible prefix, synchronised across heads --------------------
     if p.sync_heads:
-        P_all = [int(min(P_h.min(), M, N))] * H
+        P_sync = int(min(P_h.min(), M, N))
+        if prefix_bound is not None:
+            P_sync = min(P_sync, max(0, int(prefix_bound)))
+        P_all = [P_sync] * H
     else:
+        assert prefix_bound is None, "a prefix bound needs synchronised heads"
         P_all = [int(min(P_h[hh], M, N)) for hh in range(H)]
     admitted = []
     for hh in range(H):

@@ -288,6 +288,33 @@ def test_independent_heads_equal_one_head_banks():
         np.testing.assert_array_equal(together[hh].rho0, alone.rho0)
 
 
+@pytest.mark.parametrize("tau", [2.0, 1.2])
+def test_head_split_with_min_exchange_equals_the_whole_layer(tau):
+    """Head-parallel admission: each group of heads computes its own prefix
+    min(min_h P_h, M, N), the groups exchange the MIN, and each admits under that
+    bound.  The banks equal those of one admit over every head, step after step."""
+    blocks = _random_blocks(4, H=4)
+    p = dkv.Params(capacity=20, tau=tau, eps=0.5, s=2.0)
+    groups = [(0, 1), (1, 4)]
+    whole = [dkv.HeadBank.empty(4) for _ in range(4)]
+    split = [dkv.HeadBank.empty(4) for _ in range(4)]
+    bound_used = False
+    for ids, K, V in blocks:
+        r = dkv.admit(whole, ids, K, V, p)
+        own = [min(int(dkv.admit(split[a:b], ids, K[a:b], V[a:b], p).P_h.min()), p.capacity, ids.size)
+               for a, b in groups]
+        m = min(own)
+        bound_used |= max(own) > m
+        new = []
+        for a, b in groups:
+            new += dkv.admit(split[a:b], ids, K[a:b], V[a:b], p, prefix_bound=m).banks
+        for x, y in zip(r.banks, new):
+            np.testing.assert_array_equal(x.ids, y.ids)
+            np.testing.assert_array_equal(x.rho0, y.rho0)
+        whole, split = r.banks, new
+    assert bound_used or tau == 2.0     # tau 1.2 makes the groups' prefixes differ
+
+
 def test_incremental_update_equals_from_scratch():
     """The CUDA path keeps densities incrementally (App. B.1, O(N M d_k) exact update):
     survivors rho + sum_A phi - sum_E phi; new c: rho_B(c) - sum_E phi + sum_{A, c' != c} phi."""
