@@ -4,8 +4,9 @@
 //   count     per head: mean frozen baseline of the bank, number of candidates
 //             whose disturbance score rho_B(c) / mean rho0 is <= tau
 //   select    P = min over heads (synchronised prefix) of the feasible counts,
-//             capped by M and N; each head keeps its P lowest (score, id) keys
-//             (radix select over 64-bit composite keys: exact, tie-free)
+//             capped by M and N (and by an outside bound when the layer's heads
+//             are split across banks); each head keeps its P lowest (score, id)
+//             keys (radix select over 64-bit composite keys: exact, tie-free)
 //   evict     projected ratio (rho_i + sum_A phi) / rho0_i; every entry above tau
 //             is evicted, then max(0, |B| - mandatory + P - M) more by (ratio
 //             descending, id ascending) -- another radix select
