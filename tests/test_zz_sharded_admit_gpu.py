@@ -54,6 +54,16 @@ def test_two_bank_head_split_matches_oracle():
             bank.admit_finish(0, bound)
         torch.cuda.synchronize()
         assert all(bank.status() == 0 for bank in gb)
+        banks = r.banks   # the next step starts from the oracle's banks whatever happens here
+        # one shared P on both halves; it can differ from the oracle's only through
+        # a feasibility decision within the near-tie margin (one flip in the head
+        # that sets the minimum moves every head's cut), and then the step is not compared
+        P_gpu = {st["admitted"] for bank in gb for st in bank.stats(0)}
+        assert len(P_gpu) == 1
+        P_gpu = P_gpu.pop()
+        if P_gpu != r.P:
+            assert abs(P_gpu - r.P) <= sum(len(t) for t in r.tie_cand_ids), (P_gpu, r.P)
+            continue
         all_exact = True
         for (h0, h1), bank, pre in zip(SPLIT, gb, prefix):
             if not any(r.tie_cand_ids[h0:h1]):
@@ -76,7 +86,6 @@ def test_two_bank_head_split_matches_oracle():
                 np.testing.assert_allclose(g[j]["rho0"][go], ob.rho0[oo], rtol=RTOL)
                 assert st[j]["admitted"] == len(r.admitted[hh]) == r.P
         exact_steps += int(all_exact)
-        banks = r.banks
     assert exact_steps >= (w.n_chunks - 1) // 2
     for bank in gb:
         bank.close()
