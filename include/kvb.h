@@ -227,7 +227,8 @@ KVB_API kvb_status kvb_bank_export(kvb_bank* bank, int32_t layer, int32_t head, 
 
 /* Load one (layer, head) DensityKV bank from caller device buffers (size <= M):
  * ids, rho (current density within the bank), rho0 (frozen baselines), K, V.
- * Replaces the bank's contents; used for checkpoint/resume and stepwise tests. */
+ * Replaces the bank's contents; used for checkpoint/resume and stepwise tests.
+ * A Forcing-KV bank returns KVB_E_STATE: its history is exported, not restored. */
 KVB_API kvb_status kvb_bank_import(kvb_bank* bank, int32_t layer, int32_t head, const int32_t* ids,
                            const float* rho, const float* rho0, const void* K, const void* V,
                            int32_t size, void* stream);
