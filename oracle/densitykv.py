@@ -55,6 +55,17 @@ Ablation switches of App. E (off by default; each replaces one default above):
 
 Nothing here is incremental: the CUDA path's incremental maintenance (the exact
 O(N M d_k) update of App. B.1) is checked against these from-scratch values.
+
+Near ties.  A decision is a near tie when the value that decides it lies within a
+relative margin ``tie_margin`` (1e-4) of its threshold or of the value across its
+cut (``_margins``, ``_tie_ids``).  Another implementation that rounds differently
+may legitimately take such a decision the other way.  ``admit(..., forced=...)``
+replays a step with such an outcome: it takes every head's admitted and evicted id
+sets as given, but first checks that they are an outcome of the rule under a
+relative perturbation below the margin of every value that decides them
+(``_forced_violations``), and raises ``ValueError`` otherwise.  The densities,
+baselines and bank contents of the replay then follow from those sets exactly as
+in an ordinary step.
 """
 from __future__ import annotations
 
@@ -117,6 +128,7 @@ class AdmitResult:
     margins: dict
     tie_cand_ids: List[set] = None   # per head: candidate ids in a near-tie decision
     tie_bank_ids: List[set] = None   # per head: old bank ids in a near-tie decision
+    forced: bool = False             # the decisions were given (a replay), not taken
 
 
 def _lex_order(primary: np.ndarray, ids: np.ndarray) -> np.ndarray:
@@ -125,12 +137,18 @@ def _lex_order(primary: np.ndarray, ids: np.ndarray) -> np.ndarray:
 
 
 def admit(banks: List[HeadBank], cand_ids: np.ndarray, candK: np.ndarray, candV: np.ndarray,
-          p: Params, tie_margin: float = 1e-4, prefix_bound: Optional[int] = None) -> AdmitResult:
+          p: Params, tie_margin: float = 1e-4, prefix_bound: Optional[int] = None,
+          forced=None) -> AdmitResult:
     """One admit step for one layer.  candK/candV [H][N][d] (storage precision).
 
     ``prefix_bound`` caps the synchronised P from outside: the prefix the other
     heads of the layer allow when ``banks`` holds only some of them (heads split
-    across processes); the shared P is then min(own prefix, prefix_bound)."""
+    across processes); the shared P is then min(own prefix, prefix_bound).
+
+    ``forced = (admitted_ids, evicted_ids)``, one id collection per head, replays
+    the step with those decisions instead of taking them (see the module's note on
+    near ties); ``ValueError`` if they are not an outcome of the rule within
+    ``tie_margin``."""
     H = len(banks)
     cand_ids = np.asarray(cand_ids, dtype=np.int64)
     N = cand_ids.shape[0]
@@ -164,6 +182,9 @@ def admit(banks: List[HeadBank], cand_ids: np.ndarray, candK: np.ndarray, candV:
     for hh in range(H):
         order = _lex_order(_cand_key(p, score[hh]), cand_ids)
         admitted.append(order[:P_all[hh]])
+    if forced is not None:
+        admitted = [_positions(cand_ids, forced[0][hh], "admitted candidate") for hh in range(H)]
+        P_all = [len(a) for a in admitted]
 
     # -- step 4: projected growth, threshold-first and capacity eviction ---------------
     rho_cur, proj, ratio, mand, evicted, n_cap, cutv = [], [], [], [], [], [], []
@@ -182,6 +203,10 @@ def admit(banks: List[HeadBank], cand_ids: np.ndarray, candK: np.ndarray, candV:
             rest = np.nonzero(~md)[0]
             order = _lex_order(-_cut_value(p, rt, rhat, b.ids)[rest], b.ids[rest])
             ev[rest[order[:ecap]]] = True
+        if forced is not None:
+            ev = np.zeros(b.size, bool)
+            ev[_positions(b.ids, forced[1][hh], "evicted entry")] = True
+            ecap = int((ev & ~md).sum())
         rho_cur.append(rcur)
         proj.append(pj)
         ratio.append(rt)
@@ -189,6 +214,13 @@ def admit(banks: List[HeadBank], cand_ids: np.ndarray, candK: np.ndarray, candV:
         mand.append(md)
         evicted.append(ev)
         n_cap.append(ecap)
+
+    if forced is not None:
+        bad = _forced_violations(p, tie_margin, banks, cand_ids, score, admitted, ratio,
+                                 [rc + pj for rc, pj in zip(rho_cur, proj)], evicted, prefix_bound)
+        if bad:
+            raise ValueError("forced decisions are not an outcome of the rule within the near-tie "
+                             "margin: " + "; ".join(bad[:8]))
 
     # -- step 5: new bank, baselines of co-admitted entries set together ---------------
     new_banks, rho_new = [], []
@@ -209,7 +241,153 @@ def admit(banks: List[HeadBank], cand_ids: np.ndarray, candK: np.ndarray, candV:
     near = sum(int((m < tie_margin).sum()) for m in margins.values())
     tc, tb = _tie_ids(p, score, P_h, P_all, ratio, mand, n_cap, banks, cand_ids, tie_margin, cutv)
     return AdmitResult(new_banks, P_all[0] if p.sync_heads else -1, P_h, rho_cand, score, admitted,
-                       rho_cur, proj, ratio, mand, evicted, np.array(n_cap), rho_new, near, margins, tc, tb)
+                       rho_cur, proj, ratio, mand, evicted, np.array(n_cap), rho_new, near, margins, tc, tb,
+                       forced is not None)
+
+
+def _positions(ids: np.ndarray, want, what: str) -> np.ndarray:
+    """Positions in ``ids`` of the ids in ``want`` (each must occur, once)."""
+    want = np.asarray(sorted(int(v) for v in want), np.int64)
+    if np.unique(want).size != want.size:
+        raise ValueError(f"forced decisions: a repeated {what} id")
+    pos = {int(v): k for k, v in enumerate(np.asarray(ids).tolist())}
+    missing = [int(v) for v in want if int(v) not in pos]
+    if missing:
+        raise ValueError(f"forced decisions: {what} ids not present: {missing[:8]}")
+    return np.array([pos[int(v)] for v in want], np.int64)
+
+
+def _clearly_below(a, b, m):
+    """a is below b by a relative margin of at least m (a < b and a <= (1 - m) b,
+    values >= 0): no perturbation of relative size below m makes a >= b."""
+    a, b = np.asarray(a), np.asarray(b)
+    return (a < b) & (a <= (1.0 - m) * b)
+
+
+def _order_violations(key_first: np.ndarray, ids_first: np.ndarray, key_rest: np.ndarray,
+                      ids_rest: np.ndarray, m: float) -> int:
+    """How many pairs (x in first, y in rest) break the order "x before y" by
+    (key descending, id ascending) beyond the margin: key(x) clearly below key(y),
+    or equal keys with id(x) > id(y).  Equal keys are taken exactly (no margin): the
+    same inputs give the same value in any precision, and the id then decides."""
+    if key_first.size == 0 or key_rest.size == 0:
+        return 0
+    n = int(_clearly_below(key_first[:, None], key_rest[None, :], m).sum())
+    eq = key_first[:, None] == key_rest[None, :]
+    n += int((eq & (ids_first[:, None] > ids_rest[None, :])).sum())
+    return n
+
+
+def feasible_bounds(p: Params, score: np.ndarray, cand_ids: np.ndarray, m: float):
+    """(clear, possible): a head's feasible count with tau shrunk and grown by the
+    relative margin m -- the range in which another rounding of its scores may put
+    it (DensityKV App. E feasible prefix, either candidate order)."""
+    return (_feasible_prefix(p, score <= p.tau * (1.0 - m), cand_ids),
+            _feasible_prefix(p, score < p.tau * (1.0 + m), cand_ids))
+
+
+def mandatory_bounds(p: Params, ratio: np.ndarray, m: float):
+    """(clear, possible): the number of threshold evictions (ratio > tau) with tau
+    grown and shrunk by the relative margin m; (0, 0) for densest-only."""
+    if p.eviction == "densest":
+        return 0, 0
+    return int((ratio >= p.tau * (1.0 + m)).sum()), int((ratio > p.tau * (1.0 - m)).sum())
+
+
+def _forced_violations(p, m, banks, cand_ids, score, admitted, ratio, rhat, evicted, prefix_bound):
+    """Decisions of a replay (admitted candidate positions per head, evicted flags
+    per old entry) that no relative perturbation below ``m`` of the deciding values
+    could produce under the rule.  Returns one message per violated condition.
+
+    Admission, per head with scores S (all 0 when the bank is empty or its mean
+    baseline is 0):
+      * a head's feasible count lies between the counts with tau shrunk and grown
+        by m; the shared P (synchronised heads) lies between the minima of those
+        counts (capped by M, N and the outside bound);
+      * every admitted candidate has S < tau (1 + m);
+      * disturbance order: no rejected candidate precedes an admitted one by
+        (S ascending, id ascending) beyond the margin; source order: the admitted
+        candidates are exactly the P lowest ids.
+    Eviction, per head with projected ratios R under the admitted set:
+      * the bank fits: |B| - |E| + P <= M;
+      * threshold modes: no survivor has R >= tau (1 + m); |E| lies between
+        max(#{R >= tau (1+m)}, need) and max(#{R > tau (1-m)}, need), need =
+        max(0, |B| + P - M); an evicted entry with R <= tau (1 - m) is a capacity
+        eviction, so there are only as many evictions as make room, and it precedes
+        every survivor by (R descending, id ascending)
+        beyond the margin (ratio order) or has a smaller id than every survivor
+        (source-order completion);
+      * densest-only: |E| = need, and the evicted precede the survivors by
+        (R-hat descending, id ascending) beyond the margin."""
+    H = len(banks)
+    M = p.capacity
+    N = cand_ids.shape[0]
+    out = []
+    lo_h, hi_h = [], []
+    for hh in range(H):
+        lo, hi = feasible_bounds(p, score[hh], cand_ids, m)
+        lo_h.append(lo)
+        hi_h.append(hi)
+    P_all = [len(a) for a in admitted]
+    if p.sync_heads:
+        cap = min(M, N) if prefix_bound is None else min(M, N, max(0, int(prefix_bound)))
+        lo, hi = min(min(lo_h), cap), min(min(hi_h), cap)
+        if len(set(P_all)) != 1:
+            out.append(f"admitted counts differ across synchronised heads: {P_all}")
+        elif not lo <= P_all[0] <= hi:
+            out.append(f"shared P {P_all[0]} outside [{lo}, {hi}]")
+    else:
+        for hh in range(H):
+            lo, hi = min(lo_h[hh], M, N), min(hi_h[hh], M, N)
+            if not lo <= P_all[hh] <= hi:
+                out.append(f"head {hh}: P {P_all[hh]} outside [{lo}, {hi}]")
+    for hh in range(H):
+        S = score[hh]
+        A = np.asarray(admitted[hh], np.int64)
+        rej = np.setdiff1d(np.arange(N), A)
+        if (S[A] >= p.tau * (1.0 + m)).any():
+            out.append(f"head {hh}: an admitted candidate is clearly infeasible")
+        if p.cand_order == "source":
+            if set(cand_ids[A].tolist()) != set(np.sort(cand_ids)[:A.size].tolist()):
+                out.append(f"head {hh}: source order admits other than the {A.size} lowest ids")
+        else:
+            # by (S ascending, id ascending) no rejected candidate r may precede an
+            # admitted a: S(r) clearly below S(a), or equal scores and the smaller id
+            SR, SA, iR, iA = S[rej][:, None], S[A][None, :], cand_ids[rej][:, None], cand_ids[A][None, :]
+            n = int((_clearly_below(SR, SA, m) | ((SR == SA) & (iR < iA))).sum())
+            if n:
+                out.append(f"head {hh}: {n} (admitted, rejected) pairs out of order")
+    for hh in range(H):
+        b = banks[hh]
+        R, Rh, ev = ratio[hh], rhat[hh], evicted[hh]
+        P = P_all[hh]
+        surv = ~ev
+        if b.size - int(ev.sum()) + P > M:
+            out.append(f"head {hh}: the bank exceeds M")
+        need = max(0, b.size + P - M)
+        if p.eviction == "densest":
+            if int(ev.sum()) != need:
+                out.append(f"head {hh}: densest-only evicts {int(ev.sum())}, not {need}")
+            if _order_violations(Rh[ev], b.ids[ev], Rh[surv], b.ids[surv], m):
+                out.append(f"head {hh}: an evicted entry is clearly less dense than a survivor")
+            continue
+        clear_mand = R >= p.tau * (1.0 + m)
+        maybe_mand = R > p.tau * (1.0 - m)
+        if (clear_mand & surv).any():
+            out.append(f"head {hh}: a survivor is clearly above tau")
+        E = int(ev.sum())
+        n_lo, n_hi = mandatory_bounds(p, R, m)
+        if not max(n_lo, need) <= E <= max(n_hi, need):
+            out.append(f"head {hh}: {E} evictions outside [{max(n_lo, need)}, {max(n_hi, need)}]")
+        capv = ev & ~maybe_mand            # evicted entries that can only be capacity evictions
+        if capv.any() and E > need:
+            out.append(f"head {hh}: {E} evictions where {need} make room, one of them not above tau")
+        if p.eviction == "source":
+            if capv.any() and surv.any() and b.ids[capv].max() > b.ids[surv].min():
+                out.append(f"head {hh}: a capacity eviction is younger than a survivor")
+        elif _order_violations(R[capv], b.ids[capv], R[surv], b.ids[surv], m):
+            out.append(f"head {hh}: a capacity eviction clearly ranks below a survivor")
+    return out
 
 
 def _feasible_prefix(p: Params, feasible: np.ndarray, cand_ids: np.ndarray) -> int:

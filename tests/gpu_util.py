@@ -124,3 +124,75 @@ def check_admit_sampled(w, pre, post, stats, cand_ids, candK, rng, rtol=1e-4, n=
             if evicted.size:
                 re_ = ratio(rng.choice(evicted, min(n, evicted.size), replace=False))
                 assert re_.min() >= rs.max() * (1 - rtol)
+
+
+def import_step_state(bank, banks, params, w, layer=0):
+    """Load the oracle's banks before a step into the GPU bank (the stepwise
+    tests start every GPU step from the oracle's state, so a near-tie decision
+    taken the other way never cascades into the next step)."""
+    import_oracle_banks(bank, banks, params, w, layer=layer)
+
+
+def check_admit_step(bank, w, p, banks_pre, x, r, layer=0, m=1e-4, rtol=1e-4, label=""):
+    """One GPU admit step against the oracle's step r on the same inputs and the
+    same starting banks (banks_pre, imported into the GPU bank before the step).
+
+    * The GPU's decisions (admitted candidates, evicted entries per head) must be
+      the oracle's, or an outcome of the rule within the near-tie margin m: the
+      oracle then replays the step with them (admit(..., forced=...), which raises
+      unless every differing decision is a near tie, a shared P moved by a near-tie
+      feasibility included).
+    * Against that oracle step or replay, every head's bank must match: id set,
+      K rows bit for bit, V paired with its id, rho and rho0 within rtol; and the
+      counters: admitted, size, evictions, feasible and mandatory within the
+      ranges the margin allows.
+    * At most 2 flips per oracle near-tie decision plus 3 per head and unit of P
+      moved (a shared P one higher admits one more candidate per head and may
+      evict one more entry).
+    Returns (flipped decisions, oracle near-tie decisions)."""
+    import kvgen
+    from oracle import densitykv as dkv
+    H = len(banks_pre)
+    cand_ids = np.asarray(x["cand_ids"], np.int64)
+    cset = set(cand_ids.tolist())
+    # ``bank`` may be a list of (bank, h0, h1): heads h0..h1-1 of the layer held by
+    # each of several banks (a head-parallel split)
+    parts = bank if isinstance(bank, (list, tuple)) else [(bank, 0, H)]
+    g, st = [], []
+    for b, h0, h1 in parts:
+        g += export_banks(b, layer, h1 - h0)
+        st += b.stats(layer)
+    assert len(g) == H
+    A_gpu, E_gpu, flips = [], [], 0
+    for hh in range(H):
+        got = set(g[hh]["ids"].tolist())
+        A = sorted(got & cset)
+        E = sorted(set(banks_pre[hh].ids.tolist()) - got)
+        assert len(got) == g[hh]["ids"].size, f"{label} head {hh}: repeated ids in the GPU bank"
+        A_or = set(cand_ids[r.admitted[hh]].tolist())
+        E_or = set(banks_pre[hh].ids[r.evicted[hh]].tolist())
+        flips += len(set(A) ^ A_or) + len(set(E) ^ E_or)
+        A_gpu.append(A)
+        E_gpu.append(E)
+    ref = r
+    if flips:
+        ref = dkv.admit(banks_pre, cand_ids, x["candK"], x["candV"], p, tie_margin=m, forced=(A_gpu, E_gpu))
+    dP = abs(len(A_gpu[0]) - (r.P if r.P >= 0 else len(r.admitted[0])))
+    assert flips <= 2 * r.near_ties + 3 * H * dP, \
+        f"{label}: {flips} flipped decisions for {r.near_ties} near ties and a P moved by {dP}"
+    for hh in range(H):
+        gb, ob = g[hh], ref.banks[hh]
+        assert set(gb["ids"].tolist()) == set(ob.ids.tolist()), f"{label} head {hh}: bank ids"
+        np.testing.assert_array_equal(kvgen.untag_ids(gb["V"]), gb["ids"])
+        go, oo = np.argsort(gb["ids"]), np.argsort(ob.ids)
+        np.testing.assert_array_equal(gb["K"][go], ob.K[oo].astype(np.float32))
+        np.testing.assert_allclose(gb["rho"][go], ref.rho_new[hh][oo], rtol=rtol, err_msg=f"{label} head {hh} rho")
+        np.testing.assert_allclose(gb["rho0"][go], ob.rho0[oo], rtol=rtol, err_msg=f"{label} head {hh} rho0")
+        s = st[hh]
+        assert s["admitted"] == len(A_gpu[hh]) and s["size"] == ob.size
+        assert s["mandatory"] + s["capacity_evicted"] == len(E_gpu[hh])
+        lo, hi = dkv.feasible_bounds(p, r.score[hh], cand_ids, m)
+        assert lo <= s["feasible"] <= hi, f"{label} head {hh}: feasible {s['feasible']} outside [{lo}, {hi}]"
+        mlo, mhi = dkv.mandatory_bounds(p, ref.ratio[hh], m)
+        assert mlo <= s["mandatory"] <= mhi, f"{label} head {hh}: mandatory {s['mandatory']} outside [{mlo}, {mhi}]"
+    return flips, r.near_ties

@@ -5,20 +5,18 @@ The four heads of the mid workload are split over two banks (heads 0-1 and
 prefix, the host takes the MIN (what the ranks' all-reduce computes), and
 kvb_admit_finish completes both halves.  Stepwise against the oracle's
 synchronised admit over all four heads, with the parity bar of the other
-DensityKV tests (ids exact except near ties, densities within 1e-4).  No kernel
+DensityKV tests (tests.gpu_util.check_admit_step: decisions equal to the
+oracle's or a near-tie outcome it replays, then ids, K, rho and rho0 on every
+step).  No kernel
 waits on another: the two banks run one after the other on one stream."""
-import dataclasses
-
-import numpy as np
 import pytest
 
 import kvgen
 from oracle import densitykv as dkv
-from tests.gpu_util import dev_ids, dev_tensor, export_banks, import_oracle_banks
+from tests.gpu_util import check_admit_step, dev_ids, dev_tensor, import_oracle_banks
 
 pytestmark = pytest.mark.gpu
 
-RTOL = 1e-4
 SPLIT = [(0, 2), (2, 4)]
 
 
@@ -39,7 +37,7 @@ def test_two_bank_head_split_matches_oracle():
     banks = [dkv.HeadBank.empty(w.head_dim) for _ in range(w.heads)]
     gb = [kvb.Bank(_cfg(w, h1 - h0, tau)) for h0, h1 in SPLIT]
     prefix = [torch.full((1,), -1, dtype=torch.int32, device="cuda") for _ in SPLIT]
-    exact_steps = 0
+    counts = []
     for i in range(1, w.n_chunks):
         x = L.step(i)
         r = dkv.admit(banks, x["cand_ids"], x["candK"], x["candV"], p)
@@ -54,39 +52,21 @@ def test_two_bank_head_split_matches_oracle():
             bank.admit_finish(0, bound)
         torch.cuda.synchronize()
         assert all(bank.status() == 0 for bank in gb)
-        banks = r.banks   # the next step starts from the oracle's banks whatever happens here
-        # one shared P on both halves; it can differ from the oracle's only through
-        # a feasibility decision within the near-tie margin (one flip in the head
-        # that sets the minimum moves every head's cut), and then the step is not compared
-        P_gpu = {st["admitted"] for bank in gb for st in bank.stats(0)}
-        assert len(P_gpu) == 1
-        P_gpu = P_gpu.pop()
-        if P_gpu != r.P:
-            assert abs(P_gpu - r.P) <= sum(len(t) for t in r.tie_cand_ids), (P_gpu, r.P)
-            continue
-        all_exact = True
-        for (h0, h1), bank, pre in zip(SPLIT, gb, prefix):
-            if not any(r.tie_cand_ids[h0:h1]):
-                N = len(x["cand_ids"])
-                assert int(pre.item()) == min(int(r.P_h[h0:h1].min()), w.capacity, N)
-            g = export_banks(bank, 0, h1 - h0)
-            st = bank.stats(0)
-            for j, hh in enumerate(range(h0, h1)):
-                ob = r.banks[hh]
-                diff = set(g[j]["ids"].tolist()) ^ set(ob.ids.tolist())
-                ties = r.tie_cand_ids[hh] | r.tie_bank_ids[hh]
-                assert diff <= ties, f"head {hh}: ids differ outside near ties: {sorted(diff - ties)[:10]}"
-                np.testing.assert_array_equal(kvgen.untag_ids(g[j]["V"]), g[j]["ids"])
-                if diff:
-                    all_exact = False
-                    continue
-                go, oo = np.argsort(g[j]["ids"]), np.argsort(ob.ids)
-                np.testing.assert_array_equal(g[j]["K"][go], ob.K[oo].astype(np.float32))
-                np.testing.assert_allclose(g[j]["rho"][go], r.rho_new[hh][oo], rtol=RTOL)
-                np.testing.assert_allclose(g[j]["rho0"][go], ob.rho0[oo], rtol=RTOL)
-                assert st[j]["admitted"] == len(r.admitted[hh]) == r.P
-        exact_steps += int(all_exact)
-    assert exact_steps >= (w.n_chunks - 1) // 2
+        # each half's prefix: min(its heads' feasible counts, M, N), within the
+        # ranges the near-tie margin allows
+        N = len(x["cand_ids"])
+        for (h0, h1), pre in zip(SPLIT, prefix):
+            lo = min(min(dkv.feasible_bounds(p, r.score[hh], x["cand_ids"], 1e-4)[0] for hh in range(h0, h1)),
+                     w.capacity, N)
+            hi = min(min(dkv.feasible_bounds(p, r.score[hh], x["cand_ids"], 1e-4)[1] for hh in range(h0, h1)),
+                     w.capacity, N)
+            assert lo <= int(pre.item()) <= hi, (i, h0, int(pre.item()), lo, hi)
+        # the layer as a whole against the oracle's synchronised step over all four
+        # heads: one shared P, decisions equal or a near-tie outcome it replays
+        parts = [(bank, h0, h1) for bank, (h0, h1) in zip(gb, SPLIT)]
+        counts.append(check_admit_step(parts, w, p, banks, x, r, label=f"head split step {i}"))
+        banks = r.banks
+    print(f"\nhead split: per step (flips, oracle near ties): {counts}")
     for bank in gb:
         bank.close()
 
