@@ -269,7 +269,10 @@ def kernel_units(w, name, N, st_before, st_after, n_frames, labels):
     moved = sum(s.get("moved", 0) for s in st_after)
     size = sum(s["size"] for s in st_after)
     if name == "gram_bf16_kernel":
-        return "tensor", 2.0 * w.head_dim * sum(pairs), "2*d flops per pair over the four density passes"
+        # the method's own work (DensityKV App. B.1): N*|B| + P^2 + E*(|B| - E + P)
+        # pairs; the projected-growth pass recomputes |B|*P pairs on top (executed)
+        return "tensor", density_flops_algorithmic(w, N, st_before, st_after), \
+            "2*d flops per pair over N*|B| + P^2 + E*(|B|-E+P) pairs (executed: + |B|*P of the growth pass)"
     if name == "attend_bf16_kernel":
         return "tensor", attention_flops(w, [s["size"] for s in st_after]), "4*Nq*(Ls+|B_h|+Lw)*d flops"
     if name == "aug_rows_kernel":
@@ -287,9 +290,11 @@ def kernel_units(w, name, N, st_before, st_after, n_frames, labels):
     return "latency", None, "selection (one CTA per head)"
 
 
-def kernel_table(w, records, steps, per_step_units, peaks):
+def kernel_table(w, records, steps, per_step_units, peaks, executed=None):
     """Per-kernel live timing (library launch trace, CUDA events on the launch
-    stream) against its roofline."""
+    stream) against its roofline.  `executed`: flops per step a kernel executes
+    beyond its algorithmic count (the density Gram's recomputed growth pass),
+    reported beside the algorithmic fraction."""
     agg = {}
     for n, ms in records:
         a = agg.setdefault(n, [0, 0.0])
@@ -306,6 +311,10 @@ def kernel_table(w, records, steps, per_step_units, peaks):
                 ach = units / (ms / steps * 1e-3) / 1e12
                 e.update(achieved=round(ach, 2), unit="TFLOP/s", peak=peaks["bf16_tflops"],
                          frac=round(ach / peaks["bf16_tflops"], 4))
+                ex = (executed or {}).get(n)
+                if ex:
+                    ach_x = ex / (ms / steps * 1e-3) / 1e12
+                    e.update(executed_tflops=round(ach_x, 2), executed_frac=round(ach_x / peaks["bf16_tflops"], 4))
             else:
                 ach = units / (ms / steps * 1e-3) / 1e9
                 e.update(achieved=round(ach, 1), unit="GB/s", peak=peaks["hbm_gbs"],
@@ -362,8 +371,9 @@ def run_workload(args, w, rank, world):
     barrier(world)
     torch.cuda.synchronize()
     sampler.start()
-    per_step, upd_ms, att_ms, att_fl, den_fl, den_alg = [], [], [], [], [], []
+    per_step, upd_ms, att_ms, att_fl, den_fl, den_alg, ties = [], [], [], [], [], [], []
     units = {}
+    gram_exec = 0.0
     launches0 = kvb.kvb_launch_count()
     timed_end = first + args.warmup + args.steps
     launches = None
@@ -397,7 +407,10 @@ def run_workload(args, w, rank, world):
             if not w.forcing:
                 den_fl.append(density_flops(w, N, st_before, st))
                 den_alg.append(density_flops_algorithmic(w, N, st_before, st))
+                ties.append(sum(s_["near_ties"] for s_ in st))
             continue
+        if not w.forcing:
+            gram_exec += density_flops(w, N, st_before, st)
         for name in ("gram_bf16_kernel", "attend_bf16_kernel", "aug_rows_kernel", "gather_admitted_kernel",
                      "gather_evicted_kernel", "compact_kernel", "finalize_kernel", "gram_reduce_kernel",
                      "admit_count_kernel", "admit_select_kernel", "evict_select_kernel", "seg_cosine_kernel",
@@ -413,32 +426,68 @@ def run_workload(args, w, rank, world):
         raise RuntimeError(f"device status {status}")
     total_ms = max_over_ranks(sum(per_step), world)
 
-    # end-to-end: host (pinned) inputs in, result out, every step
-    Oh = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+    # end-to-end: every step's inputs go in from pinned host memory and its output
+    # comes back, inside the timed region.  Two device input sets and two outputs
+    # let the copies overlap the compute: step j+1's inputs travel on an upload
+    # stream while step j runs, and step j's output on a download stream once it
+    # is done (copies in the two directions use separate engines).
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    keys = sorted(hosted)
+    proto = hosted[keys[0]]
+    bufs = [{k: torch.empty_like(v, device="cuda") for k, v in proto.items()} for _ in range(2)]
+    outs = [O, torch.empty_like(O)]
+    Oh = [torch.empty(O.shape, dtype=O.dtype).pin_memory() for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_back = [torch.cuda.Event() for _ in range(2)]
     h2d = d2h = 0
-    dev_bufs = {k: torch.empty_like(v, device="cuda") for k, v in next(iter(hosted.values())).items()}
+
+    def upload(j, b):
+        nonlocal h2d
+        for k, v in hosted[keys[j]].items():
+            if bufs[b][k].shape != v.shape:
+                raise RuntimeError("end-to-end inputs change shape between steps")
+            bufs[b][k].copy_(v, non_blocking=True)
+            h2d += v.numel() * v.element_size()
+        ev_in[b].record(up)
+
     barrier(world)
     torch.cuda.synchronize()
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e_start.record(stream)
-    for i in sorted(hosted):
-        hx = hosted[i]
-        for k, v in hx.items():
-            if dev_bufs[k].shape != v.shape:
-                dev_bufs[k] = torch.empty_like(v, device="cuda")
-            dev_bufs[k].copy_(v, non_blocking=True)
-            h2d += v.numel() * v.element_size()
-        step(dev_bufs)
-        Oh.copy_(O, non_blocking=True)
+    up.wait_event(e_start)
+    down.wait_event(e_start)
+    with torch.cuda.stream(up):
+        upload(0, 0)
+    for j in range(len(keys)):
+        b = j % 2
+        stream.wait_event(ev_in[b])
+        if j >= 2:
+            stream.wait_event(ev_back[b])       # outs[b] has been read back
+        x = bufs[b]
+        update(x)
+        bank.attend(0, x["Q"], x["sinkK"], x["sinkV"], x["winK"], x["winV"], outs[b], lse, stream)
+        ev_done[b].record(stream)
+        if j + 1 < len(keys):
+            if j >= 1:
+                up.wait_event(ev_done[1 - b])   # step j-1 no longer reads bufs[1-b]
+            with torch.cuda.stream(up):
+                upload(j + 1, 1 - b)
+        down.wait_event(ev_done[b])
+        with torch.cuda.stream(down):
+            Oh[b].copy_(outs[b], non_blocking=True)
+            ev_back[b].record(down)
         d2h += O.numel() * O.element_size()
+    stream.wait_stream(down)
     e_end.record(stream)
     torch.cuda.synchronize()
     e2e_total = max_over_ranks(e_start.elapsed_time(e_end), world)
-    nh = len(hosted)
+    nh = len(keys)
 
     peaks, peak_src = load_peaks()
     per_step_units = {n: (b, (u / n_trace if u is not None else None), t) for n, (b, u, t) in units.items()}
-    kernels = kernel_table(w, records, n_trace, per_step_units, peaks)
+    kernels = kernel_table(w, records, n_trace, per_step_units, peaks,
+                           executed={"gram_bf16_kernel": gram_exec / n_trace} if not w.forcing else None)
     att_achieved = statistics.mean(f / (t * 1e-3) for f, t in zip(att_fl, att_ms)) / 1e12
     bf16_peak = peaks["bf16_tflops"]
 
@@ -450,6 +499,8 @@ def run_workload(args, w, rank, world):
              "launches_per_step": k["launches_per_step"], "ms_per_launch": k["ms_per_launch"],
              "peak_source": f"{peak_src} " + ("bf16 burst" if k["bound"] == "tensor" else "HBM copy"),
              "algorithmic": k["algorithmic"]}
+        if "executed_tflops" in k:
+            r.update(executed_tflops=k["executed_tflops"], executed_frac=k["executed_frac"])
         return r
 
     # the dominant kernel: largest share of the step's device time (traced steps)
@@ -472,6 +523,9 @@ def run_workload(args, w, rank, world):
                          density_algorithmic_gflop=round(statistics.mean(den_alg) / 1e9, 1),
                          density_executed_gflop=round(statistics.mean(den_fl) / 1e9, 1),
                          admitted=[s["admitted"] for s in bank.stats(0)][:1])
+        near_ties = {"per_step": ties, "total": int(sum(ties)),
+                     "what": "admit/evict decisions within 1e-4 (relative) of their threshold or cut, "
+                             "counted by the kernels from their fp32 values, summed over heads"}
     else:
         breakdown.update(static_heads=[int(v) for v in labels])
     return {
@@ -483,6 +537,7 @@ def run_workload(args, w, rank, world):
         "roofline_other": others,
         "kernels": kernels,
         "breakdown": breakdown,
+        "near_ties": None if w.forcing else near_ties,
         "gen_s": round(gen_s, 1),
         "first_timed_chunk": first + args.warmup,
     }
@@ -770,6 +825,7 @@ def run_kvb(args, w, rank, world, local):
         "roofline_other": r["roofline_other"],
         "kernels": r["kernels"],
         "breakdown": r["breakdown"],
+        "near_ties": r["near_ties"],
         "clocks": r["clocks"],
         "cpu_baseline": cpu,
     }

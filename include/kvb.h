@@ -146,7 +146,12 @@ typedef struct {
   int32_t capacity_evicted;
   int32_t size;          /* bank size after the update (ring size for Forcing-KV) */
   int32_t moved;         /* DensityKV: surviving entries moved from the tail into holes */
-  int32_t reserved[2];
+  int32_t near_ties;     /* DensityKV: decisions of this step whose deciding value, as the
+                            kernels compute it in fp32, lies within 1e-4 (relative) of its
+                            threshold (a score or projected ratio vs tau) or of the value
+                            across its cut (the shared-prefix cut, the capacity cut):
+                            the decisions another rounding could take the other way */
+  int32_t reserved;
 } kvb_admit_stats;
 
 typedef struct kvb_bank kvb_bank; /* opaque, host-side */
@@ -318,10 +323,15 @@ KVB_API kvb_status kvb_density(const void* rows, int32_t n_rows, const void* col
  *   256 + 64*H*n_rows + 64*H*n_cols + 64*H*n_rows  (each term rounded up to
  *   256 bytes)  <=  4 MiB.
  * The first call on a device looks up the array's address with that device
- * current: make it before any stream capture.  All calls on a device share the
- * array (it keeps the last call's contents); calls that overlap on the GPU race,
- * so order them on one stream.  status_out: device int32 (may be NULL) that
- * receives this call's device status (zeroed by the call). */
+ * current: make it before any stream capture.  The address is kept for the life
+ * of the process; after a cudaDeviceReset of that device it is stale, so do not
+ * call this entry point on a device that has been reset.  All calls on a device
+ * share the array (it keeps the last call's contents); calls that overlap on the
+ * GPU race, so order them on one stream.  status_out: device int32 that receives
+ * this call's device status (zeroed by the call).  It may be NULL: a device-side
+ * failure (a bounded wait that gave up) is then written to a word inside the
+ * shared array that no call reads back, so it goes unreported and `out` may hold
+ * partial sums; pass status_out to learn of it. */
 KVB_API kvb_status kvb_density_noalloc(const void* rows, int32_t n_rows, const void* cols, int32_t n_cols,
                                        int32_t heads, int32_t head_dim, kvb_dtype dtype, float dist_scale,
                                        float eps, float s, int32_t exclude_diagonal, float* out,

@@ -66,6 +66,37 @@ __device__ __forceinline__ float block_sum(float v, SelShared* S) {
   return t;
 }
 
+// block-wide max (min via negation); every thread receives the result
+__device__ __forceinline__ float block_max(float v, SelShared* S) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) S->fred[w] = v;
+  __syncthreads();
+  float t = -INFINITY;
+  if (w == 0) {
+    t = (l < static_cast<int>(blockDim.x >> 5)) ? S->fred[l] : -INFINITY;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, o));
+    if (l == 0) S->fred[0] = t;
+  }
+  __syncthreads();
+  t = S->fred[0];
+  __syncthreads();
+  return t;
+}
+
+// Near-tie accounting (the decisions another rounding could take the other way):
+// a value within kTieMargin, relative, of its threshold, or a cut whose two sides
+// (last value taken, first value left) are that close.  Counted per head into
+// kvb_admit_stats.near_ties from the kernels' own fp32 values.
+constexpr float kTieMargin = 1e-4f;
+__device__ __forceinline__ bool near_tau(float v, float tau) { return fabsf(v - tau) < kTieMargin * tau; }
+__device__ __forceinline__ bool near_cut(float taken, float left) {
+  return taken != 0.f && fabsf(left - taken) < kTieMargin * fabsf(taken);
+}
+
 // exclusive scan over the block; *total receives the sum
 __device__ __forceinline__ int block_excl_scan(int v, SelShared* S, int* total) {
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
@@ -207,10 +238,17 @@ __global__ void __launch_bounds__(kSelThreads) admit_count_kernel(const AdmitPla
   }
   int total;
   block_excl_scan(cnt, &S, &total);
+  // admission-threshold near ties (scores exist only against a bank with a mean baseline)
+  int nt = 0;
+  if (n > 0 && mean0 > 0.f)
+    for (int c = threadIdx.x; c < p.N; c += blockDim.x) nt += near_tau(score_of(rb[c], mean0), p.tau) ? 1 : 0;
+  int ties;
+  block_excl_scan(nt, &S, &ties);
   if (threadIdx.x == 0) {
     p.mean0[h] = mean0;
     p.feasible[h] = total;
     p.n_old[h] = n;
+    p.stats[h].near_ties = ties;
   }
 }
 
@@ -238,6 +276,18 @@ __global__ void __launch_bounds__(kSelThreads) admit_select_kernel(const AdmitPl
     const unsigned long long prefix = S.prefix, mask = S.mask;
     const int got = block_compact(0, p.N, [&](int c) { return (key(c) & mask) <= prefix; }, out, &S);
     if (threadIdx.x == 0 && got != P) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
+    if (!by_source && P < p.feasible[h]) {
+      // the cut inside the feasible set: last admitted score vs first rejected one
+      float lo = -INFINITY, nhi = -INFINITY;
+      for (int c = threadIdx.x; c < p.N; c += blockDim.x) {
+        const float sc = score_of(rb[c], mean0);
+        if ((key(c) & mask) <= prefix) lo = fmaxf(lo, sc);
+        else nhi = fmaxf(nhi, -sc);
+      }
+      lo = block_max(lo, &S);
+      nhi = block_max(nhi, &S);
+      if (threadIdx.x == 0 && near_cut(lo, -nhi)) p.stats[h].near_ties += 1;
+    }
   }
   if (threadIdx.x == 0) {
     p.P[h] = P;
@@ -328,6 +378,27 @@ __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPl
     }
   }
   __syncthreads();
+  // near ties: projected ratios within the margin of tau, and the capacity cut
+  // (last capacity eviction vs first non-mandatory survivor by the cut value)
+  {
+    int nt = 0;
+    if (mode != KVB_EVICT_DENSEST)
+      for (int i = threadIdx.x; i < n; i += blockDim.x) nt += near_tau(ratio(i), p.tau) ? 1 : 0;
+    int ties;
+    block_excl_scan(nt, &S, &ties);
+    if (ecap > 0 && ecap < n_free && mode != KVB_EVICT_THRESHOLD_SOURCE) {
+      float lo = -INFINITY, hi = -INFINITY;  // lo holds -min over the evicted
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const float v = (mode == KVB_EVICT_DENSEST) ? rho[i] + proj[i] : ratio(i);
+        if (evflag[i] == 2) lo = fmaxf(lo, -v);
+        else if (evflag[i] == 0) hi = fmaxf(hi, v);
+      }
+      lo = block_max(lo, &S);
+      hi = block_max(hi, &S);
+      if (near_cut(-lo, hi)) ties += 1;
+    }
+    if (threadIdx.x == 0) p.stats[h].near_ties += ties;
+  }
   const int E = n_mand + min(ecap, n_free);
   const int n_new = n - E + Ph;
   int* ev = p.ev_slot + base;

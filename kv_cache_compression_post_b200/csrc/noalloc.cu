@@ -14,12 +14,15 @@
 //  * Sizes whose scratch does not fit are rejected with KVB_E_WORKSPACE before
 //    anything is launched (see kvb_density_noalloc in kvb.h for the formula).
 //  * The first call on a device looks up the array's device address with that
-//    device current; make that first call before any stream capture begins.
+//    device current; make that first call before any stream capture begins.  The
+//    address is cached for the life of the process: a cudaDeviceReset of that
+//    device makes it stale, and the entry point must not be used there again.
 //  * Every call on a device shares the one array, which keeps the last call's
 //    contents.  Calls whose kernels overlap on the GPU (different streams without
 //    ordering between them) race on it; serialise them.
 //  * Device-side failures (a bounded wait that gave up) are latched into the
-//    caller's `status_out` word when one is passed (zeroed by the call).
+//    caller's `status_out` word when one is passed (zeroed by the call); without
+//    one they land in a status word inside the array that nothing reads back.
 #include <cmath>
 #include <mutex>
 

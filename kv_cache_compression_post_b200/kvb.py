@@ -64,7 +64,7 @@ class kvb_config(ctypes.Structure):
 class kvb_admit_stats(ctypes.Structure):
     _fields_ = [("admitted", ctypes.c_int32), ("feasible", ctypes.c_int32), ("mandatory", ctypes.c_int32),
                 ("capacity_evicted", ctypes.c_int32), ("size", ctypes.c_int32), ("moved", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 2)]
+                ("near_ties", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 def make_config(**kw) -> kvb_config:
@@ -216,7 +216,8 @@ def kvb_read_stats(bank: int, layer: int, heads: int, stream=None):
     arr = (kvb_admit_stats * heads)()
     _check(lib.kvb_read_stats(bank, layer, arr, _stream(stream)), "kvb_read_stats")
     return [dict(admitted=a.admitted, feasible=a.feasible, mandatory=a.mandatory,
-                 capacity_evicted=a.capacity_evicted, size=a.size, moved=a.moved) for a in arr]
+                 capacity_evicted=a.capacity_evicted, size=a.size, moved=a.moved, near_ties=a.near_ties)
+            for a in arr]
 
 
 def kvb_bank_export(bank: int, layer: int, head: int, ids, rho, rho0, K, V, stream=None) -> int:

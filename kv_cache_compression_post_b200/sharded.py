@@ -30,8 +30,18 @@ def admit_sharded(bank, layer: int, candK, candV, cand_ids, prefix, group=None, 
     ``admit_begin`` / ``admit_finish``); candK/candV are this rank's head slices
     [H_rank][N][d]; cand_ids [N] is the same on every rank; ``prefix`` is a
     one-element int32 tensor on this rank's device, reused across calls.  Every
-    rank of ``group`` must call this for the same layer and block."""
+    rank of ``group`` must call this for the same layer and block.
+
+    ``stream`` (a torch.cuda.Stream or None for the current stream) carries the
+    whole step: the collective is issued with it as torch's current stream, so
+    torch orders the all-reduce after the prefix is written and the second half
+    after the reduced value has landed."""
+    import contextlib
+
+    import torch
     import torch.distributed as dist
-    bank.admit_begin(layer, candK, candV, cand_ids, prefix, stream)
-    dist.all_reduce(prefix, op=dist.ReduceOp.MIN, group=group)
-    bank.admit_finish(layer, prefix, stream)
+    ctx = torch.cuda.stream(stream) if (stream is not None and prefix.is_cuda) else contextlib.nullcontext()
+    with ctx:
+        bank.admit_begin(layer, candK, candV, cand_ids, prefix, stream)
+        dist.all_reduce(prefix, op=dist.ReduceOp.MIN, group=group)
+        bank.admit_finish(layer, prefix, stream)

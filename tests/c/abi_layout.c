@@ -41,6 +41,7 @@ int main(void) {
   FIELD(kvb_admit_stats, capacity_evicted);
   FIELD(kvb_admit_stats, size);
   FIELD(kvb_admit_stats, moved);
+  FIELD(kvb_admit_stats, near_ties);
   FIELD(kvb_admit_stats, reserved);
   printf("sizeof.kvb_trace_record %zu\n", sizeof(kvb_trace_record));
   FIELD(kvb_trace_record, kernel);

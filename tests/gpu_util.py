@@ -195,4 +195,9 @@ def check_admit_step(bank, w, p, banks_pre, x, r, layer=0, m=1e-4, rtol=1e-4, la
         assert lo <= s["feasible"] <= hi, f"{label} head {hh}: feasible {s['feasible']} outside [{lo}, {hi}]"
         mlo, mhi = dkv.mandatory_bounds(p, ref.ratio[hh], m)
         assert mlo <= s["mandatory"] <= mhi, f"{label} head {hh}: mandatory {s['mandatory']} outside [{mlo}, {mhi}]"
+    # the kernels' own near-tie count (fp32 values) against the oracle's (fp64): a
+    # value right at the margin may fall on either side, and a flipped decision
+    # moves its cut
+    gpu_ties = sum(s["near_ties"] for s in st)
+    assert abs(gpu_ties - r.near_ties) <= 2 + 2 * flips, f"{label}: near ties {gpu_ties} (GPU) vs {r.near_ties}"
     return flips, r.near_ties

@@ -102,3 +102,49 @@ def test_begin_finish_state_errors():
     torch.cuda.synchronize()
     assert indep.status() == 0
     indep.close()
+
+
+def test_admit_sharded_on_a_side_stream():
+    """admit_sharded with a stream that is not torch's current one (a one-rank
+    NCCL group): the all-reduce must see the prefix written on that stream and the
+    second half the reduced value, so the bank equals a plain kvb_admit's."""
+    import os
+    import socket
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import kv_cache_compression_post_b200 as kvb
+    from kv_cache_compression_post_b200.sharded import admit_sharded
+    from tests.gpu_util import export_banks
+    w = kvgen.WORKLOADS["mid"]
+    L = kvgen.LayerInputs(w, 0, tagged=True)
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    store = dist.TCPStore("127.0.0.1", port, 1, True)
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1)
+    try:
+        side = torch.cuda.Stream()
+        a, b = kvb.Bank(_cfg(w, w.heads, 1.0)), kvb.Bank(_cfg(w, w.heads, 1.0))
+        prefix = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+        for i in range(1, 4):
+            x = L.step(i)
+            K, V, ids = dev_tensor(x["candK"]), dev_tensor(x["candV"]), dev_ids(x["cand_ids"])
+            torch.cuda.synchronize()
+            with torch.cuda.stream(side):
+                # a long kernel on the side stream first, so that a collective not
+                # ordered after it would read the prefix early
+                busy = torch.randn(4096, 4096, device="cuda")
+                for _ in range(8):
+                    busy = busy @ busy * 1e-3
+            admit_sharded(a, 0, K, V, ids, prefix, stream=side)
+            b.admit(0, K, V, ids)
+            torch.cuda.synchronize()
+            assert a.status() == 0 and b.status() == 0
+            for ga, gb_ in zip(export_banks(a, 0, w.heads), export_banks(b, 0, w.heads)):
+                np.testing.assert_array_equal(np.sort(ga["ids"]), np.sort(gb_["ids"]))
+        a.close()
+        b.close()
+    finally:
+        dist.destroy_process_group()
