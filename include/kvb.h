@@ -110,6 +110,10 @@ typedef struct {
   int32_t cand_order;       /* kvb_cand_order */
   int32_t baselines;        /* kvb_baselines */
   int32_t evict_order;      /* kvb_evict_order */
+  /* Forcing-KV variants (reading notes §3.4, §3.5); 0 is the per-frame, per-layer
+   * rule, so a zero-filled tail keeps it. */
+  int32_t bottomk_scope;    /* kvb_bottomk_scope */
+  int32_t sim_source;       /* kvb_sim_source */
 } kvb_config;
 
 /* Candidate ordering (App. E, candidate ordering).
@@ -135,6 +139,26 @@ typedef enum { KVB_BASELINES_FIXED = 0, KVB_BASELINES_REFRESH = 1 } kvb_baseline
  *  KVB_EVICT_THRESHOLD_SOURCE: every ratio_i > tau, then the capacity evictions
  *    by id ascending (oldest source position first). */
 typedef enum { KVB_EVICT_THRESHOLD_RATIO = 0, KVB_EVICT_DENSEST = 1, KVB_EVICT_THRESHOLD_SOURCE = 2 } kvb_evict_order;
+
+/* Scope of Forcing-KV's BottomK (reading notes §3.4 formula vs the §3.5 listing).
+ *  KVB_BOTTOMK_FRAME: each frame keeps its floor(r n) least similar segments.
+ *  KVB_BOTTOMK_CALL: the (frame, segment) pairs of all frames one
+ *    kvb_prune_hybrid call pushes are ranked together and the
+ *    floor(r n n_frames) least similar are kept (ties: the lower frame, then the
+ *    lower segment), so a frame may keep more or fewer than floor(r n).
+ *    Requires max_new_frames * n_segments <= 4096. */
+typedef enum { KVB_BOTTOMK_FRAME = 0, KVB_BOTTOMK_CALL = 1 } kvb_bottomk_scope;
+
+/* Where Forcing-KV's segment similarities come from (reading notes §3.4
+ * implementation notes: a first-block proxy with shared indices).
+ *  KVB_SIM_PER_LAYER: every layer's dynamic heads rank their own keys.
+ *  KVB_SIM_FIRST_LAYER: layer 0's call computes the similarities of every head
+ *    (static ones too) from its own keys; a later layer's call reuses them, so
+ *    head h of every layer keeps the segments head h of layer 0 selects, filled
+ *    with that layer's own K and V.  Layer 0 must be pruned first with each new
+ *    chunk: a call for layer > 0 returns KVB_E_STATE before layer 0 has been
+ *    pruned, or when its n_frames differs from layer 0's last call. */
+typedef enum { KVB_SIM_PER_LAYER = 0, KVB_SIM_FIRST_LAYER = 1 } kvb_sim_source;
 
 /* Per-(layer, head) counters of the last kvb_admit / kvb_prune_hybrid. */
 typedef struct {

@@ -233,16 +233,17 @@ __global__ void __launch_bounds__(kSelThreads) admit_count_kernel(const AdmitPla
     __syncthreads();
     const unsigned int bad = s_first_bad;
     for (int c = threadIdx.x; c < p.N; c += blockDim.x) cnt += (static_cast<unsigned int>(p.cand_ids[c]) < bad) ? 1 : 0;
-  } else {
-    for (int c = threadIdx.x; c < p.N; c += blockDim.x) cnt += (score_of(rb[c], mean0) <= p.tau) ? 1 : 0;
   }
-  int total;
-  block_excl_scan(cnt, &S, &total);
   // admission-threshold near ties (scores exist only against a bank with a mean baseline)
+  const bool scored = n > 0 && mean0 > 0.f;
   int nt = 0;
-  if (n > 0 && mean0 > 0.f)
-    for (int c = threadIdx.x; c < p.N; c += blockDim.x) nt += near_tau(score_of(rb[c], mean0), p.tau) ? 1 : 0;
-  int ties;
+  for (int c = threadIdx.x; c < p.N; c += blockDim.x) {
+    const float sc = score_of(rb[c], mean0);
+    if (p.cand_order != KVB_ORDER_SOURCE) cnt += (sc <= p.tau) ? 1 : 0;
+    nt += (scored && near_tau(sc, p.tau)) ? 1 : 0;
+  }
+  int total, ties;
+  block_excl_scan(cnt, &S, &total);
   block_excl_scan(nt, &S, &ties);
   if (threadIdx.x == 0) {
     p.mean0[h] = mean0;
@@ -349,17 +350,20 @@ __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPl
     else if (mode == KVB_EVICT_DENSEST) hi = ~float_key(rho[i] + proj[i]);
     return (hi << 32) | static_cast<unsigned int>(ids[i]);
   };
-  // mandatory evictions: projected growth above tau (none when densest-only)
-  int cnt = 0;
+  // mandatory evictions: projected growth above tau (none when densest-only);
+  // near ties at the threshold are counted on the way
+  int cnt = 0, nt = 0;
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     const float r = ratio(i);
     const bool m = mode != KVB_EVICT_DENSEST && r > p.tau;
     evflag[i] = m ? 1 : 0;
     cnt += m ? 1 : 0;
+    nt += (mode != KVB_EVICT_DENSEST && near_tau(r, p.tau)) ? 1 : 0;
     if (SKEYS) s_key[i] = m ? ~0ull : cut_key(i, r);
   }
-  int n_mand;
+  int n_mand, ties;
   block_excl_scan(cnt, &S, &n_mand);
+  block_excl_scan(nt, &S, &ties);
   const int ecap = max(0, n - n_mand + Ph - p.M);
   const int n_free = n - n_mand;
   if (ecap > 0) {
@@ -381,17 +385,16 @@ __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPl
   // near ties: projected ratios within the margin of tau, and the capacity cut
   // (last capacity eviction vs first non-mandatory survivor by the cut value)
   {
-    int nt = 0;
-    if (mode != KVB_EVICT_DENSEST)
-      for (int i = threadIdx.x; i < n; i += blockDim.x) nt += near_tau(ratio(i), p.tau) ? 1 : 0;
-    int ties;
-    block_excl_scan(nt, &S, &ties);
     if (ecap > 0 && ecap < n_free && mode != KVB_EVICT_THRESHOLD_SOURCE) {
       float lo = -INFINITY, hi = -INFINITY;  // lo holds -min over the evicted
       for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const float v = (mode == KVB_EVICT_DENSEST) ? rho[i] + proj[i] : ratio(i);
-        if (evflag[i] == 2) lo = fmaxf(lo, -v);
-        else if (evflag[i] == 0) hi = fmaxf(hi, v);
+        const int f = evflag[i];
+        if (f == 1) continue;
+        // the cut value: read back from the key when the keys are in shared memory
+        const float v = SKEYS ? key_float(~static_cast<uint32_t>(s_key[i] >> 32))
+                              : ((mode == KVB_EVICT_DENSEST) ? rho[i] + proj[i] : ratio(i));
+        if (f == 2) lo = fmaxf(lo, -v);
+        else hi = fmaxf(hi, v);
       }
       lo = block_max(lo, &S);
       hi = block_max(hi, &S);

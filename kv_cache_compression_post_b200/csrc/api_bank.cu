@@ -10,6 +10,7 @@
 #include "admit.cuh"
 #include "attend.cuh"
 #include "bank.h"
+#include "forcing.cuh"
 #include "gram.cuh"
 #include "small_kernels.cuh"
 
@@ -37,6 +38,11 @@ bool config_ok(const kvb_config* c) {
     if (c->frame_h < 1 || c->frame_w < 1 || c->seg_h < 1 || c->seg_w < 1) return false;
     if (c->hist_frames < 1 || c->max_new_frames < 1) return false;
     if (!(c->retention >= 0.f && c->retention <= 1.f)) return false;
+    if (c->bottomk_scope != KVB_BOTTOMK_FRAME && c->bottomk_scope != KVB_BOTTOMK_CALL) return false;
+    if (c->sim_source != KVB_SIM_PER_LAYER && c->sim_source != KVB_SIM_FIRST_LAYER) return false;
+    const long long n_seg = static_cast<long long>((c->frame_h + c->seg_h - 1) / c->seg_h) *
+                            ((c->frame_w + c->seg_w - 1) / c->seg_w);
+    if (c->bottomk_scope == KVB_BOTTOMK_CALL && n_seg * c->max_new_frames > kPruneMaxPairs) return false;
   }
   return true;
 }

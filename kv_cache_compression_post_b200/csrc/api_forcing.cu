@@ -84,13 +84,20 @@ extern "C" kvb_status kvb_prune_hybrid(kvb_bank* b, int32_t layer, const uint8_t
   const SegGeom sg = geom(g.frame_h, g.frame_w, g.seg_h, g.seg_w);
   const size_t lh = static_cast<size_t>(layer) * H;
 
+  // first-block proxy: layer 0 computes every head's similarities, later layers
+  // reuse them (they must follow a layer-0 prune of the same chunk)
+  const bool proxy = g.sim_source == KVB_SIM_FIRST_LAYER;
+  if (proxy && layer > 0 && b->proxy_frames != n_frames) return KVB_E_STATE;
+
   PrunePlan p;
   p.H = H;
   p.d = g.head_dim;
   p.n_frames = n_frames;
   p.hist_frames = g.hist_frames;
   p.ring_cap = b->ring_cap;
-  p.keep = keep_count(sg.n_seg, g.retention);
+  p.scope = g.bottomk_scope;
+  p.keep = g.bottomk_scope == KVB_BOTTOMK_CALL ? keep_count(sg.n_seg * n_frames, g.retention)
+                                               : keep_count(sg.n_seg, g.retention);
   p.row_bytes = b->row_bytes;
   p.g = sg;
   p.static_mask = mask;
@@ -121,8 +128,11 @@ extern "C" kvb_status kvb_prune_hybrid(kvb_bank* b, int32_t layer, const uint8_t
 
   cudaError_t e = cudaSuccess;
   const unsigned long long all = (H >= 64) ? ~0ull : ((1ull << H) - 1);
-  if ((mask & all) != all)
+  if (proxy && layer == 0)
+    e = launch_seg_cosine_ld(newK, nextK, g.dtype, H, n_frames, g.head_dim, sg, 0ull, b->sims, p.ld_sims, st);
+  else if (!proxy && (mask & all) != all)
     e = launch_seg_cosine_ld(newK, nextK, g.dtype, H, n_frames, g.head_dim, sg, mask, b->sims, p.ld_sims, st);
+  if (proxy && layer == 0) b->proxy_frames = e == cudaSuccess ? n_frames : -1;
   if (e == cudaSuccess) e = launch_prune_plan(p, st);
   if (e == cudaSuccess) e = launch_prune_gather(p, st);
   if (e == cudaSuccess && mask) e = launch_static_copy(p, st);

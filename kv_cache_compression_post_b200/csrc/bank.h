@@ -86,6 +86,9 @@ struct kvb_bank {
   int* seg_list = nullptr;  // [F] token index (row-major) in segment-major order
   int* plan = nullptr;      // [H][max_new_frames*F][2] (source row, ring position) pairs
   int* plan_n = nullptr;    // [H]
+  // KVB_SIM_FIRST_LAYER: frames of layer 0's last prune, whose similarities (left
+  // in `sims`) the later layers reuse; -1 before the first one
+  int proxy_frames = -1;
 
   size_t layout(void* base);  // carve (base may be null to measure); returns bytes
 };

@@ -6,7 +6,9 @@
 //                each seg_h x seg_w segment (one CTA per row of segments, a
 //                lane group of 16-byte loads per token, fixed-order segment sums)
 //   prune_plan   per dynamic head: per frame the BottomK(floor(r n)) least
-//                similar segments (ties: lower index), kept segments ascending,
+//                similar segments (ties: lower index) -- or, in the call scope,
+//                the floor(r n n_frames) least similar (frame, segment) pairs of
+//                all the call's frames ranked together -- kept segments ascending,
 //                tokens row-major inside each; the frame is pushed into a FIFO of
 //                hist_frames frames stored as a token ring (the oldest frame is
 //                dropped when the FIFO is full); emits (source row, ring slot)
@@ -133,7 +135,8 @@ __device__ __forceinline__ int2 plan_scan2(int a, int b, int2* warp_tot, int* ta
 }
 
 __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePlan p) {
-  __shared__ float s_sim[kPlanMaxSeg];
+  // similarities: one frame's (per-frame scope) or every frame's of the call
+  __shared__ float s_sim[kPruneMaxPairs];
   __shared__ int s_tok[kPlanMaxSeg + 1];  // token offset of each segment (segment-major list)
   __shared__ int s_kept[kPlanMaxSeg];     // kept segments of the current frame, ascending
   __shared__ int s_off[kPlanMaxSeg + 1];  // token offset of each kept segment in the frame
@@ -156,10 +159,15 @@ __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePla
     }
     return;
   }
-  if (n_seg > kPlanMaxSeg) {
+  const bool call = p.scope == KVB_BOTTOMK_CALL;
+  const int n_pairs = p.n_frames * n_seg;
+  if (n_seg > kPlanMaxSeg || (call && n_pairs > kPruneMaxPairs)) {
     if (threadIdx.x == 0) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
     return;
   }
+  if (call)  // the call's (frame, segment) pairs are ranked together: all of them at hand
+    for (int q = threadIdx.x; q < n_pairs; q += blockDim.x)
+      s_sim[q] = p.sims[static_cast<size_t>(h) * p.ld_sims + q];
   if (threadIdx.x < 4) s_state[threadIdx.x] = rs[threadIdx.x];
   if (threadIdx.x == 0) s_total = 0;
   for (int j = threadIdx.x; j <= n_seg; j += blockDim.x) s_tok[j] = p.seg_tok[j];
@@ -168,19 +176,26 @@ __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePla
   const int per = (n_seg + kPlanThreads - 1) / kPlanThreads;
   const int j0 = threadIdx.x * per, j1 = min(n_seg, j0 + per);
   for (int t = 0; t < p.n_frames; ++t) {
-    const float* sg = p.sims + static_cast<size_t>(h) * p.ld_sims + static_cast<size_t>(t) * n_seg;
-    for (int j = threadIdx.x; j < n_seg; j += blockDim.x) s_sim[j] = sg[j];
+    if (!call) {
+      const float* sg = p.sims + static_cast<size_t>(h) * p.ld_sims + static_cast<size_t>(t) * n_seg;
+      for (int j = threadIdx.x; j < n_seg; j += blockDim.x) s_sim[j] = sg[j];
+    }
     __syncthreads();
-    // BottomK: segment j is kept iff fewer than `keep` segments precede it in
-    // (similarity ascending, index ascending) order
+    // BottomK: segment j is kept iff fewer than `keep` entries precede it in
+    // (similarity ascending, position ascending) order, among the frame's
+    // segments (per-frame scope) or among the call's (frame, segment) pairs,
+    // position t * n_seg + j (call scope)
+    const int q0 = call ? t * n_seg : 0;
+    const int nq = call ? n_pairs : n_seg;
     int nk = 0, ntok = 0;
     unsigned int kept_bits = 0;  // per <= 32 segments per thread
     for (int j = j0; j < j1; ++j) {
-      const float sj = s_sim[j];
+      const int qj = q0 + j;
+      const float sj = s_sim[qj];
       int rank = 0;
-      for (int i = 0; i < n_seg; ++i) {
+      for (int i = 0; i < nq; ++i) {
         const float si = s_sim[i];
-        rank += (si < sj) || (si == sj && i < j);
+        rank += (si < sj) || (si == sj && i < qj);
       }
       if (rank < p.keep) {
         kept_bits |= 1u << (j - j0);

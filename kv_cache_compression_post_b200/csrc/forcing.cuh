@@ -23,9 +23,13 @@ cudaError_t launch_seg_cosine_ld(const void* K, const void* nextK, kvb_dtype dty
                                  const SegGeom& g, unsigned long long skip_mask, float* sim, int ld_sim,
                                  cudaStream_t st);
 
+// Most (frame, segment) pairs one call may rank together (KVB_BOTTOMK_CALL).
+constexpr int kPruneMaxPairs = 4096;
+
 // One layer's Forcing-KV state and the prune step's scratch.
 struct PrunePlan {
   int H = 0, d = 0, n_frames = 0, hist_frames = 0, ring_cap = 0, keep = 0, row_bytes = 0;
+  int scope = KVB_BOTTOMK_FRAME;  // kvb_bottomk_scope; `keep` counts segments per frame or pairs per call
   SegGeom g;
   unsigned long long static_mask = 0;
   const void* newK = nullptr;

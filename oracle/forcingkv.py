@@ -27,8 +27,18 @@ Variant (off by default): ``bottomk_scope="global"`` follows the reading notes'
 §3.5 listing instead of the §3.4 formula: the similarities of all frames pushed
 by one call are ranked together and floor(r * n_frames * n) (frame, segment)
 pairs are kept, so a frame can keep more or fewer than floor(r n) segments; ties
-go to the lower (frame, segment) position.  The CUDA path implements only the
-per-frame scope.
+go to the lower (frame, segment) position.
+
+Variant (off by default): the first-block similarity proxy of the reading notes'
+implementation notes (§3.4, and the §3.5 listing's comment): the segment
+similarities are computed on the first DiT block's keys only, and the indices
+they select are reused by the later blocks.  ``prune_hybrid(..., sim_keys=...)``
+takes those first-block keys; a layer then keeps, in each of its frames, the
+segments the first block's similarities select, and stores its own K and V at
+those positions.  Reading: the sharing is per head (head h of every layer reuses
+head h's selection of the first layer), and the first layer computes the
+similarities of every head, whatever its own static/dynamic label, so that a
+head that is dynamic only in a later layer has a selection to reuse.
 """
 from __future__ import annotations
 
@@ -107,11 +117,13 @@ class HeadState:
         self.kept: list = []                   # last prune's kept segment lists
 
 
-def prune_hybrid(states: List[HeadState], p: Params, newK, newV, new_ids, nextK):
+def prune_hybrid(states: List[HeadState], p: Params, newK, newV, new_ids, nextK, sim_keys=None):
     """Push the frames of a finalised chunk into each head's history.
 
     newK/newV [H][n_frames*F][d], new_ids [n_frames*F], nextK [H][F][d] (the first
-    frame of the next chunk: the successor of the last new frame)."""
+    frame of the next chunk: the successor of the last new frame).  ``sim_keys``
+    = (newK0, nextK0): the first block's keys of the same frames, from which the
+    similarities are computed instead of this layer's own (first-block proxy)."""
     F = p.F
     segs = segments(p.frame_h, p.frame_w, p.seg_h, p.seg_w)
     kkeep = keep_count(len(segs), p.retention)
@@ -124,8 +136,12 @@ def prune_hybrid(states: List[HeadState], p: Params, newK, newV, new_ids, nextK)
             st.transition = Frame(ids[-1], K[-1], V[-1])
             continue
         st.sims, st.kept = [], []
-        sims = [segment_similarity(K[t], K[t + 1] if t + 1 < n_frames else np.asarray(nextK[hh], np.float64), segs)
-                for t in range(n_frames)]
+        if sim_keys is None:
+            Ks, nxt = K, np.asarray(nextK[hh], np.float64)
+        else:
+            Ks = np.asarray(sim_keys[0][hh], np.float64).reshape(n_frames, F, -1)
+            nxt = np.asarray(sim_keys[1][hh], np.float64)
+        sims = [segment_similarity(Ks[t], Ks[t + 1] if t + 1 < n_frames else nxt, segs) for t in range(n_frames)]
         keeps = _keep_sets(p, sims, kkeep)
         for t in range(n_frames):
             sim, keep = sims[t], keeps[t]

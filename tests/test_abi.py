@@ -88,11 +88,21 @@ def test_config_validation_and_workspace_sizes():
     assert kvb.kvb_workspace_size(kvb.make_config(dtype=kvb.KVB_F32)) > base
     f = kvb.make_config(method=kvb.KVB_FORCINGKV, frame_h=30, frame_w=52)
     assert kvb.kvb_workspace_size(f) > 0
-    for kw in [dict(frame_h=0), dict(seg_w=0), dict(hist_frames=0), dict(retention=1.5), dict(max_new_frames=0)]:
+    for kw in [dict(frame_h=0), dict(seg_w=0), dict(hist_frames=0), dict(retention=1.5), dict(max_new_frames=0),
+               dict(bottomk_scope=2), dict(bottomk_scope=-1), dict(sim_source=2),
+               # the call scope ranks max_new_frames * n_seg <= 4096 pairs at once: 40 x 104 > 4096
+               dict(bottomk_scope=kvb.KVB_BOTTOMK_CALL, max_new_frames=40)]:
         c = kvb.make_config(method=kvb.KVB_FORCINGKV, frame_h=30, frame_w=52)
         for k, v in kw.items():
             setattr(c, k, v)
         assert kvb.kvb_workspace_size(c) == 0, kw
+    # the Forcing-KV variants change no buffer
+    for kw in [dict(bottomk_scope=kvb.KVB_BOTTOMK_CALL), dict(sim_source=kvb.KVB_SIM_FIRST_LAYER),
+               dict(bottomk_scope=kvb.KVB_BOTTOMK_CALL, max_new_frames=39)]:
+        c = kvb.make_config(method=kvb.KVB_FORCINGKV, frame_h=30, frame_w=52, **kw)
+        assert kvb.kvb_workspace_size(c) == kvb.kvb_workspace_size(
+            kvb.make_config(method=kvb.KVB_FORCINGKV, frame_h=30, frame_w=52,
+                            max_new_frames=kw.get("max_new_frames", 3))), kw
 
 
 def test_entry_points_reject_bad_arguments_before_any_launch():

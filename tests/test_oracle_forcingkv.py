@@ -177,3 +177,47 @@ def test_dynamic_direction_uses_successor_frame():
     np.testing.assert_allclose(st[0].sims[0], [1, 0, -1, 1 / math.sqrt(2)], atol=1e-15)
     np.testing.assert_array_equal(st[0].kept[0], [1, 2])
     np.testing.assert_array_equal(st[0].ring[0].ids, [1, 2])
+
+
+def _two_layer_chunk():
+    """One head, one new frame of 2 x 4 tokens in 2 x 2 segments (segment 0 =
+    tokens {0, 1, 4, 5}, segment 1 = {2, 3, 6, 7}), r = 0.5 (one segment kept).
+    Layer 0: segment 0 turns 90 degrees towards the next frame (cos 0), segment 1
+    stays (cos 1).  Layer 1: the opposite.  Values carry (layer, token)."""
+    base = np.array([[1.0, 0.0]] * 8)
+    turned = lambda toks: np.array([[0.0, 1.0] if i in toks else [1.0, 0.0] for i in range(8)])
+    K = [base[None], 2.0 * base[None]]
+    nxt = [turned({0, 1, 4, 5})[None], 2.0 * turned({2, 3, 6, 7})[None]]
+    V = [np.array([[10 * l + i, 0.0] for i in range(8)])[None] for l in (0, 1)]
+    return K, V, nxt, np.arange(100, 108)
+
+
+def test_first_block_proxy_selects_by_the_first_layers_keys():
+    K, V, nxt, ids = _two_layer_chunk()
+    p = fkv.Params(2, 4, 2, 2, 0.5, hist_frames=4)
+    own = [fkv.HeadState(False)]
+    fkv.prune_hybrid(own, p, K[1], V[1], ids, nxt[1])
+    np.testing.assert_array_equal(own[0].kept[0], [1])            # layer 1 on its own keys: segment 1
+    proxy = [fkv.HeadState(False)]
+    fkv.prune_hybrid(proxy, p, K[1], V[1], ids, nxt[1], sim_keys=(K[0], nxt[0]))
+    np.testing.assert_array_equal(proxy[0].kept[0], [0])          # the first layer's choice: segment 0
+    hid, hK, hV = fkv.history(proxy[0], 2)
+    np.testing.assert_array_equal(hid, ids[[0, 1, 4, 5]])
+    np.testing.assert_array_equal(hK, K[1][0][[0, 1, 4, 5]])      # this layer's own keys and values
+    np.testing.assert_array_equal(hV[:, 0], [10, 11, 14, 15])
+    np.testing.assert_allclose(proxy[0].sims[0], [0.0, 1.0], atol=1e-15)
+
+
+def test_first_block_proxy_with_its_own_keys_is_the_plain_prune():
+    w = kvgen.WORKLOADS["forcing_mid"]
+    L = kvgen.LayerInputs(w, 0, n_chunks=4, heads=range(2))
+    p = fkv.Params(w.frame_h, w.frame_w, w.seg_h, w.seg_w, w.retention, w.hist_frames)
+    a, b = [fkv.HeadState(False) for _ in range(2)], [fkv.HeadState(False) for _ in range(2)]
+    for i in range(1, 3):
+        x = L.step(i, forcing=True)
+        fkv.prune_hybrid(a, p, x["newK"], x["newV"], x["new_ids"], x["nextK"])
+        fkv.prune_hybrid(b, p, x["newK"], x["newV"], x["new_ids"], x["nextK"], sim_keys=(x["newK"], x["nextK"]))
+    for sa, sb in zip(a, b):
+        for fa, fb in zip(sa.ring, sb.ring):
+            np.testing.assert_array_equal(fa.ids, fb.ids)
+            np.testing.assert_array_equal(fa.K, fb.K)

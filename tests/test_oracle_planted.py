@@ -134,7 +134,23 @@ def _segment_sum(Kt, Knext, segs):
     return np.array([c[s].sum() for s in segs])
 
 
+_plain_prune = fkv.prune_hybrid
+
+
+def _proxy_ignored(states, p, newK, newV, new_ids, nextK, sim_keys=None):
+    return _plain_prune(states, p, newK, newV, new_ids, nextK)
+
+
+def _proxy_keys_kept(states, p, newK, newV, new_ids, nextK, sim_keys=None):
+    # the first layer's keys stored instead of this layer's own
+    if sim_keys is None:
+        return _plain_prune(states, p, newK, newV, new_ids, nextK)
+    return _plain_prune(states, p, sim_keys[0], newV, new_ids, sim_keys[1])
+
+
 FORCING_MISTAKES = {
+    "first-block proxy ignored": {"prune_hybrid": _proxy_ignored},
+    "first-block keys stored": {"prune_hybrid": _proxy_keys_kept},
     "ties to the higher index": {"bottom_k": _bottom_k_ties_high},
     "keeps the most similar": {"bottom_k": _top_k},
     "ceil(r n)": {"keep_count": lambda n, r: int(math.ceil(r * n - 1e-9))},
