@@ -214,6 +214,8 @@ __device__ __forceinline__ float ratio_of(float rho, float proj, float rho0) {
 
 // -------------------------------------------------------------------- kernels
 __global__ void __launch_bounds__(kSelThreads) admit_count_kernel(const AdmitPlan p) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ SelShared S;
   const int h = blockIdx.x;
   const int n = p.size[h];
@@ -254,6 +256,8 @@ __global__ void __launch_bounds__(kSelThreads) admit_count_kernel(const AdmitPla
 }
 
 __global__ void __launch_bounds__(kSelThreads) admit_select_kernel(const AdmitPlan p) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ SelShared S;
   const int h = blockIdx.x;
   int Pt = p.feasible[h];
@@ -298,6 +302,8 @@ __global__ void __launch_bounds__(kSelThreads) admit_select_kernel(const AdmitPl
 }
 
 __global__ void feasible_min_kernel(const AdmitPlan p, int* out) {
+  pdl_wait();
+  pdl_trigger();
   int v = min(p.M, p.N);
   for (int h = threadIdx.x; h < p.H; h += 32) v = min(v, p.feasible[h]);
   for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -310,6 +316,8 @@ __device__ __forceinline__ void copy_aug(uint16_t* dst, const uint16_t* src, con
 }
 
 __global__ void gather_admitted_kernel(const AdmitPlan p) {
+  pdl_wait();
+  pdl_trigger();
   const int h = blockIdx.y;
   const RowGroup g = row_group(p.row_bytes);
   const int P = p.P[h];
@@ -327,6 +335,8 @@ __global__ void gather_admitted_kernel(const AdmitPlan p) {
 // mandatory evictions get the largest key, so the selection needs no flags.
 template <bool SKEYS>
 __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPlan p) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ SelShared S;
   extern __shared__ unsigned long long s_key[];  // [n] (SKEYS)
   const int h = blockIdx.x;
@@ -439,6 +449,8 @@ __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPl
 }
 
 __global__ void gather_evicted_kernel(const AdmitPlan p) {
+  pdl_wait();
+  pdl_trigger();
   const int h = blockIdx.y;
   const RowGroup g = row_group(p.row_bytes);
   const int E = p.E[h];
@@ -454,6 +466,8 @@ __global__ void gather_evicted_kernel(const AdmitPlan p) {
 
 // moves: [0, P) admitted candidates, [P, P + ntail) surviving tail entries
 __global__ void compact_kernel(const AdmitPlan p) {
+  pdl_wait();
+  pdl_trigger();
   const int h = blockIdx.y;
   const RowGroup g = row_group(p.row_bytes);
   const int P = p.P[h], nt = p.ntail[h], nh = p.nhole[h], n_old = p.n_old[h];
@@ -502,6 +516,8 @@ __global__ void compact_kernel(const AdmitPlan p) {
 }
 
 __global__ void finalize_kernel(const AdmitPlan p) {
+  pdl_wait();
+  pdl_trigger();
   const int h = blockIdx.y;
   const int s = blockIdx.x * blockDim.x + threadIdx.x;
   const int n_new = p.size[h];
@@ -524,24 +540,20 @@ __global__ void finalize_kernel(const AdmitPlan p) {
 
 cudaError_t launch_admit_count(const AdmitPlan& p, cudaStream_t st) {
   LaunchTrace trace("admit_count_kernel", st);
-  admit_count_kernel<<<p.H, kSelThreads, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(admit_count_kernel, dim3(p.H), dim3(kSelThreads), 0, st, p);
 }
 cudaError_t launch_feasible_min(const AdmitPlan& p, int* out, cudaStream_t st) {
   LaunchTrace trace("feasible_min_kernel", st);
-  feasible_min_kernel<<<1, 32, 0, st>>>(p, out);
-  return cudaGetLastError();
+  return launch_pdl(feasible_min_kernel, dim3(1), dim3(32), 0, st, p, out);
 }
 cudaError_t launch_admit_select(const AdmitPlan& p, cudaStream_t st) {
   LaunchTrace trace("admit_select_kernel", st);
-  admit_select_kernel<<<p.H, kSelThreads, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(admit_select_kernel, dim3(p.H), dim3(kSelThreads), 0, st, p);
 }
 cudaError_t launch_gather_admitted(const AdmitPlan& p, int maxP, cudaStream_t st) {
   if (maxP <= 0) return cudaSuccess;
   LaunchTrace trace("gather_admitted_kernel", st);
-  gather_admitted_kernel<<<dim3(mover_blocks(maxP, p.row_bytes, p.H), p.H), 256, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(gather_admitted_kernel, dim3(mover_blocks(maxP, p.row_bytes, p.H), p.H), dim3(256), 0, st, p);
 }
 cudaError_t launch_evict_select(const AdmitPlan& p, cudaStream_t st) {
   const size_t keys = sizeof(unsigned long long) * static_cast<size_t>(p.M);
@@ -550,27 +562,23 @@ cudaError_t launch_evict_select(const AdmitPlan& p, cudaStream_t st) {
                                          static_cast<int>(keys));
     if (e != cudaSuccess) return e;
     LaunchTrace trace("evict_select_kernel", st);
-    evict_select_kernel<true><<<p.H, kSelThreads, keys, st>>>(p);
+    return launch_pdl(evict_select_kernel<true>, dim3(p.H), dim3(kSelThreads), keys, st, p);
   } else {
     LaunchTrace trace("evict_select_kernel", st);
-    evict_select_kernel<false><<<p.H, kSelThreads, 0, st>>>(p);
+    return launch_pdl(evict_select_kernel<false>, dim3(p.H), dim3(kSelThreads), 0, st, p);
   }
-  return cudaGetLastError();
 }
 cudaError_t launch_gather_evicted(const AdmitPlan& p, cudaStream_t st) {
   LaunchTrace trace("gather_evicted_kernel", st);
-  gather_evicted_kernel<<<dim3(mover_blocks(p.M, p.row_bytes, p.H), p.H), 256, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(gather_evicted_kernel, dim3(mover_blocks(p.M, p.row_bytes, p.H), p.H), dim3(256), 0, st, p);
 }
 cudaError_t launch_compact(const AdmitPlan& p, cudaStream_t st) {
   LaunchTrace trace("compact_kernel", st);
-  compact_kernel<<<dim3(mover_blocks(p.N + p.M, p.row_bytes, p.H), p.H), 256, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(compact_kernel, dim3(mover_blocks(p.N + p.M, p.row_bytes, p.H), p.H), dim3(256), 0, st, p);
 }
 cudaError_t launch_finalize(const AdmitPlan& p, cudaStream_t st) {
   LaunchTrace trace("finalize_kernel", st);
-  finalize_kernel<<<dim3((p.M + 255) / 256, p.H), 256, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(finalize_kernel, dim3((p.M + 255) / 256, p.H), dim3(256), 0, st, p);
 }
 
 }  // namespace kvb

@@ -210,6 +210,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int H = a.H;
   const int nqt = (a.Nq + kTile - 1) / kTile;
 
+  // the segment lengths (bank sizes) come from the previous kernels
+  pdl_wait();
+  pdl_trigger();
+
   // ---------------------------------------------------------------- schedule
   if (tid < H) sch.T[tid] = head_tiles(a, tid);
   __syncthreads();
@@ -649,6 +653,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr int kF32MaxD = 128;
 
 __global__ void attend_f32_kernel(const AttnArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int h = blockIdx.y;
   const int qi = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -721,8 +727,7 @@ cudaError_t launch_attend_bf16(const AttnArgs& a, cudaStream_t st) {
   // persistent: one CTA per SM; the kernel itself uses fewer when the work is small
   const int grid = dev.n_sm < kAttnMaxCtas ? dev.n_sm : kAttnMaxCtas;
   LaunchTrace trace("attend_bf16_kernel", st);
-  attend_bf16_kernel<<<grid, kThreads, smem, st>>>(maps, a);
-  return cudaGetLastError();
+  return launch_pdl(attend_bf16_kernel, dim3(grid), dim3(kThreads), smem, st, maps, a);
 }
 
 cudaError_t launch_attend_f32(const AttnArgs& a, cudaStream_t st) {
@@ -730,8 +735,7 @@ cudaError_t launch_attend_f32(const AttnArgs& a, cudaStream_t st) {
   if (a.d > kF32MaxD) return cudaErrorInvalidValue;
   dim3 grid((a.Nq + 3) / 4, a.H);
   LaunchTrace trace("attend_f32_kernel", st);
-  attend_f32_kernel<<<grid, 128, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(attend_f32_kernel, grid, dim3(128), 0, st, a);
 }
 
 }  // namespace kvb

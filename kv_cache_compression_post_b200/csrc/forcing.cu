@@ -57,6 +57,8 @@ __device__ __forceinline__ void acc_words(uint4 a, uint4 b, float& dot, float& n
 template <typename T>
 __global__ void seg_cosine_kernel(const T* __restrict__ K, const T* __restrict__ nextK, int n_frames, int d,
                                   SegGeom g, unsigned long long skip_mask, float* __restrict__ sim, int ld_sim) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ float cosv[];  // [seg_h * frame_w]
   const int sr = blockIdx.x, t = blockIdx.y, h = blockIdx.z;
   if ((skip_mask >> h) & 1ull) return;
@@ -135,6 +137,8 @@ __device__ __forceinline__ int2 plan_scan2(int a, int b, int2* warp_tot, int* ta
 }
 
 __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePlan p) {
+  pdl_wait();
+  pdl_trigger();
   // similarities: one frame's (per-frame scope) or every frame's of the call
   __shared__ float s_sim[kPruneMaxPairs];
   __shared__ int s_tok[kPlanMaxSeg + 1];  // token offset of each segment (segment-major list)
@@ -277,6 +281,8 @@ __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePla
 }
 
 __global__ void prune_gather_kernel(const PrunePlan p) {
+  pdl_wait();
+  pdl_trigger();
   const int h = blockIdx.y;
   if ((p.static_mask >> h) & 1ull) return;
   const RowGroup g = row_group(p.row_bytes);
@@ -299,6 +305,8 @@ __global__ void prune_gather_kernel(const PrunePlan p) {
 }
 
 __global__ void static_copy_kernel(const PrunePlan p) {
+  pdl_wait();
+  pdl_trigger();
   const int h = blockIdx.y;
   if (!((p.static_mask >> h) & 1ull)) return;
   const RowGroup g = row_group(p.row_bytes);
@@ -332,31 +340,26 @@ cudaError_t launch_seg_cosine_ld(const void* K, const void* nextK, kvb_dtype dty
   const size_t smem = sizeof(float) * g.seg_h * g.frame_w;
   LaunchTrace trace("seg_cosine_kernel", st);
   if (dtype == KVB_BF16)
-    seg_cosine_kernel<<<grid, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(K),
-                                               static_cast<const __nv_bfloat16*>(nextK), n_frames, d, g, skip_mask,
-                                               sim, ld_sim);
-  else
-    seg_cosine_kernel<<<grid, 256, smem, st>>>(static_cast<const float*>(K), static_cast<const float*>(nextK),
-                                               n_frames, d, g, skip_mask, sim, ld_sim);
-  return cudaGetLastError();
+    return launch_pdl(seg_cosine_kernel<__nv_bfloat16>, grid, dim3(256), smem, st,
+                      static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(nextK), n_frames, d, g,
+                      skip_mask, sim, ld_sim);
+  return launch_pdl(seg_cosine_kernel<float>, grid, dim3(256), smem, st, static_cast<const float*>(K),
+                    static_cast<const float*>(nextK), n_frames, d, g, skip_mask, sim, ld_sim);
 }
 
 cudaError_t launch_prune_plan(const PrunePlan& p, cudaStream_t st) {
   LaunchTrace trace("prune_plan_kernel", st);
-  prune_plan_kernel<<<p.H, kPlanThreads, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(prune_plan_kernel, dim3(p.H), dim3(kPlanThreads), 0, st, p);
 }
 
 cudaError_t launch_prune_gather(const PrunePlan& p, cudaStream_t st) {
   LaunchTrace trace("prune_gather_kernel", st);
-  prune_gather_kernel<<<dim3(mover_blocks(p.ld_plan, p.row_bytes, p.H), p.H), 256, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(prune_gather_kernel, dim3(mover_blocks(p.ld_plan, p.row_bytes, p.H), p.H), dim3(256), 0, st, p);
 }
 
 cudaError_t launch_static_copy(const PrunePlan& p, cudaStream_t st) {
   LaunchTrace trace("static_copy_kernel", st);
-  static_copy_kernel<<<dim3(mover_blocks(p.g.F, p.row_bytes, p.H), p.H), 256, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(static_copy_kernel, dim3(mover_blocks(p.g.F, p.row_bytes, p.H), p.H), dim3(256), 0, st, p);
 }
 
 }  // namespace kvb

@@ -207,6 +207,10 @@ __global__ void __launch_bounds__(kGramThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
+  // everything above touched only shared memory and TMEM: from here on the
+  // previous kernel's results are read
+  pdl_wait();
+  pdl_trigger();
 
   const long long T = total_steps(a);
   const int G = active_grid(a, T);
@@ -420,6 +424,8 @@ constexpr int kF32Warps = 8;
 constexpr int kF32Cols = 32;
 
 __global__ void __launch_bounds__(kF32Warps * 32) gram_f32_kernel(const GramArgs a) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ float sh[];  // [kF32Warps][d] rows + [kF32Cols][d + 1] cols
   const int d = a.d;
   float* sRow = sh;
@@ -464,6 +470,8 @@ __global__ void __launch_bounds__(kF32Warps * 32) gram_f32_kernel(const GramArgs
 }
 
 __global__ void gram_reduce_kernel(const GramArgs a, float* out, int ldOut) {
+  pdl_wait();
+  pdl_trigger();
   const int h = blockIdx.y;
   const int r = blockIdx.x * blockDim.x + threadIdx.x;
   const int nR = set_n(a.rows, h);
@@ -516,19 +524,19 @@ cudaError_t launch_gram_bf16(const GramArgs& a, const CUtensorMap& tmR, const CU
     e = cudaFuncSetAttribute(gram_bf16_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     LaunchTrace trace("gram_bf16_kernel", st);
-    gram_bf16_kernel<2><<<grid, kGramThreads, smem, st>>>(tmR, tmC, tmRa, tmCa, a);
+    e = launch_pdl(gram_bf16_kernel<2>, dim3(grid), dim3(kGramThreads), smem, st, tmR, tmC, tmRa, tmCa, a);
   } else if (a.s == 1.f) {
     e = cudaFuncSetAttribute(gram_bf16_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     LaunchTrace trace("gram_bf16_kernel", st);
-    gram_bf16_kernel<1><<<grid, kGramThreads, smem, st>>>(tmR, tmC, tmRa, tmCa, a);
+    e = launch_pdl(gram_bf16_kernel<1>, dim3(grid), dim3(kGramThreads), smem, st, tmR, tmC, tmRa, tmCa, a);
   } else {
     e = cudaFuncSetAttribute(gram_bf16_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     LaunchTrace trace("gram_bf16_kernel", st);
-    gram_bf16_kernel<0><<<grid, kGramThreads, smem, st>>>(tmR, tmC, tmRa, tmCa, a);
+    e = launch_pdl(gram_bf16_kernel<0>, dim3(grid), dim3(kGramThreads), smem, st, tmR, tmC, tmRa, tmCa, a);
   }
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_gram_f32(const GramArgs& a, cudaStream_t st) {
@@ -536,16 +544,14 @@ cudaError_t launch_gram_f32(const GramArgs& a, cudaStream_t st) {
   dim3 grid((maxR + kF32Warps - 1) / kF32Warps, a.H);
   const size_t smem = sizeof(float) * (kF32Warps * a.d + kF32Cols * (a.d + 1));
   LaunchTrace trace("gram_f32_kernel", st);
-  gram_f32_kernel<<<grid, kF32Warps * 32, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(gram_f32_kernel, grid, dim3(kF32Warps * 32), smem, st, a);
 }
 
 cudaError_t launch_gram_reduce(const GramArgs& a, float* out, int ldOut, cudaStream_t st) {
   const int maxR = a.max_rows;
   dim3 grid((maxR + 255) / 256, a.H);
   LaunchTrace trace("gram_reduce_kernel", st);
-  gram_reduce_kernel<<<grid, 256, 0, st>>>(a, out, ldOut);
-  return cudaGetLastError();
+  return launch_pdl(gram_reduce_kernel, grid, dim3(256), 0, st, a, out, ldOut);
 }
 
 }  // namespace kvb

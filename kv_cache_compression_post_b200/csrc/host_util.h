@@ -45,6 +45,28 @@ class LaunchTrace {
   int slot_ = -1;
 };
 
+// Launch with programmatic dependent launch: the kernel's CTAs may be scheduled,
+// and run their prologue, while the previous kernel on the stream is finishing.
+// Every kernel launched this way executes pdl_wait() (kvb_device.cuh) before it
+// touches global memory that earlier work on the stream writes or reads, so the
+// stream's ordering is kept; it also calls pdl_trigger() to let its own
+// successor be scheduled early.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // CTAs per head of a row-moving kernel (256 threads, row_group lanes per row):
 // enough for `rows` rows, capped so that the grid stays near one wave (about
 // 1024 CTAs over all heads).

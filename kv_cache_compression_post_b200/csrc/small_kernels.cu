@@ -13,6 +13,8 @@ namespace {
 template <typename T>
 __global__ void aug_rows_kernel(const T* __restrict__ X, long long ldX, int d, int n_uni, const int* n_dev,
                                 uint16_t* __restrict__ out, long long ldOut, float* norm_max) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float s_max[32];
   const int h = blockIdx.y;
   const int n = n_dev ? n_dev[h] : n_uni;
@@ -81,11 +83,10 @@ cudaError_t launch_aug_rows(const void* X, kvb_dtype dtype, int H, long long ldX
   dim3 grid(mover_blocks(max_n, d * (dtype == KVB_BF16 ? 2 : 4), H), H);
   LaunchTrace trace("aug_rows_kernel", st);
   if (dtype == KVB_BF16)
-    aug_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), ldX, d, n_uni, n_dev, out, ldOut,
-                                          norm_max);
-  else
-    aug_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const float*>(X), ldX, d, n_uni, n_dev, out, ldOut, norm_max);
-  return cudaGetLastError();
+    return launch_pdl(aug_rows_kernel<__nv_bfloat16>, grid, dim3(256), 0, st, static_cast<const __nv_bfloat16*>(X),
+                      ldX, d, n_uni, n_dev, out, ldOut, norm_max);
+  return launch_pdl(aug_rows_kernel<float>, grid, dim3(256), 0, st, static_cast<const float*>(X), ldX, d, n_uni,
+                    n_dev, out, ldOut, norm_max);
 }
 
 

@@ -3,11 +3,18 @@ keys) at reduced depth: 2 layers of one bank, 6 chunks, all 12 heads at full
 per-head size, inputs from the GPU generator (kvgen.gpu).  Every step of both
 layers must keep the device status clean; the last two steps of each layer are
 checked on sampled outputs and invariants against the oracle (the same checks as
-the full-size step test)."""
+the full-size step test), and sampled attention rows against the oracle's
+attention over the step's keys.
+
+A chunk captured once as a CUDA graph (every layer's admit + attend, kernels
+chained by programmatic dependent launch) and replayed for later chunks must give
+the same banks and outputs, bit for bit, as the same calls made one by one."""
 import numpy as np
 import pytest
 
 import kvgen
+from oracle import densitykv as dkv
+from oracle.attention import attention
 from tests.gpu_util import check_admit_sampled, export_banks, host
 
 pytestmark = pytest.mark.gpu
@@ -38,5 +45,81 @@ def test_rollout_layers_sampled():
             if check:
                 post = export_banks(bank, l, w.heads)
                 check_admit_sampled(w, pre, post, bank.stats(l), host(x["cand_ids"]), host(x["candK"]), rng, n=6)
+                # sampled queries of two heads against the oracle over [sink | bank | window]
+                Oh = host(O)
+                for hh in rng.choice(w.heads, 2, replace=False):
+                    b = post[hh]
+                    bank_h = dkv.HeadBank(b["ids"], b["K"].astype(np.float64), b["V"].astype(np.float64), b["rho0"])
+                    K, V = dkv.attention_set(bank_h, host(x["sinkK"][hh]), host(x["sinkV"][hh]),
+                                             host(x["winK"][hh]), host(x["winV"][hh]))
+                    rows = np.sort(rng.choice(w.chunk_tokens, 8, replace=False))
+                    ref, _ = attention(host(x["Q"][hh])[rows], K, V)
+                    np.testing.assert_allclose(Oh[hh][rows], ref, atol=2e-2, rtol=0)
     assert np.isfinite(host(O)).all()
     bank.close()
+
+
+def test_chunk_graph_replay_matches_eager_calls():
+    """Two banks of 2 layers (the mid workload's sizes with the long rollout's
+    key generator): one runs every call eagerly, the other captures chunk 2's
+    calls (both layers' admit + attend) as one CUDA graph and replays it for
+    chunks 2..5 with the inputs copied into the graph's buffers.  Banks (ids, K,
+    V, rho, rho0) and attention outputs must be identical."""
+    import dataclasses
+    import torch
+    import kv_cache_compression_post_b200 as kvb
+    from kvgen.gpu import GpuLayerStream
+    w = dataclasses.replace(kvgen.WORKLOADS["mid"], name="mid_rollout", background_rows=6, ar_a_bg=0.95,
+                            ar_a_fg=0.5)
+    n_layers, steps = 2, 5
+    cfg = kvb.make_config(method=kvb.KVB_DENSITYKV, dtype=kvb.KVB_BF16, layers=n_layers, heads=w.heads,
+                          head_dim=w.head_dim, capacity=w.capacity, max_candidates=w.chunk_tokens, tau=w.tau,
+                          eps=w.eps, s=w.s, sync_heads=1, max_queries=w.chunk_tokens)
+    eager, graphed = kvb.Bank(cfg), kvb.Bank(cfg)
+    streams = [GpuLayerStream(w, l, tagged=True) for l in range(n_layers)]
+    Oe = torch.empty(w.heads, w.chunk_tokens, w.head_dim, dtype=torch.bfloat16, device="cuda")
+    Og = torch.empty_like(Oe)
+    static, graph = None, None
+    for i in range(1, steps + 1):
+        xs = [streams[l].step(i) for l in range(n_layers)]
+        outs_e = []
+        for l, x in enumerate(xs):
+            eager.admit(l, x["candK"], x["candV"], x["cand_ids"])
+            eager.attend(l, x["Q"], x["sinkK"], x["sinkV"], x["winK"], x["winV"], Oe)
+            outs_e.append(Oe.clone())
+        if i == 1:   # a 2-frame candidate block: eager on both banks
+            outs_g = []
+            for l, x in enumerate(xs):
+                graphed.admit(l, x["candK"], x["candV"], x["cand_ids"])
+                graphed.attend(l, x["Q"], x["sinkK"], x["sinkV"], x["winK"], x["winV"], Og)
+                outs_g.append(Og.clone())
+        else:
+            if graph is None:
+                static = [{k: v.clone() for k, v in x.items()} for x in xs]
+                outs_static = [torch.empty_like(Og) for _ in range(n_layers)]
+                cap = torch.cuda.Stream()
+                cap.wait_stream(torch.cuda.current_stream())
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph, stream=cap, capture_error_mode="relaxed"):
+                    st = torch.cuda.current_stream()
+                    for l in range(n_layers):
+                        x = static[l]
+                        graphed.admit(l, x["candK"], x["candV"], x["cand_ids"], st)
+                        graphed.attend(l, x["Q"], x["sinkK"], x["sinkV"], x["winK"], x["winV"], outs_static[l],
+                                       None, st)
+            else:
+                for l, x in enumerate(xs):
+                    for k, v in x.items():
+                        static[l][k].copy_(v)
+            graph.replay()
+            outs_g = [o.clone() for o in outs_static]
+        torch.cuda.synchronize()
+        assert eager.status() == 0 and graphed.status() == 0
+        for l in range(n_layers):
+            np.testing.assert_array_equal(host(outs_g[l]), host(outs_e[l]))
+            for a, b in zip(export_banks(eager, l, w.heads), export_banks(graphed, l, w.heads)):
+                for k in ("ids", "K", "V", "rho", "rho0"):
+                    np.testing.assert_array_equal(a[k], b[k], err_msg=f"chunk {i} layer {l} {k}")
+    del graph
+    eager.close()
+    graphed.close()
