@@ -183,7 +183,12 @@ typedef struct kvb_bank kvb_bank; /* opaque, host-side */
 /* Bytes of device workspace kvb_bank_create needs for `cfg`; 0 if cfg is invalid. */
 KVB_API size_t kvb_workspace_size(const kvb_config* cfg);
 
-/* Bind a bank to a caller-owned workspace (>= kvb_workspace_size bytes, 256-B
+/* A bank holds the retained history of every (layer, head): for DensityKV an
+ * independent bank of at most M exact (id, K, V) entries per layer and head with
+ * their densities and insertion baselines (DensityKV App. B.1 "Online Bank
+ * Update", App. D); for Forcing-KV each static head's transition frame and each
+ * dynamic head's FIFO of pruned frames (Forcing-KV reading notes §3.3, §3.4).
+ * Bind a bank to a caller-owned workspace (>= kvb_workspace_size bytes, 256-B
  * aligned).  Clears the status word and every bank to empty with async memsets
  * on `stream`.  *out receives a host handle.  KVB_E_INVAL / KVB_E_WORKSPACE /
  * KVB_E_UNSUPPORTED on bad config or workspace; KVB_E_CUDA if the device is not
@@ -233,7 +238,11 @@ KVB_API kvb_status kvb_prune_hybrid(kvb_bank* bank, int32_t layer, const uint8_t
                             const void* newK, const void* newV, const void* nextK,
                             const int32_t* new_ids, int32_t n_frames, void* stream);
 
-/* Attention of the current chunk's queries over [sink | history(layer) | window]:
+/* Attention of the current chunk's queries over [sink | history(layer) | window]
+ * -- the retained states read directly by the model's native attention (DensityKV
+ * Fig. 2 and §5; Forcing-KV reading notes §3.3 and the §3.5 listing: static heads
+ * over [sink, transition frame, current chunk], dynamic heads over [sink, retained
+ * history, current chunk]):
  * Q, O: device [H][Nq][d]; sinkK/V [H][Ls][d]; winK/V [H][Lw][d]; lse: device
  * [H][Nq] f32 (natural log) or NULL.  O = softmax(Q K^T / sqrt(d)) V, no mask.
  * History is the DensityKV bank, or for Forcing-KV the transition frame (static

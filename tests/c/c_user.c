@@ -3,7 +3,8 @@
  * of the chunk's queries over [sink | bank | window], the per-head counters and
  * the device status.  Inputs are zero-filled (the point is the calling
  * sequence, argument layout and error handling, not the numbers).  Built by
- * tests/test_abi.py as a compile-and-link check; it runs on any CUDA GPU with
+ * tests/test_abi.py as a compile-and-link check and run on the GPU by
+ * tests/test_gpu_c_user.py; it needs a GPU with
  * sm_100a: ./c_user */
 #include <stdio.h>
 #include <stdlib.h>

@@ -103,6 +103,17 @@ def test_golden_hand_scenarios(name):
         prev_banks = r.banks
 
 
+def test_golden_values_are_reproduced_by_their_exact_derivation():
+    """tests/golden/derive_densitykv_hand.py re-derives every stored expected value
+    of densitykv_hand.json in exact fractions, independently of the oracle."""
+    import importlib.util
+    path = os.path.join(os.path.dirname(__file__), "golden", "derive_densitykv_hand.py")
+    spec = importlib.util.spec_from_file_location("derive_densitykv_hand", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    assert mod.mismatches(json.load(open(GOLDEN))) == []
+
+
 def _tiny_rollout(steps=7, tagged=True, **kw):
     w = kvgen.WORKLOADS["tiny"]
     L = kvgen.LayerInputs(w, 0, tagged=tagged)
