@@ -169,9 +169,9 @@ def test_admit_argument_errors():
     bank.close()
 
 
-@pytest.mark.parametrize("name,H,steps", [("wan480", 2, 4), ("wan1080", 1, 3)])
+@pytest.mark.parametrize("name,H,steps", [("wan480", 12, 4), ("wan1080", 1, 3)])
 def test_full_size_step_sampled(name, H, steps):
-    """Full 480P / 1080P sizes (fewer heads): the GPU runs the rollout from an empty
+    """Full 480P (all 12 heads) / 1080P (one head): the GPU runs the rollout from an empty
     bank; the last step (bank full, evictions) is checked on sampled outputs the
     oracle computes one by one and on the rule's invariants (check_admit_sampled)."""
     import dataclasses

@@ -1,6 +1,7 @@
 """The long streaming rollout (30 layers x 80 chunks at 480P, background-correlated
-keys) at reduced depth: 2 layers of one bank, 6 chunks, all 12 heads at full
-per-head size, inputs from the GPU generator (kvgen.gpu).  Every step of both
+keys) at reduced depth: the workload's layers 0, 15 and 29 (their own generator
+streams) in one 3-layer bank, 6 chunks, all 12 heads at full per-head size, inputs
+from the GPU generator (kvgen.gpu).  Every step of both
 layers must keep the device status clean; the last two steps of each layer are
 checked on sampled outputs and invariants against the oracle (the same checks as
 the full-size step test), and sampled attention rows against the oracle's
@@ -25,12 +26,13 @@ def test_rollout_layers_sampled():
     import kv_cache_compression_post_b200 as kvb
     from kvgen.gpu import GpuLayerStream
     w = kvgen.WORKLOADS["rollout"]
-    n_layers, steps = 2, 6
+    layers, steps = (0, 15, 29), 6
+    n_layers = len(layers)
     cfg = kvb.make_config(method=kvb.KVB_DENSITYKV, dtype=kvb.KVB_BF16, layers=n_layers, heads=w.heads,
                           head_dim=w.head_dim, capacity=w.capacity, max_candidates=w.chunk_tokens, tau=w.tau,
                           eps=w.eps, s=w.s, sync_heads=1, max_queries=w.chunk_tokens)
     bank = kvb.Bank(cfg)
-    streams = [GpuLayerStream(w, l, tagged=True) for l in range(n_layers)]
+    streams = [GpuLayerStream(w, l, tagged=True) for l in layers]
     rng = np.random.default_rng(3)
     O = torch.empty(w.heads, w.chunk_tokens, w.head_dim, dtype=torch.bfloat16, device="cuda")
     for i in range(1, steps + 1):
