@@ -56,7 +56,11 @@ def test_rollout_layers_sampled():
                                              host(x["winK"][hh]), host(x["winV"][hh]))
                     rows = np.sort(rng.choice(w.chunk_tokens, 8, replace=False))
                     ref, _ = attention(host(x["Q"][hh])[rows], K, V)
-                    np.testing.assert_allclose(Oh[hh][rows], ref, atol=2e-2, rtol=0)
+                    # V's first 3 channels carry the token id (values up to 255): a
+                    # bf16 output holds them to its rounding, 2^-8 relative; the
+                    # N(0, 1) channels are held to the 2e-2 absolute bar
+                    np.testing.assert_allclose(Oh[hh][rows][:, 3:], ref[:, 3:], atol=2e-2, rtol=0)
+                    np.testing.assert_allclose(Oh[hh][rows][:, :3], ref[:, :3], rtol=2.0 ** -8, atol=2e-2)
     assert np.isfinite(host(O)).all()
     bank.close()
 
