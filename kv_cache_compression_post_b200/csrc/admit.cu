@@ -41,6 +41,7 @@ constexpr size_t kEvictKeyBytes = 200 * 1024;
 
 struct SelShared {
   unsigned int hist[256];
+  unsigned long long kmin[32], kmax[32];
   unsigned long long prefix, mask;
   int kRem;
   int done;
@@ -148,27 +149,79 @@ __device__ int block_compact(int lo, int hi, Pred pred, int* out, SelShared* S) 
 // Radix select of the k smallest 64-bit keys among {i < n : keep(i)} (1 <= k <
 // count).  On return S->prefix / S->mask define the selection:
 // keep(i) && (key(i) & mask) <= prefix.  Keys are unique (they carry the id).
+// A key of all ones is a sentinel for entries that are never among the k
+// smallest (they are larger than every other key).
+//
+// The bits every candidate key shares (the common prefix of the smallest and the
+// largest non-sentinel key) are skipped: at these sizes the keys of one call often
+// agree on their top byte (ratios in [1, 2), say), and a pass over it would send
+// every key to one histogram bin.  Histogram increments are aggregated per warp
+// (lanes with the same bin add once), so a crowded bin costs one atomic per warp.
 template <class KeyFn, class KeepFn>
 __device__ void block_radix_select(int n, int k, KeyFn key, KeepFn keep, SelShared* S) {
-  if (threadIdx.x == 0) {
-    S->prefix = 0ull;
-    S->mask = 0ull;
-    S->kRem = k;
-    S->done = 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = static_cast<int>(blockDim.x >> 5);
+  unsigned long long lo = ~0ull, hi = 0ull;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    if (!keep(i)) continue;
+    const unsigned long long kk = key(i);
+    if (kk == ~0ull) continue;
+    lo = kk < lo ? kk : lo;
+    hi = kk > hi ? kk : hi;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long a = __shfl_xor_sync(0xffffffffu, lo, o), b = __shfl_xor_sync(0xffffffffu, hi, o);
+    lo = a < lo ? a : lo;
+    hi = b > hi ? b : hi;
+  }
+  if (lane == 0) {
+    S->kmin[warp] = lo;
+    S->kmax[warp] = hi;
   }
   __syncthreads();
-  for (int shift = 56; shift >= 0; shift -= 8) {
+  if (threadIdx.x == 0) {
+    unsigned long long mn = ~0ull, mx = 0ull;
+    for (int w = 0; w < nwarps; ++w) {
+      mn = S->kmin[w] < mn ? S->kmin[w] : mn;
+      mx = S->kmax[w] > mx ? S->kmax[w] : mx;
+    }
+    S->kRem = k;
+    S->done = 0;
+    if (mn >= mx) {  // one candidate key: it is the selection
+      S->prefix = mn;
+      S->mask = ~0ull;
+      S->done = 1;
+    } else {
+      // digits start at the byte holding the highest bit where min and max differ
+      const int top = 63 - __clzll(static_cast<long long>(mn ^ mx));
+      const int shift0 = (top / 8) * 8;
+      const unsigned long long above = shift0 >= 56 ? 0ull : ~((1ull << (shift0 + 8)) - 1ull);
+      S->prefix = mn & above;
+      S->mask = above;
+      S->kmin[0] = static_cast<unsigned long long>(shift0);
+    }
+  }
+  __syncthreads();
+  if (S->done) return;
+  const int shift0 = static_cast<int>(S->kmin[0]);
+  for (int shift = shift0; shift >= 0; shift -= 8) {
     for (int i = threadIdx.x; i < 256; i += blockDim.x) S->hist[i] = 0u;
     __syncthreads();
     const unsigned long long prefix = S->prefix, mask = S->mask;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      if (!keep(i)) continue;
-      const unsigned long long kk = key(i);
-      if ((kk & mask) == prefix) atomicAdd(&S->hist[(kk >> shift) & 0xFFull], 1u);
+    // warp-uniform trip count: every lane reaches the match
+    for (int i0 = warp * 32; i0 < n; i0 += blockDim.x) {
+      const int i = i0 + lane;
+      unsigned int bin = 256u;
+      if (i < n && keep(i)) {
+        const unsigned long long kk = key(i);
+        if ((kk & mask) == prefix) bin = static_cast<unsigned int>((kk >> shift) & 0xFFull);
+      }
+      const unsigned int peers = __match_any_sync(0xffffffffu, bin);
+      if (bin < 256u && lane == __ffs(peers) - 1) atomicAdd(&S->hist[bin], static_cast<unsigned int>(__popc(peers)));
     }
     __syncthreads();
     if (threadIdx.x < 32) {
-      const int lane = threadIdx.x;
       unsigned int loc[8];
       unsigned int s = 0;
 #pragma unroll
@@ -310,23 +363,34 @@ __global__ void feasible_min_kernel(const AdmitPlan p, int* out) {
   if (threadIdx.x == 0) out[0] = v;
 }
 
-// 64-byte augmented row, the group's lanes 0..3
-__device__ __forceinline__ void copy_aug(uint16_t* dst, const uint16_t* src, const RowGroup& g) {
-  if (g.sub < 4) reinterpret_cast<uint4*>(dst)[g.sub] = reinterpret_cast<const uint4*>(src)[g.sub];
-}
-
+// Two rows per lane group and iteration, every load before the first store.
 __global__ void gather_admitted_kernel(const AdmitPlan p) {
   pdl_wait();
   pdl_trigger();
   const int h = blockIdx.y;
   const RowGroup g = row_group(p.row_bytes);
   const int P = p.P[h];
-  for (int w = g.first; w < P; w += g.stride) {
-    const int c = p.adm_idx[static_cast<size_t>(h) * p.ldN + w];
-    const size_t dst = static_cast<size_t>(h) * p.ldEA + p.M + w;
-    copy_row(static_cast<char*>(p.EA) + dst * p.row_bytes,
-             static_cast<const char*>(p.candK) + (static_cast<size_t>(h) * p.N + c) * p.row_bytes, p.row_bytes, g);
-    copy_aug(p.EAaug + dst * 32, p.caug + (static_cast<size_t>(h) * p.ldN + c) * 32, g);
+  const char* cK = static_cast<const char*>(p.candK);
+  char* EA = static_cast<char*>(p.EA);
+  for (int w0 = g.first; w0 < P; w0 += 2 * g.stride) {
+    RowWords rw[2];
+    int c[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int w = w0 + u * g.stride;
+      c[u] = w < P ? p.adm_idx[static_cast<size_t>(h) * p.ldN + w] : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+      if (c[u] >= 0)
+        load_rows(rw[u], cK + (static_cast<size_t>(h) * p.N + c[u]) * p.row_bytes, nullptr,
+                  p.caug + (static_cast<size_t>(h) * p.ldN + c[u]) * 32, p.row_bytes, g);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (c[u] < 0) continue;
+      const size_t dst = static_cast<size_t>(h) * p.ldEA + p.M + w0 + u * g.stride;
+      store_rows(rw[u], EA + dst * p.row_bytes, nullptr, p.EAaug + dst * 32, p.row_bytes, g);
+    }
   }
 }
 
@@ -454,17 +518,35 @@ __global__ void gather_evicted_kernel(const AdmitPlan p) {
   const int h = blockIdx.y;
   const RowGroup g = row_group(p.row_bytes);
   const int E = p.E[h];
-  for (int w = g.first; w < E; w += g.stride) {
-    const int slot = p.ev_slot[static_cast<size_t>(h) * p.M + w];
-    const size_t src = static_cast<size_t>(h) * p.M + slot;
-    const size_t dst = static_cast<size_t>(h) * p.ldEA + (p.M - E) + w;
-    copy_row(static_cast<char*>(p.EA) + dst * p.row_bytes, static_cast<const char*>(p.K) + src * p.row_bytes,
-             p.row_bytes, g);
-    copy_aug(p.EAaug + dst * 32, p.aug + src * 32, g);
+  const char* K = static_cast<const char*>(p.K);
+  char* EA = static_cast<char*>(p.EA);
+  for (int w0 = g.first; w0 < E; w0 += 2 * g.stride) {
+    RowWords rw[2];
+    int slot[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int w = w0 + u * g.stride;
+      slot[u] = w < E ? p.ev_slot[static_cast<size_t>(h) * p.M + w] : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+      if (slot[u] >= 0) {
+        const size_t src = static_cast<size_t>(h) * p.M + slot[u];
+        load_rows(rw[u], K + src * p.row_bytes, nullptr, p.aug + src * 32, p.row_bytes, g);
+      }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (slot[u] < 0) continue;
+      const size_t dst = static_cast<size_t>(h) * p.ldEA + (p.M - E) + w0 + u * g.stride;
+      store_rows(rw[u], EA + dst * p.row_bytes, nullptr, p.EAaug + dst * 32, p.row_bytes, g);
+    }
   }
 }
 
-// moves: [0, P) admitted candidates, [P, P + ntail) surviving tail entries
+// moves: [0, P) admitted candidates, [P, P + ntail) surviving tail entries.  Two
+// moves per lane group and iteration, every load before the first store (sources
+// and destinations are disjoint: destinations are evicted slots or slots past the
+// old size, sources candidates or survivors at or past the new size).
 __global__ void compact_kernel(const AdmitPlan p) {
   pdl_wait();
   pdl_trigger();
@@ -473,43 +555,60 @@ __global__ void compact_kernel(const AdmitPlan p) {
   const int P = p.P[h], nt = p.ntail[h], nh = p.nhole[h], n_old = p.n_old[h];
   const size_t base = static_cast<size_t>(h) * p.M;
   const int* hole = p.ev_slot + base;  // evicted slots ascending: the first nh are holes
-  for (int w = g.first; w < P + nt; w += g.stride) {
-    if (w < P) {
-      const int dst = (w < nh) ? hole[w] : n_old + (w - nh);
-      if (dst < 0 || dst >= p.M) {
-        if (g.sub == 0) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
-        continue;
+  char* K = static_cast<char*>(p.K);
+  char* V = static_cast<char*>(p.V);
+  const char* cK = static_cast<const char*>(p.candK);
+  const char* cV = static_cast<const char*>(p.candV);
+  for (int w0 = g.first; w0 < P + nt; w0 += 2 * g.stride) {
+    int src[2], dst[2];  // src: candidate index (admitted) or bank slot (tail); -1: nothing to move
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int w = w0 + u * g.stride;
+      src[u] = dst[u] = -1;
+      if (w < P) {
+        dst[u] = (w < nh) ? hole[w] : n_old + (w - nh);
+        src[u] = p.adm_idx[static_cast<size_t>(h) * p.ldN + w];
+      } else if (w < P + nt) {
+        src[u] = p.tail[base + (w - P)];
+        dst[u] = hole[w];
+        if (src[u] < 0 || src[u] >= p.M) dst[u] = -1;
       }
-      const int c = p.adm_idx[static_cast<size_t>(h) * p.ldN + w];
-      const size_t srow = static_cast<size_t>(h) * p.N + c;
-      copy_row(static_cast<char*>(p.K) + (base + dst) * p.row_bytes,
-               static_cast<const char*>(p.candK) + srow * p.row_bytes, p.row_bytes, g);
-      copy_row(static_cast<char*>(p.V) + (base + dst) * p.row_bytes,
-               static_cast<const char*>(p.candV) + srow * p.row_bytes, p.row_bytes, g);
-      copy_aug(p.aug + (base + dst) * 32, p.caug + (static_cast<size_t>(h) * p.ldN + c) * 32, g);
-      if (g.sub == 0) {
-        p.ids[base + dst] = p.cand_ids[c];
-        p.rho[base + dst] = p.rhoB[static_cast<size_t>(h) * p.ldN + c];
-        p.newp[base + dst] = w;
+      if (dst[u] < 0 || dst[u] >= p.M) {
+        if (w < P + nt && g.sub == 0) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
+        src[u] = dst[u] = -1;
       }
-    } else {
-      const int k = w - P;
-      const int src = p.tail[base + k];
-      const int dst = hole[P + k];
-      if (src < 0 || src >= p.M || dst < 0 || dst >= p.M) {
-        if (g.sub == 0) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
-        continue;
+    }
+    RowWords rw[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (src[u] < 0) continue;
+      if (w0 + u * g.stride < P) {
+        const size_t srow = static_cast<size_t>(h) * p.N + src[u];
+        load_rows(rw[u], cK + srow * p.row_bytes, cV + srow * p.row_bytes,
+                  p.caug + (static_cast<size_t>(h) * p.ldN + src[u]) * 32, p.row_bytes, g);
+      } else {
+        const size_t sb = base + src[u];
+        load_rows(rw[u], K + sb * p.row_bytes, V + sb * p.row_bytes, p.aug + sb * 32, p.row_bytes, g);
       }
-      copy_row(static_cast<char*>(p.K) + (base + dst) * p.row_bytes,
-               static_cast<const char*>(p.K) + (base + src) * p.row_bytes, p.row_bytes, g);
-      copy_row(static_cast<char*>(p.V) + (base + dst) * p.row_bytes,
-               static_cast<const char*>(p.V) + (base + src) * p.row_bytes, p.row_bytes, g);
-      copy_aug(p.aug + (base + dst) * 32, p.aug + (base + src) * 32, g);
-      if (g.sub == 0) {
-        p.ids[base + dst] = p.ids[base + src];
-        p.rho0[base + dst] = p.rho0[base + src];
-        p.rho[base + dst] = p.rho[base + src] + p.proj[base + src];
-        p.newp[base + dst] = -2;
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (src[u] < 0) continue;
+      const int w = w0 + u * g.stride;
+      const size_t db = base + dst[u];
+      store_rows(rw[u], K + db * p.row_bytes, V + db * p.row_bytes, p.aug + db * 32, p.row_bytes, g);
+      if (g.sub != 0) continue;
+      if (w < P) {
+        const int c = src[u];
+        p.ids[db] = p.cand_ids[c];
+        p.rho[db] = p.rhoB[static_cast<size_t>(h) * p.ldN + c];
+        p.newp[db] = w;
+      } else {
+        const size_t sb = base + src[u];
+        p.ids[db] = p.ids[sb];
+        p.rho0[db] = p.rho0[sb];
+        p.rho[db] = p.rho[sb] + p.proj[sb];
+        p.newp[db] = -2;
       }
     }
   }

@@ -280,6 +280,7 @@ __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePla
   }
 }
 
+// Two kept tokens per lane group and iteration, every load before the first store.
 __global__ void prune_gather_kernel(const PrunePlan p) {
   pdl_wait();
   pdl_trigger();
@@ -288,19 +289,38 @@ __global__ void prune_gather_kernel(const PrunePlan p) {
   const RowGroup g = row_group(p.row_bytes);
   const int n = min(p.plan_n[h], p.ld_plan);
   const int* plan = p.plan + static_cast<size_t>(h) * p.ld_plan * 2;
-  for (int e = g.first; e < n; e += g.stride) {
-    const int src = plan[2 * e], dst = plan[2 * e + 1];
-    if (src < 0 || src >= p.n_frames * p.g.F || dst < 0 || dst >= p.ring_cap) {
-      if (g.sub == 0) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
-      continue;
+  const char* nK = static_cast<const char*>(p.newK);
+  const char* nV = static_cast<const char*>(p.newV);
+  for (int e0 = g.first; e0 < n; e0 += 2 * g.stride) {
+    int src[2], dst[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int e = e0 + u * g.stride;
+      src[u] = dst[u] = -1;
+      if (e < n) {
+        src[u] = plan[2 * e];
+        dst[u] = plan[2 * e + 1];
+        if (src[u] < 0 || src[u] >= p.n_frames * p.g.F || dst[u] < 0 || dst[u] >= p.ring_cap) {
+          if (g.sub == 0) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
+          src[u] = -1;
+        }
+      }
     }
-    const size_t s = static_cast<size_t>(h) * p.n_frames * p.g.F + src;
-    const size_t t = static_cast<size_t>(h) * p.ring_cap + dst;
-    copy_row(static_cast<char*>(p.rK) + t * p.row_bytes, static_cast<const char*>(p.newK) + s * p.row_bytes,
-             p.row_bytes, g);
-    copy_row(static_cast<char*>(p.rV) + t * p.row_bytes, static_cast<const char*>(p.newV) + s * p.row_bytes,
-             p.row_bytes, g);
-    if (g.sub == 0) p.rids[t] = p.new_ids[src];
+    RowWords rw[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (src[u] < 0) continue;
+      const size_t s = static_cast<size_t>(h) * p.n_frames * p.g.F + src[u];
+      load_rows(rw[u], nK + s * p.row_bytes, nV + s * p.row_bytes, nullptr, p.row_bytes, g);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (src[u] < 0) continue;
+      const size_t t = static_cast<size_t>(h) * p.ring_cap + dst[u];
+      store_rows(rw[u], static_cast<char*>(p.rK) + t * p.row_bytes, static_cast<char*>(p.rV) + t * p.row_bytes,
+                 nullptr, p.row_bytes, g);
+      if (g.sub == 0) p.rids[t] = p.new_ids[src[u]];
+    }
   }
 }
 
@@ -310,17 +330,28 @@ __global__ void static_copy_kernel(const PrunePlan p) {
   const int h = blockIdx.y;
   if (!((p.static_mask >> h) & 1ull)) return;
   const RowGroup g = row_group(p.row_bytes);
-  for (int i = g.first; i < p.g.F; i += g.stride) {
-    const int src = (p.n_frames - 1) * p.g.F + i;
-    const size_t s = static_cast<size_t>(h) * p.n_frames * p.g.F + src;
-    const size_t t = static_cast<size_t>(h) * p.g.F + i;
-    copy_row(static_cast<char*>(p.tK) + t * p.row_bytes, static_cast<const char*>(p.newK) + s * p.row_bytes,
-             p.row_bytes, g);
-    copy_row(static_cast<char*>(p.tV) + t * p.row_bytes, static_cast<const char*>(p.newV) + s * p.row_bytes,
-             p.row_bytes, g);
-    if (g.sub == 0) {
-      p.tids[t] = p.new_ids[src];
-      if (i == 0) p.tlen[h] = p.g.F;
+  const char* nK = static_cast<const char*>(p.newK);
+  const char* nV = static_cast<const char*>(p.newV);
+  for (int i0 = g.first; i0 < p.g.F; i0 += 2 * g.stride) {
+    RowWords rw[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = i0 + u * g.stride;
+      if (i >= p.g.F) continue;
+      const size_t s = static_cast<size_t>(h) * p.n_frames * p.g.F + (p.n_frames - 1) * p.g.F + i;
+      load_rows(rw[u], nK + s * p.row_bytes, nV + s * p.row_bytes, nullptr, p.row_bytes, g);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = i0 + u * g.stride;
+      if (i >= p.g.F) continue;
+      const size_t t = static_cast<size_t>(h) * p.g.F + i;
+      store_rows(rw[u], static_cast<char*>(p.tK) + t * p.row_bytes, static_cast<char*>(p.tV) + t * p.row_bytes,
+                 nullptr, p.row_bytes, g);
+      if (g.sub == 0) {
+        p.tids[t] = p.new_ids[(p.n_frames - 1) * p.g.F + i];
+        if (i == 0) p.tlen[h] = p.g.F;
+      }
     }
   }
 }

@@ -67,4 +67,38 @@ __device__ __forceinline__ void copy_row(void* dst, const void* src, int row_byt
   for (int o = g.sub; o < row_bytes / 16; o += g.L) d[o] = s[o];
 }
 
+// K and V rows (and, for the group's lanes 0..3, a 64-byte augmented row) moved
+// together: every load is issued before the first store, so a lane has all its
+// words in flight at once (rows of at most 32 words of 16 bytes per lane group:
+// 512 bytes).  Null pointers skip that row.
+struct RowWords {
+  uint4 k[2], v[2], a;
+};
+__device__ __forceinline__ void load_rows(RowWords& w, const void* k, const void* v, const void* aug, int row_bytes,
+                                          const RowGroup& g) {
+  const int words = row_bytes / 16;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int o = g.sub + u * g.L;
+    if (o < words) {
+      if (k) w.k[u] = __ldg(static_cast<const uint4*>(k) + o);
+      if (v) w.v[u] = __ldg(static_cast<const uint4*>(v) + o);
+    }
+  }
+  if (aug && g.sub < 4) w.a = __ldg(static_cast<const uint4*>(aug) + g.sub);
+}
+__device__ __forceinline__ void store_rows(const RowWords& w, void* k, void* v, void* aug, int row_bytes,
+                                           const RowGroup& g) {
+  const int words = row_bytes / 16;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int o = g.sub + u * g.L;
+    if (o < words) {
+      if (k) static_cast<uint4*>(k)[o] = w.k[u];
+      if (v) static_cast<uint4*>(v)[o] = w.v[u];
+    }
+  }
+  if (aug && g.sub < 4) static_cast<uint4*>(aug)[g.sub] = w.a;
+}
+
 }  // namespace kvb

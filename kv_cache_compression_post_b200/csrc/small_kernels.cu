@@ -20,47 +20,59 @@ __global__ void aug_rows_kernel(const T* __restrict__ X, long long ldX, int d, i
   const int n = n_dev ? n_dev[h] : n_uni;
   const int row_bytes = d * static_cast<int>(sizeof(T));
   const RowGroup g = row_group(row_bytes);
-  const __nv_bfloat16 one = __float2bfloat16_rn(1.f), zero = __float2bfloat16_rn(0.f);
   float gmax = 0.f;
-  // the loop runs warp-uniformly (every lane reaches the shuffles); a group whose
-  // row is past the end only skips its loads and stores
+  // rows of at most 32 words of 16 bytes: one word per lane of a group (g.L = words).
+  // Two rows per group in flight; the loop runs warp-uniformly (every lane
+  // reaches the shuffles), a group whose row is past the end only skips its load
+  // and store
   const int lane_group = (threadIdx.x & 31) / g.L;
-  for (int r0 = g.first - lane_group; r0 < n; r0 += g.stride) {
-    const int r = r0 + lane_group;
-    const bool live = r < n;
-    float acc = 0.f;
-    if (live) {
-      const uint4* x = reinterpret_cast<const uint4*>(X + (static_cast<long long>(h) * ldX + r) * d);
-      for (int w = g.sub; w < row_bytes / 16; w += g.L) {
-        const uint4 u = __ldg(x + w);
-        const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+  for (int r0 = g.first - lane_group; r0 < n; r0 += 2 * g.stride) {
+    float acc[2] = {0.f, 0.f};
+    uint4 u[2];
+    bool live[2];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          if (sizeof(T) == 2) {
-            const float lo = __uint_as_float(q[k] << 16), hi = __uint_as_float(q[k] & 0xFFFF0000u);
-            acc = fmaf(lo, lo, fmaf(hi, hi, acc));
-          } else {
-            const float v = __uint_as_float(q[k]);
-            acc = fmaf(v, v, acc);
-          }
+    for (int k = 0; k < 2; ++k) {
+      const int r = r0 + lane_group + k * g.stride;
+      live[k] = r < n;
+      if (live[k] && g.sub < row_bytes / 16)
+        u[k] = __ldg(reinterpret_cast<const uint4*>(X + (static_cast<long long>(h) * ldX + r) * d) + g.sub);
+      else
+        u[k] = make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint32_t q[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (sizeof(T) == 2) {
+          const float lo = __uint_as_float(q[j] << 16), hi = __uint_as_float(q[j] & 0xFFFF0000u);
+          acc[k] = fmaf(lo, lo, fmaf(hi, hi, acc[k]));
+        } else {
+          const float v = __uint_as_float(q[j]);
+          acc[k] = fmaf(v, v, acc[k]);
         }
       }
+      for (int o = g.L >> 1; o > 0; o >>= 1) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], o);
     }
-    for (int o = g.L >> 1; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (!live) continue;
-    gmax = fmaxf(gmax, acc);
-    // 32 entries: row form [hi, mid, lo, 1, 1, 1, 0...], column form [1, 1, 1, hi, mid, lo, 0...]
-    const float nrm = -0.5f * acc;
-    const __nv_bfloat16 hi = __float2bfloat16_rn(nrm);
-    const __nv_bfloat16 mid = __float2bfloat16_rn(nrm - __bfloat162float(hi));
-    const __nv_bfloat16 lo = __float2bfloat16_rn(nrm - __bfloat162float(hi) - __bfloat162float(mid));
-    for (int e = g.sub; e < 32; e += g.L) {
-      const int c = e & 15;
-      const bool colform = e >= 16;
-      __nv_bfloat16 v = zero;
-      if (c < 3) v = colform ? one : (c == 0 ? hi : (c == 1 ? mid : lo));
-      else if (c < 6) v = colform ? (c == 3 ? hi : (c == 4 ? mid : lo)) : one;
-      out[(static_cast<long long>(h) * ldOut + r) * 32 + e] = *reinterpret_cast<uint16_t*>(&v);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      if (!live[k]) continue;
+      gmax = fmaxf(gmax, acc[k]);
+      // 32 entries: row form [hi, mid, lo, 1, 1, 1, 0...], column form [1, 1, 1, hi, mid, lo, 0...];
+      // lanes 0..3 of the group write one 16-byte word each
+      if (g.sub >= 4) continue;
+      const float nrm = -0.5f * acc[k];
+      const __nv_bfloat16 bhi = __float2bfloat16_rn(nrm);
+      const __nv_bfloat16 bmid = __float2bfloat16_rn(nrm - __bfloat162float(bhi));
+      const __nv_bfloat16 blo = __float2bfloat16_rn(nrm - __bfloat162float(bhi) - __bfloat162float(bmid));
+      const uint32_t one = 0x3F80u;  // bf16 1.0
+      const uint32_t hi = *reinterpret_cast<const uint16_t*>(&bhi), mid = *reinterpret_cast<const uint16_t*>(&bmid),
+                     lo = *reinterpret_cast<const uint16_t*>(&blo);
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (g.sub == 0) w = make_uint4(hi | (mid << 16), lo | (one << 16), one | (one << 16), 0u);
+      else if (g.sub == 2) w = make_uint4(one | (one << 16), one | (hi << 16), mid | (lo << 16), 0u);
+      const int r = r0 + lane_group + k * g.stride;
+      reinterpret_cast<uint4*>(out + (static_cast<long long>(h) * ldOut + r) * 32)[g.sub] = w;
     }
   }
   if (!norm_max) return;
