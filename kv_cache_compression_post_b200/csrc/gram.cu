@@ -15,18 +15,15 @@
 // The clamp t >= eps is applied only when the largest key norm makes the fp32
 // rounding of x comparable to eps (a per-launch flag).
 //
-// Work = the sequence of (head, 256-row block, 128-column tile) steps, split evenly
+// Work = the sequence of (head, 256-row block, 256-column tile) steps, split evenly
 // over a persistent grid (one CTA per SM).  A CTA keeps its 256 rows (two 128-row
-// MMA tiles) in shared memory and streams 128-column tiles through a 4-stage TMA
-// ring.  TMEM holds four 128 x 128 fp32 accumulators, one per (step parity, row
-// tile): the tensor core fills the two of a step while the epilogue drains the two
-// of the step before, so each accumulator has three other MMA groups' time to be
-// read out before it is needed again (with two 256-column accumulators the
-// read-out, not the MMA, set the pace).
-// Warp roles: 0 = TMA producer, 1 = MMA issuer, 2 = TMEM owner, 4..19 epilogue:
-// four warps (the four TMEM lane quarters) per accumulator, one thread per row, so
-// row sums need no cross-thread reduction; each parity keeps its own partial sum
-// of a row and writes it as one partial slot.
+// MMA tiles) in shared memory and streams 256-column tiles through a 2-stage TMA
+// ring.  Each row tile has one 128 x 256 fp32 accumulator in TMEM (N = 256 MMAs run
+// at full tensor rate); the two row tiles ping-pong: while the tensor core fills
+// one, the 8 epilogue warps of the other drain it.
+// Warp roles: 0 = TMA producer, 1 = MMA issuer, 2 = TMEM owner, 4..11 epilogue of
+// row tile 0, 12..19 of row tile 1 (4 TMEM lane quarters x 2 column halves; one
+// thread per row and half, so row sums need no cross-thread reduction).
 #include <climits>
 
 #include "gram.cuh"
@@ -39,16 +36,15 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kStages = 4;
-constexpr int kColTile = kGramColTile;   // columns per MMA (N) and per step
-constexpr int kAcc = 4;                  // TMEM accumulators: (step parity, row tile)
-constexpr int kEpiWarpsPerAcc = 4;
+constexpr int kStages = 2;
+constexpr int kColTile = 256;   // columns per MMA (N) and per step
+constexpr int kEpiWarpsPerTile = 8;
 constexpr uint32_t kAugRowBytes = 32;  // 16 bf16 of the augmented row per operand row
 
 struct alignas(8) GramBars {
   uint64_t a_full, a_empty;
   uint64_t full[kStages], empty[kStages];
-  uint64_t acc_full[kAcc], acc_empty[kAcc];
+  uint64_t acc_full[2], acc_empty[2];   // per row tile
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
@@ -177,7 +173,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nbox = a.d / 64;
   const uint32_t aBytes = static_cast<uint32_t>(kGramRowTile) * a.d * 2;   // one 128-row tile
-  const uint32_t bBytes = static_cast<uint32_t>(kColTile) * a.d * 2;       // one column tile
+  const uint32_t bBytes = static_cast<uint32_t>(kColTile) * a.d * 2;       // one 256-row column tile
   const uint32_t aAug = kGramRowTile * kAugRowBytes, bAug = kColTile * kAugRowBytes;
   uint8_t* sA = smem;                          // 2 row tiles
   uint8_t* sB = sA + 2 * aBytes;               // kStages column tiles
@@ -195,9 +191,9 @@ __global__ void __launch_bounds__(kGramThreads, 1)
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
-    for (int g = 0; g < kAcc; ++g) {
-      mbar_init(&bars->acc_full[g], 1);
-      mbar_init(&bars->acc_empty[g], kEpiWarpsPerAcc);
+    for (int r = 0; r < 2; ++r) {
+      mbar_init(&bars->acc_full[r], 1);
+      mbar_init(&bars->acc_empty[r], kEpiWarpsPerTile);
     }
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
@@ -269,7 +265,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
       const uint32_t aBase = smem_u32(sA), bBase = smem_u32(sB);
       const uint32_t aaBase = smem_u32(sAa), baBase = smem_u32(sBa);
       int it = 0, aload = 0;
-      int tr[kAcc] = {0, 0, 0, 0};  // tiles issued into each accumulator
+      int tr[2] = {0, 0};  // tiles issued into each row tile's accumulator
       bool ok = true;
       Cursor c;
       if (L0 < L1) cursor_seek(a, L0, c);
@@ -283,11 +279,10 @@ __global__ void __launch_bounds__(kGramThreads, 1)
         const int s = it % kStages;
         if (!(ok = mbar_wait(&bars->full[s], (it / kStages) & 1, abort, a.status))) break;
         for (int r = 0; r < nact && ok; ++r) {
-          // accumulator (step parity, row tile): free once its 4 epilogue warps hold it in registers
-          const int g = ((it & 1) << 1) | r;
-          if (!(ok = mbar_wait(&bars->acc_empty[g], (tr[g] & 1) ^ 1, abort, a.status))) break;
+          // the row tile's accumulator is free once its 8 epilogue warps hold it in registers
+          if (!(ok = mbar_wait(&bars->acc_empty[r], (tr[r] & 1) ^ 1, abort, a.status))) break;
           tc_fence_after();
-          const uint32_t dcol = tmem + static_cast<uint32_t>(g * kColTile);
+          const uint32_t dcol = tmem + static_cast<uint32_t>(r * kColTile);
           for (int kk = 0; kk < a.d / 16; ++kk) {
             const uint32_t ka = static_cast<uint32_t>((kk >> 2) * (kGramRowTile * 128) + (kk & 3) * 32);
             const uint32_t kb = static_cast<uint32_t>((kk >> 2) * (kColTile * 128) + (kk & 3) * 32);
@@ -296,8 +291,8 @@ __global__ void __launch_bounds__(kGramThreads, 1)
           }
           // the norm terms: one more K=16 step over the augmented rows
           mma_f16_ss(dcol, sdesc_sw32(aaBase + r * aAug, 256), sdesc_sw32(baBase + s * bAug, 256), idesc, 1u);
-          mma_commit(&bars->acc_full[g]);
-          ++tr[g];
+          mma_commit(&bars->acc_full[r]);
+          ++tr[r];
         }
         if (!ok) break;
         mma_commit(&bars->empty[s]);
@@ -306,7 +301,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
         if (last_of_block) mma_commit(&bars->a_empty);
         cursor_next(a, c);
       }
-      if (!ok && (tr[0] + tr[1] + tr[2] + tr[3]) > 0) {
+      if (!ok && (tr[0] + tr[1]) > 0) {
         // abort path: no MMA may still write TMEM when it is freed (the commit
         // arrives once every MMA issued by this thread has completed)
         mma_commit(&bars->mma_done);
@@ -316,16 +311,15 @@ __global__ void __launch_bounds__(kGramThreads, 1)
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
     const int e = warp - 4;
-    const int acc = e >> 2;          // accumulator: (step parity, row tile)
-    const int par = acc >> 1;        // steps of this parity (CTA-local step index)
-    const int r = acc & 1;           // row tile
+    const int r = e >> 3;            // row tile
     const int q = warp & 3;          // TMEM lane quarter (warp_id % 4)
+    const int hf = (e >> 2) & 1;     // column half of the 256-column tile
     const int row_in_tile = q * 32 + lane;
     const float ks = a.kscale, eps = a.eps, nhs = -0.5f * a.s;
     const float2 ks2 = make_float2(ks, ks), eps2 = make_float2(eps, eps);
     // clamp t >= eps only when fp32 rounding of x could reach eps / 2 (see header)
     const bool clamp = a.norm_max ? (*a.norm_max) * 1e-4f >= eps * (-2.f / ks) : true;
-    int t = 0;                       // tiles seen by this accumulator (phase of its barriers)
+    int t = 0;                       // tiles seen by this row tile (phase of its barriers)
     bool ok = true;
     Cursor c;
     if (L0 < L1) cursor_seek(a, L0, c);
@@ -334,7 +328,6 @@ __global__ void __launch_bounds__(kGramThreads, 1)
     bool active = false, valid_row = false;
     long long Lblock = L0;  // first step of the current row block
     for (long long L = L0; L < L1; ++L) {
-      const bool mine = ((L - L0) & 1) == par;
       if (L == L0 || c.j == 0) {
         Lblock = L - c.j;
         rt0 = c.rb * kGramRowBlock + r * kGramRowTile;
@@ -346,16 +339,17 @@ __global__ void __launch_bounds__(kGramThreads, 1)
         acc_pos = 0.f;
         acc_neg = 0.f;
       }
-      if (active && mine) {
-        if (!(ok = mbar_wait(&bars->acc_full[acc], t & 1, abort, a.status))) break;
+      if (active) {
+        if (!(ok = mbar_wait(&bars->acc_full[r], t & 1, abort, a.status))) break;
         tc_fence_after();
-        const int c0 = c.j * kColTile;  // first column of the tile
-        const bool tail = c0 + kColTile > c.nC;
-        const bool allneg = c0 + kColTile <= nneg;
+        const int c0 = c.j * kColTile + hf * 128;  // first column of this thread's half
+        const bool tail = c0 + 128 > c.nC;
+        const bool allneg = c0 + 128 <= nneg;
         const bool mixed = (c0 < nneg) && !allneg;
-        const bool diag_hit = a.use_diag && (rt0 + diag < c0 + kColTile) && (rt0 + diag + kGramRowTile > c0);
+        const bool diag_hit = a.use_diag && (rt0 + diag < c0 + 128) && (rt0 + diag + kGramRowTile > c0);
         const bool masked = tail || mixed || diag_hit;
-        const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kColTile);
+        const uint32_t taddr =
+            tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(r * kColTile + hf * 128);
         float2 acc2 = make_float2(0.f, 0.f);
         float accs = 0.f;
         // masked tiles (ragged end, self pair, sign change) take an exact scalar path
@@ -375,7 +369,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
             }
           }
         };
-        // 8 chunks of 16 columns (kColTile = 128); chunk c+1 is in flight while chunk c is processed
+        // 8 chunks of 16 columns; chunk c+1 is in flight while chunk c is processed
         uint32_t va[16], vb[16];
         tmem_ld16(taddr + 0, va);
         tmem_wait_ld_reg16(va);
@@ -390,7 +384,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
             // every column this warp needs is in registers: hand the accumulator back
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->acc_empty[acc]);
+            if (lane == 0) mbar_arrive(&bars->acc_empty[r]);
           }
           chunk(vb, cc + 1);
           if (cc + 2 < 8) tmem_wait_ld_reg16(va);
@@ -406,7 +400,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
       }
       const bool last_of_block = (L + 1 == L1) || (c.j + 1 == c.CT);
       if (last_of_block && valid_row) {
-        const int slot = 2 * (cta - cta_of(Lblock, T, G)) + par;
+        const int slot = 2 * (cta - cta_of(Lblock, T, G)) + hf;
         if (slot >= 0 && slot < a.slots)
           a.partial[(static_cast<size_t>(slot) * a.H + c.h) * a.ldOut + row] = acc_pos - acc_neg;
         else
@@ -496,7 +490,7 @@ __global__ void gram_reduce_kernel(const GramArgs a, float* out, int ldOut) {
     }
     const long long Lb = before + static_cast<long long>(r / kGramRowBlock) * CT;
     const int first = cta_of(Lb, T, G), last = cta_of(Lb + CT - 1, T, G);
-    const int n = 2 * (last - first + 1);  // two step parities per CTA
+    const int n = 2 * (last - first + 1);  // two column halves per CTA
     for (int sl = 0; sl < n && sl < a.slots; ++sl)
       acc += a.partial[(static_cast<size_t>(sl) * a.H + h) * a.ldOut + r];
   }
@@ -513,7 +507,7 @@ size_t gram_smem_bytes(int d) {
 
 void gram_plan(GramArgs& a, int max_col_tiles, int n_sm) {
   // at most 8 CTAs cover a row block (every active CTA takes >= min_steps steps);
-  // each CTA writes one partial per step parity
+  // each CTA writes one partial per column half
   a.grid = n_sm;
   a.slots = 16;
   const int m = (max_col_tiles + 6) / 7;

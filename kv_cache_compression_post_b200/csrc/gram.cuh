@@ -9,8 +9,8 @@
 namespace kvb {
 
 constexpr int kGramRowTile = 128;      // rows per TMEM accumulator (M of the MMA)
-constexpr int kGramRowBlock = 256;     // rows per work unit (two row tiles)
-constexpr int kGramColTile = 128;      // columns per MMA (N) and per work step
+constexpr int kGramRowBlock = 256;     // rows per work unit (two accumulators)
+constexpr int kGramColTile = 256;      // columns per MMA (N) and per work step
 constexpr int kGramThreads = 640;      // 4 control warps + 16 epilogue warps
 
 // A set of rows/cols: per head a count and a start row inside its buffer.  Each
@@ -37,7 +37,7 @@ struct GramArgs {
   float s = 2.f;
   int max_rows = 0;                // upper bound of the row count of any head
   int grid = 0;                    // CTAs launched
-  int slots = 0;                   // partial slots per row block (two step parities per CTA)
+  int slots = 0;                   // partial slots per row block (two column halves per CTA)
   int min_steps = 1;               // every active CTA takes at least this many steps
   float* partial = nullptr;        // [slots][H][ldOut]
   int ldOut = 0;
@@ -52,7 +52,7 @@ struct GramArgs {
 
 // bf16 operands through TMA: tensor maps over [H][rows][d] and over the augmented
 // rows [H][rows][32] (see launch_aug_rows); row maps use 128-row boxes, column maps
-// kGramColTile-row boxes.  The MMA accumulates a.b - (||a||^2 + ||b||^2)/2 =
+// 256-row boxes (kGramColTile).  The MMA accumulates a.b - (||a||^2 + ||b||^2)/2 =
 // -||a - b||^2 / 2 directly.
 cudaError_t launch_gram_bf16(const GramArgs& a, const CUtensorMap& tmR, const CUtensorMap& tmC,
                              const CUtensorMap& tmRa, const CUtensorMap& tmCa, cudaStream_t st);
