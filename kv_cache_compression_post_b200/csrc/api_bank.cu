@@ -321,7 +321,7 @@ cudaError_t admit_phase1(kvb_bank* b, const AdmitPlan& p, const DeviceInfo& dev,
   cudaError_t e = cudaSuccess;
   if (g.dtype == KVB_BF16)
     e = launch_aug_rows(candK, g.dtype, H, N, d, N, nullptr, N, b->caug, b->ldN, reinterpret_cast<float*>(b->status + 1),
-                        st);
+                        -0.5f * g.eps * b->h, st);
 
   // pass 1: candidate density against the bank, rho_B(c)
   if (e == cudaSuccess) {
@@ -506,7 +506,8 @@ kvb_status kvb_bank_import(kvb_bank* b, int32_t layer, int32_t head, const int32
                           cudaMemcpyDeviceToDevice, st);
     if (e == cudaSuccess && b->cfg.dtype == KVB_BF16)
       e = launch_aug_rows(b->K + slot0 * b->row_bytes, b->cfg.dtype, 1, size, b->cfg.head_dim, size, nullptr, size,
-                          b->aug + slot0 * 32, size, reinterpret_cast<float*>(b->status + 1), st);
+                          b->aug + slot0 * 32, size, reinterpret_cast<float*>(b->status + 1),
+                          -0.5f * b->cfg.eps * b->h, st);
   }
   // the size word comes from host memory; the call synchronises before returning
   int host_size = size;

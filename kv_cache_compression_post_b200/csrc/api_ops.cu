@@ -109,9 +109,9 @@ kvb_status kvb_density(const void* rows, int32_t n_rows, const void* cols, int32
   }
   if (n_cols == 0) return cuda_status(cudaMemsetAsync(out, 0, sizeof(float) * heads * n_rows, st));
   cudaError_t e =
-      launch_aug_rows(rows, dtype, heads, n_rows, head_dim, n_rows, nullptr, n_rows, L.rowAug, n_rows, norm_max, st);
+      launch_aug_rows(rows, dtype, heads, n_rows, head_dim, n_rows, nullptr, n_rows, L.rowAug, n_rows, norm_max, -0.5f * eps * h, st);
   if (e == cudaSuccess)
-    e = launch_aug_rows(cols, dtype, heads, n_cols, head_dim, n_cols, nullptr, n_cols, L.colAug, n_cols, norm_max, st);
+    e = launch_aug_rows(cols, dtype, heads, n_cols, head_dim, n_cols, nullptr, n_cols, L.colAug, n_cols, norm_max, -0.5f * eps * h, st);
   a.norm_max = norm_max;
   if (e != cudaSuccess) return KVB_E_CUDA;
   CUtensorMap tmR, tmC, tmRa, tmCa;

@@ -6,14 +6,16 @@
 //     -||a - b||^2 / 2 = a.b - ||a||^2/2 - ||b||^2/2
 // the whole right-hand side is one bf16 contraction: each key carries 32 extra
 // bf16 values ("augmented row": -||k||^2/2 split exactly into three bf16 parts,
-// plus ones), and one extra K=16 MMA step adds both norm terms, so the fp32 TMEM
-// accumulator holds -||a - b||^2 / 2 for every pair.  The epilogue on CUDA cores is
-// t = acc * (-2/h) + eps and phi(t).  For the default s = 2 four reciprocals share
-// one MUFU op,
-//     1/t0 + 1/t1 + 1/t2 + 1/t3 = ((t0+t1) t2 t3 + (t2+t3) t0 t1) / (t0 t1 t2 t3),
-// and the arithmetic runs two pairs per instruction (packed f32x2 FMA/MUL/ADD).
-// The clamp t >= eps is applied only when the largest key norm makes the fp32
-// rounding of x comparable to eps (a per-launch flag).
+// the constant -eps h/2 split into two, and ones), and one extra K=16 MMA step adds
+// the norm terms and the regulariser, so the fp32 TMEM accumulator holds
+//     D = -||a - b||^2 / 2 - eps h / 2 = -(h/2) t,   t = ||a - b||^2 / h + eps,
+// for every pair.  The epilogue on CUDA cores sums 1/D directly (phi = 1/t =
+// -(h/2)/D for the default s = 2): four reciprocals share one MUFU op,
+//     1/D0 + 1/D1 + 1/D2 + 1/D3 = ((D0+D1) D2 D3 + (D2+D3) D0 D1) / (D0 D1 D2 D3),
+// the arithmetic runs two pairs per instruction (packed f32x2 ADD/MUL/FMA), and the
+// tile's sum is scaled by -h/2 once.  Other exponents take t = D (-2/h) per pair.
+// The clamp t >= eps (D <= -eps h/2) is applied only when the largest key norm
+// makes the fp32 rounding of x comparable to eps (a per-launch flag).
 //
 // Work = the sequence of (head, 256-row block, 256-column tile) steps, split evenly
 // over a persistent grid (one CTA per SM).  A CTA keeps its 256 rows (two 128-row
@@ -138,26 +140,26 @@ __device__ __forceinline__ float phi_t(float t, float nhs) {
 
 __device__ __forceinline__ float2 f2(uint32_t x, uint32_t y) { return make_float2(__uint_as_float(x), __uint_as_float(y)); }
 
-// Sum of phi over 16 accumulator columns (s = 2, packed f32x2, 4 MUFU ops):
-// t = acc * ks + eps; pairs (t_{2i}, t_{2i+1}) travel together, and each lane of a
-// float2 folds four reciprocals into one.
+// Sum of 1/D over 16 accumulator columns (s = 2, packed f32x2, 4 MUFU ops): pairs
+// (D_{2i}, D_{2i+1}) travel together, and each lane of a float2 folds four
+// reciprocals into one.  dmax = -eps h/2 is the clamp (D <= dmax).
 template <bool CLAMP>
-__device__ __forceinline__ float2 sum_recip16(const uint32_t (&v)[16], float2 ks2, float2 eps2, float eps, float2 acc) {
+__device__ __forceinline__ float2 sum_recip16(const uint32_t (&v)[16], float dmax, float2 acc) {
 #pragma unroll
   for (int k = 0; k < 16; k += 8) {
-    float2 A = __ffma2_rn(f2(v[k + 0], v[k + 1]), ks2, eps2);
-    float2 B = __ffma2_rn(f2(v[k + 2], v[k + 3]), ks2, eps2);
-    float2 C = __ffma2_rn(f2(v[k + 4], v[k + 5]), ks2, eps2);
-    float2 D = __ffma2_rn(f2(v[k + 6], v[k + 7]), ks2, eps2);
+    float2 A = f2(v[k + 0], v[k + 1]);
+    float2 B = f2(v[k + 2], v[k + 3]);
+    float2 C = f2(v[k + 4], v[k + 5]);
+    float2 D = f2(v[k + 6], v[k + 7]);
     if constexpr (CLAMP) {
-      A = make_float2(fmaxf(A.x, eps), fmaxf(A.y, eps));
-      B = make_float2(fmaxf(B.x, eps), fmaxf(B.y, eps));
-      C = make_float2(fmaxf(C.x, eps), fmaxf(C.y, eps));
-      D = make_float2(fmaxf(D.x, eps), fmaxf(D.y, eps));
+      A = make_float2(fminf(A.x, dmax), fminf(A.y, dmax));
+      B = make_float2(fminf(B.x, dmax), fminf(B.y, dmax));
+      C = make_float2(fminf(C.x, dmax), fminf(C.y, dmax));
+      D = make_float2(fminf(D.x, dmax), fminf(D.y, dmax));
     }
-    const float2 s = __fadd2_rn(A, B), p = __fmul2_rn(A, B);     // lane x: t0+t2, t0 t2; lane y: t1+t3, t1 t3
+    const float2 s = __fadd2_rn(A, B), p = __fmul2_rn(A, B);     // lane x: D0+D2, D0 D2; lane y: D1+D3, D1 D3
     const float2 s2 = __fadd2_rn(C, D), p2 = __fmul2_rn(C, D);
-    const float2 num = __ffma2_rn(s, p2, __fmul2_rn(s2, p));      // (ta+tb) tc td + (tc+td) ta tb
+    const float2 num = __ffma2_rn(s, p2, __fmul2_rn(s2, p));      // (Da+Db) Dc Dd + (Dc+Dd) Da Db
     const float2 den = __fmul2_rn(p, p2);
     acc = __ffma2_rn(num, make_float2(rcp_approx(den.x), rcp_approx(den.y)), acc);
   }
@@ -316,7 +318,8 @@ __global__ void __launch_bounds__(kGramThreads, 1)
     const int hf = (e >> 2) & 1;     // column half of the 256-column tile
     const int row_in_tile = q * 32 + lane;
     const float ks = a.kscale, eps = a.eps, nhs = -0.5f * a.s;
-    const float2 ks2 = make_float2(ks, ks), eps2 = make_float2(eps, eps);
+    const float kinv = 1.f / ks;     // -h/2: sum of 1/D -> sum of phi (s = 2)
+    const float dmax = eps * kinv;   // -eps h/2: D <= dmax <=> t >= eps
     // clamp t >= eps only when fp32 rounding of x could reach eps / 2 (see header)
     const bool clamp = a.norm_max ? (*a.norm_max) * 1e-4f >= eps * (-2.f / ks) : true;
     int t = 0;                       // tiles seen by this row tile (phase of its barriers)
@@ -356,12 +359,12 @@ __global__ void __launch_bounds__(kGramThreads, 1)
         auto chunk = [&](const uint32_t (&v)[16], int cc) {
           const int cb = c0 + cc * 16;
           if (SMODE == 2 && !masked) {
-            acc2 = clamp ? sum_recip16<true>(v, ks2, eps2, eps, acc2) : sum_recip16<false>(v, ks2, eps2, eps, acc2);
+            acc2 = clamp ? sum_recip16<true>(v, dmax, acc2) : sum_recip16<false>(v, dmax, acc2);
           } else {
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
               const int col = cb + k;
-              const float tv = fmaxf(fmaf(__uint_as_float(v[k]), ks, eps), eps);
+              const float tv = fmaxf(__uint_as_float(v[k]) * ks, eps);
               const bool valid = (col < c.nC) && (col != row + diag);
               const float ph = valid ? phi_t<SMODE>(tv, nhs) : 0.f;
               if (masked && col < nneg) acc_neg += ph;
@@ -390,7 +393,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
           if (cc + 2 < 8) tmem_wait_ld_reg16(va);
         }
         if (!masked) {
-          const float tile = acc2.x + acc2.y + accs;
+          const float tile = (acc2.x + acc2.y) * kinv + accs;
           if (allneg) acc_neg += tile;
           else acc_pos += tile;
         } else {

@@ -103,9 +103,9 @@ extern "C" kvb_status kvb_density_noalloc(const void* rows, int32_t n_rows, cons
 
   const float h = dist_scale > 0.f ? dist_scale : static_cast<float>(head_dim);
   cudaError_t e =
-      launch_aug_rows(rows, dtype, heads, n_rows, head_dim, n_rows, nullptr, n_rows, rowAug, n_rows, norm_max, st);
+      launch_aug_rows(rows, dtype, heads, n_rows, head_dim, n_rows, nullptr, n_rows, rowAug, n_rows, norm_max, -0.5f * eps * h, st);
   if (e == cudaSuccess)
-    e = launch_aug_rows(cols, dtype, heads, n_cols, head_dim, n_cols, nullptr, n_cols, colAug, n_cols, norm_max, st);
+    e = launch_aug_rows(cols, dtype, heads, n_cols, head_dim, n_cols, nullptr, n_cols, colAug, n_cols, norm_max, -0.5f * eps * h, st);
   if (e != cudaSuccess) return KVB_E_CUDA;
   CUtensorMap tmR, tmC, tmRa, tmCa;
   if (!make_tmap_bf16(&tmR, rows, head_dim, n_rows, heads, 128) ||

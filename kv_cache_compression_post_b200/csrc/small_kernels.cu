@@ -12,7 +12,7 @@ namespace {
 // norm_max with a single atomic (per-row atomics on one word serialise).
 template <typename T>
 __global__ void aug_rows_kernel(const T* __restrict__ X, long long ldX, int d, int n_uni, const int* n_dev,
-                                uint16_t* __restrict__ out, long long ldOut, float* norm_max) {
+                                uint16_t* __restrict__ out, long long ldOut, float* norm_max, float reg) {
   pdl_wait();
   pdl_trigger();
   __shared__ float s_max[32];
@@ -58,19 +58,23 @@ __global__ void aug_rows_kernel(const T* __restrict__ X, long long ldX, int d, i
     for (int k = 0; k < 2; ++k) {
       if (!live[k]) continue;
       gmax = fmaxf(gmax, acc[k]);
-      // 32 entries: row form [hi, mid, lo, 1, 1, 1, 0...], column form [1, 1, 1, hi, mid, lo, 0...];
+      // 32 entries: row form [hi, mid, lo, 1, 1, 1, rhi, rlo, 0...], column form
+      // [1, 1, 1, hi, mid, lo, 1, 1, 0...];
       // lanes 0..3 of the group write one 16-byte word each
       if (g.sub >= 4) continue;
       const float nrm = -0.5f * acc[k];
       const __nv_bfloat16 bhi = __float2bfloat16_rn(nrm);
       const __nv_bfloat16 bmid = __float2bfloat16_rn(nrm - __bfloat162float(bhi));
       const __nv_bfloat16 blo = __float2bfloat16_rn(nrm - __bfloat162float(bhi) - __bfloat162float(bmid));
+      const __nv_bfloat16 brh = __float2bfloat16_rn(reg);
+      const __nv_bfloat16 brl = __float2bfloat16_rn(reg - __bfloat162float(brh));
       const uint32_t one = 0x3F80u;  // bf16 1.0
       const uint32_t hi = *reinterpret_cast<const uint16_t*>(&bhi), mid = *reinterpret_cast<const uint16_t*>(&bmid),
                      lo = *reinterpret_cast<const uint16_t*>(&blo);
+      const uint32_t rh = *reinterpret_cast<const uint16_t*>(&brh), rl = *reinterpret_cast<const uint16_t*>(&brl);
       uint4 w = make_uint4(0u, 0u, 0u, 0u);
-      if (g.sub == 0) w = make_uint4(hi | (mid << 16), lo | (one << 16), one | (one << 16), 0u);
-      else if (g.sub == 2) w = make_uint4(one | (one << 16), one | (hi << 16), mid | (lo << 16), 0u);
+      if (g.sub == 0) w = make_uint4(hi | (mid << 16), lo | (one << 16), one | (one << 16), rh | (rl << 16));
+      else if (g.sub == 2) w = make_uint4(one | (one << 16), one | (hi << 16), mid | (lo << 16), one | (one << 16));
       const int r = r0 + lane_group + k * g.stride;
       reinterpret_cast<uint4*>(out + (static_cast<long long>(h) * ldOut + r) * 32)[g.sub] = w;
     }
@@ -90,15 +94,15 @@ __global__ void aug_rows_kernel(const T* __restrict__ X, long long ldX, int d, i
 }  // namespace
 
 cudaError_t launch_aug_rows(const void* X, kvb_dtype dtype, int H, long long ldX, int d, int n_uni, const int* n_dev,
-                            int max_n, uint16_t* out, long long ldOut, float* norm_max, cudaStream_t st) {
+                            int max_n, uint16_t* out, long long ldOut, float* norm_max, float reg, cudaStream_t st) {
   if (max_n <= 0 || H <= 0) return cudaSuccess;
   dim3 grid(mover_blocks(max_n, d * (dtype == KVB_BF16 ? 2 : 4), H), H);
   LaunchTrace trace("aug_rows_kernel", st);
   if (dtype == KVB_BF16)
     return launch_pdl(aug_rows_kernel<__nv_bfloat16>, grid, dim3(256), 0, st, static_cast<const __nv_bfloat16*>(X),
-                      ldX, d, n_uni, n_dev, out, ldOut, norm_max);
+                      ldX, d, n_uni, n_dev, out, ldOut, norm_max, reg);
   return launch_pdl(aug_rows_kernel<float>, grid, dim3(256), 0, st, static_cast<const float*>(X), ldX, d, n_uni,
-                    n_dev, out, ldOut, norm_max);
+                    n_dev, out, ldOut, norm_max, reg);
 }
 
 
