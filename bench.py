@@ -196,7 +196,8 @@ def _cfg(w, kvb):
                                max_queries=w.chunk_tokens)
     return kvb.make_config(method=kvb.KVB_DENSITYKV, dtype=dt, layers=1, heads=w.heads, head_dim=w.head_dim,
                            capacity=w.capacity, max_candidates=w.chunk_tokens, tau=w.tau, eps=w.eps, s=w.s,
-                           sync_heads=1, max_queries=w.chunk_tokens)
+                           sync_heads=1, max_queries=w.chunk_tokens,
+                           storage=kvb.KVB_STORE_FP8_E4M3 if STORAGE["fp8"] else kvb.KVB_STORE_NATIVE)
 
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
@@ -206,6 +207,9 @@ DRAM_TRAFFIC = {
     # the four density passes of one 480P admit: 54.12 + 54.13 + 54.71 + 18.16 MB
     ("wan480", "gram_bf16_kernel"): (181.12e6 / 4, "profiles/gram_bf16_kernel_wan480.md"),
 }
+
+# bank K/V storage of the DensityKV workloads (--storage)
+STORAGE = {"fp8": False}
 
 # first timed chunk: steady state (DensityKV bank full; Forcing-KV ring of 21 frames full)
 FIRST_TIMED = {"wan480": 19, "wan1080": 9, "mid": 4, "tiny": 4, "forcing480": 8, "forcing_mid": 4}
@@ -848,6 +852,9 @@ def workload_config(w, args, world):
                 f"queries over sink {w.F} + bank (M={w.capacity}) + window {w.chunk_tokens}; {w.heads} heads, "
                 f"d={w.head_dim}, 1 layer, {chunks}")
         extra = {"M": w.capacity, "tau": w.tau}
+        if STORAGE["fp8"]:
+            text += "; bank K/V stored in FP8 E4M3 (the layer decompressed into a bf16 working copy)"
+            extra["storage"] = "fp8_e4m3"
     cfg = {"workload": text, "heads": w.heads, "head_dim": w.head_dim, "F": w.F, "N": w.chunk_tokens}
     cfg.update(extra)
     cfg.update({"parallelism": f"replicas x{world}", "l2": "flushed (256 MB write) before each step"})
@@ -862,9 +869,12 @@ def main():
     ap.add_argument("--workload", default="wan480")
     ap.add_argument("--impl", default="kvb", choices=["kvb", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--storage", default="native", choices=["native", "fp8"],
+                    help="DensityKV bank K/V storage: the bank dtype (native) or FP8 E4M3")
     ap.add_argument("--graph", action="store_true",
                     help="rollout workload: one CUDA graph per chunk over all layers, replayed")
     args = ap.parse_args()
+    STORAGE["fp8"] = args.storage == "fp8"
     if args.warmup < 3:
         args.warmup = 3
     w = kvgen.WORKLOADS[args.workload]

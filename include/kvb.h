@@ -114,6 +114,8 @@ typedef struct {
    * rule, so a zero-filled tail keeps it. */
   int32_t bottomk_scope;    /* kvb_bottomk_scope */
   int32_t sim_source;       /* kvb_sim_source */
+  /* storage of the retained K/V (0: the bank's dtype) */
+  int32_t storage;          /* kvb_storage */
 } kvb_config;
 
 /* Candidate ordering (App. E, candidate ordering).
@@ -159,6 +161,23 @@ typedef enum { KVB_BOTTOMK_FRAME = 0, KVB_BOTTOMK_CALL = 1 } kvb_bottomk_scope;
  *    chunk: a call for layer > 0 returns KVB_E_STATE before layer 0 has been
  *    pruned, or when its n_frames differs from layer 0's last call. */
 typedef enum { KVB_SIM_PER_LAYER = 0, KVB_SIM_FIRST_LAYER = 1 } kvb_sim_source;
+
+/* Storage of a DensityKV bank's K and V (bf16 banks).  The Forcing-KV reading
+ * notes report the method combined with FP8 (results); this library's reading is
+ * the retained history held in FP8 E4M3.
+ *  KVB_STORE_NATIVE: K and V in the bank's dtype.
+ *  KVB_STORE_FP8_E4M3: every layer's bank K and V are held in FP8 E4M3 (1 sign,
+ *    4 exponent bits with bias 7, 3 mantissa bits; one byte per element).
+ *    kvb_admit first rounds the candidates' K and V to E4M3 (to nearest, ties
+ *    to even, saturating at +-448), so every density, score, ratio and baseline
+ *    of the step and of later steps is computed from the values the bank stores;
+ *    kvb_bank_import rounds what it is given the same way and kvb_bank_export
+ *    returns the stored values as bf16.  The layer being updated or attended is
+ *    decompressed into one bf16 working copy (one layer's K and V, shared by the
+ *    layers) that the density and attention kernels read; the persistent
+ *    per-layer storage is half that of bf16.  An f32 bank returns KVB_E_INVAL
+ *    from kvb_workspace_size / kvb_bank_create with this storage. */
+typedef enum { KVB_STORE_NATIVE = 0, KVB_STORE_FP8_E4M3 = 1 } kvb_storage;
 
 /* Per-(layer, head) counters of the last kvb_admit / kvb_prune_hybrid. */
 typedef struct {

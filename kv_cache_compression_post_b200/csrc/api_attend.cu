@@ -38,7 +38,10 @@ extern "C" kvb_status kvb_attend(kvb_bank* b, int32_t layer, const void* Q, int3
     ++n;
   }
   if (g.method == KVB_DENSITYKV) {
-    const size_t lo = static_cast<size_t>(layer) * H * g.capacity;
+    // E4M3 storage: attention reads the bf16 working copy, made to hold the layer
+    const bool fp8 = g.storage == KVB_STORE_FP8_E4M3;
+    if (fp8 && kvb_work_layer(b, layer, st) != cudaSuccess) return KVB_E_CUDA;
+    const size_t lo = fp8 ? 0 : static_cast<size_t>(layer) * H * g.capacity;
     a.seg[n].K = b->K + lo * b->row_bytes;
     a.seg[n].V = b->V + lo * b->row_bytes;
     a.seg[n].ld = g.capacity;

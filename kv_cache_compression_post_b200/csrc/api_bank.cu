@@ -11,6 +11,7 @@
 #include "attend.cuh"
 #include "bank.h"
 #include "forcing.cuh"
+#include "fp8.cuh"
 #include "gram.cuh"
 #include "small_kernels.cuh"
 
@@ -25,6 +26,9 @@ bool config_ok(const kvb_config* c) {
   if (c->layers < 1 || c->heads < 1 || c->heads > 64) return false;
   if (c->head_dim != 64 && c->head_dim != 128) return false;
   if (c->max_queries < 1) return false;
+  if (c->storage != KVB_STORE_NATIVE && c->storage != KVB_STORE_FP8_E4M3) return false;
+  // E4M3 storage: DensityKV banks of bf16 keys and values
+  if (c->storage == KVB_STORE_FP8_E4M3 && (c->method != KVB_DENSITYKV || c->dtype != KVB_BF16)) return false;
   if (c->method == KVB_DENSITYKV) {
     if (c->capacity < 1 || c->max_candidates < 1) return false;
     if (!(c->eps > 0.f) || !std::isfinite(c->eps) || !(c->s >= 0.f) || !std::isfinite(c->s)) return false;
@@ -61,8 +65,17 @@ size_t kvb_bank::layout(void* base) {
     ldN = static_cast<int>(N);
     ldEA = static_cast<int>(M + N);
     ldPart = static_cast<int>(M > N ? M : N);
-    K = c.take<char>(L * H * M * d * elem);
-    V = c.take<char>(L * H * M * d * elem);
+    if (g.storage == KVB_STORE_FP8_E4M3) {
+      // one layer's bf16 working copy, every layer's E4M3 codes, the rounded candidates
+      K = c.take<char>(H * M * d * elem);
+      V = c.take<char>(H * M * d * elem);
+      K8 = c.take<uint8_t>(L * H * M * d);
+      V8 = c.take<uint8_t>(L * H * M * d);
+      candQ = c.take<char>(2 * H * N * d * elem);
+    } else {
+      K = c.take<char>(L * H * M * d * elem);
+      V = c.take<char>(L * H * M * d * elem);
+    }
     ids = c.take<int>(L * H * M);
     rho = c.take<float>(L * H * M);
     rho0 = c.take<float>(L * H * M);
@@ -164,10 +177,17 @@ kvb_status kvb_bank_create(const kvb_config* cfg, void* workspace, size_t worksp
   if (cfg->method == KVB_DENSITYKV) {
     // rows past a bank's size are read by full attention tiles (and masked): keep
     // them finite by starting from zeros
-    const size_t kv = LH * cfg->capacity * static_cast<size_t>(b->row_bytes);
+    const bool fp8 = cfg->storage == KVB_STORE_FP8_E4M3;
+    const size_t kv = (fp8 ? static_cast<size_t>(cfg->heads) : LH) * cfg->capacity * static_cast<size_t>(b->row_bytes);
     if (e == cudaSuccess) e = cudaMemsetAsync(b->size, 0, LH * sizeof(int), st);
     if (e == cudaSuccess) e = cudaMemsetAsync(b->K, 0, kv, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(b->V, 0, kv, st);
+    if (fp8) {
+      const size_t codes = LH * cfg->capacity * static_cast<size_t>(cfg->head_dim);
+      if (e == cudaSuccess) e = cudaMemsetAsync(b->K8, 0, codes, st);
+      if (e == cudaSuccess) e = cudaMemsetAsync(b->V8, 0, codes, st);
+      b->work_layer = -1;
+    }
   } else if (e == cudaSuccess) {
     const kvb_status fs = kvb_forcing_init(b, st);
     if (fs != KVB_OK) {
@@ -191,7 +211,50 @@ kvb_status kvb_bank_destroy(kvb_bank* bank) {
 
 }  // extern "C"
 
+// E4M3 storage: make the bf16 working copy hold `layer` (decompressing its codes
+// if it holds another layer or none).  Nothing to do for native storage.
+cudaError_t kvb_work_layer(kvb_bank* b, int layer, cudaStream_t st) {
+  if (b->cfg.method != KVB_DENSITYKV || b->cfg.storage != KVB_STORE_FP8_E4M3 || b->work_layer == layer)
+    return cudaSuccess;
+  const size_t n = static_cast<size_t>(b->cfg.heads) * b->cfg.capacity * b->cfg.head_dim;
+  b->work_layer = -1;
+  cudaError_t e = launch_dequant(b->K8 + static_cast<size_t>(layer) * n, b->K, n, st);
+  if (e == cudaSuccess) e = launch_dequant(b->V8 + static_cast<size_t>(layer) * n, b->V, n, st);
+  if (e == cudaSuccess) b->work_layer = layer;
+  return e;
+}
+
 namespace {
+
+// E4M3 storage: write the working copy's rows [0, size) back into `layer`'s codes
+// (its values are E4M3 values already, so the rounding is exact).
+cudaError_t store_work_layer(kvb_bank* b, int layer, cudaStream_t st) {
+  if (b->cfg.storage != KVB_STORE_FP8_E4M3) return cudaSuccess;
+  const kvb_config& g = b->cfg;
+  const size_t n = static_cast<size_t>(g.heads) * g.capacity * g.head_dim;
+  const int* size = b->size + static_cast<size_t>(layer) * g.heads;
+  cudaError_t e = launch_quant_rows(b->K, b->K8 + static_cast<size_t>(layer) * n, g.heads, g.capacity, g.head_dim, size, st);
+  if (e == cudaSuccess)
+    e = launch_quant_rows(b->V, b->V8 + static_cast<size_t>(layer) * n, g.heads, g.capacity, g.head_dim, size, st);
+  return e;
+}
+
+// E4M3 storage: the step's candidates rounded to E4M3 (once per step, `round`)
+// replace the caller's in the plan.
+cudaError_t use_rounded_candidates(kvb_bank* b, AdmitPlan& p, bool round, cudaStream_t st) {
+  if (b->cfg.storage != KVB_STORE_FP8_E4M3) return cudaSuccess;
+  const size_t n = static_cast<size_t>(p.H) * p.N * p.d;
+  char* qK = b->candQ;
+  char* qV = b->candQ + static_cast<size_t>(p.H) * b->cfg.max_candidates * p.d * b->elem;
+  cudaError_t e = cudaSuccess;
+  if (round) {
+    e = launch_round_e4m3(p.candK, qK, n, st);
+    if (e == cudaSuccess) e = launch_round_e4m3(p.candV, qV, n, st);
+  }
+  p.candK = qK;
+  p.candV = qV;
+  return e;
+}
 
 // One density pass: out[h][r] = sum over the column set of sign * phi, through the
 // tcgen05 kernel (bf16) or the CUDA-core kernel (f32).
@@ -258,6 +321,10 @@ kvb_status admit_plan(kvb_bank* b, int32_t layer, const void* candK, const void*
   if (g.method != KVB_DENSITYKV) return KVB_E_STATE;
   if (layer < 0 || layer >= g.layers || N < 1 || N > g.max_candidates) return KVB_E_INVAL;
   if (!candK || !candV || !cand_ids) return KVB_E_INVAL;
+  // the rounding kernels move 16-byte words
+  if (g.storage == KVB_STORE_FP8_E4M3 &&
+      ((reinterpret_cast<uintptr_t>(candK) | reinterpret_cast<uintptr_t>(candV)) & 15) != 0)
+    return KVB_E_INVAL;
   const int H = g.heads, M = g.capacity, d = g.head_dim;
   const size_t lo = static_cast<size_t>(layer) * H * M;  // slot offset of this layer
 
@@ -274,8 +341,10 @@ kvb_status admit_plan(kvb_bank* b, int32_t layer, const void* candK, const void*
   p.cand_order = g.cand_order;
   p.baselines = g.baselines;
   p.evict_order = g.evict_order;
-  p.K = b->K + lo * b->row_bytes;
-  p.V = b->V + lo * b->row_bytes;
+  // E4M3 storage: the kernels work on the bf16 working copy of the layer
+  const size_t klo = g.storage == KVB_STORE_FP8_E4M3 ? 0 : lo;
+  p.K = b->K + klo * b->row_bytes;
+  p.V = b->V + klo * b->row_bytes;
   p.ids = b->ids + lo;
   p.rho = b->rho + lo;
   p.rho0 = b->rho0 + lo;
@@ -383,8 +452,11 @@ extern "C" kvb_status kvb_admit(kvb_bank* b, int32_t layer, const void* candK, c
   if (!current_device(&dev)) return KVB_E_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   b->pending.layer = -1;  // the scratch of a begun step is overwritten
-  cudaError_t e = admit_phase1(b, p, dev, st);
+  cudaError_t e = kvb_work_layer(b, layer, st);
+  if (e == cudaSuccess) e = use_rounded_candidates(b, p, true, st);
+  if (e == cudaSuccess) e = admit_phase1(b, p, dev, st);
   if (e == cudaSuccess) e = admit_phase2(b, p, dev, st);
+  if (e == cudaSuccess) e = store_work_layer(b, layer, st);
   return cuda_status(e);
 }
 
@@ -398,7 +470,9 @@ extern "C" kvb_status kvb_admit_begin(kvb_bank* b, int32_t layer, const void* ca
   if (!current_device(&dev)) return KVB_E_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   b->pending.layer = -1;
-  cudaError_t e = admit_phase1(b, p, dev, st);
+  cudaError_t e = kvb_work_layer(b, layer, st);
+  if (e == cudaSuccess) e = use_rounded_candidates(b, p, true, st);
+  if (e == cudaSuccess) e = admit_phase1(b, p, dev, st);
   if (e == cudaSuccess) e = launch_feasible_min(p, prefix_out, st);
   if (e != cudaSuccess) return cuda_status(e);
   b->pending.layer = layer;
@@ -421,7 +495,11 @@ extern "C" kvb_status kvb_admit_finish(kvb_bank* b, int32_t layer, const int32_t
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   p.p_bound = prefix_bound;
   b->pending.layer = -1;
-  return cuda_status(admit_phase2(b, p, dev, st));
+  // the working copy and the rounded candidates of the begun step are still in place
+  cudaError_t e = use_rounded_candidates(b, p, false, st);
+  if (e == cudaSuccess) e = admit_phase2(b, p, dev, st);
+  if (e == cudaSuccess) e = store_work_layer(b, layer, st);
+  return cuda_status(e);
 }
 
 extern "C" {
@@ -458,6 +536,10 @@ kvb_status kvb_bank_export(kvb_bank* b, int32_t layer, int32_t head, int32_t* id
   if (b->cfg.method == KVB_FORCINGKV) return kvb_forcing_export(b, layer, head, ids, K, V, size, st);
   const int M = b->cfg.capacity;
   const size_t slot0 = (static_cast<size_t>(layer) * b->cfg.heads + head) * M;
+  // K/V rows: the layer's own (native storage) or the working copy, made to hold it (E4M3)
+  const bool fp8 = b->cfg.storage == KVB_STORE_FP8_E4M3;
+  const size_t kslot0 = fp8 ? static_cast<size_t>(head) * M : slot0;
+  if (fp8 && kvb_work_layer(b, layer, st) != cudaSuccess) return KVB_E_CUDA;
   int n = 0;
   cudaError_t e = cudaMemcpyAsync(&n, b->size + static_cast<size_t>(layer) * b->cfg.heads + head, sizeof(int),
                                   cudaMemcpyDeviceToHost, st);
@@ -473,10 +555,10 @@ kvb_status kvb_bank_export(kvb_bank* b, int32_t layer, int32_t head, int32_t* id
   if (rho0 && e == cudaSuccess)
     e = cudaMemcpyAsync(rho0, b->rho0 + slot0, sizeof(float) * n, cudaMemcpyDeviceToDevice, st);
   if (K && e == cudaSuccess)
-    e = cudaMemcpyAsync(K, b->K + slot0 * b->row_bytes, static_cast<size_t>(n) * b->row_bytes,
+    e = cudaMemcpyAsync(K, b->K + kslot0 * b->row_bytes, static_cast<size_t>(n) * b->row_bytes,
                         cudaMemcpyDeviceToDevice, st);
   if (V && e == cudaSuccess)
-    e = cudaMemcpyAsync(V, b->V + slot0 * b->row_bytes, static_cast<size_t>(n) * b->row_bytes,
+    e = cudaMemcpyAsync(V, b->V + kslot0 * b->row_bytes, static_cast<size_t>(n) * b->row_bytes,
                         cudaMemcpyDeviceToDevice, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   return cuda_status(e);
@@ -492,20 +574,29 @@ kvb_status kvb_bank_import(kvb_bank* b, int32_t layer, int32_t head, const int32
   if (size > 0 && (!ids || !rho || !rho0 || !K || !V)) return KVB_E_INVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t slot0 = (static_cast<size_t>(layer) * b->cfg.heads + head) * M;
-  cudaError_t e = cudaSuccess;
-  if (size > 0) {
+  // E4M3 storage: K/V go into the working copy of the layer, rounded to E4M3, and
+  // from there into the layer's codes
+  const bool fp8 = b->cfg.storage == KVB_STORE_FP8_E4M3;
+  const size_t kslot0 = fp8 ? static_cast<size_t>(head) * M : slot0;
+  if (fp8 && size > 0 && ((reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(V)) & 15) != 0)
+    return KVB_E_INVAL;
+  cudaError_t e = fp8 ? kvb_work_layer(b, layer, st) : cudaSuccess;
+  if (size > 0 && e == cudaSuccess) {
     e = cudaMemcpyAsync(b->ids + slot0, ids, sizeof(int) * size, cudaMemcpyDeviceToDevice, st);
     if (e == cudaSuccess) e = cudaMemcpyAsync(b->rho + slot0, rho, sizeof(float) * size, cudaMemcpyDeviceToDevice, st);
     if (e == cudaSuccess)
       e = cudaMemcpyAsync(b->rho0 + slot0, rho0, sizeof(float) * size, cudaMemcpyDeviceToDevice, st);
+    const size_t elems = static_cast<size_t>(size) * b->cfg.head_dim;
     if (e == cudaSuccess)
-      e = cudaMemcpyAsync(b->K + slot0 * b->row_bytes, K, static_cast<size_t>(size) * b->row_bytes,
-                          cudaMemcpyDeviceToDevice, st);
+      e = fp8 ? launch_round_e4m3(K, b->K + kslot0 * b->row_bytes, elems, st)
+              : cudaMemcpyAsync(b->K + kslot0 * b->row_bytes, K, static_cast<size_t>(size) * b->row_bytes,
+                                cudaMemcpyDeviceToDevice, st);
     if (e == cudaSuccess)
-      e = cudaMemcpyAsync(b->V + slot0 * b->row_bytes, V, static_cast<size_t>(size) * b->row_bytes,
-                          cudaMemcpyDeviceToDevice, st);
+      e = fp8 ? launch_round_e4m3(V, b->V + kslot0 * b->row_bytes, elems, st)
+              : cudaMemcpyAsync(b->V + kslot0 * b->row_bytes, V, static_cast<size_t>(size) * b->row_bytes,
+                                cudaMemcpyDeviceToDevice, st);
     if (e == cudaSuccess && b->cfg.dtype == KVB_BF16)
-      e = launch_aug_rows(b->K + slot0 * b->row_bytes, b->cfg.dtype, 1, size, b->cfg.head_dim, size, nullptr, size,
+      e = launch_aug_rows(b->K + kslot0 * b->row_bytes, b->cfg.dtype, 1, size, b->cfg.head_dim, size, nullptr, size,
                           b->aug + slot0 * 32, size, reinterpret_cast<float*>(b->status + 1),
                           -0.5f * b->cfg.eps * b->h, st);
   }
@@ -514,6 +605,7 @@ kvb_status kvb_bank_import(kvb_bank* b, int32_t layer, int32_t head, const int32
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(b->size + static_cast<size_t>(layer) * b->cfg.heads + head, &host_size, sizeof(int),
                         cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess && fp8) e = store_work_layer(b, layer, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   return cuda_status(e);
 }

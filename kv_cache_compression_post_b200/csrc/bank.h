@@ -25,8 +25,12 @@ struct kvb_bank {
   unsigned int attn_epoch = 0;  // launches so far (the kernel's epoch tag, never 0)
 
   // ---- DensityKV, per layer: base pointers of layer 0 and strides
-  char* K = nullptr;        // [L][H][M][d]
+  char* K = nullptr;        // [L][H][M][d]; E4M3 storage: the bf16 working copy of one layer, [H][M][d]
   char* V = nullptr;
+  uint8_t* K8 = nullptr;    // E4M3 storage: [L][H][M][d] codes (null otherwise)
+  uint8_t* V8 = nullptr;
+  char* candQ = nullptr;    // E4M3 storage: the step's candidates rounded to E4M3, [2][H][Nmax][d] bf16 (K, V)
+  int work_layer = -1;      // E4M3 storage: the layer the working copy holds (-1: none)
   int* ids = nullptr;       // [L][H][M]
   float* rho = nullptr;
   float* rho0 = nullptr;
@@ -92,3 +96,6 @@ struct kvb_bank {
 
   size_t layout(void* base);  // carve (base may be null to measure); returns bytes
 };
+
+// E4M3 storage: make the bank's bf16 working copy hold `layer` (api_bank.cu).
+cudaError_t kvb_work_layer(kvb_bank* b, int layer, cudaStream_t st);

@@ -18,6 +18,7 @@ __all__ = [
     "KVB_ORDER_DISTURBANCE", "KVB_ORDER_SOURCE", "KVB_BASELINES_FIXED", "KVB_BASELINES_REFRESH",
     "KVB_EVICT_THRESHOLD_RATIO", "KVB_EVICT_DENSEST", "KVB_EVICT_THRESHOLD_SOURCE",
     "KVB_BOTTOMK_FRAME", "KVB_BOTTOMK_CALL", "KVB_SIM_PER_LAYER", "KVB_SIM_FIRST_LAYER",
+    "KVB_STORE_NATIVE", "KVB_STORE_FP8_E4M3",
     "kvb_workspace_size", "kvb_bank_create", "kvb_bank_destroy", "kvb_admit", "kvb_prune_hybrid",
     "kvb_attend", "kvb_read_stats", "kvb_bank_export", "kvb_bank_import", "kvb_device_status",
     "kvb_status_string", "kvb_launch_count", "kvb_trace_enable", "kvb_trace_read", "kvb_density_workspace_size", "kvb_density", "kvb_density_noalloc", "kvb_segment_cosine",
@@ -33,6 +34,7 @@ KVB_BASELINES_FIXED, KVB_BASELINES_REFRESH = 0, 1
 KVB_EVICT_THRESHOLD_RATIO, KVB_EVICT_DENSEST, KVB_EVICT_THRESHOLD_SOURCE = 0, 1, 2
 KVB_BOTTOMK_FRAME, KVB_BOTTOMK_CALL = 0, 1
 KVB_SIM_PER_LAYER, KVB_SIM_FIRST_LAYER = 0, 1
+KVB_STORE_NATIVE, KVB_STORE_FP8_E4M3 = 0, 1
 
 # The Soft-Riesz parameters the DensityKV pages select (§4 parameter sensitivity,
 # App. E parameter sweeps: width sigma = 8, decay p = 2, regulariser eps fixed
@@ -61,7 +63,7 @@ class kvb_config(ctypes.Structure):
         ("seg_w", ctypes.c_int32), ("hist_frames", ctypes.c_int32), ("max_new_frames", ctypes.c_int32),
         ("retention", ctypes.c_float), ("max_queries", ctypes.c_int32),
         ("cand_order", ctypes.c_int32), ("baselines", ctypes.c_int32), ("evict_order", ctypes.c_int32),
-        ("bottomk_scope", ctypes.c_int32), ("sim_source", ctypes.c_int32),
+        ("bottomk_scope", ctypes.c_int32), ("sim_source", ctypes.c_int32), ("storage", ctypes.c_int32),
     ]
 
 
@@ -79,7 +81,7 @@ def make_config(**kw) -> kvb_config:
                     frame_h=0, frame_w=0, seg_h=4, seg_w=4, hist_frames=21, max_new_frames=3,
                     retention=0.7, max_queries=4680, cand_order=KVB_ORDER_DISTURBANCE,
                     baselines=KVB_BASELINES_FIXED, evict_order=KVB_EVICT_THRESHOLD_RATIO,
-                    bottomk_scope=KVB_BOTTOMK_FRAME, sim_source=KVB_SIM_PER_LAYER)
+                    bottomk_scope=KVB_BOTTOMK_FRAME, sim_source=KVB_SIM_PER_LAYER, storage=KVB_STORE_NATIVE)
     defaults.update(kw)
     for k, v in defaults.items():
         setattr(c, k, v)

@@ -36,6 +36,7 @@ int main(void) {
   FIELD(kvb_config, evict_order);
   FIELD(kvb_config, bottomk_scope);
   FIELD(kvb_config, sim_source);
+  FIELD(kvb_config, storage);
   printf("sizeof.kvb_admit_stats %zu\n", sizeof(kvb_admit_stats));
   FIELD(kvb_admit_stats, admitted);
   FIELD(kvb_admit_stats, feasible);

@@ -133,7 +133,7 @@ def import_step_state(bank, banks, params, w, layer=0):
     import_oracle_banks(bank, banks, params, w, layer=layer)
 
 
-def check_admit_step(bank, w, p, banks_pre, x, r, layer=0, m=1e-4, rtol=1e-4, label=""):
+def check_admit_step(bank, w, p, banks_pre, x, r, layer=0, m=1e-4, rtol=1e-4, label="", tagged=True):
     """One GPU admit step against the oracle's step r on the same inputs and the
     same starting banks (banks_pre, imported into the GPU bank before the step).
 
@@ -143,7 +143,8 @@ def check_admit_step(bank, w, p, banks_pre, x, r, layer=0, m=1e-4, rtol=1e-4, la
       unless every differing decision is a near tie, a shared P moved by a near-tie
       feasibility included).
     * Against that oracle step or replay, every head's bank must match: id set,
-      K rows bit for bit, V paired with its id, rho and rho0 within rtol; and the
+      K and V rows bit for bit (by id), V carrying its own id when the inputs are
+      tagged, rho and rho0 within rtol; and the
       counters: admitted, size, evictions, feasible and mandatory within the
       ranges the margin allows.
     * At most 2 flips per oracle near-tie decision plus 3 per head and unit of P
@@ -183,9 +184,11 @@ def check_admit_step(bank, w, p, banks_pre, x, r, layer=0, m=1e-4, rtol=1e-4, la
     for hh in range(H):
         gb, ob = g[hh], ref.banks[hh]
         assert set(gb["ids"].tolist()) == set(ob.ids.tolist()), f"{label} head {hh}: bank ids"
-        np.testing.assert_array_equal(kvgen.untag_ids(gb["V"]), gb["ids"])
+        if tagged:
+            np.testing.assert_array_equal(kvgen.untag_ids(gb["V"]), gb["ids"])
         go, oo = np.argsort(gb["ids"]), np.argsort(ob.ids)
         np.testing.assert_array_equal(gb["K"][go], ob.K[oo].astype(np.float32))
+        np.testing.assert_array_equal(gb["V"][go], ob.V[oo].astype(np.float32))
         np.testing.assert_allclose(gb["rho"][go], ref.rho_new[hh][oo], rtol=rtol, err_msg=f"{label} head {hh} rho")
         np.testing.assert_allclose(gb["rho0"][go], ob.rho0[oo], rtol=rtol, err_msg=f"{label} head {hh} rho0")
         s = st[hh]

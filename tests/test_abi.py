@@ -77,6 +77,16 @@ def test_config_validation_and_workspace_sizes():
            dict(cand_order=2), dict(cand_order=-1), dict(baselines=2), dict(evict_order=3), dict(evict_order=-1)]
     for kw in bad:
         assert kvb.kvb_workspace_size(kvb.make_config(**kw)) == 0, kw
+    # E4M3 storage: DensityKV banks of bf16 only; it halves the per-layer K/V storage
+    for kw in [dict(storage=2), dict(storage=-1), dict(storage=kvb.KVB_STORE_FP8_E4M3, dtype=kvb.KVB_F32)]:
+        assert kvb.kvb_workspace_size(kvb.make_config(**kw)) == 0, kw
+    assert kvb.kvb_workspace_size(kvb.make_config(method=kvb.KVB_FORCINGKV, frame_h=30, frame_w=52,
+                                                  storage=kvb.KVB_STORE_FP8_E4M3)) == 0
+    L, H, M, N, d = 30, 12, 9360, 4680, 128
+    native = kvb.kvb_workspace_size(kvb.make_config(layers=L))
+    fp8 = kvb.kvb_workspace_size(kvb.make_config(layers=L, storage=kvb.KVB_STORE_FP8_E4M3))
+    # per layer 2*H*M*d bytes less, plus one bf16 working layer and the rounded candidates
+    assert abs((native - fp8) - (2 * L * H * M * d - 4 * H * M * d - 4 * H * N * d)) <= 4096
     # the ablation switches change no buffer
     for kw in [dict(cand_order=kvb.KVB_ORDER_SOURCE), dict(baselines=kvb.KVB_BASELINES_REFRESH),
                dict(evict_order=kvb.KVB_EVICT_DENSEST), dict(evict_order=kvb.KVB_EVICT_THRESHOLD_SOURCE)]:
