@@ -204,8 +204,6 @@ def _cfg(w, kvb):
 # ncu captures summarised under profiles/, by (workload, kernel); valid only for
 # the kernel versions those files name.
 DRAM_TRAFFIC = {
-    # the four density passes of one 480P admit: 54.12 + 54.13 + 54.71 + 18.16 MB
-    ("wan480", "gram_bf16_kernel"): (181.12e6 / 4, "profiles/gram_bf16_kernel_wan480.md"),
 }
 
 # bank K/V storage of the DensityKV workloads (--storage)
