@@ -436,7 +436,13 @@ def run_workload(args, w, rank, world):
     up, down = torch.cuda.Stream(), torch.cuda.Stream()
     keys = sorted(hosted)
     proto = hosted[keys[0]]
-    bufs = [{k: torch.empty_like(v, device="cuda") for k, v in proto.items()} for _ in range(2)]
+    # the sink frame (frame 0) is the same for every step: it is uploaded once, before
+    # the timed region, and stays resident like the bank; every other input of a
+    # step is copied in during it
+    resident = ("sinkK", "sinkV")
+    sink = {k: proto[k].to("cuda") for k in resident if k in proto}
+    bufs = [{k: (sink[k] if k in sink else torch.empty_like(v, device="cuda")) for k, v in proto.items()}
+            for _ in range(2)]
     outs = [O, torch.empty_like(O)]
     Oh = [torch.empty(O.shape, dtype=O.dtype).pin_memory() for _ in range(2)]
     ev_in = [torch.cuda.Event() for _ in range(2)]
@@ -447,6 +453,8 @@ def run_workload(args, w, rank, world):
     def upload(j, b):
         nonlocal h2d
         for k, v in hosted[keys[j]].items():
+            if k in sink:
+                continue
             if bufs[b][k].shape != v.shape:
                 raise RuntimeError("end-to-end inputs change shape between steps")
             bufs[b][k].copy_(v, non_blocking=True)
@@ -909,7 +917,11 @@ def run_kvb(args, w, rank, world, local):
         else "f32", "data": "synthetic",
         "config": workload_config(w, args, world),
         "e2e": {"value": round(r["e2e_ms"], 4), "unit": UNIT, "h2d_bytes_per_step": r["h2d"],
-                "d2h_bytes_per_step": r["d2h"]},
+                "d2h_bytes_per_step": r["d2h"],
+                "what": "kvb_admit / kvb_prune_hybrid + kvb_attend with each step's inputs (candidates or new "
+                        "frames, queries, window) copied in from pinned host memory and the output copied out, "
+                        "inside the timed region, overlapped with the compute on two copy streams; the sink "
+                        "frame, the same every step, is resident like the bank"},
         "gpu_launches": r["launches"],
         "roofline": r["roofline"],
         "roofline_other": r["roofline_other"],
