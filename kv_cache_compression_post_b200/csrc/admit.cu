@@ -36,8 +36,8 @@ namespace kvb {
 namespace {
 
 constexpr int kSelThreads = 1024;
-// banks up to this many bytes of 64-bit keys keep them in shared memory
-constexpr size_t kEvictKeyBytes = 200 * 1024;
+// banks whose 64-bit keys and flag bytes fit in this many bytes keep them in shared memory
+constexpr size_t kEvictKeyBytes = 216 * 1024;
 
 struct SelShared {
   unsigned int hist[256];
@@ -394,15 +394,53 @@ __global__ void gather_admitted_kernel(const AdmitPlan p) {
   }
 }
 
+// Exclusive scan of three counts packed in one 64-bit word (21 bits each: counts
+// below 2^21) over the block; returns this thread's offsets, *total the totals.
+__device__ __forceinline__ unsigned long long block_excl_scan3(unsigned long long v, SelShared* S,
+                                                               unsigned long long* total) {
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  unsigned long long incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (l >= o) incl += t;
+  }
+  __syncthreads();
+  if (l == 31) S->kmin[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    const int nw = blockDim.x >> 5;
+    const unsigned long long x = (l < nw) ? S->kmin[l] : 0ull;
+    unsigned long long xi = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long t = __shfl_up_sync(0xffffffffu, xi, o);
+      if (l >= o) xi += t;
+    }
+    if (l < nw) S->kmin[l] = xi - x;   // exclusive warp offsets
+    if (l == nw - 1) S->kmax[0] = xi;  // totals
+  }
+  __syncthreads();
+  const unsigned long long res = S->kmin[w] + incl - v;
+  *total = S->kmax[0];
+  __syncthreads();
+  return res;
+}
+
 // SKEYS: every entry's 64-bit key is computed once into shared memory (the radix
-// passes then read 8 bytes of shared memory instead of recomputing the ratio);
-// mandatory evictions get the largest key, so the selection needs no flags.
+// passes then read 8 bytes of shared memory instead of recomputing the ratio), and
+// its eviction flag (0 survivor, 1 above tau, 2 capacity) sits beside it, so the
+// lists built at the end (evicted slots, holes, tail survivors) come from one pass
+// over shared memory; mandatory evictions get the largest key, so the selection
+// needs no flags.  Without SKEYS (banks too large for shared memory) keys are
+// recomputed and flags live in global memory.
 template <bool SKEYS>
 __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPlan p) {
   pdl_wait();
   pdl_trigger();
   __shared__ SelShared S;
-  extern __shared__ unsigned long long s_key[];  // [n] (SKEYS)
+  extern __shared__ unsigned long long s_key[];  // [M] keys, then [M] flag bytes (SKEYS)
+  uint8_t* s_flag = reinterpret_cast<uint8_t*>(s_key + p.M);
   const int h = blockIdx.x;
   const int n = p.n_old[h];
   const int Ph = p.P[h];
@@ -411,7 +449,12 @@ __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPl
   const float* rho0 = p.rho0 + base;
   const float* proj = p.proj + base;
   const int* ids = p.ids + base;
-  int* evflag = p.tail + base;  // per-slot flags live in the tail array until the tail list is built
+  int* evflag = p.tail + base;  // global flags (no SKEYS) live in the tail array until the tail list is built
+  auto getf = [&](int i) -> int { return SKEYS ? static_cast<int>(s_flag[i]) : evflag[i]; };
+  auto setf = [&](int i, int v) {
+    if (SKEYS) s_flag[i] = static_cast<uint8_t>(v);
+    else evflag[i] = v;
+  };
   auto ratio = [&](int i) { return ratio_of(rho[i], proj[i], rho0[i]); };
   const int mode = p.evict_order;
   // the capacity-cut key of a non-mandatory entry (ascending = evicted first):
@@ -430,7 +473,7 @@ __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPl
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     const float r = ratio(i);
     const bool m = mode != KVB_EVICT_DENSEST && r > p.tau;
-    evflag[i] = m ? 1 : 0;
+    setf(i, m ? 1 : 0);
     cnt += m ? 1 : 0;
     nt += (mode != KVB_EVICT_DENSEST && near_tau(r, p.tau)) ? 1 : 0;
     if (SKEYS) s_key[i] = m ? ~0ull : cut_key(i, r);
@@ -447,12 +490,12 @@ __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPl
     };
     auto keep = [&](int i) { return SKEYS || evflag[i] == 0; };
     if (ecap >= n_free) {
-      for (int i = threadIdx.x; i < n; i += blockDim.x) evflag[i] = 1;
+      for (int i = threadIdx.x; i < n; i += blockDim.x) setf(i, 1);
     } else {
       block_radix_select(n, ecap, key, keep, &S);
       const unsigned long long prefix = S.prefix, mask = S.mask;
       for (int i = threadIdx.x; i < n; i += blockDim.x)
-        if (evflag[i] == 0 && (key(i) & mask) <= prefix) evflag[i] = 2;
+        if (getf(i) == 0 && (key(i) & mask) <= prefix) setf(i, 2);
     }
   }
   __syncthreads();
@@ -462,7 +505,7 @@ __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPl
     if (ecap > 0 && ecap < n_free && mode != KVB_EVICT_THRESHOLD_SOURCE) {
       float lo = -INFINITY, hi = -INFINITY;  // lo holds -min over the evicted
       for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const int f = evflag[i];
+        const int f = getf(i);
         if (f == 1) continue;
         // the cut value: read back from the key when the keys are in shared memory
         const float v = SKEYS ? key_float(~static_cast<uint32_t>(s_key[i] >> 32))
@@ -479,28 +522,59 @@ __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPl
   const int E = n_mand + min(ecap, n_free);
   const int n_new = n - E + Ph;
   int* ev = p.ev_slot + base;
-  const int gotE = block_compact(0, n, [&](int i) { return evflag[i] != 0; }, ev, &S);
-  const int nh = block_compact(0, n, [&](int i) { return evflag[i] != 0 && i < n_new; }, nullptr, &S);
-  // survivors at or above the new size move into holes; list them (ascending)
-  __shared__ int s_ntail;
-  {
-    // count first (flags are still needed), then write the list over the flag array
-    const int nt = block_compact(n_new < n ? n_new : n, n, [&](int i) { return evflag[i] == 0; }, nullptr, &S);
-    if (threadIdx.x == 0) s_ntail = nt;
-  }
-  __syncthreads();
-  // the tail list is short; build it in the newp scratch and copy it over the flags
   int* tmp = p.newp + base;
-  block_compact(n_new < n ? n_new : n, n, [&](int i) { return evflag[i] == 0; }, tmp, &S);
-  for (int k = threadIdx.x; k < s_ntail; k += blockDim.x) evflag[k] = tmp[k];
-  __syncthreads();
+  __shared__ int s_ntail, s_gotE, s_nh;
+  if (SKEYS) {
+    // one ordered pass over contiguous chunks: the evicted slots (ascending), the
+    // number of them below the new size (holes), and the survivors at or above
+    // the new size (they move into holes), listed ascending into the tail array
+    const int chunk = (n + blockDim.x - 1) / blockDim.x;
+    const int b0 = threadIdx.x * chunk, b1 = min(n, b0 + chunk);
+    unsigned long long c3 = 0ull;
+    for (int i = b0; i < b1; ++i) {
+      const int f = s_flag[i];
+      c3 += (f != 0) ? 1ull : 0ull;
+      c3 += (f != 0 && i < n_new) ? (1ull << 21) : 0ull;
+      c3 += (f == 0 && i >= n_new) ? (1ull << 42) : 0ull;
+    }
+    unsigned long long tot;
+    const unsigned long long off = block_excl_scan3(c3, &S, &tot);
+    int pe = static_cast<int>(off & 0x1FFFFFull), pt = static_cast<int>((off >> 42) & 0x1FFFFFull);
+    for (int i = b0; i < b1; ++i) {
+      const int f = s_flag[i];
+      if (f != 0) ev[pe++] = i;
+      else if (i >= n_new) evflag[pt++] = i;
+    }
+    if (threadIdx.x == 0) {
+      s_gotE = static_cast<int>(tot & 0x1FFFFFull);
+      s_nh = static_cast<int>((tot >> 21) & 0x1FFFFFull);
+      s_ntail = static_cast<int>((tot >> 42) & 0x1FFFFFull);
+    }
+    __syncthreads();
+  } else {
+    const int gotE = block_compact(0, n, [&](int i) { return evflag[i] != 0; }, ev, &S);
+    const int nh = block_compact(0, n, [&](int i) { return evflag[i] != 0 && i < n_new; }, nullptr, &S);
+    // survivors at or above the new size move into holes; list them (ascending):
+    // count first (flags are still needed), then write the list over the flag array
+    const int ntl = block_compact(n_new < n ? n_new : n, n, [&](int i) { return evflag[i] == 0; }, nullptr, &S);
+    if (threadIdx.x == 0) {
+      s_ntail = ntl;
+      s_gotE = gotE;
+      s_nh = nh;
+    }
+    __syncthreads();
+    // the tail list is short; build it in the newp scratch and copy it over the flags
+    block_compact(n_new < n ? n_new : n, n, [&](int i) { return evflag[i] == 0; }, tmp, &S);
+    for (int k = threadIdx.x; k < s_ntail; k += blockDim.x) evflag[k] = tmp[k];
+    __syncthreads();
+  }
   // every slot of the new bank starts as an old, unmoved entry
   const int top = max(n, n_new);
   for (int i = threadIdx.x; i < top; i += blockDim.x) tmp[i] = -1;
   if (threadIdx.x == 0) {
-    if (gotE != E) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
+    if (s_gotE != E) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
     p.E[h] = E;
-    p.nhole[h] = nh;
+    p.nhole[h] = s_nh;
     p.ntail[h] = s_ntail;
     p.EAoff[h] = p.M - E;
     p.EAcnt[h] = E;
@@ -655,7 +729,8 @@ cudaError_t launch_gather_admitted(const AdmitPlan& p, int maxP, cudaStream_t st
   return launch_pdl(gather_admitted_kernel, dim3(mover_blocks(maxP, p.row_bytes, p.H), p.H), dim3(256), 0, st, p);
 }
 cudaError_t launch_evict_select(const AdmitPlan& p, cudaStream_t st) {
-  const size_t keys = sizeof(unsigned long long) * static_cast<size_t>(p.M);
+  // keys (8 bytes) and flags (1 byte) of every entry in shared memory
+  const size_t keys = (sizeof(unsigned long long) + 1) * static_cast<size_t>(p.M);
   if (keys <= kEvictKeyBytes) {
     cudaError_t e = cudaFuncSetAttribute(evict_select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(keys));

@@ -63,7 +63,7 @@ cudaError_t launch_gram_f32(const GramArgs& a, cudaStream_t st);
 // tile range covered the row's block (fixed order: deterministic).
 cudaError_t launch_gram_reduce(const GramArgs& a, float* out, int ldOut, cudaStream_t st);
 
-// Work of a launch is the sequence of (head, 256-row block, 128-column tile)
+// Work of a launch is the sequence of (head, 256-row block, 256-column tile)
 // steps, T in total (known only on the device).  Only G_eff = clamp(T / min_steps,
 // 1, grid) CTAs work; CTA b takes steps [T b / G_eff, T (b+1) / G_eff), so a row
 // block is covered by at most `slots` CTAs.  Fills grid/slots/min_steps.
