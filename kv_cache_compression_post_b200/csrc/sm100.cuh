@@ -177,6 +177,16 @@ __device__ __forceinline__ void tmem_wait_ld_reg16(uint32_t (&r)[16]) {
       :
       : "memory");
 }
+// an empty statement that marks r as written here: placed right after a
+// tcgen05.wait::ld, it keeps every use of r (the destination of an earlier
+// tcgen05.ld) after that wait (volatile statements keep their order)
+__device__ __forceinline__ void reg_fence16(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 32 lanes x 32 consecutive 32-bit columns: thread t of the warp gets lane (base+t),
