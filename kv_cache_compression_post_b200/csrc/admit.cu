@@ -39,8 +39,13 @@ constexpr int kSelThreads = 1024;
 // banks whose 64-bit keys and flag bytes fit in this many bytes keep them in shared memory
 constexpr size_t kEvictKeyBytes = 216 * 1024;
 
+// the radix histogram is split in kHistCopies copies (warp w counts into copy
+// w % kHistCopies): keys that share a digit then contend on an address only
+// within their group of warps
+constexpr int kHistCopies = 8;
+
 struct SelShared {
-  unsigned int hist[256];
+  unsigned int hist[kHistCopies][256];
   unsigned long long kmin[32], kmax[32];
   unsigned long long prefix, mask;
   int kRem;
@@ -155,8 +160,9 @@ __device__ int block_compact(int lo, int hi, Pred pred, int* out, SelShared* S) 
 // The bits every candidate key shares (the common prefix of the smallest and the
 // largest non-sentinel key) are skipped: at these sizes the keys of one call often
 // agree on their top byte (ratios in [1, 2), say), and a pass over it would send
-// every key to one histogram bin.  Histogram increments are aggregated per warp
-// (lanes with the same bin add once), so a crowded bin costs one atomic per warp.
+// every key to one histogram bin.  Each warp counts into one of kHistCopies
+// copies of the histogram, so a crowded bin is contended only within a group of
+// warps; the copies are summed when the digit is chosen.
 template <class KeyFn, class KeepFn>
 __device__ void block_radix_select(int n, int k, KeyFn key, KeepFn keep, SelShared* S) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -206,10 +212,9 @@ __device__ void block_radix_select(int n, int k, KeyFn key, KeepFn keep, SelShar
   if (S->done) return;
   const int shift0 = static_cast<int>(S->kmin[0]);
   for (int shift = shift0; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) S->hist[i] = 0u;
+    for (int i = threadIdx.x; i < kHistCopies * 256; i += blockDim.x) (&S->hist[0][0])[i] = 0u;
     __syncthreads();
     const unsigned long long prefix = S->prefix, mask = S->mask;
-    // warp-uniform trip count: every lane reaches the match
     for (int i0 = warp * 32; i0 < n; i0 += blockDim.x) {
       const int i = i0 + lane;
       unsigned int bin = 256u;
@@ -217,8 +222,9 @@ __device__ void block_radix_select(int n, int k, KeyFn key, KeepFn keep, SelShar
         const unsigned long long kk = key(i);
         if ((kk & mask) == prefix) bin = static_cast<unsigned int>((kk >> shift) & 0xFFull);
       }
-      const unsigned int peers = __match_any_sync(0xffffffffu, bin);
-      if (bin < 256u && lane == __ffs(peers) - 1) atomicAdd(&S->hist[bin], static_cast<unsigned int>(__popc(peers)));
+      // one shared-memory atomic per key: with the histogram copies this measured
+      // faster than aggregating equal digits per warp with __match_any_sync
+      if (bin < 256u) atomicAdd(&S->hist[warp % kHistCopies][bin], 1u);
     }
     __syncthreads();
     if (threadIdx.x < 32) {
@@ -226,7 +232,10 @@ __device__ void block_radix_select(int n, int k, KeyFn key, KeepFn keep, SelShar
       unsigned int s = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        loc[j] = S->hist[lane * 8 + j];
+        unsigned int b = 0u;
+#pragma unroll
+        for (int c = 0; c < kHistCopies; ++c) b += S->hist[c][lane * 8 + j];
+        loc[j] = b;
         s += loc[j];
       }
       unsigned int incl = s;
@@ -461,22 +470,42 @@ __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const AdmitPl
   // ratio descending (default), projected density descending (densest-only), or
   // nothing (source order); id ascending breaks ties.  Ratios and densities are
   // >= 0, so no such key has the top byte 0xFF of the mandatory entries' key.
-  auto cut_key = [&](int i, float r) -> unsigned long long {
+  auto cut_key_of = [&](float r, float dens, int id) -> unsigned long long {
     unsigned long long hi = 0ull;
     if (mode == KVB_EVICT_THRESHOLD_RATIO) hi = ~float_key(r);
-    else if (mode == KVB_EVICT_DENSEST) hi = ~float_key(rho[i] + proj[i]);
-    return (hi << 32) | static_cast<unsigned int>(ids[i]);
+    else if (mode == KVB_EVICT_DENSEST) hi = ~float_key(dens);
+    return (hi << 32) | static_cast<unsigned int>(id);
   };
+  auto cut_key = [&](int i, float r) { return cut_key_of(r, rho[i] + proj[i], ids[i]); };
   // mandatory evictions: projected growth above tau (none when densest-only);
-  // near ties at the threshold are counted on the way
+  // near ties at the threshold are counted on the way.  Each thread takes four
+  // entries per round and issues all their loads before using any (one memory
+  // latency per round instead of one per entry)
   int cnt = 0, nt = 0;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const float r = ratio(i);
-    const bool m = mode != KVB_EVICT_DENSEST && r > p.tau;
-    setf(i, m ? 1 : 0);
-    cnt += m ? 1 : 0;
-    nt += (mode != KVB_EVICT_DENSEST && near_tau(r, p.tau)) ? 1 : 0;
-    if (SKEYS) s_key[i] = m ? ~0ull : cut_key(i, r);
+  constexpr int kU = 4;
+  for (int i0 = threadIdx.x; i0 < n; i0 += kU * static_cast<int>(blockDim.x)) {
+    float rv[kU], pv[kU], r0v[kU];
+    int idv[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = i0 + u * static_cast<int>(blockDim.x);
+      const bool in = i < n;
+      rv[u] = in ? __ldg(rho + i) : 0.f;
+      pv[u] = in ? __ldg(proj + i) : 0.f;
+      r0v[u] = in ? __ldg(rho0 + i) : 0.f;
+      idv[u] = in ? __ldg(ids + i) : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = i0 + u * static_cast<int>(blockDim.x);
+      if (i >= n) break;
+      const float r = ratio_of(rv[u], pv[u], r0v[u]);
+      const bool m = mode != KVB_EVICT_DENSEST && r > p.tau;
+      setf(i, m ? 1 : 0);
+      cnt += m ? 1 : 0;
+      nt += (mode != KVB_EVICT_DENSEST && near_tau(r, p.tau)) ? 1 : 0;
+      if (SKEYS) s_key[i] = m ? ~0ull : cut_key_of(r, rv[u] + pv[u], idv[u]);
+    }
   }
   int n_mand, ties;
   block_excl_scan(cnt, &S, &n_mand);
