@@ -872,7 +872,7 @@ def workload_config(w, args, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="wan480")
     ap.add_argument("--impl", default="kvb", choices=["kvb", "reference"])
