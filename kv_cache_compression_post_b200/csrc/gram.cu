@@ -169,40 +169,40 @@ __device__ __forceinline__ float2 sum_recip16(const uint32_t (&v)[16], float dma
 // Sum of 1/D over a thread's 128 accumulator columns (8 chunks of 16, s = 2, no
 // masked pair), releasing the accumulator (one arrival per warp on acc_empty) as
 // soon as the last chunk is in registers.  tcgen05.wait::ld waits for every load
-// of the thread, so three 16-column buffers alternate between two loads in flight
-// over one chunk's arithmetic and one load in flight over two chunks'.
+// of the thread, so four 16-column buffers work in pairs: two loads in flight
+// over two chunks' arithmetic (a TMEM load takes ~200 clk while the other row
+// tile's MMAs run).
 template <bool CLAMP>
 __device__ __forceinline__ float2 drain_recip128(uint32_t taddr, float dmax, uint64_t* acc_empty, int lane) {
   float2 acc = make_float2(0.f, 0.f);
-  uint32_t va[16], vb[16], vc[16];
+  uint32_t va[16], vb[16], vc[16], vd[16];
   tmem_ld16(taddr + 0, va);
-  tmem_wait_ld_reg16(va);
   tmem_ld16(taddr + 16, vb);
+  tmem_wait_ld_reg16(va);
+  reg_fence16(vb);
   tmem_ld16(taddr + 32, vc);
-  acc = sum_recip16<CLAMP>(va, dmax, acc);  // chunk 0
-  tmem_wait_ld_reg16(vb);
-  reg_fence16(vc);
-  tmem_ld16(taddr + 48, va);
-  acc = sum_recip16<CLAMP>(vb, dmax, acc);  // 1
-  acc = sum_recip16<CLAMP>(vc, dmax, acc);  // 2
+  tmem_ld16(taddr + 48, vd);
+  acc = sum_recip16<CLAMP>(va, dmax, acc);
+  acc = sum_recip16<CLAMP>(vb, dmax, acc);
+  tmem_wait_ld_reg16(vc);
+  reg_fence16(vd);
+  tmem_ld16(taddr + 64, va);
+  tmem_ld16(taddr + 80, vb);
+  acc = sum_recip16<CLAMP>(vc, dmax, acc);
+  acc = sum_recip16<CLAMP>(vd, dmax, acc);
   tmem_wait_ld_reg16(va);
-  tmem_ld16(taddr + 64, vb);
-  tmem_ld16(taddr + 80, vc);
-  acc = sum_recip16<CLAMP>(va, dmax, acc);  // 3
-  tmem_wait_ld_reg16(vb);
-  reg_fence16(vc);
-  tmem_ld16(taddr + 96, va);
-  acc = sum_recip16<CLAMP>(vb, dmax, acc);  // 4
-  acc = sum_recip16<CLAMP>(vc, dmax, acc);  // 5
-  tmem_wait_ld_reg16(va);
-  tmem_ld16(taddr + 112, vb);
-  acc = sum_recip16<CLAMP>(va, dmax, acc);  // 6
-  tmem_wait_ld_reg16(vb);
-  // every column this warp needs is in registers: hand the accumulator back
+  reg_fence16(vb);
+  tmem_ld16(taddr + 96, vc);
+  tmem_ld16(taddr + 112, vd);
+  acc = sum_recip16<CLAMP>(va, dmax, acc);
+  acc = sum_recip16<CLAMP>(vb, dmax, acc);
+  tmem_wait_ld_reg16(vc);
+  reg_fence16(vd);
   tc_fence_before();
   __syncwarp();
   if (lane == 0) mbar_arrive(acc_empty);
-  return sum_recip16<CLAMP>(vb, dmax, acc);  // 7
+  acc = sum_recip16<CLAMP>(vc, dmax, acc);
+  return sum_recip16<CLAMP>(vd, dmax, acc);
 }
 
 template <int SMODE>
