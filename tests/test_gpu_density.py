@@ -64,6 +64,18 @@ def test_density_bf16_exponents_and_scale(s):
     np.testing.assert_allclose(got, _oracle(rows, cols, 64.0, 0.5, s, False), rtol=RTOL)
 
 
+def test_density_bf16_pages_preset():
+    """The pages' sigma / eps / p preset (h = sigma^2 = 64, eps = 1, s = p = 2)."""
+    import kv_cache_compression_post_b200 as kvb
+    pp = kvb.PAGES_PRESET
+    rows = _keys(2, 260, 128, 7)
+    cols = _keys(2, 390, 128, 8)
+    got = _run(rows, cols, "bf16", h=pp["dist_scale"], eps=pp["eps"], s=pp["s"])
+    np.testing.assert_allclose(got, _oracle(rows, cols, pp["dist_scale"], pp["eps"], pp["s"], False), rtol=RTOL)
+    got = _run(rows, rows, "bf16", h=pp["dist_scale"], eps=pp["eps"], s=pp["s"], diag=1)
+    np.testing.assert_allclose(got, _oracle(rows, rows, pp["dist_scale"], pp["eps"], pp["s"], True), rtol=RTOL)
+
+
 def test_density_bf16_exclude_diagonal():
     rows = _keys(4, 700, 128, 5)
     got = _run(rows, rows, "bf16", diag=1)

@@ -120,6 +120,17 @@ def test_mid_stepwise_matches_oracle(tau, sync):
     _stepwise(w, p, dict(tau=tau, sync=sync), f"mid tau {tau} sync {sync}")
 
 
+def test_mid_stepwise_pages_preset():
+    """The pages' sigma / eps / p preset (h = sigma^2 = 64, eps = 1, s = p = 2),
+    stepwise against the oracle on every step."""
+    import dataclasses
+    import kv_cache_compression_post_b200 as kvb
+    pp = kvb.PAGES_PRESET
+    w = dataclasses.replace(kvgen.WORKLOADS["mid"], eps=pp["eps"], s=pp["s"])
+    p = dkv.Params(capacity=w.capacity, tau=w.tau, eps=w.eps, s=w.s, h=pp["dist_scale"])
+    _stepwise(w, p, dict(dist_scale=pp["dist_scale"]), "mid pages preset")
+
+
 # App. E ablation switches: (tau, oracle Params fields).  tau 1.2 with source
 # candidate order gives feasible runs from 0 to N over the steps; the tau 2 cases
 # reach capacity evictions; tau 1 with refresh + densest changes admission too.
