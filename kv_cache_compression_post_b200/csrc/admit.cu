@@ -321,10 +321,18 @@ __global__ void __launch_bounds__(kSelThreads) admit_select_kernel(const AdmitPl
   pdl_wait();
   pdl_trigger();
   __shared__ SelShared S;
+  __shared__ int sPt;
   const int h = blockIdx.x;
-  int Pt = p.feasible[h];
-  if (p.sync_heads)
-    for (int g = 0; g < p.H; ++g) Pt = min(Pt, p.feasible[g]);
+  if (threadIdx.x < 32) {
+    // the shared prefix: one warp loads the heads' feasible counts side by side
+    int v = p.feasible[h];
+    if (p.sync_heads)
+      for (int g = threadIdx.x; g < p.H; g += 32) v = min(v, p.feasible[g]);
+    for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (threadIdx.x == 0) sPt = v;
+  }
+  __syncthreads();
+  int Pt = sPt;
   if (p.p_bound) Pt = min(Pt, max(0, *p.p_bound));
   const int P = min(Pt, min(p.M, p.N));
   const float mean0 = p.mean0[h];

@@ -57,28 +57,57 @@ static_assert(sizeof(GramBars) <= kBarBytes, "barrier block overflows its reserv
 __device__ __forceinline__ int set_n(const GramSet& s, int h) { return s.n_dev ? s.n_dev[h] : s.n_uni; }
 __device__ __forceinline__ int set_off(const GramSet& s, int h) { return s.off_dev ? s.off_dev[h] : s.off_uni; }
 
+// Per-head sizes of a launch, read once per CTA into shared memory: the counts
+// can live in device memory (bank sizes, admitted counts), and a walk over the
+// heads that loads them one after another costs a memory round trip per head.
+struct HeadDims {
+  int nR, nC, rOff, cOff;
+  int RB, CT;            // row blocks / column tiles
+  int nneg, diag;        // signed-column count, self-pair offset
+  long long L0;          // first step of the head; entry H holds the total
+};
+constexpr int kTabBytes = (kGramMaxHeads + 1) * static_cast<int>(sizeof(HeadDims));
+
+// Filled by one warp: each lane loads one head's sizes, a warp scan places the
+// heads' step ranges one after another.
+__device__ __forceinline__ void build_head_table(const GramArgs& a, HeadDims* tab, int lane) {
+  long long carry = 0;
+  for (int base = 0; base < a.H; base += 32) {
+    const int h = base + lane;
+    HeadDims t{};
+    long long n = 0;
+    if (h < a.H) {
+      t.nR = set_n(a.rows, h);
+      t.nC = set_n(a.cols, h);
+      t.rOff = set_off(a.rows, h);
+      t.cOff = set_off(a.cols, h);
+      t.RB = t.nC > 0 ? (t.nR + kGramRowBlock - 1) / kGramRowBlock : 0;
+      t.CT = t.nR > 0 ? (t.nC + kColTile - 1) / kColTile : 0;
+      t.nneg = a.nneg_dev ? a.nneg_dev[h] : a.nneg_uni;
+      t.diag = a.use_diag ? (a.diag_dev ? a.diag_dev[h] : a.diag_uni) : INT_MIN / 2;
+      n = static_cast<long long>(t.RB) * t.CT;
+    }
+    long long x = n;  // inclusive scan of the step counts over the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (h < a.H) {
+      t.L0 = carry + x - n;
+      tab[h] = t;
+    }
+    carry += __shfl_sync(0xffffffffu, x, 31);
+  }
+  if (lane == 0) tab[a.H].L0 = carry;
+}
+
 // Position in the (head, row block, column tile) step sequence.
 struct Cursor {
   int h, rb, j;          // current step
   int RB, CT;            // row blocks / column tiles of head h
   int nR, nC, rOff, cOff;
 };
-
-__device__ __forceinline__ void head_dims(const GramArgs& a, int h, int& RB, int& CT) {
-  const int nR = set_n(a.rows, h), nC = set_n(a.cols, h);
-  RB = nC > 0 ? (nR + kGramRowBlock - 1) / kGramRowBlock : 0;
-  CT = nR > 0 ? (nC + kColTile - 1) / kColTile : 0;
-}
-
-__device__ __forceinline__ long long total_steps(const GramArgs& a) {
-  long long T = 0;
-  for (int h = 0; h < a.H; ++h) {
-    int RB, CT;
-    head_dims(a, h, RB, CT);
-    T += static_cast<long long>(RB) * CT;
-  }
-  return T;
-}
 
 __device__ __forceinline__ int active_grid(const GramArgs& a, long long T) {
   long long g = T / a.min_steps;
@@ -87,28 +116,27 @@ __device__ __forceinline__ int active_grid(const GramArgs& a, long long T) {
   return static_cast<int>(g);
 }
 
-__device__ __forceinline__ void cursor_load_head(const GramArgs& a, Cursor& c) {
-  head_dims(a, c.h, c.RB, c.CT);
-  c.nR = set_n(a.rows, c.h);
-  c.nC = set_n(a.cols, c.h);
-  c.rOff = set_off(a.rows, c.h);
-  c.cOff = set_off(a.cols, c.h);
+__device__ __forceinline__ void cursor_load_head(const HeadDims* tab, Cursor& c) {
+  const HeadDims& t = tab[c.h];
+  c.RB = t.RB;
+  c.CT = t.CT;
+  c.nR = t.nR;
+  c.nC = t.nC;
+  c.rOff = t.rOff;
+  c.cOff = t.cOff;
 }
 
-// position the cursor at step L (0 <= L < T)
-__device__ __forceinline__ void cursor_seek(const GramArgs& a, long long L, Cursor& c) {
-  for (c.h = 0; c.h < a.H; ++c.h) {
-    head_dims(a, c.h, c.RB, c.CT);
-    const long long n = static_cast<long long>(c.RB) * c.CT;
-    if (L < n) break;
-    L -= n;
-  }
-  cursor_load_head(a, c);
+// position the cursor at step L (0 <= L < total)
+__device__ __forceinline__ void cursor_seek(const GramArgs& a, const HeadDims* tab, long long L, Cursor& c) {
+  c.h = 0;
+  while (c.h + 1 < a.H && L >= tab[c.h + 1].L0) ++c.h;
+  cursor_load_head(tab, c);
+  L -= tab[c.h].L0;
   c.rb = static_cast<int>(L / c.CT);
   c.j = static_cast<int>(L % c.CT);
 }
 
-__device__ __forceinline__ void cursor_next(const GramArgs& a, Cursor& c) {
+__device__ __forceinline__ void cursor_next(const GramArgs& a, const HeadDims* tab, Cursor& c) {
   if (++c.j < c.CT) return;
   c.j = 0;
   if (++c.rb < c.RB) return;
@@ -116,9 +144,8 @@ __device__ __forceinline__ void cursor_next(const GramArgs& a, Cursor& c) {
   do {
     ++c.h;
     if (c.h >= a.H) return;
-    head_dims(a, c.h, c.RB, c.CT);
-  } while (c.RB * c.CT == 0);
-  cursor_load_head(a, c);
+  } while (tab[c.h].RB * tab[c.h].CT == 0);
+  cursor_load_head(tab, c);
 }
 
 // the CTA (of G_eff) whose range contains step L
@@ -221,6 +248,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
   uint8_t* sAa = sB + kStages * bBytes;        // 2 augmented row tiles
   uint8_t* sBa = sAa + 2 * aAug;               // kStages augmented column tiles
   GramBars* bars = reinterpret_cast<GramBars*>(sBa + kStages * bAug);
+  HeadDims* tab = reinterpret_cast<HeadDims*>(reinterpret_cast<uint8_t*>(bars) + kBarBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -252,8 +280,10 @@ __global__ void __launch_bounds__(kGramThreads, 1)
   // previous kernel's results are read
   pdl_wait();
   pdl_trigger();
+  if (warp == 3) build_head_table(a, tab, lane);
+  __syncthreads();
 
-  const long long T = total_steps(a);
+  const long long T = tab[a.H].L0;
   const int G = active_grid(a, T);
   const int cta = blockIdx.x;
   const long long L0 = (cta < G) ? (T * cta) / G : 0;
@@ -269,8 +299,8 @@ __global__ void __launch_bounds__(kGramThreads, 1)
       int it = 0, aload = 0;
       bool ok = true;
       Cursor c;
-      if (L0 < L1) cursor_seek(a, L0, c);
-      for (long long L = L0; L < L1; ++L, cursor_next(a, c)) {
+      if (L0 < L1) cursor_seek(a, tab, L0, c);
+      for (long long L = L0; L < L1; ++L, cursor_next(a, tab, c)) {
         if (L == L0 || c.j == 0) {
           if (aload > 0 && !(ok = mbar_wait(&bars->a_empty, (aload - 1) & 1, abort, a.status))) break;
           const int nact = nact_of(c);
@@ -309,7 +339,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
       int tr[2] = {0, 0};  // tiles issued into each row tile's accumulator
       bool ok = true;
       Cursor c;
-      if (L0 < L1) cursor_seek(a, L0, c);
+      if (L0 < L1) cursor_seek(a, tab, L0, c);
       for (long long L = L0; L < L1 && ok; ++L) {
         const int nact = nact_of(c);
         if (L == L0 || c.j == 0) {
@@ -340,7 +370,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
         ++it;
         const bool last_of_block = (L + 1 == L1) || (c.j + 1 == c.CT);
         if (last_of_block) mma_commit(&bars->a_empty);
-        cursor_next(a, c);
+        cursor_next(a, tab, c);
       }
       if (!ok && (tr[0] + tr[1]) > 0) {
         // abort path: no MMA may still write TMEM when it is freed (the commit
@@ -364,7 +394,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
     int t = 0;                       // tiles seen by this row tile (phase of its barriers)
     bool ok = true;
     Cursor c;
-    if (L0 < L1) cursor_seek(a, L0, c);
+    if (L0 < L1) cursor_seek(a, tab, L0, c);
     float acc_pos = 0.f, acc_neg = 0.f;
     int row = 0, nneg = 0, diag = 0, rt0 = 0;
     bool active = false, valid_row = false;
@@ -376,8 +406,8 @@ __global__ void __launch_bounds__(kGramThreads, 1)
         row = rt0 + row_in_tile;
         active = r < nact_of(c);
         valid_row = active && row < c.nR;
-        nneg = a.nneg_dev ? a.nneg_dev[c.h] : a.nneg_uni;
-        diag = a.use_diag ? (a.diag_dev ? a.diag_dev[c.h] : a.diag_uni) : INT_MIN / 2;
+        nneg = tab[c.h].nneg;
+        diag = tab[c.h].diag;
         acc_pos = 0.f;
         acc_neg = 0.f;
       }
@@ -453,7 +483,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
         else
           latch_status(a.status, 5 /* KVB_E_DEVICE_BOUNDS */);
       }
-      cursor_next(a, c);
+      cursor_next(a, tab, c);
     }
   }
 
@@ -516,31 +546,33 @@ __global__ void __launch_bounds__(kF32Warps * 32) gram_f32_kernel(const GramArgs
   if (lane == 0 && row < nR) a.partial[static_cast<size_t>(h) * a.ldOut + row] = acc;
 }
 
-__global__ void gram_reduce_kernel(const GramArgs a, float* out, int ldOut) {
+// One CTA per (256-row block, head): the block's partials were written by the
+// CTAs whose step ranges covered it, two column halves each, in slot order.
+__global__ void __launch_bounds__(kGramRowBlock) gram_reduce_kernel(const GramArgs a, float* out, int ldOut) {
+  __shared__ HeadDims tab[kGramMaxHeads + 1];
+  __shared__ int nslots;
   pdl_wait();
   pdl_trigger();
-  const int h = blockIdx.y;
-  const int r = blockIdx.x * blockDim.x + threadIdx.x;
-  const int nR = set_n(a.rows, h);
-  if (r >= nR) return;
-  int RB, CT;
-  head_dims(a, h, RB, CT);
-  float acc = 0.f;
-  if (CT > 0) {
-    const long long T = total_steps(a);
-    const int G = active_grid(a, T);
-    long long before = 0;
-    for (int g = 0; g < h; ++g) {
-      int rb2, ct2;
-      head_dims(a, g, rb2, ct2);
-      before += static_cast<long long>(rb2) * ct2;
+  const int h = blockIdx.y, rb = blockIdx.x;
+  if (threadIdx.x < 32) build_head_table(a, tab, threadIdx.x);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const HeadDims& t = tab[h];
+    int n = 0;
+    if (t.CT > 0 && rb < t.RB) {
+      const long long T = tab[a.H].L0;
+      const int G = active_grid(a, T);
+      const long long Lb = t.L0 + static_cast<long long>(rb) * t.CT;
+      n = 2 * (cta_of(Lb + t.CT - 1, T, G) - cta_of(Lb, T, G) + 1);
     }
-    const long long Lb = before + static_cast<long long>(r / kGramRowBlock) * CT;
-    const int first = cta_of(Lb, T, G), last = cta_of(Lb + CT - 1, T, G);
-    const int n = 2 * (last - first + 1);  // two column halves per CTA
-    for (int sl = 0; sl < n && sl < a.slots; ++sl)
-      acc += a.partial[(static_cast<size_t>(sl) * a.H + h) * a.ldOut + r];
+    nslots = n < a.slots ? n : a.slots;
   }
+  __syncthreads();
+  const int r = rb * kGramRowBlock + threadIdx.x;
+  if (r >= tab[h].nR) return;
+  const int n = nslots;
+  float acc = 0.f;
+  for (int sl = 0; sl < n; ++sl) acc += a.partial[(static_cast<size_t>(sl) * a.H + h) * a.ldOut + r];
   out[static_cast<size_t>(h) * ldOut + r] = acc;
 }
 
@@ -549,7 +581,7 @@ __global__ void gram_reduce_kernel(const GramArgs a, float* out, int ldOut) {
 size_t gram_smem_bytes(int d) {
   const size_t a = static_cast<size_t>(kGramRowTile) * (d * 2 + kAugRowBytes);
   const size_t b = static_cast<size_t>(kColTile) * (d * 2 + kAugRowBytes);
-  return 1024 + 2 * a + kStages * b + kBarBytes;
+  return 1024 + 2 * a + kStages * b + kBarBytes + kTabBytes;
 }
 
 void gram_plan(GramArgs& a, int max_col_tiles, int n_sm) {
@@ -563,6 +595,7 @@ void gram_plan(GramArgs& a, int max_col_tiles, int n_sm) {
 
 cudaError_t launch_gram_bf16(const GramArgs& a, const CUtensorMap& tmR, const CUtensorMap& tmC,
                              const CUtensorMap& tmRa, const CUtensorMap& tmCa, cudaStream_t st) {
+  if (a.H < 1 || a.H > kGramMaxHeads) return cudaErrorInvalidValue;
   const size_t smem = gram_smem_bytes(a.d);
   const int grid = a.grid;
   if (grid <= 0) return cudaSuccess;
@@ -595,10 +628,11 @@ cudaError_t launch_gram_f32(const GramArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_gram_reduce(const GramArgs& a, float* out, int ldOut, cudaStream_t st) {
+  if (a.H < 1 || a.H > kGramMaxHeads) return cudaErrorInvalidValue;
   const int maxR = a.max_rows;
-  dim3 grid((maxR + 255) / 256, a.H);
+  dim3 grid((maxR + kGramRowBlock - 1) / kGramRowBlock, a.H);
   LaunchTrace trace("gram_reduce_kernel", st);
-  return launch_pdl(gram_reduce_kernel, grid, dim3(256), 0, st, a, out, ldOut);
+  return launch_pdl(gram_reduce_kernel, grid, dim3(kGramRowBlock), 0, st, a, out, ldOut);
 }
 
 }  // namespace kvb

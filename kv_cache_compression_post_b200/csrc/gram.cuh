@@ -12,6 +12,7 @@ constexpr int kGramRowTile = 128;      // rows per TMEM accumulator (M of the MM
 constexpr int kGramRowBlock = 256;     // rows per work unit (two accumulators)
 constexpr int kGramColTile = 256;      // columns per MMA (N) and per work step
 constexpr int kGramThreads = 640;      // 4 control warps + 16 epilogue warps
+constexpr int kGramMaxHeads = 64;      // heads of one launch
 
 // A set of rows/cols: per head a count and a start row inside its buffer.  Each
 // field is either a uniform value or (if the pointer is non-null) a device array
