@@ -431,7 +431,7 @@ def run_workload(args, w, rank, world):
     total_ms = max_over_ranks(sum(per_step), world)
 
     # end-to-end: every step's inputs go in from pinned host memory and its output
-    # comes back, inside the timed region.  Two device input sets and two outputs
+    # comes back, inside the timed region.  Three device input sets and two outputs
     # let the copies overlap the compute: step j+1's inputs travel on an upload
     # stream while step j runs, and step j's output on a download stream once it
     # is done (copies in the two directions use separate engines).
@@ -439,29 +439,47 @@ def run_workload(args, w, rank, world):
     keys = sorted(hosted)
     proto = hosted[keys[0]]
     # the sink frame (frame 0) is the same for every step: it is uploaded once, before
-    # the timed region, and stays resident like the bank; every other input of a
-    # step is copied in during it
+    # the timed region, and stays resident like the bank
     resident = ("sinkK", "sinkV")
     sink = {k: proto[k].to("cuda") for k in resident if k in proto}
-    bufs = [{k: (sink[k] if k in sink else torch.empty_like(v, device="cuda")) for k, v in proto.items()}
-            for _ in range(2)]
+    # the finalised chunk's tensors that are the previous step's window, bit for
+    # bit (its values, and for Forcing-KV its keys too, which keep their true frame
+    # index): a step reads them from the window the previous step uploaded, as a
+    # rollout does; DensityKV candidate keys carry the memory rotation (frame index
+    # 0) and are copied in
+    carry = {"newK": "winK", "newV": "winV"} if w.forcing else {"candV": "winV"}
+    before = inputs[keys[0] - 1]   # the last device-timed step, resident before the timed region
+    for j, i in enumerate(keys):
+        for k, src in carry.items():
+            ref = hosted[keys[j - 1]][src] if j > 0 else before[src].cpu()
+            if not torch.equal(hosted[i][k], ref):
+                raise RuntimeError(f"step {i}: {k} is not the previous window's {src}")
+    nb = 3
+    bufs = [{k: (sink[k] if k in sink else torch.empty_like(v, device="cuda")) for k, v in proto.items()
+             if k not in carry} for _ in range(nb)]
     outs = [O, torch.empty_like(O)]
     Oh = [torch.empty(O.shape, dtype=O.dtype).pin_memory() for _ in range(2)]
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(nb)]
+    ev_done = [torch.cuda.Event() for _ in range(nb)]
     ev_back = [torch.cuda.Event() for _ in range(2)]
     h2d = d2h = 0
 
     def upload(j, b):
         nonlocal h2d
         for k, v in hosted[keys[j]].items():
-            if k in sink:
+            if k in sink or k in carry:
                 continue
             if bufs[b][k].shape != v.shape:
                 raise RuntimeError("end-to-end inputs change shape between steps")
             bufs[b][k].copy_(v, non_blocking=True)
             h2d += v.numel() * v.element_size()
         ev_in[b].record(up)
+
+    def inputs_of(j):
+        x = dict(bufs[j % nb])
+        for k, src in carry.items():
+            x[k] = bufs[(j - 1) % nb][src] if j > 0 else before[src]
+        return x
 
     barrier(world)
     torch.cuda.synchronize()
@@ -472,23 +490,25 @@ def run_workload(args, w, rank, world):
     with torch.cuda.stream(up):
         upload(0, 0)
     for j in range(len(keys)):
-        b = j % 2
+        b, ob = j % nb, j % 2
         stream.wait_event(ev_in[b])
         if j >= 2:
-            stream.wait_event(ev_back[b])       # outs[b] has been read back
-        x = bufs[b]
+            stream.wait_event(ev_back[ob])      # outs[ob] has been read back
+        x = inputs_of(j)
         update(x)
-        bank.attend(0, x["Q"], x["sinkK"], x["sinkV"], x["winK"], x["winV"], outs[b], lse, stream)
+        bank.attend(0, x["Q"], x["sinkK"], x["sinkV"], x["winK"], x["winV"], outs[ob], lse, stream)
         ev_done[b].record(stream)
         if j + 1 < len(keys):
             if j >= 1:
-                up.wait_event(ev_done[1 - b])   # step j-1 no longer reads bufs[1-b]
+                # bufs[(j+1) % 3] was read by step j-2 (its inputs) and step j-1 (the
+                # carried window): both are done once step j-1 is
+                up.wait_event(ev_done[(j - 1) % nb])
             with torch.cuda.stream(up):
-                upload(j + 1, 1 - b)
+                upload(j + 1, (j + 1) % nb)
         down.wait_event(ev_done[b])
         with torch.cuda.stream(down):
-            Oh[b].copy_(outs[b], non_blocking=True)
-            ev_back[b].record(down)
+            Oh[ob].copy_(outs[ob], non_blocking=True)
+            ev_back[ob].record(down)
         d2h += O.numel() * O.element_size()
     stream.wait_stream(down)
     e_end.record(stream)
@@ -920,10 +940,13 @@ def run_kvb(args, w, rank, world, local):
         "config": workload_config(w, args, world),
         "e2e": {"value": round(r["e2e_ms"], 4), "unit": UNIT, "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"],
-                "what": "kvb_admit / kvb_prune_hybrid + kvb_attend with each step's inputs (candidates or new "
-                        "frames, queries, window) copied in from pinned host memory and the output copied out, "
-                        "inside the timed region, overlapped with the compute on two copy streams; the sink "
-                        "frame, the same every step, is resident like the bank"},
+                "what": "kvb_admit / kvb_prune_hybrid + kvb_attend with each step's new inputs (queries, "
+                        "window K/V, DensityKV candidate keys and ids or the Forcing-KV successor frame and ids) "
+                        "copied in from pinned host memory and the output copied out, inside the timed region, "
+                        "overlapped with the compute on two copy streams; the finalised chunk's values (and "
+                        "Forcing-KV keys), identical to the previous step's window, are read from that window "
+                        "on the device (checked bit for bit on the host); the sink frame, the same every step, "
+                        "is resident like the bank"},
         "gpu_launches": r["launches"],
         "roofline": r["roofline"],
         "roofline_other": r["roofline_other"],

@@ -45,6 +45,12 @@ def test_token_ids_and_chunk_bookkeeping():
     assert x2["sinkK"].shape == (w.heads, w.F, w.head_dim)
     # the window of step 1 is the candidate block of step 2 (same raw keys, other rotation)
     np.testing.assert_array_equal(x1["winV"], x2["candV"])
+    # Forcing-KV: the frames entering the history are the previous window, keys and
+    # values alike (true frame index), and the successor frame opens the window
+    f1, f2 = L.step(1, forcing=True), L.step(2, forcing=True)
+    np.testing.assert_array_equal(f1["winK"], f2["newK"])
+    np.testing.assert_array_equal(f1["winV"], f2["newV"])
+    np.testing.assert_array_equal(f2["nextK"], f2["winK"][:, :w.F])
 
 
 def test_memory_keys_are_rotated_with_frame_zero():
