@@ -263,9 +263,8 @@ def kernel_units(w, name, N, st_before, st_after, n_frames, labels):
                 "dynamic heads x (n_frames+1 frames of K read + segment means written)"
         if name == "prune_gather_kernel":
             kept = sum(st_after[h]["admitted"] for h in dyn)
-            return "hbm", kept * (4 * row + 8), "kept tokens x (K,V read+write + id read+write)"
-        if name == "static_copy_kernel":
-            return "hbm", len(sta) * w.F * (4 * row + 8), "static heads x F x (K,V read+write + id)"
+            return "hbm", (kept + len(sta) * w.F) * (4 * row + 8), \
+                "(dynamic heads' kept tokens + static heads x F) x (K,V read+write + id read+write)"
         return "latency", None, "per-head bookkeeping (one CTA per head)"
     pairs = gram_pairs(N, st_before, st_after)
     P = sum(s["admitted"] for s in st_after)
@@ -418,7 +417,7 @@ def run_workload(args, w, rank, world):
         for name in ("gram_bf16_kernel", "attend_bf16_kernel", "aug_rows_kernel", "gather_admitted_kernel",
                      "gather_evicted_kernel", "compact_kernel", "finalize_kernel", "gram_reduce_kernel",
                      "admit_count_kernel", "admit_select_kernel", "evict_select_kernel", "seg_cosine_kernel",
-                     "prune_plan_kernel", "prune_gather_kernel", "static_copy_kernel"):
+                     "prune_plan_kernel", "prune_gather_kernel"):
             b, u, text = kernel_units(w, name, N, st_before, st, nf, labels)
             prev = units.get(name)
             units[name] = (b, None if u is None else (u + (prev[1] or 0.0) if prev else u), text)

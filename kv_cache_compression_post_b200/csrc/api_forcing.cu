@@ -134,8 +134,7 @@ extern "C" kvb_status kvb_prune_hybrid(kvb_bank* b, int32_t layer, const uint8_t
     e = launch_seg_cosine_ld(newK, nextK, g.dtype, H, n_frames, g.head_dim, sg, mask, b->sims, p.ld_sims, st);
   if (proxy && layer == 0) b->proxy_frames = e == cudaSuccess ? n_frames : -1;
   if (e == cudaSuccess) e = launch_prune_plan(p, st);
-  if (e == cudaSuccess) e = launch_prune_gather(p, st);
-  if (e == cudaSuccess && mask) e = launch_static_copy(p, st);
+  if (e == cudaSuccess) e = launch_prune_gather(p, st);  // static heads' transition frames too
   return cuda_status(e);
 }
 

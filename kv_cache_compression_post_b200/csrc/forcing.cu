@@ -12,9 +12,9 @@
 //                tokens row-major inside each; the frame is pushed into a FIFO of
 //                hist_frames frames stored as a token ring (the oldest frame is
 //                dropped when the FIFO is full); emits (source row, ring slot)
-//   prune_gather kept tokens' K, V rows and ids into the ring (lane groups of 16
-//                bytes per lane, grid-strided)
-//   static_copy  static heads: the last new frame becomes the transition frame
+//   prune_gather dynamic heads: kept tokens' K, V rows and ids into the ring;
+//                static heads: the last new frame becomes the transition frame
+//                (lane groups of 16 bytes per lane, grid-strided)
 #include <cuda_bf16.h>
 
 #include "forcing.cuh"
@@ -51,12 +51,19 @@ __device__ __forceinline__ void acc_words(uint4 a, uint4 b, float& dot, float& n
   }
 }
 
+constexpr int kSegThreads = 512;
+constexpr int kSegRound = 4;  // tokens per lane group and round
+
 // One CTA per (row of segments, frame, head).  A token's two rows are read by a
-// group of L lanes with 16-byte loads (L = row bytes / 16, at most 32), so a warp
-// covers 32/L tokens at once, two rounds in flight per iteration.
+// group of L lanes with 16-byte loads (L = the largest power of two up to the
+// row's 16-byte word count, at most 32: lane groups are aligned inside a warp),
+// so the CTA covers blockDim / L tokens per pass; a round takes kSegRound passes
+// and, when a lane holds exactly one word of each row (the word count a power of
+// two up to 32), issues every load of the round before the first product.
 template <typename T>
-__global__ void seg_cosine_kernel(const T* __restrict__ K, const T* __restrict__ nextK, int n_frames, int d,
-                                  SegGeom g, unsigned long long skip_mask, float* __restrict__ sim, int ld_sim) {
+__global__ void __launch_bounds__(kSegThreads)
+    seg_cosine_kernel(const T* __restrict__ K, const T* __restrict__ nextK, int n_frames, int d, SegGeom g,
+                      unsigned long long skip_mask, float* __restrict__ sim, int ld_sim) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ float cosv[];  // [seg_h * frame_w]
@@ -66,26 +73,44 @@ __global__ void seg_cosine_kernel(const T* __restrict__ K, const T* __restrict__
   const int nrows = min(g.seg_h, g.frame_h - r0);
   const int ntok = nrows * g.frame_w;
   const int chunks = d * static_cast<int>(sizeof(T)) / 16;  // 16-byte chunks per row
-  const int L = chunks < 32 ? chunks : 32;                  // lanes per token
+  int L = 1;                                                 // lanes per token
+  while (2 * L <= chunks && L < 32) L *= 2;
   const int per_pass = blockDim.x / L;                       // tokens per pass of the CTA
   const int slot = threadIdx.x / L, sub = threadIdx.x % L;
   const size_t Fd = static_cast<size_t>(g.F) * d;
   const T* base = K + static_cast<size_t>(h) * n_frames * Fd + static_cast<size_t>(t) * Fd;
   const T* succ = (t + 1 < n_frames) ? base + Fd : nextK + static_cast<size_t>(h) * Fd;
   const size_t first = static_cast<size_t>(r0) * g.frame_w;  // segment rows are contiguous tokens
-  for (int i0 = 0; i0 < ntok; i0 += 2 * per_pass) {
-    float dot[2] = {0.f, 0.f}, na[2] = {0.f, 0.f}, nb[2] = {0.f, 0.f};
+  for (int i0 = 0; i0 < ntok; i0 += kSegRound * per_pass) {
+    float dot[kSegRound], na[kSegRound], nb[kSegRound];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int i = i0 + u * per_pass + slot;
-      if (i < ntok) {
-        const uint4* a = reinterpret_cast<const uint4*>(base + (first + i) * d);
-        const uint4* b = reinterpret_cast<const uint4*>(succ + (first + i) * d);
-        for (int c = sub; c < chunks; c += L) acc_words(__ldg(a + c), __ldg(b + c), dot[u], na[u], nb[u], T());
+    for (int u = 0; u < kSegRound; ++u) dot[u] = na[u] = nb[u] = 0.f;
+    if (chunks == L) {
+      uint4 wa[kSegRound], wb[kSegRound];
+#pragma unroll
+      for (int u = 0; u < kSegRound; ++u) {
+        const int i = i0 + u * per_pass + slot;
+        wa[u] = wb[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (i < ntok) {
+          wa[u] = __ldg(reinterpret_cast<const uint4*>(base + (first + i) * d) + sub);
+          wb[u] = __ldg(reinterpret_cast<const uint4*>(succ + (first + i) * d) + sub);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kSegRound; ++u) acc_words(wa[u], wb[u], dot[u], na[u], nb[u], T());
+    } else {
+#pragma unroll
+      for (int u = 0; u < kSegRound; ++u) {
+        const int i = i0 + u * per_pass + slot;
+        if (i < ntok) {
+          const uint4* a = reinterpret_cast<const uint4*>(base + (first + i) * d);
+          const uint4* b = reinterpret_cast<const uint4*>(succ + (first + i) * d);
+          for (int c = sub; c < chunks; c += L) acc_words(__ldg(a + c), __ldg(b + c), dot[u], na[u], nb[u], T());
+        }
       }
     }
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < kSegRound; ++u) {
       const float dd = group_sum(dot[u], L), aa = group_sum(na[u], L), bb = group_sum(nb[u], L);
       const int i = i0 + u * per_pass + slot;
       if (sub == 0 && i < ntok) cosv[i] = dd / fmaxf(sqrtf(aa) * sqrtf(bb), 1e-8f);
@@ -104,6 +129,7 @@ __global__ void seg_cosine_kernel(const T* __restrict__ K, const T* __restrict__
 
 constexpr int kPlanThreads = 256;
 constexpr int kPlanMaxSeg = 1024;
+constexpr int kPlanMaxHist = 256;
 
 // Exclusive scan of two ints over the CTA (kPlanThreads threads); returns the
 // totals through *ta / *tb.
@@ -145,6 +171,7 @@ __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePla
   __shared__ int s_kept[kPlanMaxSeg];     // kept segments of the current frame, ascending
   __shared__ int s_off[kPlanMaxSeg + 1];  // token offset of each kept segment in the frame
   __shared__ int2 s_wtot[kPlanThreads / 32];
+  __shared__ int s_fc[kPlanMaxHist];      // the FIFO's frame token counts (histories up to kPlanMaxHist)
   __shared__ int s_state[4];
   __shared__ int s_fs, s_total;
   const int h = blockIdx.x;
@@ -169,9 +196,16 @@ __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePla
     if (threadIdx.x == 0) latch_status(p.status, KVB_E_DEVICE_BOUNDS);
     return;
   }
-  if (call)  // the call's (frame, segment) pairs are ranked together: all of them at hand
+  // every frame's similarities at hand from the start when they fit (always in the
+  // call scope, whose pairs are ranked together), and the FIFO's frame counts:
+  // no global load on the per-frame path
+  const bool sims_at_hand = n_pairs <= kPruneMaxPairs;
+  const bool fc_at_hand = p.hist_frames <= kPlanMaxHist;
+  if (sims_at_hand)
     for (int q = threadIdx.x; q < n_pairs; q += blockDim.x)
       s_sim[q] = p.sims[static_cast<size_t>(h) * p.ld_sims + q];
+  if (fc_at_hand)
+    for (int k = threadIdx.x; k < p.hist_frames; k += blockDim.x) s_fc[k] = p.fcount[h * p.hist_frames + k];
   if (threadIdx.x < 4) s_state[threadIdx.x] = rs[threadIdx.x];
   if (threadIdx.x == 0) s_total = 0;
   for (int j = threadIdx.x; j <= n_seg; j += blockDim.x) s_tok[j] = p.seg_tok[j];
@@ -180,7 +214,7 @@ __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePla
   const int per = (n_seg + kPlanThreads - 1) / kPlanThreads;
   const int j0 = threadIdx.x * per, j1 = min(n_seg, j0 + per);
   for (int t = 0; t < p.n_frames; ++t) {
-    if (!call) {
+    if (!sims_at_hand) {
       const float* sg = p.sims + static_cast<size_t>(h) * p.ld_sims + static_cast<size_t>(t) * n_seg;
       for (int j = threadIdx.x; j < n_seg; j += blockDim.x) s_sim[j] = sg[j];
     }
@@ -188,17 +222,20 @@ __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePla
     // BottomK: segment j is kept iff fewer than `keep` entries precede it in
     // (similarity ascending, position ascending) order, among the frame's
     // segments (per-frame scope) or among the call's (frame, segment) pairs,
-    // position t * n_seg + j (call scope)
+    // position t * n_seg + j (call scope); the frame's similarities start at
+    // sbase in shared memory
+    const int sbase = sims_at_hand ? t * n_seg : 0;
     const int q0 = call ? t * n_seg : 0;
     const int nq = call ? n_pairs : n_seg;
+    const int ib = call ? 0 : sbase;   // shared-memory index of position 0 of the ranking
     int nk = 0, ntok = 0;
     unsigned int kept_bits = 0;  // per <= 32 segments per thread
     for (int j = j0; j < j1; ++j) {
       const int qj = q0 + j;
-      const float sj = s_sim[qj];
+      const float sj = s_sim[ib + qj];
       int rank = 0;
       for (int i = 0; i < nq; ++i) {
-        const float si = s_sim[i];
+        const float si = s_sim[ib + i];
         rank += (si < sj) || (si == sj && i < qj);
       }
       if (rank < p.keep) {
@@ -224,7 +261,7 @@ __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePla
       // FIFO: drop the oldest frame when full, then append this one
       int first = s_state[0], held = s_state[1], tstart = s_state[2], theld = s_state[3];
       if (held == p.hist_frames) {
-        const int c = p.fcount[h * p.hist_frames + first];
+        const int c = fc_at_hand ? s_fc[first] : p.fcount[h * p.hist_frames + first];
         tstart = (tstart + c) % p.ring_cap;
         theld -= c;
         first = (first + 1) % p.hist_frames;
@@ -234,6 +271,7 @@ __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePla
       s_fs = (tstart + theld) % p.ring_cap;
       p.fstart[h * p.hist_frames + slot] = s_fs;
       p.fcount[h * p.hist_frames + slot] = tot_tok;
+      if (fc_at_hand) s_fc[slot] = tot_tok;
       s_state[0] = first;
       s_state[1] = held + 1;
       s_state[2] = tstart;
@@ -280,13 +318,46 @@ __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePla
   }
 }
 
-// Two kept tokens per lane group and iteration, every load before the first store.
+// Static heads: the last new frame becomes the transition frame.
+__device__ __forceinline__ void static_copy(const PrunePlan& p, int h, const RowGroup& g) {
+  const char* nK = static_cast<const char*>(p.newK);
+  const char* nV = static_cast<const char*>(p.newV);
+  for (int i0 = g.first; i0 < p.g.F; i0 += 2 * g.stride) {
+    RowWords rw[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = i0 + u * g.stride;
+      if (i >= p.g.F) continue;
+      const size_t s = static_cast<size_t>(h) * p.n_frames * p.g.F + (p.n_frames - 1) * p.g.F + i;
+      load_rows(rw[u], nK + s * p.row_bytes, nV + s * p.row_bytes, nullptr, p.row_bytes, g);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = i0 + u * g.stride;
+      if (i >= p.g.F) continue;
+      const size_t t = static_cast<size_t>(h) * p.g.F + i;
+      store_rows(rw[u], static_cast<char*>(p.tK) + t * p.row_bytes, static_cast<char*>(p.tV) + t * p.row_bytes,
+                 nullptr, p.row_bytes, g);
+      if (g.sub == 0) {
+        p.tids[t] = p.new_ids[(p.n_frames - 1) * p.g.F + i];
+        if (i == 0) p.tlen[h] = p.g.F;
+      }
+    }
+  }
+}
+
+// Row moves of a prune: dynamic heads' kept tokens into their rings (two per
+// lane group and iteration, every load before the first store), static heads'
+// transition frame; one grid row per head.
 __global__ void prune_gather_kernel(const PrunePlan p) {
   pdl_wait();
   pdl_trigger();
   const int h = blockIdx.y;
-  if ((p.static_mask >> h) & 1ull) return;
   const RowGroup g = row_group(p.row_bytes);
+  if ((p.static_mask >> h) & 1ull) {
+    static_copy(p, h, g);
+    return;
+  }
   const int n = min(p.plan_n[h], p.ld_plan);
   const int* plan = p.plan + static_cast<size_t>(h) * p.ld_plan * 2;
   const char* nK = static_cast<const char*>(p.newK);
@@ -324,38 +395,6 @@ __global__ void prune_gather_kernel(const PrunePlan p) {
   }
 }
 
-__global__ void static_copy_kernel(const PrunePlan p) {
-  pdl_wait();
-  pdl_trigger();
-  const int h = blockIdx.y;
-  if (!((p.static_mask >> h) & 1ull)) return;
-  const RowGroup g = row_group(p.row_bytes);
-  const char* nK = static_cast<const char*>(p.newK);
-  const char* nV = static_cast<const char*>(p.newV);
-  for (int i0 = g.first; i0 < p.g.F; i0 += 2 * g.stride) {
-    RowWords rw[2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int i = i0 + u * g.stride;
-      if (i >= p.g.F) continue;
-      const size_t s = static_cast<size_t>(h) * p.n_frames * p.g.F + (p.n_frames - 1) * p.g.F + i;
-      load_rows(rw[u], nK + s * p.row_bytes, nV + s * p.row_bytes, nullptr, p.row_bytes, g);
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int i = i0 + u * g.stride;
-      if (i >= p.g.F) continue;
-      const size_t t = static_cast<size_t>(h) * p.g.F + i;
-      store_rows(rw[u], static_cast<char*>(p.tK) + t * p.row_bytes, static_cast<char*>(p.tV) + t * p.row_bytes,
-                 nullptr, p.row_bytes, g);
-      if (g.sub == 0) {
-        p.tids[t] = p.new_ids[(p.n_frames - 1) * p.g.F + i];
-        if (i == 0) p.tlen[h] = p.g.F;
-      }
-    }
-  }
-}
-
 }  // namespace
 
 cudaError_t launch_seg_cosine(const void* K, const void* nextK, kvb_dtype dtype, int H, int n_frames, int d,
@@ -371,10 +410,10 @@ cudaError_t launch_seg_cosine_ld(const void* K, const void* nextK, kvb_dtype dty
   const size_t smem = sizeof(float) * g.seg_h * g.frame_w;
   LaunchTrace trace("seg_cosine_kernel", st);
   if (dtype == KVB_BF16)
-    return launch_pdl(seg_cosine_kernel<__nv_bfloat16>, grid, dim3(256), smem, st,
+    return launch_pdl(seg_cosine_kernel<__nv_bfloat16>, grid, dim3(kSegThreads), smem, st,
                       static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(nextK), n_frames, d, g,
                       skip_mask, sim, ld_sim);
-  return launch_pdl(seg_cosine_kernel<float>, grid, dim3(256), smem, st, static_cast<const float*>(K),
+  return launch_pdl(seg_cosine_kernel<float>, grid, dim3(kSegThreads), smem, st, static_cast<const float*>(K),
                     static_cast<const float*>(nextK), n_frames, d, g, skip_mask, sim, ld_sim);
 }
 
@@ -388,9 +427,5 @@ cudaError_t launch_prune_gather(const PrunePlan& p, cudaStream_t st) {
   return launch_pdl(prune_gather_kernel, dim3(mover_blocks(p.ld_plan, p.row_bytes, p.H), p.H), dim3(256), 0, st, p);
 }
 
-cudaError_t launch_static_copy(const PrunePlan& p, cudaStream_t st) {
-  LaunchTrace trace("static_copy_kernel", st);
-  return launch_pdl(static_copy_kernel, dim3(mover_blocks(p.g.F, p.row_bytes, p.H), p.H), dim3(256), 0, st, p);
-}
 
 }  // namespace kvb

@@ -61,6 +61,5 @@ struct PrunePlan {
 
 cudaError_t launch_prune_plan(const PrunePlan& p, cudaStream_t st);
 cudaError_t launch_prune_gather(const PrunePlan& p, cudaStream_t st);
-cudaError_t launch_static_copy(const PrunePlan& p, cudaStream_t st);
 
 }  // namespace kvb

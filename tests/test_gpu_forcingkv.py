@@ -204,3 +204,29 @@ def test_forcing_mid_first_block_proxy():
                     np.testing.assert_array_equal(gK[gf == f], oK[of == f].astype(np.float32))
                     np.testing.assert_array_equal(gV[gf == f], oV[of == f].astype(np.float32))
     bank.close()
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 48), ("f32", 20), ("bf16", 80), ("f32", 72), ("bf16", 256)])
+def test_segment_cosine_row_widths(dtype, d):
+    """Rows whose 16-byte word count is not a power of two (a lane holds several
+    words, or a lane group is narrower than the row), and wide rows; a 7 x 9 frame
+    in 2 x 3 segments, partial at both edges."""
+    import torch
+    import kv_cache_compression_post_b200 as kvb
+    H, nf, fh, fw, sh, sw = 3, 2, 7, 9, 2, 3
+    rng = np.random.default_rng(d)
+    K = rng.standard_normal((H, nf * fh * fw, d)).astype(np.float32)
+    nxt = rng.standard_normal((H, fh * fw, d)).astype(np.float32)
+    if dtype == "bf16":  # the stored values, rounded on the host
+        K, nxt = (torch.from_numpy(a).to(torch.bfloat16).float().numpy() for a in (K, nxt))
+    segs = fkv.segments(fh, fw, sh, sw)
+    sim = torch.full((H, nf, len(segs)), float("nan"), device="cuda")
+    kvb.kvb_segment_cosine(dev_tensor(K, dtype), dev_tensor(nxt, dtype), H, nf, fh, fw, sh, sw, d,
+                           kvb.KVB_BF16 if dtype == "bf16" else kvb.KVB_F32, sim)
+    torch.cuda.synchronize()
+    got = host(sim)
+    for hh in range(H):
+        Kf = K[hh].reshape(nf, fh * fw, d)
+        for t in range(nf):
+            succ = Kf[t + 1] if t + 1 < nf else nxt[hh]
+            np.testing.assert_allclose(got[hh, t], fkv.segment_similarity(Kf[t], succ, segs), atol=2e-6, rtol=0)
