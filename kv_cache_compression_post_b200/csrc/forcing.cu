@@ -52,55 +52,67 @@ __device__ __forceinline__ void acc_words(uint4 a, uint4 b, float& dot, float& n
 }
 
 constexpr int kSegThreads = 512;
-constexpr int kSegRound = 4;  // tokens per lane group and round
 
 // One CTA per (row of segments, frame, head).  A token's two rows are read by a
-// group of L lanes with 16-byte loads (L = the largest power of two up to the
-// row's 16-byte word count, at most 32: lane groups are aligned inside a warp),
-// so the CTA covers blockDim / L tokens per pass; a round takes kSegRound passes
-// and, when a lane holds exactly one word of each row (the word count a power of
-// two up to 32), issues every load of the round before the first product.
-template <typename T>
+// group of L lanes with 16-byte loads.  With CPL > 0 each lane holds CPL words of
+// each row (L = words / CPL, a power of two, 4 for the rows of up to 64 words the
+// banks use), and a round issues every load of its U tokens per group before the
+// first product; the three sums per token then need log2(L) shuffle steps.
+// CPL = 0 takes any row: L = the largest power of two up to min(words, 32) and a
+// loop over each lane's words.
+template <typename T, int CPL>
 __global__ void __launch_bounds__(kSegThreads)
     seg_cosine_kernel(const T* __restrict__ K, const T* __restrict__ nextK, int n_frames, int d, SegGeom g,
                       unsigned long long skip_mask, float* __restrict__ sim, int ld_sim) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ float cosv[];  // [seg_h * frame_w]
+  constexpr int U = CPL > 0 ? (CPL >= 8 ? 1 : 8 / CPL) : 2;  // tokens per lane group and round
   const int sr = blockIdx.x, t = blockIdx.y, h = blockIdx.z;
   if ((skip_mask >> h) & 1ull) return;
   const int r0 = sr * g.seg_h;
   const int nrows = min(g.seg_h, g.frame_h - r0);
   const int ntok = nrows * g.frame_w;
-  const int chunks = d * static_cast<int>(sizeof(T)) / 16;  // 16-byte chunks per row
+  const int chunks = d * static_cast<int>(sizeof(T)) / 16;  // 16-byte words per row
   int L = 1;                                                 // lanes per token
-  while (2 * L <= chunks && L < 32) L *= 2;
+  if (CPL > 0) {
+    L = chunks / CPL;
+  } else {
+    while (2 * L <= chunks && L < 32) L *= 2;
+  }
   const int per_pass = blockDim.x / L;                       // tokens per pass of the CTA
   const int slot = threadIdx.x / L, sub = threadIdx.x % L;
   const size_t Fd = static_cast<size_t>(g.F) * d;
   const T* base = K + static_cast<size_t>(h) * n_frames * Fd + static_cast<size_t>(t) * Fd;
   const T* succ = (t + 1 < n_frames) ? base + Fd : nextK + static_cast<size_t>(h) * Fd;
   const size_t first = static_cast<size_t>(r0) * g.frame_w;  // segment rows are contiguous tokens
-  for (int i0 = 0; i0 < ntok; i0 += kSegRound * per_pass) {
-    float dot[kSegRound], na[kSegRound], nb[kSegRound];
+  for (int i0 = 0; i0 < ntok; i0 += U * per_pass) {
+    float dot[U], na[U], nb[U];
 #pragma unroll
-    for (int u = 0; u < kSegRound; ++u) dot[u] = na[u] = nb[u] = 0.f;
-    if (chunks == L) {
-      uint4 wa[kSegRound], wb[kSegRound];
+    for (int u = 0; u < U; ++u) dot[u] = na[u] = nb[u] = 0.f;
+    if constexpr (CPL > 0) {
+      uint4 wa[U][CPL], wb[U][CPL];
 #pragma unroll
-      for (int u = 0; u < kSegRound; ++u) {
+      for (int u = 0; u < U; ++u) {
         const int i = i0 + u * per_pass + slot;
-        wa[u] = wb[u] = make_uint4(0u, 0u, 0u, 0u);
-        if (i < ntok) {
-          wa[u] = __ldg(reinterpret_cast<const uint4*>(base + (first + i) * d) + sub);
-          wb[u] = __ldg(reinterpret_cast<const uint4*>(succ + (first + i) * d) + sub);
+        const uint4* a = reinterpret_cast<const uint4*>(base + (first + i) * d);
+        const uint4* b = reinterpret_cast<const uint4*>(succ + (first + i) * d);
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) {
+          wa[u][k] = wb[u][k] = make_uint4(0u, 0u, 0u, 0u);
+          if (i < ntok) {
+            wa[u][k] = __ldg(a + sub + k * L);
+            wb[u][k] = __ldg(b + sub + k * L);
+          }
         }
       }
 #pragma unroll
-      for (int u = 0; u < kSegRound; ++u) acc_words(wa[u], wb[u], dot[u], na[u], nb[u], T());
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) acc_words(wa[u][k], wb[u][k], dot[u], na[u], nb[u], T());
     } else {
 #pragma unroll
-      for (int u = 0; u < kSegRound; ++u) {
+      for (int u = 0; u < U; ++u) {
         const int i = i0 + u * per_pass + slot;
         if (i < ntok) {
           const uint4* a = reinterpret_cast<const uint4*>(base + (first + i) * d);
@@ -110,7 +122,7 @@ __global__ void __launch_bounds__(kSegThreads)
       }
     }
 #pragma unroll
-    for (int u = 0; u < kSegRound; ++u) {
+    for (int u = 0; u < U; ++u) {
       const float dd = group_sum(dot[u], L), aa = group_sum(na[u], L), bb = group_sum(nb[u], L);
       const int i = i0 + u * per_pass + slot;
       if (sub == 0 && i < ntok) cosv[i] = dd / fmaxf(sqrtf(aa) * sqrtf(bb), 1e-8f);
@@ -402,6 +414,34 @@ cudaError_t launch_seg_cosine(const void* K, const void* nextK, kvb_dtype dtype,
   return launch_seg_cosine_ld(K, nextK, dtype, H, n_frames, d, g, skip_mask, sim, n_frames * g.n_seg, st);
 }
 
+template <typename T>
+cudaError_t launch_seg_typed(const void* K, const void* nextK, int n_frames, int d, const SegGeom& g,
+                             unsigned long long skip_mask, float* sim, int ld_sim, dim3 grid, size_t smem,
+                             cudaStream_t st) {
+  // four lanes per token when a row is 4, 8, 16 or 32 words long (each lane holds a
+  // fixed number of words); any other row takes the looping form
+  const int words = d * static_cast<int>(sizeof(T)) / 16;
+  const T* k = static_cast<const T*>(K);
+  const T* n = static_cast<const T*>(nextK);
+  switch (words) {
+    case 4:
+      return launch_pdl(seg_cosine_kernel<T, 1>, grid, dim3(kSegThreads), smem, st, k, n, n_frames, d, g, skip_mask,
+                        sim, ld_sim);
+    case 8:
+      return launch_pdl(seg_cosine_kernel<T, 2>, grid, dim3(kSegThreads), smem, st, k, n, n_frames, d, g, skip_mask,
+                        sim, ld_sim);
+    case 16:
+      return launch_pdl(seg_cosine_kernel<T, 4>, grid, dim3(kSegThreads), smem, st, k, n, n_frames, d, g, skip_mask,
+                        sim, ld_sim);
+    case 32:
+      return launch_pdl(seg_cosine_kernel<T, 8>, grid, dim3(kSegThreads), smem, st, k, n, n_frames, d, g, skip_mask,
+                        sim, ld_sim);
+    default:
+      return launch_pdl(seg_cosine_kernel<T, 0>, grid, dim3(kSegThreads), smem, st, k, n, n_frames, d, g, skip_mask,
+                        sim, ld_sim);
+  }
+}
+
 cudaError_t launch_seg_cosine_ld(const void* K, const void* nextK, kvb_dtype dtype, int H, int n_frames, int d,
                                  const SegGeom& g, unsigned long long skip_mask, float* sim, int ld_sim,
                                  cudaStream_t st) {
@@ -410,11 +450,8 @@ cudaError_t launch_seg_cosine_ld(const void* K, const void* nextK, kvb_dtype dty
   const size_t smem = sizeof(float) * g.seg_h * g.frame_w;
   LaunchTrace trace("seg_cosine_kernel", st);
   if (dtype == KVB_BF16)
-    return launch_pdl(seg_cosine_kernel<__nv_bfloat16>, grid, dim3(kSegThreads), smem, st,
-                      static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(nextK), n_frames, d, g,
-                      skip_mask, sim, ld_sim);
-  return launch_pdl(seg_cosine_kernel<float>, grid, dim3(kSegThreads), smem, st, static_cast<const float*>(K),
-                    static_cast<const float*>(nextK), n_frames, d, g, skip_mask, sim, ld_sim);
+    return launch_seg_typed<__nv_bfloat16>(K, nextK, n_frames, d, g, skip_mask, sim, ld_sim, grid, smem, st);
+  return launch_seg_typed<float>(K, nextK, n_frames, d, g, skip_mask, sim, ld_sim, grid, smem, st);
 }
 
 cudaError_t launch_prune_plan(const PrunePlan& p, cudaStream_t st) {
