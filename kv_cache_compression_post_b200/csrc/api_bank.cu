@@ -124,7 +124,6 @@ size_t kvb_bank::layout(void* base) {
     sims = c.take<float>(H * nf * n_seg);
     keep = c.take<int>(H * nf * n_seg);
     seg_tok = c.take<int>(n_seg + 1);
-    seg_list = c.take<int>(F);
     plan = c.take<int>(2 * H * nf * F);  // (source row, ring slot) pairs
     plan_n = c.take<int>(H);
   }

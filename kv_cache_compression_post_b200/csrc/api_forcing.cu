@@ -38,20 +38,19 @@ extern "C" kvb_status kvb_forcing_init(kvb_bank* b, cudaStream_t st) {
   if (sg.n_seg > 1024) return KVB_E_UNSUPPORTED;
   // segment-major token order: segment j (row-major over segments) lists its
   // tokens row-major; seg_tok[j] is its first position in that order
-  std::vector<int> tok(sg.n_seg + 1), list(sg.F);
+  std::vector<int> tok(sg.n_seg + 1);
   int pos = 0;
   for (int sr = 0; sr < sg.seg_rows; ++sr)
     for (int sc = 0; sc < sg.seg_cols; ++sc) {
       tok[sr * sg.seg_cols + sc] = pos;
-      for (int r = sr * sg.seg_h; r < std::min((sr + 1) * sg.seg_h, sg.frame_h); ++r)
-        for (int c = sc * sg.seg_w; c < std::min((sc + 1) * sg.seg_w, sg.frame_w); ++c) list[pos++] = r * sg.frame_w + c;
+      const int rows = std::min((sr + 1) * sg.seg_h, sg.frame_h) - sr * sg.seg_h;
+      const int cols = std::min((sc + 1) * sg.seg_w, sg.frame_w) - sc * sg.seg_w;
+      pos += rows * cols;
     }
   tok[sg.n_seg] = pos;
   const size_t LH = static_cast<size_t>(g.layers) * g.heads;
   cudaError_t e = cudaMemcpyAsync(b->seg_tok, tok.data(), sizeof(int) * tok.size(), cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(b->seg_list, list.data(), sizeof(int) * list.size(), cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(st);  // host vectors go out of scope
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);  // the host vector goes out of scope
   // rows past a history's length are read by full attention tiles (and masked):
   // keep them finite by starting from zeros
   if (e == cudaSuccess) e = cudaMemsetAsync(b->tK, 0, LH * b->F * static_cast<size_t>(b->row_bytes), st);
@@ -106,7 +105,6 @@ extern "C" kvb_status kvb_prune_hybrid(kvb_bank* b, int32_t layer, const uint8_t
   p.new_ids = new_ids;
   p.sims = b->sims;
   p.seg_tok = b->seg_tok;
-  p.seg_list = b->seg_list;
   p.plan = b->plan;
   p.plan_n = b->plan_n;
   p.keep_list = b->keep;

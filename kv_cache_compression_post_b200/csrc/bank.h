@@ -87,7 +87,6 @@ struct kvb_bank {
   float* sims = nullptr;    // [H][max_new_frames][n_seg]
   int* keep = nullptr;      // [H][max_new_frames][n_seg] kept segment ids, ascending
   int* seg_tok = nullptr;   // [n_seg + 1] token offsets of each segment in segment-major order
-  int* seg_list = nullptr;  // [F] token index (row-major) in segment-major order
   int* plan = nullptr;      // [H][max_new_frames*F][2] (source row, ring position) pairs
   int* plan_n = nullptr;    // [H]
   // KVB_SIM_FIRST_LAYER: frames of layer 0's last prune, whose similarities (left

@@ -141,6 +141,17 @@ __global__ void __launch_bounds__(kSegThreads)
 
 constexpr int kPlanThreads = 256;
 constexpr int kPlanMaxSeg = 1024;
+
+// Token (row-major position in the frame) of the m-th token of segment j, tokens
+// numbered row-major inside the segment; segments are seg_h x seg_w tiles
+// numbered row-major, partial at the right and bottom edges.
+__device__ __forceinline__ int seg_token(const SegGeom& g, int j, int m) {
+  const int sr = j / g.seg_cols, sc = j - sr * g.seg_cols;
+  const int c0 = sc * g.seg_w;
+  const int w = min(c0 + g.seg_w, g.frame_w) - c0;
+  const int r = sr * g.seg_h + m / w;
+  return r * g.frame_w + c0 + (m - (m / w) * w);
+}
 constexpr int kPlanMaxHist = 256;
 
 // Exclusive scan of two ints over the CTA (kPlanThreads threads); returns the
@@ -184,6 +195,7 @@ __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePla
   __shared__ int s_off[kPlanMaxSeg + 1];  // token offset of each kept segment in the frame
   __shared__ int2 s_wtot[kPlanThreads / 32];
   __shared__ int s_fc[kPlanMaxHist];      // the FIFO's frame token counts (histories up to kPlanMaxHist)
+  __shared__ uint8_t s_kflag[kPruneMaxPairs];  // kept flag of every (frame, segment) pair
   __shared__ int s_state[4];
   __shared__ int s_fs, s_total;
   const int h = blockIdx.x;
@@ -222,35 +234,49 @@ __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePla
   if (threadIdx.x == 0) s_total = 0;
   for (int j = threadIdx.x; j <= n_seg; j += blockDim.x) s_tok[j] = p.seg_tok[j];
   int* plan = p.plan + static_cast<size_t>(h) * p.ld_plan * 2;
+  // BottomK: a pair is kept iff fewer than `keep` entries precede it in
+  // (similarity ascending, position ascending) order, among its frame's segments
+  // (per-frame scope) or among the call's (frame, segment) pairs, position
+  // t * n_seg + j (call scope).  With every similarity at hand all pairs are
+  // ranked at once, before the frames are placed one after another.
+  if (sims_at_hand) {
+    __syncthreads();
+    for (int q = threadIdx.x; q < n_pairs; q += blockDim.x) {
+      const int lo = call ? 0 : (q / n_seg) * n_seg, hi = call ? n_pairs : lo + n_seg;
+      const float sq = s_sim[q];
+      int rank = 0;
+      for (int i = lo; i < hi; ++i) {
+        const float si = s_sim[i];
+        rank += (si < sq) || (si == sq && i < q);
+      }
+      s_kflag[q] = rank < p.keep ? 1 : 0;
+    }
+  }
   // each thread owns a run of consecutive segments (for the ordered scans)
   const int per = (n_seg + kPlanThreads - 1) / kPlanThreads;
   const int j0 = threadIdx.x * per, j1 = min(n_seg, j0 + per);
   for (int t = 0; t < p.n_frames; ++t) {
-    if (!sims_at_hand) {
+    if (!sims_at_hand) {  // per-frame scope: this frame's similarities only
       const float* sg = p.sims + static_cast<size_t>(h) * p.ld_sims + static_cast<size_t>(t) * n_seg;
       for (int j = threadIdx.x; j < n_seg; j += blockDim.x) s_sim[j] = sg[j];
     }
     __syncthreads();
-    // BottomK: segment j is kept iff fewer than `keep` entries precede it in
-    // (similarity ascending, position ascending) order, among the frame's
-    // segments (per-frame scope) or among the call's (frame, segment) pairs,
-    // position t * n_seg + j (call scope); the frame's similarities start at
-    // sbase in shared memory
-    const int sbase = sims_at_hand ? t * n_seg : 0;
-    const int q0 = call ? t * n_seg : 0;
-    const int nq = call ? n_pairs : n_seg;
-    const int ib = call ? 0 : sbase;   // shared-memory index of position 0 of the ranking
     int nk = 0, ntok = 0;
     unsigned int kept_bits = 0;  // per <= 32 segments per thread
     for (int j = j0; j < j1; ++j) {
-      const int qj = q0 + j;
-      const float sj = s_sim[ib + qj];
-      int rank = 0;
-      for (int i = 0; i < nq; ++i) {
-        const float si = s_sim[ib + i];
-        rank += (si < sj) || (si == sj && i < qj);
+      bool kept;
+      if (sims_at_hand) {
+        kept = s_kflag[t * n_seg + j] != 0;
+      } else {
+        const float sj = s_sim[j];
+        int rank = 0;
+        for (int i = 0; i < n_seg; ++i) {
+          const float si = s_sim[i];
+          rank += (si < sj) || (si == sj && i < j);
+        }
+        kept = rank < p.keep;
       }
-      if (rank < p.keep) {
+      if (kept) {
         kept_bits |= 1u << (j - j0);
         ++nk;
         ntok += s_tok[j + 1] - s_tok[j];
@@ -306,7 +332,7 @@ __global__ void __launch_bounds__(kPlanThreads) prune_plan_kernel(const PrunePla
       const int m = e - s_off[lo];
       const int g = base + e;
       if (g < p.ld_plan) {
-        plan[2 * g] = t * p.g.F + p.seg_list[s_tok[j] + m];
+        plan[2 * g] = t * p.g.F + seg_token(p.g, j, m);
         plan[2 * g + 1] = (s_fs + e) % p.ring_cap;
       }
     }

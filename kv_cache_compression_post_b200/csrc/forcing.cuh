@@ -37,7 +37,6 @@ struct PrunePlan {
   const int* new_ids = nullptr;
   const float* sims = nullptr;     // [H][max_new_frames][n_seg]
   const int* seg_tok = nullptr;    // [n_seg + 1]
-  const int* seg_list = nullptr;   // [F]
   int* plan = nullptr;             // [H][max_new_frames * F][2] (source row, ring position)
   int* plan_n = nullptr;           // [H]
   int* keep_list = nullptr;        // [H][max_new_frames][n_seg]
