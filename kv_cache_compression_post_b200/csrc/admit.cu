@@ -281,8 +281,21 @@ __global__ void __launch_bounds__(kSelThreads) admit_count_kernel(const AdmitPla
   __shared__ SelShared S;
   const int h = blockIdx.x;
   const int n = p.size[h];
+  // each thread adds its baselines in index order; four loads in flight per round
+  constexpr int kU = 4;
+  const float* r0h = p.rho0 + static_cast<size_t>(h) * p.M;
   float s = 0.f;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) s += p.rho0[static_cast<size_t>(h) * p.M + i];
+  for (int i0 = threadIdx.x; i0 < n; i0 += kU * static_cast<int>(blockDim.x)) {
+    float v[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = i0 + u * static_cast<int>(blockDim.x);
+      v[u] = i < n ? __ldg(r0h + i) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      if (i0 + u * static_cast<int>(blockDim.x) < n) s += v[u];
+  }
   const float sum = block_sum(s, &S);
   const float mean0 = n > 0 ? sum / static_cast<float>(n) : 0.f;
   const float* rb = p.rhoB + static_cast<size_t>(h) * p.ldN;
@@ -301,10 +314,20 @@ __global__ void __launch_bounds__(kSelThreads) admit_count_kernel(const AdmitPla
   // admission-threshold near ties (scores exist only against a bank with a mean baseline)
   const bool scored = n > 0 && mean0 > 0.f;
   int nt = 0;
-  for (int c = threadIdx.x; c < p.N; c += blockDim.x) {
-    const float sc = score_of(rb[c], mean0);
-    if (p.cand_order != KVB_ORDER_SOURCE) cnt += (sc <= p.tau) ? 1 : 0;
-    nt += (scored && near_tau(sc, p.tau)) ? 1 : 0;
+  for (int c0 = threadIdx.x; c0 < p.N; c0 += kU * static_cast<int>(blockDim.x)) {
+    float v[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int c = c0 + u * static_cast<int>(blockDim.x);
+      v[u] = c < p.N ? rb[c] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      if (c0 + u * static_cast<int>(blockDim.x) >= p.N) break;
+      const float sc = score_of(v[u], mean0);
+      if (p.cand_order != KVB_ORDER_SOURCE) cnt += (sc <= p.tau) ? 1 : 0;
+      nt += (scored && near_tau(sc, p.tau)) ? 1 : 0;
+    }
   }
   int total, ties;
   block_excl_scan(cnt, &S, &total);
