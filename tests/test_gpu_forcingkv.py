@@ -206,11 +206,13 @@ def test_forcing_mid_first_block_proxy():
     bank.close()
 
 
-@pytest.mark.parametrize("dtype,d", [("bf16", 48), ("f32", 20), ("bf16", 80), ("f32", 72), ("bf16", 256)])
+@pytest.mark.parametrize("dtype,d", [("bf16", 48), ("f32", 20), ("bf16", 80), ("f32", 72), ("bf16", 256),
+                                     ("bf16", 32), ("bf16", 64), ("f32", 64), ("f32", 128)])
 def test_segment_cosine_row_widths(dtype, d):
-    """Rows whose 16-byte word count is not a power of two (a lane holds several
-    words, or a lane group is narrower than the row), and wide rows; a 7 x 9 frame
-    in 2 x 3 segments, partial at both edges."""
+    """Every row form of the kernel: 4, 8, 16 and 32 words of 16 bytes (a lane
+    holds 1, 2, 4 or 8 words of each row), word counts that are not a power of
+    two (a lane group narrower than the row, looping), and wide rows; a 7 x 9
+    frame in 2 x 3 segments, partial at both edges."""
     import torch
     import kv_cache_compression_post_b200 as kvb
     H, nf, fh, fw, sh, sw = 3, 2, 7, 9, 2, 3
