@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(kSegThreads)
   const int ntok = nrows * g.frame_w;
   const int chunks = d * static_cast<int>(sizeof(T)) / 16;  // 16-byte words per row
   int L = 1;                                                 // lanes per token
-  if (CPL > 0) {
+  if constexpr (CPL > 0) {
     L = chunks / CPL;
   } else {
     while (2 * L <= chunks && L < 32) L *= 2;
