@@ -410,6 +410,9 @@ __global__ void gather_admitted_kernel(const AdmitPlan p) {
   const int h = blockIdx.y;
   const RowGroup g = row_group(p.row_bytes);
   const int P = p.P[h];
+  // bf16: a head that admits every candidate has its admitted block read in place
+  // by the density passes (the admitted indices are then 0..N-1)
+  if (p.dtype == KVB_BF16 && P >= p.N) return;
   const char* cK = static_cast<const char*>(p.candK);
   char* EA = static_cast<char*>(p.EA);
   for (int w0 = g.first; w0 < P; w0 += 2 * g.stride) {

@@ -272,6 +272,20 @@ struct Pass {
   int nneg = 0;
   float* out;
   int ldOut;
+  // rows per head of Raug / Caug when they differ from ldR / ldC (0: the same)
+  long long ldRaug = 0, ldCaug = 0;
+  // bf16: alternate operands for heads whose row (column) count is alt_rows_n
+  // (alt_cols_n): read from row 0 of R2 / C2 instead (null: none)
+  const void* R2 = nullptr;
+  long long ldR2 = 0;
+  const uint16_t* Raug2 = nullptr;
+  long long ldRaug2 = 0;
+  int alt_rows_n = -1;
+  const void* C2 = nullptr;
+  long long ldC2 = 0;
+  const uint16_t* Caug2 = nullptr;
+  long long ldCaug2 = 0;
+  int alt_cols_n = -1;
 };
 
 cudaError_t run_pass(kvb_bank* b, const Pass& ps, const DeviceInfo& dev, cudaStream_t st) {
@@ -298,16 +312,33 @@ cudaError_t run_pass(kvb_bank* b, const Pass& ps, const DeviceInfo& dev, cudaStr
     a.ldOut = ps.ldOut;
     return launch_gram_f32(a, st);
   }
-  CUtensorMap tmR, tmC, tmRa, tmCa;
-  if (!make_tmap_bf16(&tmR, ps.R, g.head_dim, ps.ldR, g.heads, 128) ||
-      !make_tmap_bf16(&tmC, ps.C, g.head_dim, ps.ldC, g.heads, kGramColTile) ||
-      !make_tmap_aug(&tmRa, ps.Raug, ps.ldR, g.heads, 128) || !make_tmap_aug(&tmCa, ps.Caug, ps.ldC, g.heads, kGramColTile))
+  GramMaps m;
+  if (!make_tmap_bf16(&m.R, ps.R, g.head_dim, ps.ldR, g.heads, 128) ||
+      !make_tmap_bf16(&m.C, ps.C, g.head_dim, ps.ldC, g.heads, kGramColTile) ||
+      !make_tmap_aug(&m.Ra, ps.Raug, ps.ldRaug ? ps.ldRaug : ps.ldR, g.heads, 128) ||
+      !make_tmap_aug(&m.Ca, ps.Caug, ps.ldCaug ? ps.ldCaug : ps.ldC, g.heads, kGramColTile))
     return cudaErrorInvalidValue;
+  m.R2 = m.R;
+  m.Ra2 = m.Ra;
+  m.C2 = m.C;
+  m.Ca2 = m.Ca;
+  if (ps.R2) {
+    if (!make_tmap_bf16(&m.R2, ps.R2, g.head_dim, ps.ldR2, g.heads, 128) ||
+        !make_tmap_aug(&m.Ra2, ps.Raug2, ps.ldRaug2 ? ps.ldRaug2 : ps.ldR2, g.heads, 128))
+      return cudaErrorInvalidValue;
+    a.alt_rows_n = ps.alt_rows_n;
+  }
+  if (ps.C2) {
+    if (!make_tmap_bf16(&m.C2, ps.C2, g.head_dim, ps.ldC2, g.heads, kGramColTile) ||
+        !make_tmap_aug(&m.Ca2, ps.Caug2, ps.ldCaug2 ? ps.ldCaug2 : ps.ldC2, g.heads, kGramColTile))
+      return cudaErrorInvalidValue;
+    a.alt_cols_n = ps.alt_cols_n;
+  }
   a.partial = b->partial;
   a.ldOut = b->ldPart;
   a.norm_max = reinterpret_cast<const float*>(b->status + 1);
   gram_plan(a, (ps.max_cols + kGramColTile - 1) / kGramColTile, dev.n_sm);
-  cudaError_t e = launch_gram_bf16(a, tmR, tmC, tmRa, tmCa, st);
+  cudaError_t e = launch_gram_bf16(a, m, st);
   if (e == cudaSuccess) e = launch_gram_reduce(a, ps.out, ps.ldOut, st);
   return e;
 }
@@ -394,6 +425,7 @@ cudaError_t admit_phase1(kvb_bank* b, const AdmitPlan& p, const DeviceInfo& dev,
   // pass 1: candidate density against the bank, rho_B(c)
   if (e == cudaSuccess) {
     Pass ps{candK, N, GramSet{N, nullptr, 0, nullptr}, b->caug, p.K, M, GramSet{0, p.size, 0, nullptr}, p.aug, N, M};
+    ps.ldRaug = b->ldN;  // the candidates' augmented rows are laid out for max_candidates
     ps.out = b->rhoB;
     ps.ldOut = b->ldN;
     e = run_pass(b, ps, dev, st);
@@ -413,6 +445,14 @@ cudaError_t admit_phase2(kvb_bank* b, const AdmitPlan& p, const DeviceInfo& dev,
     Pass ps{p.K, M, GramSet{0, p.size, 0, nullptr}, p.aug, b->EA, b->ldEA, GramSet{0, b->P, M, nullptr}, b->EAaug, M, N};
     ps.out = b->proj;
     ps.ldOut = M;
+    if (b->cfg.dtype == KVB_BF16) {
+      // a head that admits every candidate (P = N, in candidate order) reads them in place
+      ps.C2 = p.candK;
+      ps.ldC2 = N;
+      ps.Caug2 = b->caug;
+      ps.ldCaug2 = b->ldN;
+      ps.alt_cols_n = N;
+    }
     e = run_pass(b, ps, dev, st);
   }
   if (e == cudaSuccess) e = launch_evict_select(p, st);
@@ -434,6 +474,13 @@ cudaError_t admit_phase2(kvb_bank* b, const AdmitPlan& p, const DeviceInfo& dev,
     ps.use_diag = 1;
     ps.out = b->coadm;
     ps.ldOut = b->ldN;
+    if (b->cfg.dtype == KVB_BF16) {
+      ps.R2 = ps.C2 = p.candK;
+      ps.ldR2 = ps.ldC2 = N;
+      ps.Raug2 = ps.Caug2 = b->caug;
+      ps.ldRaug2 = ps.ldCaug2 = b->ldN;
+      ps.alt_rows_n = ps.alt_cols_n = N;
+    }
     e = run_pass(b, ps, dev, st);
   }
   if (e == cudaSuccess) e = launch_finalize(p, st);

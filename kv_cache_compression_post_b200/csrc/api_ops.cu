@@ -114,15 +114,19 @@ kvb_status kvb_density(const void* rows, int32_t n_rows, const void* cols, int32
     e = launch_aug_rows(cols, dtype, heads, n_cols, head_dim, n_cols, nullptr, n_cols, L.colAug, n_cols, norm_max, -0.5f * eps * h, st);
   a.norm_max = norm_max;
   if (e != cudaSuccess) return KVB_E_CUDA;
-  CUtensorMap tmR, tmC, tmRa, tmCa;
-  if (!make_tmap_bf16(&tmR, rows, head_dim, n_rows, heads, 128) ||
-      !make_tmap_bf16(&tmC, cols, head_dim, n_cols, heads, kGramColTile) || !make_tmap_aug(&tmRa, L.rowAug, n_rows, heads, 128) ||
-      !make_tmap_aug(&tmCa, L.colAug, n_cols, heads, kGramColTile))
+  GramMaps m;
+  if (!make_tmap_bf16(&m.R, rows, head_dim, n_rows, heads, 128) ||
+      !make_tmap_bf16(&m.C, cols, head_dim, n_cols, heads, kGramColTile) || !make_tmap_aug(&m.Ra, L.rowAug, n_rows, heads, 128) ||
+      !make_tmap_aug(&m.Ca, L.colAug, n_cols, heads, kGramColTile))
     return KVB_E_INVAL;
   a.partial = L.partial;
   a.ldOut = n_rows;
   gram_plan(a, (n_cols + kGramColTile - 1) / kGramColTile, dev.n_sm);
-  e = launch_gram_bf16(a, tmR, tmC, tmRa, tmCa, st);
+  m.R2 = m.R;  // no alternate operands
+  m.C2 = m.C;
+  m.Ra2 = m.Ra;
+  m.Ca2 = m.Ca;
+  e = launch_gram_bf16(a, m, st);
   if (e == cudaSuccess) e = launch_gram_reduce(a, out, n_rows, st);
   return cuda_status(e);
 }

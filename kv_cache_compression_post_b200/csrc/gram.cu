@@ -64,6 +64,7 @@ struct HeadDims {
   int nR, nC, rOff, cOff;
   int RB, CT;            // row blocks / column tiles
   int nneg, diag;        // signed-column count, self-pair offset
+  int altR, altC;        // rows / columns through the alternate maps (offset 0)
   long long L0;          // first step of the head; entry H holds the total
 };
 constexpr int kTabBytes = (kGramMaxHeads + 1) * static_cast<int>(sizeof(HeadDims));
@@ -79,8 +80,10 @@ __device__ __forceinline__ void build_head_table(const GramArgs& a, HeadDims* ta
     if (h < a.H) {
       t.nR = set_n(a.rows, h);
       t.nC = set_n(a.cols, h);
-      t.rOff = set_off(a.rows, h);
-      t.cOff = set_off(a.cols, h);
+      t.altR = (a.alt_rows_n >= 0 && t.nR == a.alt_rows_n) ? 1 : 0;
+      t.altC = (a.alt_cols_n >= 0 && t.nC == a.alt_cols_n) ? 1 : 0;
+      t.rOff = t.altR ? 0 : set_off(a.rows, h);
+      t.cOff = t.altC ? 0 : set_off(a.cols, h);
       t.RB = t.nC > 0 ? (t.nR + kGramRowBlock - 1) / kGramRowBlock : 0;
       t.CT = t.nR > 0 ? (t.nC + kColTile - 1) / kColTile : 0;
       t.nneg = a.nneg_dev ? a.nneg_dev[h] : a.nneg_uni;
@@ -234,9 +237,7 @@ __device__ __forceinline__ float2 drain_recip128(uint32_t taddr, float dmax, uin
 
 template <int SMODE>
 __global__ void __launch_bounds__(kGramThreads, 1)
-    gram_bf16_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmC,
-                     const __grid_constant__ CUtensorMap tmRa, const __grid_constant__ CUtensorMap tmCa,
-                     const GramArgs a) {
+    gram_bf16_kernel(const __grid_constant__ GramMaps maps, const GramArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nbox = a.d / 64;
@@ -292,10 +293,14 @@ __global__ void __launch_bounds__(kGramThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      prefetch_tmap(&tmR);
-      prefetch_tmap(&tmC);
-      prefetch_tmap(&tmRa);
-      prefetch_tmap(&tmCa);
+      prefetch_tmap(&maps.R);
+      prefetch_tmap(&maps.C);
+      prefetch_tmap(&maps.Ra);
+      prefetch_tmap(&maps.Ca);
+      prefetch_tmap(&maps.R2);
+      prefetch_tmap(&maps.C2);
+      prefetch_tmap(&maps.Ra2);
+      prefetch_tmap(&maps.Ca2);
       int it = 0, aload = 0;
       bool ok = true;
       Cursor c;
@@ -304,12 +309,15 @@ __global__ void __launch_bounds__(kGramThreads, 1)
         if (L == L0 || c.j == 0) {
           if (aload > 0 && !(ok = mbar_wait(&bars->a_empty, (aload - 1) & 1, abort, a.status))) break;
           const int nact = nact_of(c);
+          const bool alt = tab[c.h].altR != 0;
+          const CUtensorMap* mR = alt ? &maps.R2 : &maps.R;
+          const CUtensorMap* mRa = alt ? &maps.Ra2 : &maps.Ra;
           mbar_arrive_expect_tx(&bars->a_full, nact * (aBytes + aAug));
           for (int r = 0; r < nact; ++r) {
             const int y = c.rOff + c.rb * kGramRowBlock + r * kGramRowTile;
             for (int k = 0; k < nbox; ++k)
-              tma_load_3d(sA + r * aBytes + k * (kGramRowTile * 128), &tmR, &bars->a_full, k * 64, y, c.h);
-            tma_load_3d(sAa + r * aAug, &tmRa, &bars->a_full, 0, y, c.h);  // row form
+              tma_load_3d(sA + r * aBytes + k * (kGramRowTile * 128), mR, &bars->a_full, k * 64, y, c.h);
+            tma_load_3d(sAa + r * aAug, mRa, &bars->a_full, 0, y, c.h);  // row form
           }
           ++aload;
         }
@@ -317,9 +325,12 @@ __global__ void __launch_bounds__(kGramThreads, 1)
         if (!(ok = mbar_wait(&bars->empty[s], ((it / kStages) & 1) ^ 1, abort, a.status))) break;
         mbar_arrive_expect_tx(&bars->full[s], bBytes + bAug);
         const int y = c.cOff + c.j * kColTile;
+        const bool alt = tab[c.h].altC != 0;
+        const CUtensorMap* mC = alt ? &maps.C2 : &maps.C;
+        const CUtensorMap* mCa = alt ? &maps.Ca2 : &maps.Ca;
         for (int k = 0; k < nbox; ++k)
-          tma_load_3d(sB + s * bBytes + k * (kColTile * 128), &tmC, &bars->full[s], k * 64, y, c.h);
-        tma_load_3d(sBa + s * bAug, &tmCa, &bars->full[s], 16, y, c.h);  // column form
+          tma_load_3d(sB + s * bBytes + k * (kColTile * 128), mC, &bars->full[s], k * 64, y, c.h);
+        tma_load_3d(sBa + s * bAug, mCa, &bars->full[s], 16, y, c.h);  // column form
         ++it;
       }
       if (!ok) {
@@ -593,8 +604,7 @@ void gram_plan(GramArgs& a, int max_col_tiles, int n_sm) {
   a.min_steps = m < 1 ? 1 : m;
 }
 
-cudaError_t launch_gram_bf16(const GramArgs& a, const CUtensorMap& tmR, const CUtensorMap& tmC,
-                             const CUtensorMap& tmRa, const CUtensorMap& tmCa, cudaStream_t st) {
+cudaError_t launch_gram_bf16(const GramArgs& a, const GramMaps& m, cudaStream_t st) {
   if (a.H < 1 || a.H > kGramMaxHeads) return cudaErrorInvalidValue;
   const size_t smem = gram_smem_bytes(a.d);
   const int grid = a.grid;
@@ -604,17 +614,17 @@ cudaError_t launch_gram_bf16(const GramArgs& a, const CUtensorMap& tmR, const CU
     e = cudaFuncSetAttribute(gram_bf16_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     LaunchTrace trace("gram_bf16_kernel", st);
-    e = launch_pdl(gram_bf16_kernel<2>, dim3(grid), dim3(kGramThreads), smem, st, tmR, tmC, tmRa, tmCa, a);
+    e = launch_pdl(gram_bf16_kernel<2>, dim3(grid), dim3(kGramThreads), smem, st, m, a);
   } else if (a.s == 1.f) {
     e = cudaFuncSetAttribute(gram_bf16_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     LaunchTrace trace("gram_bf16_kernel", st);
-    e = launch_pdl(gram_bf16_kernel<1>, dim3(grid), dim3(kGramThreads), smem, st, tmR, tmC, tmRa, tmCa, a);
+    e = launch_pdl(gram_bf16_kernel<1>, dim3(grid), dim3(kGramThreads), smem, st, m, a);
   } else {
     e = cudaFuncSetAttribute(gram_bf16_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     LaunchTrace trace("gram_bf16_kernel", st);
-    e = launch_pdl(gram_bf16_kernel<0>, dim3(grid), dim3(kGramThreads), smem, st, tmR, tmC, tmRa, tmCa, a);
+    e = launch_pdl(gram_bf16_kernel<0>, dim3(grid), dim3(kGramThreads), smem, st, m, a);
   }
   return e;
 }

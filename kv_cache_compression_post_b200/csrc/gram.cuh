@@ -45,6 +45,9 @@ struct GramArgs {
   int* status = nullptr;
   // largest ||k||^2 among the rows and columns (null: unknown, always clamp t >= eps)
   const float* norm_max = nullptr;
+  // a head whose row (column) count equals alt_rows_n (alt_cols_n) reads its rows
+  // (columns) through the alternate tensor maps, from row 0; -1: never
+  int alt_rows_n = -1, alt_cols_n = -1;
   // f32 SIMT path only
   const float* R32 = nullptr;      // [H][ldR][d]
   const float* C32 = nullptr;      // [H][ldC][d]
@@ -54,9 +57,13 @@ struct GramArgs {
 // bf16 operands through TMA: tensor maps over [H][rows][d] and over the augmented
 // rows [H][rows][32] (see launch_aug_rows); row maps use 128-row boxes, column maps
 // 256-row boxes (kGramColTile).  The MMA accumulates a.b - (||a||^2 + ||b||^2)/2 =
-// -||a - b||^2 / 2 directly.
-cudaError_t launch_gram_bf16(const GramArgs& a, const CUtensorMap& tmR, const CUtensorMap& tmC,
-                             const CUtensorMap& tmRa, const CUtensorMap& tmCa, cudaStream_t st);
+// -||a - b||^2 / 2 directly.  R2 .. Ca2 are the alternate maps (GramArgs
+// alt_rows_n / alt_cols_n); callers without alternates repeat R .. Ca.
+struct GramMaps {
+  CUtensorMap R, C, Ra, Ca;
+  CUtensorMap R2, C2, Ra2, Ca2;
+};
+cudaError_t launch_gram_bf16(const GramArgs& a, const GramMaps& m, cudaStream_t st);
 // f32 operands, CUDA-core direct differences (small problems).
 cudaError_t launch_gram_f32(const GramArgs& a, cudaStream_t st);
 

@@ -80,10 +80,11 @@ def test_tiny_rollout_matches_oracle_exactly():
     bank.close()
 
 
-def _stepwise(w, p, cfg_kw, label, seed_offset=None):
+def _stepwise(w, p, cfg_kw, label, seed_offset=None, n_cands=None):
     """Every step of the workload's rollout: import the oracle's banks, run one GPU
-    admit, check it against the oracle's step (check_admit_step).  Returns the
-    per-step (near ties, flips)."""
+    admit, check it against the oracle's step (check_admit_step).  n_cands(i, N), if
+    given, keeps only the first n of step i's N candidates.  Returns the per-step
+    (near ties, flips)."""
     import torch
     import kv_cache_compression_post_b200 as kvb
     L = kvgen.LayerInputs(w, 0, tagged=True, seed_offset=seed_offset)
@@ -93,6 +94,9 @@ def _stepwise(w, p, cfg_kw, label, seed_offset=None):
     dtype = "bf16" if w.dtype == "bf16" else "f32"
     for i in range(1, w.n_chunks):
         x = L.step(i)
+        if n_cands is not None:
+            n = n_cands(i, x["cand_ids"].shape[0])
+            x = dict(x, cand_ids=x["cand_ids"][:n], candK=x["candK"][:, :n], candV=x["candV"][:, :n])
         r = dkv.admit(banks, x["cand_ids"], x["candK"], x["candV"], p)
         import_step_state(bank, banks, p, w)
         bank.admit(0, dev_tensor(x["candK"], dtype), dev_tensor(x["candV"], dtype), dev_ids(x["cand_ids"]))
@@ -118,6 +122,17 @@ def test_mid_stepwise_matches_oracle(tau, sync):
     w = kvgen.WORKLOADS["mid"]
     p = dkv.Params(capacity=w.capacity, tau=tau, eps=w.eps, s=w.s, sync_heads=bool(sync))
     _stepwise(w, p, dict(tau=tau, sync=sync), f"mid tau {tau} sync {sync}")
+
+
+def test_mid_stepwise_fewer_candidates():
+    """Steps that pass fewer candidates than max_candidates (the first N' of the
+    chunk's candidates, N' ragged) to a bank that is not empty: the step's
+    per-candidate scratch keeps its max_candidates layout while the candidate
+    block itself is N' rows per head."""
+    w = kvgen.WORKLOADS["mid"]
+    p = dkv.Params(capacity=w.capacity, tau=w.tau, eps=w.eps, s=w.s)
+    _stepwise(w, p, {}, "mid fewer candidates",
+              n_cands=lambda i, N: N - 37 * (i % 3) - (i % 2) * (N // 3))
 
 
 def test_mid_stepwise_pages_preset():
