@@ -122,3 +122,31 @@ def test_attend_full_size_sampled_rows(name, H):
         np.testing.assert_allclose(O[hh][idx], O_ref, atol=ATOL_BF16, rtol=0)
         np.testing.assert_allclose(lse[hh][idx], lse_ref, atol=2e-3, rtol=0)
     bank.close()
+
+
+@pytest.mark.parametrize("nq", [1, 129, 300])
+def test_attend_fewer_queries_than_max(nq):
+    """Nq below max_queries (one query; a ragged second tile; three tiles, so one
+    unit holds a lone tile) with the full window and a bank of ragged sizes."""
+    import kv_cache_compression_post_b200 as kvb
+    w = kvgen.WORKLOADS["mid"]
+    L = kvgen.LayerInputs(w, 0)
+    x = dict(L.step(3))
+    x["Q"] = x["Q"][:, :nq]
+    rng = np.random.default_rng(nq)
+    banks = []
+    for hh in range(w.heads):
+        n = 200 + 37 * hh
+        K = kvgen.round_bf16(rng.standard_normal((n, w.head_dim)).astype(np.float32))
+        V = kvgen.round_bf16(rng.standard_normal((n, w.head_dim)).astype(np.float32))
+        banks.append(dkv.HeadBank(np.arange(n) + 10 ** 6, K.astype(np.float64), V.astype(np.float64), np.ones(n)))
+    p = dkv.Params(capacity=w.capacity)
+    bank = kvb.Bank(_cfg(w))
+    import_oracle_banks(bank, banks, p, w)
+    O, lse = _attend(bank, w, x)
+    for hh in range(w.heads):
+        K, V = dkv.attention_set(banks[hh], x["sinkK"][hh], x["sinkV"][hh], x["winK"][hh], x["winV"][hh])
+        O_ref, lse_ref = attention(x["Q"][hh], K, V)
+        np.testing.assert_allclose(O[hh], O_ref, atol=ATOL_BF16, rtol=0)
+        np.testing.assert_allclose(lse[hh], lse_ref, atol=2e-3, rtol=0)
+    bank.close()
